@@ -1,0 +1,541 @@
+"""Benchmark of the block-scaled quantization hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|weight_x50]
+
+A step is one pass of the whole path over one synthetic tensor of the workload:
+quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
+then dequantize each result to bf16. The default workload is the 4096 x 4096 weight
+(N(0, 0.02^2) with 0.1% entries +-U(0.1, 0.2)) under UINT4 group-128 asymmetric
+(fp16 scale + zero) and INT8 per-output-channel symmetric.
+
+value: algorithmic bytes of every kernel of a step (bytes each kernel must read plus
+bytes it must write) / step time, summed over ranks (weak scaling: each rank owns an
+independent tensor), with inputs resident in HBM. Inputs rotate over enough buffer sets
+that every step reads data last touched more than 4 x L2 ago.
+e2e: the same bytes / step time when every step also copies its input from pinned host
+memory and reads its quantized outputs and QSNR sums back.
+
+Under torchrun (N > 1) each rank drives cuda:LOCAL_RANK; times are the max over ranks.
+--impl reference times the CPU oracle (the reference of this build) on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
+KERNEL_SOURCES = ["common.cuh", "quant_ops.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu"]
+
+# workload -> (generator kwargs, list of (label, scheme args))
+WORKLOADS = {
+    "weight_outliers": [("uint4_g128_asym", ("uint4_asym", "group", 128, "fp16", False)),
+                        ("int8_row_sym", ("int8_sym", "row", 0, "fp32", False))],
+    "tiny_weight": [("int8_tensor_sym", ("int8_sym", "tensor", 0, "fp32", False)),
+                    ("int4_g64_sym", ("int4_sym", "group", 64, "fp32", False))],
+    "activations_t3": [("e4m3_tensor", ("e4m3", "tensor", 0, "fp32", False)),
+                       ("e5m2_tensor", ("e5m2", "tensor", 0, "fp32", False)),
+                       ("e4m3_token", ("e4m3", "row", 0, "fp32", False)),
+                       ("e5m2_token", ("e5m2", "row", 0, "fp32", False))],
+    "ffn_lognormal": [("mxint8", ("int8_sym", "mx", 32, "ue8m0", False)),
+                      ("mxfp8_e4m3", ("e4m3", "mx", 32, "ue8m0", False))],
+    "weight_x50": [("nvfp4", ("e2m1", "nv", 16, "e4m3", False)),
+                   ("nvint4", ("int4_sym", "nv", 16, "e4m3", False)),
+                   ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
+}
+
+
+def gen_input(workload: str, rank: int) -> torch.Tensor:
+    """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
+    if workload == "ffn_lognormal":
+        return synth.ffn_lognormal(rank)
+    gen, _, _ = synth.WORKLOADS[workload]
+    base = {"tiny_weight": 0, "weight_outliers": 1, "activations_t3": 2, "weight_x50": 4}[workload]
+    return gen(seed=base + 1000 * rank)
+
+
+# ---------------------------------------------------------------------------
+# byte accounting
+# ---------------------------------------------------------------------------
+
+def kernel_bytes(sizes, rows: int, cols: int):
+    """Algorithmic bytes of (quantize, dequantize-to-bf16) for one scheme.
+    sizes = (code, scale, zero point, tensor scale) bytes."""
+    cb, sb, zb, tb = sizes
+    x = 2 * rows * cols
+    q = x + cb + sb + zb + tb
+    dq = cb + sb + zb + tb + x
+    return q, dq
+
+
+def aggregate(bytes_per_step_per_rank: float, n_ranks: int, max_ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank moves the same bytes per step; the slowest rank sets the time."""
+    return bytes_per_step_per_rank * n_ranks / (max_ms_per_step * 1e-3) / 1e9
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+        self.t_on = self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.01)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_on(self):
+        self.t_on = time.time()
+
+    def mark_off(self):
+        self.t_off = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            rows.append((t, parts))
+        window = [p for t, p in rows if self.t_on - 0.025 <= t <= self.t_off + 0.025]
+        use = window or [p for _, p in rows]
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return math.nan
+
+        sm = [num(p[2]) for p in use]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in use:
+            for name, v in zip(names, p[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(num(p[3]) for p in use) if use else None,
+                "reasons": sorted(reasons),
+                "samples": len(use), "samples_in_timed_region": len(window)}
+
+
+# ---------------------------------------------------------------------------
+# roofline inputs
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "block_scaled_bit_bq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(label: str, workload: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, if that summary
+    was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_src_hash()
+    for line in open(p):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        kv = dict(item.split("=", 1) for item in line.split() if "=" in item)
+        if kv.get("workload") == workload and kv.get("kernel") == label and kv.get("src_hash") == cur:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import block_scaled_bit_bq_b200 as bq
+    from block_scaled_bit_bq_b200 import Scheme
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    schemes = [(lab, Scheme(*a)) for lab, a in WORKLOADS[args.workload]]
+    x_host = gen_input(args.workload, rank)
+    rows, cols = x_host.shape
+    per_scheme_bytes = [kernel_bytes(bq.bq_buffer_sizes(s, rows, cols), rows, cols) for _, s in schemes]
+    step_bytes = sum(q + d for q, d in per_scheme_bytes)
+
+    # buffer sets: inputs + outputs of every kernel, rotated so that each step touches
+    # memory last used more than 4 x L2 ago
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    set_bytes = step_bytes
+    n_sets = max(2, math.ceil(4 * l2 / set_bytes) + 1)
+    n_sets = min(n_sets, max(2, int(0.5 * torch.cuda.mem_get_info(device)[0] // max(set_bytes, 1))))
+    x_dev = x_host.to(device)
+    sets = []
+    for i in range(n_sets):
+        xi = x_dev if i == 0 else x_dev.clone()
+        outs = [bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes]
+        deqs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in schemes]
+        sets.append((xi, outs, deqs))
+    ws = bq.new_workspace(device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i, evs=None):
+        xi, outs, deqs = sets[i % n_sets]
+        k = 0
+        for (lab, s), q, dq in zip(schemes, outs, deqs):
+            if evs is not None:
+                evs[k].record(stream)
+            bq.bq_quantize(xi, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, stream)
+            if evs is not None:
+                evs[k + 1].record(stream)
+            bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, dq, stream)
+            k += 2
+        if evs is not None:
+            evs[k].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+
+    n_k = 2 * len(schemes)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_k + 1)] for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(vis.split(",")[local_rank].strip() if vis else device.index)
+    if rank == 0:
+        sampler.start()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler.mark_on()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_off()
+    barrier(device)
+    clocks = sampler.stop() if rank == 0 else None
+    ms = t0.elapsed_time(t1) / args.steps
+    ms_max = reduce_max(ms, device)
+
+    # per-kernel mean durations (events between consecutive launches on this stream)
+    per_k = [statistics.fmean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) for k in range(n_k)]
+    kernels = []
+    for j, (lab, s) in enumerate(schemes):
+        qb, db = per_scheme_bytes[j]
+        for kind, nbytes, kms in (("quantize", qb, per_k[2 * j]), ("dequantize", db, per_k[2 * j + 1])):
+            kernels.append({"kernel": f"{kind}:{lab}", "bytes": nbytes, "ms": kms,
+                            "gbs": nbytes / (kms * 1e-3) / 1e9})
+    dom = max(kernels, key=lambda k: k["ms"])
+    peak, peak_kind = measured_peaks()
+
+    # QSNR of the last step (device sums read back after timing)
+    qsnr = {}
+    xi, outs, _ = sets[(args.warmup + args.steps - 1) % n_sets]
+    for (lab, _), q in zip(schemes, outs):
+        st = q.stats.cpu().tolist()
+        qsnr[lab] = {"db": bq.bq_stats_qsnr_db(st), "mean_kappa": (st[2] / st[4]) if st[4] else None}
+
+    # end to end: pinned host input in, quantized outputs + sums out, every step
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_host.pin_memory()
+        xd, outs, deqs = sets[0]
+        host_outs = []
+        d2h = 0
+        for q in outs:
+            hs = []
+            for t in (q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats):
+                if t is None:
+                    hs.append(None)
+                    continue
+                h = torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                hs.append((t, h))
+                d2h += t.numel() * t.element_size()
+            host_outs.append(hs)
+        h2d = x_pin.numel() * x_pin.element_size()
+
+        def e2e_step():
+            xd.copy_(x_pin, non_blocking=True)
+            for (lab, s), q, dq in zip(schemes, outs, deqs):
+                bq.bq_quantize(xd, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, stream)
+                bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, dq, stream)
+            for hs in host_outs:
+                for pair in hs:
+                    if pair is not None:
+                        pair[1].copy_(pair[0], non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(1, min(args.steps, 50))
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
+        e2e = {"value": aggregate(step_bytes, world, e_ms), "unit": "GB/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, schemes_args=WORKLOADS[args.workload], x_host=x_host,
+                           budget_s=args.cpu_seconds)
+
+    value = aggregate(step_bytes, world, ms_max)
+    if rank != 0:
+        return None
+    traffic = ncu_traffic(dom["kernel"], args.workload)
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload} {rows}x{cols} bf16: " + " + ".join(l for l, _ in schemes)
+                        + "; quantize with fused QSNR/kappa, then dequantize to bf16",
+            "rows": rows, "cols": cols,
+            "bytes_per_step_per_gpu": step_bytes,
+            "l2": f"inputs larger than L2: {n_sets} rotating buffer sets of {set_bytes / 2**20:.1f} MiB",
+            "parallelism": f"dp{world} (one independent tensor per GPU, no collective on the data path)",
+        },
+        "pct_hbm_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(dom["gbs"], 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes": dom["bytes"], "peak_source": peak_kind},
+        "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kernels],
+        "qsnr": qsnr,
+        "gpu_launches": args.steps * n_k,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+    }
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_step(xb: np.ndarray, schemes_args):
+    import oracle
+    for _, a in schemes_args:
+        s = oracle.Scheme(*a)
+        r = oracle.quantize(xb, s, stats=True)
+        xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], r["tensor_scale"], xb.shape[0], xb.shape[1], s)
+        oracle.to_bf16_array(xh)
+
+
+def oracle_bytes(schemes_args, rows, cols):
+    import oracle
+    tot = 0
+    for _, a in schemes_args:
+        q, d = kernel_bytes(oracle.buffer_sizes(oracle.Scheme(*a), rows, cols), rows, cols)
+        tot += q + d
+    return tot
+
+
+def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, rows_per_step=None):
+    """Time the oracle, as it stands, on this host (one thread) over whole steps of a
+    row sample of the workload tensor, until budget_s is spent (at least 2 steps)."""
+    xb = synth.bf16_bits(x_host)
+    rows, cols = xb.shape
+    if rows_per_step is None:
+        t = time.perf_counter()
+        oracle_step(xb[: max(1, rows // 32)], schemes_args)
+        per_row = (time.perf_counter() - t) / max(1, rows // 32)
+        rows_per_step = int(min(rows, max(16, budget_s / 4 / max(per_row, 1e-9))))
+    sample = xb[:rows_per_step]
+    nbytes = oracle_bytes(schemes_args, rows_per_step, cols)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(sample, schemes_args)
+        n += 1
+        if n >= 2 and time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows_per_step} of {rows} rows of the {workload} tensor, {n} whole steps "
+                      f"(quantize + dequantize of every scheme) in {dt:.1f} s, single thread"}
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return None
+    schemes_args = WORKLOADS[args.workload]
+    x_host = gen_input(args.workload, 0)
+    xb = synth.bf16_bits(x_host)
+    rows, cols = xb.shape
+    # rows per step so that warmup + steps take about args.cpu_seconds * 6 in total
+    t = time.perf_counter()
+    oracle_step(xb[: max(1, rows // 32)], schemes_args)
+    per_row = (time.perf_counter() - t) / max(1, rows // 32)
+    total_budget = max(30.0, 6 * args.cpu_seconds)
+    rows_per_step = int(min(rows, max(16, total_budget / (args.steps + args.warmup) / max(per_row, 1e-9))))
+    sample = xb[:rows_per_step]
+    nbytes = oracle_bytes(schemes_args, rows_per_step, cols)
+    for _ in range(args.warmup):
+        oracle_step(sample, schemes_args)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sample, schemes_args)
+    dt = time.perf_counter() - t0
+    value = nbytes * args.steps / dt / 1e9
+    desc = (f"first {rows_per_step} of {rows} rows of the {args.workload} tensor per step, "
+            f"{args.steps} steps in {dt:.1f} s, single thread")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload} {rows}x{cols} bf16: " + " + ".join(l for l, _ in schemes_args)
+                   + "; quantize with QSNR/kappa, then dequantize to bf16 (CPU oracle)",
+                   "rows": rows, "cols": cols, "parallelism": "host, one thread"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="weight_outliers")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    pg = False
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        pg = True
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

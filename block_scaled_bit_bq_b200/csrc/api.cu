@@ -1,0 +1,301 @@
+// api.cu -- the C ABI of libbq.so (declared and documented in include/bq.h):
+// argument, shape and alignment checks on the host, buffer sizing, and dispatch to
+// the kernels on the caller's stream. Nothing here allocates device memory.
+#include "common.cuh"
+#include "internal.h"
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+namespace bq {
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+std::atomic<int> g_sm_count[MAX_DEVICES];
+
+struct Plan {
+    int fmt, gran, block, sdt, had;
+    bool four, asym, is_int;
+    uint64_t n;            // elements
+    uint32_t n_chunks;     // n / 16
+    uint64_t n_scales;
+    size_t code_bytes, scale_bytes, zp_bytes, ts_bytes;
+    bool needs_range;      // per-tensor and NV schemes take the range pass first
+};
+
+bool fmt_is_int(int f) { return f == BQ_INT8_SYM || f == BQ_INT8_ASYM || f == BQ_INT4_SYM || f == BQ_UINT4_ASYM; }
+bool fmt_four(int f) { return f == BQ_INT4_SYM || f == BQ_UINT4_ASYM || f == BQ_FP4_E2M1; }
+bool fmt_asym(int f) { return f == BQ_INT8_ASYM || f == BQ_UINT4_ASYM; }
+
+bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
+{
+    if (!s) return BQ_ERR_INVALID_ARG;
+    if (s->reserved != 0 || (s->hadamard != 0 && s->hadamard != 1)) return BQ_ERR_INVALID_ARG;
+    if (s->format < BQ_INT8_SYM || s->format > BQ_FP4_E2M1) return BQ_ERR_INVALID_ARG;
+    if (s->granularity < BQ_PER_TENSOR || s->granularity > BQ_NV_BLOCK) return BQ_ERR_INVALID_ARG;
+    if (s->scale_dtype < BQ_DT_BF16 || s->scale_dtype > BQ_DT_E4M3) return BQ_ERR_INVALID_ARG;
+    std::memset(p, 0, sizeof *p);
+    p->fmt = s->format; p->gran = s->granularity; p->sdt = s->scale_dtype; p->had = s->hadamard;
+    p->four = fmt_four(p->fmt); p->asym = fmt_asym(p->fmt); p->is_int = fmt_is_int(p->fmt);
+
+    switch (p->gran) {
+    case BQ_PER_TENSOR:
+    case BQ_PER_ROW:
+        if (p->fmt == BQ_FP4_E2M1) return BQ_ERR_UNSUPPORTED;
+        if (p->sdt != BQ_DT_FP32 && p->sdt != BQ_DT_FP16) return BQ_ERR_UNSUPPORTED;
+        p->block = 0;
+        break;
+    case BQ_PER_GROUP:
+        if (p->fmt == BQ_FP4_E2M1) return BQ_ERR_UNSUPPORTED;
+        if (p->sdt != BQ_DT_FP32 && p->sdt != BQ_DT_FP16) return BQ_ERR_UNSUPPORTED;
+        if (!(s->block == 16 || s->block == 32 || s->block == 64 || s->block == 128 ||
+              s->block == 256 || s->block == 512)) return BQ_ERR_UNSUPPORTED;
+        p->block = s->block;
+        break;
+    case BQ_MX_BLOCK:
+        if (!(p->fmt == BQ_INT8_SYM || p->fmt == BQ_FP8_E4M3 || p->fmt == BQ_FP8_E5M2 || p->fmt == BQ_FP4_E2M1))
+            return BQ_ERR_UNSUPPORTED;
+        if (!(s->block == 32 || s->block == 0) || p->sdt != BQ_DT_UE8M0) return BQ_ERR_UNSUPPORTED;
+        p->block = 32;
+        break;
+    case BQ_NV_BLOCK:
+        if (!(p->fmt == BQ_FP4_E2M1 || p->fmt == BQ_INT4_SYM)) return BQ_ERR_UNSUPPORTED;
+        if (!(s->block == 16 || s->block == 0) || p->sdt != BQ_DT_E4M3) return BQ_ERR_UNSUPPORTED;
+        p->block = 16;
+        break;
+    }
+    if (rows < 0 || cols <= 0 || cols % 16 != 0) return BQ_ERR_SHAPE;
+    if (p->block && cols % p->block != 0) return BQ_ERR_SHAPE;
+    if (rows > 0 && (uint64_t)rows > ((1ull << 36) - 16) / (uint64_t)cols) return BQ_ERR_SHAPE;
+    if (rows >= (1ll << 31) || cols >= (1ll << 31)) return BQ_ERR_SHAPE;
+
+    p->n = (uint64_t)rows * (uint64_t)cols;
+    p->n_chunks = (uint32_t)(p->n / 16);
+    switch (p->gran) {
+    case BQ_PER_TENSOR: p->n_scales = 1; break;
+    case BQ_PER_ROW: p->n_scales = (uint64_t)rows; break;
+    default: p->n_scales = p->n / (uint64_t)p->block; break;
+    }
+    const size_t se = (p->sdt == BQ_DT_FP32) ? 4 : (p->sdt == BQ_DT_FP16) ? 2 : 1;
+    p->code_bytes = p->four ? p->n / 2 : p->n;
+    p->scale_bytes = p->n_scales * se;
+    p->zp_bytes = p->asym ? p->n_scales * se : 0;
+    p->ts_bytes = p->gran == BQ_NV_BLOCK ? 4 : 0;
+    p->needs_range = (p->gran == BQ_PER_TENSOR || p->gran == BQ_NV_BLOCK);
+    return BQ_OK;
+}
+
+bool aligned32(const void* ptr) { return ((uintptr_t)ptr & 31u) == 0; }
+
+size_t ws_needed(const Plan& p, bool stats) { return (stats || p.needs_range) ? WS_BYTES : 0; }
+
+int kind_of(int gran)
+{
+    switch (gran) {
+    case BQ_PER_TENSOR: return K_TENSOR;
+    case BQ_PER_GROUP: return K_GROUP;
+    case BQ_MX_BLOCK: return K_MX;
+    default: return K_NV;
+    }
+}
+
+int scale_kind(const Plan& p)
+{
+    if (p.gran == BQ_MX_BLOCK) return SK_UE8M0;
+    if (p.gran == BQ_NV_BLOCK) return SK_NV;
+    return p.sdt == BQ_DT_FP16 ? SK_F16 : SK_F32;
+}
+
+DequantArgs dequant_args(const Plan& p, int64_t cols)
+{
+    DequantArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.n_chunks = p.n_chunks;
+    a.n_dtiles = (uint32_t)((p.n_chunks + 63u) / 64u);
+    uint32_t cpu = 0;
+    switch (p.gran) {
+    case BQ_PER_TENSOR: cpu = 0; break;
+    case BQ_PER_ROW: cpu = (uint32_t)(cols / 16); break;
+    default: cpu = (uint32_t)(p.block / 16); break;
+    }
+    a.chunks_per_unit = cpu;
+    if (cpu) {
+        const FastDiv f = make_fastdiv(cpu);
+        a.fd_m = f.m;
+        a.fd_s = f.s;
+    }
+    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+    return a;
+}
+
+bq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA; }
+
+}  // namespace
+
+int device_sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) dev = 0;
+    int v = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        g_sm_count[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+size_t workspace_bytes() { return WS_BYTES; }
+
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" {
+
+const char* bq_status_string(int status)
+{
+    switch (status) {
+    case BQ_OK: return "BQ_OK";
+    case BQ_ERR_INVALID_ARG: return "BQ_ERR_INVALID_ARG: null pointer or bad enum value";
+    case BQ_ERR_UNSUPPORTED: return "BQ_ERR_UNSUPPORTED: format / granularity / scale dtype combination not offered";
+    case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE: rows < 0, cols not a positive multiple of 16 (and of the block), or too large";
+    case BQ_ERR_ALIGNMENT: return "BQ_ERR_ALIGNMENT: x, codes and out must be 32-byte aligned";
+    case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE: workspace missing or too small";
+    case BQ_ERR_CUDA: return "BQ_ERR_CUDA: a CUDA launch or call failed";
+    default: return "unknown bq_status";
+    }
+}
+
+const char* bq_version(void) { return "bq 0.1 (sm_100a)"; }
+
+bq_status bq_buffer_sizes(const bq_scheme* scheme, int64_t rows, int64_t cols,
+                          size_t* code_bytes, size_t* scale_bytes,
+                          size_t* zero_point_bytes, size_t* tensor_scale_bytes)
+{
+    Plan p;
+    const bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (code_bytes) *code_bytes = p.code_bytes;
+    if (scale_bytes) *scale_bytes = p.scale_bytes;
+    if (zero_point_bytes) *zero_point_bytes = p.zp_bytes;
+    if (tensor_scale_bytes) *tensor_scale_bytes = p.ts_bytes;
+    return BQ_OK;
+}
+
+bq_status bq_workspace_size(const bq_scheme* scheme, int64_t rows, int64_t cols, int with_stats, size_t* bytes)
+{
+    Plan p;
+    const bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (!bytes) return BQ_ERR_INVALID_ARG;
+    *bytes = ws_needed(p, with_stats != 0);
+    return BQ_OK;
+}
+
+bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                      const bq_scheme* scheme,
+                      void* codes, void* scales, void* zero_points, float* tensor_scale,
+                      bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    const bool want_stats = stats != nullptr;
+    const size_t need_ws = ws_needed(p, want_stats);
+    if (need_ws && (!workspace || workspace_bytes < need_ws)) return BQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (p.n == 0) {
+        if (want_stats) return cuda_status(cudaMemsetAsync(stats, 0, sizeof(bq_stats), s));
+        return BQ_OK;
+    }
+    if (!x || !codes || !scales) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const uint32_t* xw = reinterpret_cast<const uint32_t*>(x);
+
+    if (p.needs_range) {
+        const cudaError_t e = launch_range(xw, p.n_chunks, p.had != 0, p.gran == BQ_PER_TENSOR && p.asym, ws, s);
+        if (e != cudaSuccess) return BQ_ERR_CUDA;
+    }
+    if (p.gran == BQ_PER_ROW) {
+        RowArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cpr = (uint32_t)(cols / 16);
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.inv_cols = 1.0f / (float)cols;
+        return cuda_status(launch_quant_row(p.fmt, p.had != 0, want_stats, a, s));
+    }
+    FlatArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+    a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
+    a.n_chunks = p.n_chunks;
+    a.n_dtiles = (uint32_t)((p.n_chunks + 63u) / 64u);
+    a.lanes_per_group = p.gran == BQ_PER_GROUP ? p.block / 16 : 1;
+    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+    a.n_elems = (double)p.n;
+    a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
+    return cuda_status(launch_quant_flat(p.fmt, kind_of(p.gran), p.had != 0, want_stats, a, s));
+}
+
+bq_status bq_dequantize(const void* codes, const void* scales, const void* zero_points,
+                        const float* tensor_scale, int64_t rows, int64_t cols,
+                        const bq_scheme* scheme, void* out, int32_t out_dtype, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (out_dtype != BQ_DT_BF16 && out_dtype != BQ_DT_FP32) return BQ_ERR_UNSUPPORTED;
+    if (p.n == 0) return BQ_OK;
+    if (!codes || !scales || !out) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(codes) || !aligned32(out)) return BQ_ERR_ALIGNMENT;
+    DequantArgs a = dequant_args(p, cols);
+    a.codes = reinterpret_cast<const uint8_t*>(codes);
+    a.scales = scales; a.zps = zero_points; a.tensor_scale = tensor_scale; a.out = out;
+    return cuda_status(launch_dequant(p.fmt, scale_kind(p), p.had != 0, out_dtype, a,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void* scales,
+                  const void* zero_points, const float* tensor_scale,
+                  int64_t rows, int64_t cols, const bq_scheme* scheme,
+                  bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    if (!stats) return BQ_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < WS_BYTES) return BQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (p.n == 0) return cuda_status(cudaMemsetAsync(stats, 0, sizeof(bq_stats), s));
+    if (!x || !codes || !scales) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    DequantArgs a = dequant_args(p, cols);
+    a.codes = reinterpret_cast<const uint8_t*>(codes);
+    a.scales = scales; a.zps = zero_points; a.tensor_scale = tensor_scale;
+    a.x = reinterpret_cast<const uint32_t*>(x);
+    a.stats = stats;
+    a.ws = reinterpret_cast<uint8_t*>(workspace);
+    return cuda_status(launch_qsnr(p.fmt, scale_kind(p), p.had != 0, a, s));
+}
+
+double bq_stats_qsnr_db(const bq_stats* host_stats)
+{
+    if (!host_stats) return NAN;
+    if (host_stats->err2 == 0.0) return INFINITY;
+    return -10.0 * std::log10(host_stats->err2 / host_stats->x2);
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// internal.h -- launch interface between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "bq.h"
+
+namespace bq {
+
+// Arguments of the one-pass kernels that see the tensor as a flat run of 16-element
+// chunks (per-tensor, per-group, MX and NV granularities). Groups never straddle rows
+// because cols is a multiple of the group size.
+struct FlatArgs {
+    const uint32_t* x;          // bf16 pairs
+    uint8_t* codes;
+    void* scales;
+    void* zps;
+    float* tensor_scale;
+    bq_stats* stats;
+    uint8_t* ws;
+    uint32_t n_chunks;          // rows * cols / 16
+    uint32_t n_dtiles;          // ceil(n_chunks / 64): a warp takes 64 chunks per step
+    int32_t lanes_per_group;    // per-group: block / 16 (power of two, <= 32)
+    int32_t scale_fp16;         // 1: fp16 scales and zero points
+    double n_elems;
+    float inv_unit;             // 1 / elements per scaling unit (kappa)
+};
+
+// Per-row kernel: one CTA per row at a time.
+struct RowArgs {
+    const uint32_t* x;
+    uint8_t* codes;
+    void* scales;
+    void* zps;
+    bq_stats* stats;
+    uint8_t* ws;
+    uint32_t rows;
+    uint32_t cpr;               // chunks per row = cols / 16
+    int32_t scale_fp16;
+    float inv_cols;
+};
+
+struct DequantArgs {
+    const uint8_t* codes;
+    const void* scales;
+    const void* zps;
+    const float* tensor_scale;
+    void* out;
+    const uint32_t* x;          // QSNR only
+    bq_stats* stats;            // QSNR only
+    uint8_t* ws;                // QSNR only
+    uint32_t n_chunks;
+    uint32_t n_dtiles;
+    uint32_t chunks_per_unit;   // chunks sharing one scale (0: one scale for the tensor)
+    uint32_t fd_m, fd_s;        // fast division by chunks_per_unit
+    int32_t scale_fp16;
+};
+
+// Scale kinds for dequantize / QSNR.
+enum { SK_F32 = 0, SK_F16 = 1, SK_UE8M0 = 2, SK_NV = 3 };
+
+int device_sm_count();
+size_t workspace_bytes();
+
+cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool hadamard, bool minmax,
+                         uint8_t* ws, cudaStream_t st);
+cudaError_t launch_quant_flat(int fmt, int kind, bool hadamard, bool stats, const FlatArgs& a,
+                              cudaStream_t st);
+cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& a, cudaStream_t st);
+cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
+                           cudaStream_t st);
+cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);
+
+}  // namespace bq

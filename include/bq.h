@@ -1,0 +1,192 @@
+/*
+ * bq.h -- C ABI of the block-scaled tensor quantization library (libbq.so).
+ *
+ * One NVIDIA B200 (sm_100a). Every entry point takes plain pointers and sizes; all
+ * tensors are caller-owned device memory unless a parameter says "host". Work is
+ * enqueued on the caller's CUDA stream (passed as void*, a cudaStream_t; NULL is the
+ * legacy default stream) and results are valid after the caller synchronizes that
+ * stream. No entry point allocates device memory, throws, or falls back to the CPU.
+ * Argument, shape and alignment checks run on the host before any launch; a failed
+ * check launches nothing. A launch failure returns BQ_ERR_CUDA.
+ *
+ * Method (source pages cited by title and section):
+ *  - AbsMax scale s = max|X| / Qmax and Xq = clip(round(X/s), Qmin, Qmax) * s:
+ *    "INT vs FP at fine granularity" §2.1; granularity per tensor / per channel /
+ *    per block: same page §3.1.
+ *  - Affine INT: q = round(w/scale) + zero_point, w = scale * (q - zero_point):
+ *    "INT4/INT8/FP8 quantization" §INT8; INT4 [-8, 7] groups, two codes per byte:
+ *    same page §INT4; E4M3 +-448, E5M2 +-57344: same page §FP8.
+ *  - FP element formats E2M1 / E4M3 / E5M2 and their bit layouts: "Quantization
+ *    survey" §4.1; MX (block 32, power-of-two E8M0 scale) and NV (block 16, E4M3
+ *    block scale plus an FP32 tensor scale, x = x_q * s_block * S_tensor): same page
+ *    §4.3.1 and §4.3.2.
+ *  - Hadamard rotation before quantizing: "INT vs FP at fine granularity" §4.2 and
+ *    §7.2; orthogonal rotation R^T R = I: "Quantization survey" §5.3.
+ *  - QSNR = -10 log10(||X - Xq||^2 / ||X||^2) and the crest factor kappa:
+ *    "INT vs FP at fine granularity" §4.1.
+ *
+ * Arithmetic contract (bit-exact with the library's CPU oracle):
+ *  - inputs are bf16, widened exactly to fp32; scales and quotients are fp32;
+ *  - every code is decided from the correctly rounded fp32 quotient x / s (round half
+ *    to even for INT, round-to-nearest-even with saturation to the largest finite
+ *    value for FP element formats; the sign of an FP zero is kept);
+ *  - the quantizer divides by the scale as stored (an fp16 scale is rounded first,
+ *    saturating at 65504);
+ *  - asymmetric INT: min' = min(min, 0), max' = max(max, 0), s = (max' - min') / L
+ *    (L = 255 or 15), zp = clamp(Qmin + round(-min'/s)), q = clamp(round(x/s) + zp);
+ *  - MX: the scale exponent e is the smallest integer with amax <= Qmax * 2^e,
+ *    clamped to [-127, 127] (amax = 0 gives -127), stored as e + 127;
+ *  - NV: S = A / (Qmax * 448) over the whole tensor; s_b = E4M3((amax_b / Qmax) / S);
+ *    d = s_b * S; code = enc(x / d), zero codes where d = 0; dequant (code * s_b) * S;
+ *  - Hadamard: each run of 16 elements along a row is replaced by H16 x / 4
+ *    (Sylvester order, butterfly stages h = 1, 2, 4, 8 of (a+b, a-b), then * 0.25);
+ *    the per-tensor range is taken on rotated values; dequantize applies the same
+ *    transform again (it is its own inverse).
+ *
+ * Layouts (row-major, rows x cols input):
+ *  - codes: 8-bit formats uint8 [rows, cols]; 4-bit formats uint8 [rows, cols/2], element
+ *    2j in the low nibble of byte j; INT codes are two's complement (UINT4 unsigned);
+ *  - scales: per tensor 1 value; per row [rows]; per group [rows, cols/block]; MX uint8
+ *    [rows, cols/32] (UE8M0 codes); NV uint8 [rows, cols/16] (E4M3 codes);
+ *    fp32 or fp16 as scheme.scale_dtype says for the first three;
+ *  - zero points (asymmetric formats only): same shape and dtype as the scales,
+ *    holding exact integers;
+ *  - tensor_scale: one fp32 (NV only).
+ *
+ * Shapes: rows >= 0, cols > 0, cols % 16 == 0 (and cols % block == 0); rows * cols <
+ * 2^36. rows == 0 is a valid empty call. Alignment: x, codes and out 32-byte aligned.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bq_status {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1,   /* null pointer where one is required, bad enum value */
+    BQ_ERR_UNSUPPORTED = 2,   /* format x granularity x scale dtype not offered */
+    BQ_ERR_SHAPE = 3,         /* negative rows, cols not a multiple of 16 / block, too large */
+    BQ_ERR_ALIGNMENT = 4,     /* x, codes or out not 32-byte aligned */
+    BQ_ERR_WORKSPACE = 5,     /* workspace missing or smaller than bq_workspace_size() */
+    BQ_ERR_CUDA = 6           /* a CUDA call failed (see cudaGetLastError on the caller side) */
+} bq_status;
+
+/* data and scale dtypes */
+enum { BQ_DT_BF16 = 0, BQ_DT_FP16 = 1, BQ_DT_FP32 = 2, BQ_DT_UE8M0 = 3, BQ_DT_E4M3 = 4 };
+
+/* element formats */
+enum {
+    BQ_INT8_SYM = 0,     /* [-127, 127], s = amax / 127                        */
+    BQ_INT8_ASYM = 1,    /* [-128, 127] with zero point, 255 levels            */
+    BQ_INT4_SYM = 2,     /* [-8, 7], s = amax / 7 ([-7, 7] under NV: NVINT4)   */
+    BQ_UINT4_ASYM = 3,   /* [0, 15] with zero point, 15 levels                 */
+    BQ_FP8_E4M3 = 4,     /* +-448                                              */
+    BQ_FP8_E5M2 = 5,     /* +-57344                                            */
+    BQ_FP4_E2M1 = 6      /* +-6 (MX or NV granularity only)                    */
+};
+
+/* scaling granularity */
+enum {
+    BQ_PER_TENSOR = 0,   /* one scale; per-tensor range pass first (needs a workspace) */
+    BQ_PER_ROW = 1,      /* one scale per row (output channel of a weight, or token)   */
+    BQ_PER_GROUP = 2,    /* block in {16, 32, 64, 128, 256, 512} contiguous along a row */
+    BQ_MX_BLOCK = 3,     /* block 32, UE8M0 scale: INT8_SYM, E4M3, E5M2, E2M1          */
+    BQ_NV_BLOCK = 4      /* block 16, E4M3 scale + fp32 tensor scale: E2M1, INT4_SYM    */
+};
+
+typedef struct bq_scheme {
+    int32_t format;       /* BQ_INT8_SYM ...                                     */
+    int32_t granularity;  /* BQ_PER_TENSOR ...                                   */
+    int32_t block;        /* group size for BQ_PER_GROUP; 32 for MX, 16 for NV;  */
+                          /* ignored (0) for per-tensor / per-row                */
+    int32_t scale_dtype;  /* BQ_DT_FP32 or BQ_DT_FP16 (tensor/row/group),        */
+                          /* BQ_DT_UE8M0 (MX), BQ_DT_E4M3 (NV)                    */
+    int32_t hadamard;     /* 0 or 1: rotate each 16-run by H16/4 before scaling  */
+    int32_t reserved;     /* must be 0                                           */
+} bq_scheme;
+
+/* QSNR and crest-factor sums, written by the library into caller device memory.
+ * err2 = sum (x - xhat)^2 and x2 = sum x^2 over the whole tensor (original domain);
+ * kappa_* over the scaling units (block, group, row, or the tensor), each unit's
+ * kappa = amax / sqrt(mean of squares) of the values it quantizes (rotated values
+ * when hadamard = 1); units whose sum of squares is zero are not counted. */
+typedef struct bq_stats {
+    double err2;
+    double x2;
+    double kappa_sum;
+    double kappa_max;
+    double n_units;       /* an exact integer */
+} bq_stats;
+
+/* A readable name for a status code (static storage; never NULL). */
+const char* bq_status_string(int status);
+
+/* Library version string (static storage). */
+const char* bq_version(void);
+
+/* Byte sizes of the four outputs of bq_quantize for this scheme and shape (host
+ * pointers; any may be NULL). Zero-point and tensor-scale sizes are 0 when the
+ * scheme has none. Validates the scheme and shape like bq_quantize. */
+bq_status bq_buffer_sizes(const bq_scheme* scheme, int64_t rows, int64_t cols,
+                          size_t* code_bytes, size_t* scale_bytes,
+                          size_t* zero_point_bytes, size_t* tensor_scale_bytes);
+
+/* Device workspace needed by bq_quantize / bq_qsnr for this scheme and shape (host
+ * pointer out). It is 0 when the call needs none (no stats and not per-tensor or NV).
+ * The workspace holds the cross-CTA partial sums and the per-tensor range; it must be
+ * zero-filled once after allocation (the library leaves its counters at zero after
+ * every call) and must not be used by two calls that can run at the same time. */
+bq_status bq_workspace_size(const bq_scheme* scheme, int64_t rows, int64_t cols,
+                            int with_stats, size_t* bytes);
+
+/*
+ * Quantize x [rows, cols] (device, dtype x_dtype = BQ_DT_BF16) into codes, scales,
+ * zero_points (asymmetric formats; else may be NULL) and tensor_scale (NV; else may
+ * be NULL), all device buffers of the sizes bq_buffer_sizes gives.
+ * stats (device, may be NULL): when given, the QSNR and kappa sums of this call are
+ * written there, reduced in a fixed order (bit-reproducible on a given GPU).
+ * workspace / workspace_bytes: device scratch of at least bq_workspace_size() bytes
+ * (NULL / 0 when that size is 0).
+ * Per-tensor and NV schemes take two passes over x (range, then quantize); all other
+ * schemes take one.
+ */
+bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                      const bq_scheme* scheme,
+                      void* codes, void* scales, void* zero_points, float* tensor_scale,
+                      bq_stats* stats, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * Dequantize codes (+ scales, zero_points, tensor_scale as written by bq_quantize)
+ * into out [rows, cols] (device) of dtype out_dtype = BQ_DT_BF16 (round to nearest
+ * even from the fp32 value) or BQ_DT_FP32. Applies the inverse rotation when
+ * scheme->hadamard is set. One pass; needs no workspace.
+ */
+bq_status bq_dequantize(const void* codes, const void* scales, const void* zero_points,
+                        const float* tensor_scale, int64_t rows, int64_t cols,
+                        const bq_scheme* scheme, void* out, int32_t out_dtype,
+                        void* stream);
+
+/*
+ * QSNR sums of x against the dequantized codes, computed in one pass without writing
+ * the dequantized tensor: stats->err2 and stats->x2 (original domain); the kappa
+ * fields are written as zero. Needs a workspace of bq_workspace_size(..., 1, ...).
+ */
+bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void* scales,
+                  const void* zero_points, const float* tensor_scale,
+                  int64_t rows, int64_t cols, const bq_scheme* scheme,
+                  bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
+
+/* -10 log10(err2 / x2) from a host copy of the stats (+inf when err2 = 0). */
+double bq_stats_qsnr_db(const bq_stats* host_stats);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */
