@@ -30,7 +30,9 @@
  *     saturate to the largest finite value ("satfinite"); the sign of a value that
  *     rounds to zero is kept;
  *   - asymmetric ranges include zero: min' = min(min, 0), max' = max(max, 0);
- *     zero_point = Qmin + round(-min'/s), clamped; q = clamp(round(x/s) + zp);
+ *     zero_point = Qmin + round(-min'/s), clamped; q = clamp(round(x/s) + zp); a range
+ *     whose fp32 scale would overflow saturates at the largest finite fp32 value;
+ *   - clamping applies to the rounded quotient whatever its magnitude;
  *   - the quantizer divides by the scale as stored (fp16 scales are rounded first,
  *     with saturation to 65504);
  *   - MX exponent: the smallest integer e with amax <= Qmax * 2^e, decided exactly,
@@ -49,6 +51,7 @@
  * "parity unpinned".
  */
 
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -307,6 +310,16 @@ static float read_scale(const void* arr, int64_t i, int sdt)
 
 static int clampi(int v, int lo, int hi) { return v < lo ? lo : v > hi ? hi : v; }
 
+/* clamp(round_half_even(v) + add, lo, hi) for any finite or infinite v: the clamp
+ * applies to the rounded value whatever its magnitude (no out-of-range int conversion). */
+static int round_clamp(float v, int add, int lo, int hi)
+{
+    float r = rintf(v);
+    if (r < -1.0e9f) return lo;
+    if (r > 1.0e9f) return hi;
+    return clampi((int)r + add, lo, hi);
+}
+
 static void put_code(uint8_t* codes, int64_t row, int64_t cols, int64_t j, unsigned c, int bits4)
 {
     if (!bits4) { codes[row * cols + j] = (uint8_t)c; return; }
@@ -382,7 +395,7 @@ static void quant_unit(const scheme* s, const float* y, int64_t n, unit_range ur
             float v = y[i] * p;
             float val;
             if (s->is_int) {
-                int q = clampi((int)rintf(v), s->qmin, s->qmax);
+                int q = round_clamp(v, 0, s->qmin, s->qmax);
                 code[i] = (unsigned)q & 0xFFu;
                 val = (float)q;
             } else {
@@ -405,11 +418,11 @@ static void quant_unit(const scheme* s, const float* y, int64_t n, unit_range ur
         *scale_code = (uint8_t)sbc;
         float d = sbv * S;
         for (int64_t i = 0; i < n; i++) {
-            if (d == 0.0f) { code[i] = 0; yhat[i] = 0.0f; continue; }
+            if (!(d > 0.0f)) { code[i] = 0; yhat[i] = 0.0f; continue; }
             float v = y[i] / d;
             float val;
             if (s->is_int) {
-                int q = clampi((int)rintf(v), s->qmin, s->qmax);
+                int q = round_clamp(v, 0, s->qmin, s->qmax);
                 code[i] = (unsigned)q & 0xFu;
                 val = (float)q;
             } else {
@@ -426,14 +439,15 @@ static void quant_unit(const scheme* s, const float* y, int64_t n, unit_range ur
         float mn = ur.mn < 0.0f ? ur.mn : 0.0f;
         float mx = ur.mx > 0.0f ? ur.mx : 0.0f;
         float s32 = (mx - mn) / s->qscale;
+        if (s32 > FLT_MAX) s32 = FLT_MAX;          /* a range beyond fp32 saturates */
         float sc = store_scale(s32, s->sdt);
         int zp;
-        if (sc > 0.0f) zp = clampi(s->qmin + (int)rintf(-mn / sc), s->qmin, s->qmax);
+        if (sc > 0.0f) zp = round_clamp(-mn / sc, s->qmin, s->qmin, s->qmax);
         else zp = s->qmin;
         *scale_out = sc;
         *zp_out = (float)zp;
         for (int64_t i = 0; i < n; i++) {
-            int q = sc > 0.0f ? clampi((int)rintf(y[i] / sc) + zp, s->qmin, s->qmax) : zp;
+            int q = sc > 0.0f ? round_clamp(y[i] / sc, zp, s->qmin, s->qmax) : zp;
             code[i] = (unsigned)q & (s->bits4 ? 0xFu : 0xFFu);
             yhat[i] = sc * (float)(q - zp);
         }
@@ -446,7 +460,7 @@ static void quant_unit(const scheme* s, const float* y, int64_t n, unit_range ur
         if (!(sc > 0.0f)) { code[i] = 0; yhat[i] = 0.0f; continue; }
         float v = y[i] / sc;
         if (s->is_int) {
-            int q = clampi((int)rintf(v), s->qmin, s->qmax);
+            int q = round_clamp(v, 0, s->qmin, s->qmax);
             code[i] = (unsigned)q & (s->bits4 ? 0xFu : 0xFFu);
             yhat[i] = (float)q * sc;
         } else {

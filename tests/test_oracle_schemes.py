@@ -321,3 +321,30 @@ def test_tensor_range_subset_matches_full_call():
     part = oracle.quantize(x[10:20], s, tensor_range=tr)
     assert np.array_equal(part["codes"], full["codes"][10:20])
     assert np.array_equal(part["scales"], full["scales"])
+
+
+def test_clamp_applies_to_the_rounded_quotient_at_any_magnitude():
+    # "INT vs FP at fine granularity" §2.1: clip(round(X/s), Qmin, Qmax). An fp16 scale
+    # saturates at 65504, so x / s is ~4.6e33 for x ~ 3e38: the codes saturate at
+    # +-Qmax with the sign of x.
+    big = 1.5 * 2.0 ** 127                                        # exact in bf16
+    x = _bits_of([big if i % 2 == 0 else -big for i in range(16)]).reshape(1, 16)
+    x = np.ascontiguousarray(x)
+    r = oracle.quantize(x, Scheme("int8_sym", "tensor", scale_dtype="fp16"))
+    assert r["scales"].tolist() == [0x7BFF]                      # 65504 in fp16
+    assert r["codes"].view(np.int8).reshape(-1).tolist() == [127, -127] * 8
+    r = oracle.quantize(x, Scheme("int4_sym", "group", 16, "fp16"))
+    # INT4 clamps to its full range [-8, 7] ("INT4/INT8/FP8 quantization" §INT4)
+    assert r["codes"].reshape(-1).tolist() == [0x87] * 8          # +7 low nibble, -8 high nibble
+
+
+def test_asymmetric_range_beyond_fp32_saturates():
+    # max' - min' overflows fp32 for a unit holding +-3e38: the scale saturates at the
+    # largest finite fp32 value (reading), and the codes stay in range.
+    vals = [1.5 * 2.0 ** 127, -1.5 * 2.0 ** 127] + [0.0] * 14
+    x = _bits_of(vals).reshape(1, 16)
+    r = oracle.quantize(np.ascontiguousarray(x), Scheme("int8_asym", "tensor"))
+    assert r["scales"].view(np.uint32).tolist() == [0x7F7FFFFF]
+    zp = int(r["zps"][0])
+    q = r["codes"].view(np.int8).reshape(-1).astype(int)
+    assert -128 <= zp <= 127 and q.min() >= -128 and q.max() <= 127
