@@ -88,6 +88,7 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
 }
 
 bool aligned32(const void* ptr) { return ((uintptr_t)ptr & 31u) == 0; }
+bool aligned4(const void* ptr) { return ((uintptr_t)ptr & 3u) == 0; }
 
 size_t ws_needed(const Plan& p, bool stats) { return (stats || p.needs_range) ? WS_BYTES : 0; }
 
@@ -161,7 +162,7 @@ const char* bq_status_string(int status)
     case BQ_ERR_INVALID_ARG: return "BQ_ERR_INVALID_ARG: null pointer or bad enum value";
     case BQ_ERR_UNSUPPORTED: return "BQ_ERR_UNSUPPORTED: format / granularity / scale dtype combination not offered";
     case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE: rows < 0, cols not a positive multiple of 16 (and of the block), or too large";
-    case BQ_ERR_ALIGNMENT: return "BQ_ERR_ALIGNMENT: x, codes and out must be 32-byte aligned";
+    case BQ_ERR_ALIGNMENT: return "BQ_ERR_ALIGNMENT: x, codes and out must be 32-byte aligned, scales, zero points and tensor scale 4-byte aligned";
     case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE: workspace missing or too small";
     case BQ_ERR_CUDA: return "BQ_ERR_CUDA: a CUDA launch or call failed";
     default: return "unknown bq_status";
@@ -215,6 +216,7 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
     if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
     if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points) || !aligned4(tensor_scale)) return BQ_ERR_ALIGNMENT;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     const uint32_t* xw = reinterpret_cast<const uint32_t*>(x);
 
@@ -238,7 +240,8 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
     a.n_chunks = p.n_chunks;
     a.n_dtiles = (uint32_t)((p.n_chunks + 63u) / 64u);
-    a.lanes_per_group = p.gran == BQ_PER_GROUP ? p.block / 16 : 1;
+    // units of 16 elements are lane-local (0); larger units span block / 32 lanes
+    a.lanes_per_group = (p.gran == BQ_PER_GROUP && p.block > 16) ? p.block / 32 : (p.gran == BQ_PER_GROUP ? 0 : 1);
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     a.n_elems = (double)p.n;
     a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
@@ -258,6 +261,7 @@ bq_status bq_dequantize(const void* codes, const void* scales, const void* zero_
     if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
     if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
     if (!aligned32(codes) || !aligned32(out)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points) || !aligned4(tensor_scale)) return BQ_ERR_ALIGNMENT;
     DequantArgs a = dequant_args(p, cols);
     a.codes = reinterpret_cast<const uint8_t*>(codes);
     a.scales = scales; a.zps = zero_points; a.tensor_scale = tensor_scale; a.out = out;
@@ -282,6 +286,7 @@ bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void*
     if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
     if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
     if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points) || !aligned4(tensor_scale)) return BQ_ERR_ALIGNMENT;
     DequantArgs a = dequant_args(p, cols);
     a.codes = reinterpret_cast<const uint8_t*>(codes);
     a.scales = scales; a.zps = zero_points; a.tensor_scale = tensor_scale;

@@ -34,9 +34,9 @@ enum { K_TENSOR = 0, K_GROUP = 1, K_MX = 2, K_NV = 3 };
 // to even) and leaves that integer, two's complement, in the low bits of the sum.
 constexpr float MAGIC = 12582912.0f;
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;
-// Reciprocal bracket factors 1 -+ 2^-21 (both exact in fp32).
-constexpr float BRACKET_LO = 0.999999523162841796875f;
-constexpr float BRACKET_HI = 1.000000476837158203125f;
+// Reciprocal bracket factors 1 -+ 2^-20 (both exact in fp32).
+constexpr float BRACKET_LO = 0.99999904632568359375f;
+constexpr float BRACKET_HI = 1.00000095367431640625f;
 constexpr float FP32_MIN_NORMAL = 1.17549435082228750797e-38f;
 
 // ---------------------------------------------------------------------------
@@ -200,11 +200,100 @@ __device__ __forceinline__ float exp2i(int k)
 }
 
 // ---------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 FFMA2 / FMUL2 / FADD2: two IEEE operations per
+// instruction, each rounded exactly like its scalar form).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b, rounded once (fma with -1 is exactly the subtraction)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, splat(-1.0f), a); }
+
+// max(a, |b|, |c|) in one three-input max
+__device__ __forceinline__ float amax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 16 bf16 -> 8 fp32 pairs (pair i = elements 2i, 2i+1), exactly.
+__device__ __forceinline__ void widen16x2(const uint32_t (&w)[8], float2 (&v)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
+// 16-point Walsh-Hadamard transform on pairs; the same additions in the same order as
+// fwht16 (stage h = 1 inside each pair, stages 2, 4, 8 across pairs), then * 0.25.
+__device__ __forceinline__ void fwht16x2(float2 (&v)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float a = v[i].x, b = v[i].y;
+        v[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2 * h) {
+#pragma unroll
+            for (int j = i; j < i + h; ++j) {
+                const float2 a = v[j], b = v[j + h];
+                v[j] = add2(a, b);
+                v[j + h] = sub2(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = mul2(v[i], splat(0.25f));
+}
+
+// Power-of-two p with amax * p in [1, 2) (p = 1 for amax = 0; p kept within
+// [2^-127, 2^126]) and 1 / p^2 as a double. Sums of squares are taken on values
+// scaled by p, so they neither overflow nor underflow in fp32, and are scaled back
+// exactly in double.
+struct Pow2 {
+    float p;
+    double inv_p2;
+};
+
+__device__ __forceinline__ Pow2 pow2_for(float amax)
+{
+    const uint32_t b = __float_as_uint(amax) & 0x7FFFFFFFu;
+    int k = (int)(b >> 23) - 127;           // floor(log2) for normal amax
+    if ((b >> 23) == 0) k = 0;              // zero: p = 1; subnormal: see below
+    if (b != 0 && (b >> 23) == 0) k = -126;
+    k = k > 127 ? 127 : (k < -126 ? -126 : k);
+    Pow2 r;
+    r.p = exp2i(-k);
+    r.inv_p2 = __longlong_as_double((long long)(1023 + 2 * k) << 52);
+    return r;
+}
+
+// ---------------------------------------------------------------------------
 // Division x / s decided without a per-element divide.
 //
-// r = RN(1/s); r_lo = RN(r (1 - 2^-21)) and r_hi = RN(r (1 + 2^-21)) satisfy
-// x r_lo < RN(x/s) < x r_hi for x > 0 (reversed for x < 0) whenever s and r are
-// normal: each rounding is at most 2^-24 relative. Any monotone rounding rule
+// r ~ 1/s within 2^-23; r_lo = RN(r (1 - 2^-20)) and r_hi = RN(r (1 + 2^-20))
+// satisfy x r_lo < RN(x/s) < x r_hi for x > 0 (reversed for x < 0) whenever s and r
+// are normal: RN(x/s) is within 2^-24 of x/s, and r_lo, r_hi are at least
+// 2^-20 - 2^-23 - 2^-24 away from 1/s. Any monotone rounding rule
 // (to the integer grid, or to an FP element grid) therefore returns the same value
 // on both bracket ends exactly when it returns that value for RN(x/s). When the two
 // ends disagree, the code is recomputed from a correctly rounded division.
@@ -215,11 +304,21 @@ struct Recip {
     bool fast;
 };
 
+__device__ __forceinline__ float rcp_approx(float s)
+{
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
+}
+
+// The reciprocal need not be correctly rounded: the hardware approximation is within
+// 1 ulp (2^-23 relative), and with the 1 -+ 2^-20 factors r_lo and r_hi still lie
+// strictly outside 1/s * (1 -+ 2^-24).
 __device__ __forceinline__ Recip make_recip(float s, float amax)
 {
     Recip r;
     r.s = s;
-    const float inv = __frcp_rn(s);
+    const float inv = rcp_approx(s);
     r.rlo = __fmul_rn(inv, BRACKET_LO);
     r.rhi = __fmul_rn(inv, BRACKET_HI);
     // s normal and not huge (so 1/s, r_lo, r_hi are normal); |x/s| < 2^22 keeps the
@@ -298,8 +397,12 @@ __device__ __forceinline__ WsHeader* ws_header(uint8_t* ws) { return reinterpret
 __device__ __forceinline__ RangeSlot* ws_range(uint8_t* ws) { return reinterpret_cast<RangeSlot*>(ws + WS_RANGE_OFF); }
 __device__ __forceinline__ StatSlot* ws_stats(uint8_t* ws) { return reinterpret_cast<StatSlot*>(ws + WS_STAT_OFF); }
 
+// Per-thread QSNR / crest-factor accumulators (kept small: they live in registers
+// through the whole kernel).
 struct Acc {
-    double err2 = 0.0, x2 = 0.0, ksum = 0.0, kmax = 0.0, nunits = 0.0, ss = 0.0;
+    double err2 = 0.0, x2 = 0.0, ksum = 0.0;
+    float kmax = 0.0f;
+    uint32_t nunits = 0;
 };
 
 __device__ __forceinline__ double warp_sum(double v)
@@ -332,27 +435,31 @@ __device__ __forceinline__ float warp_minf(float v)
 
 // Block-wide reduction of an Acc into thread 0 (fixed order: warp tree, then warps
 // in index order). blockDim.x must be a multiple of 32 and at most 1024.
-__device__ __forceinline__ Acc block_reduce_acc(Acc a)
+// Block totals in double (fixed order: warp tree, then warps in index order).
+struct AccD {
+    double err2 = 0.0, x2 = 0.0, ksum = 0.0, kmax = 0.0, nunits = 0.0;
+};
+
+__device__ __forceinline__ AccD block_reduce_acc(AccD a)
 {
-    __shared__ double sh[32][6];
+    __shared__ double sh[32][5];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     a.err2 = warp_sum(a.err2);
     a.x2 = warp_sum(a.x2);
     a.ksum = warp_sum(a.ksum);
     a.kmax = warp_max(a.kmax);
     a.nunits = warp_sum(a.nunits);
-    a.ss = warp_sum(a.ss);
     __syncthreads();
     if (lane == 0) {
         sh[warp][0] = a.err2; sh[warp][1] = a.x2; sh[warp][2] = a.ksum;
-        sh[warp][3] = a.kmax; sh[warp][4] = a.nunits; sh[warp][5] = a.ss;
+        sh[warp][3] = a.kmax; sh[warp][4] = a.nunits;
     }
     __syncthreads();
-    Acc t;
+    AccD t;
     if (threadIdx.x == 0) {
         for (int w = 0; w < nw; ++w) {
             t.err2 += sh[w][0]; t.x2 += sh[w][1]; t.ksum += sh[w][2];
-            t.kmax = fmax(t.kmax, sh[w][3]); t.nunits += sh[w][4]; t.ss += sh[w][5];
+            t.kmax = fmax(t.kmax, sh[w][3]); t.nunits += sh[w][4];
         }
     }
     return t;
@@ -361,17 +468,19 @@ __device__ __forceinline__ Acc block_reduce_acc(Acc a)
 // Called by every thread of every CTA at kernel end. Each CTA leaves its partial in
 // a workspace slot; the CTA that arrives last sums the slots in index order and
 // writes the result. tensor_kappa: the unit is the whole tensor; kappa = amax /
-// sqrt(ss / n_elems) is formed from the totals.
+// sqrt(x2 / n_elems) is formed from the totals.
 __device__ __forceinline__ void finish_stats(Acc mine, uint8_t* ws, bq_stats* out,
                                              bool tensor_kappa, float tensor_amax,
                                              double n_elems, bool write_kappa)
 {
     __shared__ bool is_last;
-    Acc t = block_reduce_acc(mine);
+    AccD m;
+    m.err2 = mine.err2; m.x2 = mine.x2; m.ksum = mine.ksum; m.kmax = (double)mine.kmax; m.nunits = (double)mine.nunits;
+    AccD t = block_reduce_acc(m);
     StatSlot* slots = ws_stats(ws);
     WsHeader* h = ws_header(ws);
     if (threadIdx.x == 0) {
-        StatSlot s{t.err2, t.x2, t.ksum, t.kmax, t.nunits, t.ss};
+        StatSlot s{t.err2, t.x2, t.ksum, t.kmax, t.nunits, 0.0};
         slots[blockIdx.x] = s;
         __threadfence();
         const unsigned ticket = atomicAdd(&h->counter_stats, 1u);
@@ -380,13 +489,13 @@ __device__ __forceinline__ void finish_stats(Acc mine, uint8_t* ws, bq_stats* ou
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    Acc a;
+    AccD a;
     for (unsigned i = threadIdx.x; i < gridDim.x; i += blockDim.x) {
         const double* p = reinterpret_cast<const double*>(&slots[i]);
         a.err2 += __ldcg(p + 0); a.x2 += __ldcg(p + 1); a.ksum += __ldcg(p + 2);
-        a.kmax = fmax(a.kmax, __ldcg(p + 3)); a.nunits += __ldcg(p + 4); a.ss += __ldcg(p + 5);
+        a.kmax = fmax(a.kmax, __ldcg(p + 3)); a.nunits += __ldcg(p + 4);
     }
-    Acc tot = block_reduce_acc(a);
+    AccD tot = block_reduce_acc(a);
     if (threadIdx.x == 0) {
         bq_stats r;
         r.err2 = tot.err2;
@@ -396,8 +505,8 @@ __device__ __forceinline__ void finish_stats(Acc mine, uint8_t* ws, bq_stats* ou
         r.n_units = tot.nunits;
         if (tensor_kappa) {
             r.kappa_sum = r.kappa_max = r.n_units = 0.0;
-            if (tot.ss > 0.0) {
-                const double k = (double)tensor_amax / sqrt(tot.ss / n_elems);
+            if (tot.x2 > 0.0) {
+                const double k = (double)tensor_amax / sqrt(tot.x2 / n_elems);
                 r.kappa_sum = k; r.kappa_max = k; r.n_units = 1.0;
             }
         }
@@ -413,8 +522,8 @@ __device__ __forceinline__ void kappa_add(Acc& a, float amax, float ss, float in
     if (ss > 0.0f) {
         const float k = __fmul_rn(amax, rsqrtf(__fmul_rn(ss, inv_n)));
         a.ksum += (double)k;
-        a.kmax = fmax(a.kmax, (double)k);
-        a.nunits += 1.0;
+        a.kmax = fmaxf(a.kmax, k);
+        a.nunits += 1u;
     }
 }
 

@@ -6,70 +6,95 @@
 // granularity" §2.2), the inverse Hadamard rotation (H16/4 is its own inverse), and
 // QSNR = -10 log10(||X - Xq||^2 / ||X||^2) (same page §4.1).
 //
-// Work layout as in the quantize kernels: a warp takes 64 consecutive 16-element
-// chunks per step, two per lane, codes read with one vector load per chunk, the
-// chunk's scale found by a multiply-high division of the chunk index.
-#include "common.cuh"
+// Work layout as in the quantize kernels: lane l of a warp owns two consecutive
+// 16-element chunks of the warp's 1024-element tile, reads their codes with one
+// vector load (32 bytes for 8-bit codes, 16 for 4-bit), and loads the next tile's
+// codes before decoding the current ones. A chunk's scale index is its chunk index
+// divided (multiply-high) by the chunks per scaling unit.
+#include "quant_ops.cuh"
 #include "internal.h"
 
 #include <atomic>
 
 namespace bq {
 
+template <int FMT>
+struct SpanCodes {
+    // 8-bit codes: 8 words (two chunks); 4-bit codes: 4 words
+    static constexpr int n = Fmt<FMT>::four ? 4 : 8;
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_codes(const uint8_t* codes, uint32_t span, uint32_t n_chunks,
+                                           uint32_t (&w)[SpanCodes<FMT>::n])
+{
+    constexpr int NB = Fmt<FMT>::four ? 16 : 32;   // bytes per span
+    const uint32_t c0 = 2 * span;
+    if (c0 + 1 < n_chunks) {
+        if constexpr (Fmt<FMT>::four) ld_nc_v4(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[4]>(&w));
+        else ld_nc_v8(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[8]>(&w));
+    } else {
+#pragma unroll
+        for (int i = 0; i < SpanCodes<FMT>::n; ++i) w[i] = 0u;
+        if (c0 < n_chunks) {
+            // half span: one chunk's codes
+            if constexpr (Fmt<FMT>::four) ld_nc_v2(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[2]>(&w));
+            else ld_nc_v4(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[4]>(&w));
+        }
+    }
+}
+
+// Element values of chunk h (0 or 1) of a span: integers as exact floats, FP codes decoded.
+template <int FMT>
+__device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>::n], int h, float2 (&val)[8])
+{
+    using F = Fmt<FMT>;
+    if constexpr (F::four) {
+        const uint32_t w0 = w[2 * h], w1 = w[2 * h + 1];
+        if constexpr (F::is_int) {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const uint32_t byte = ((p < 4 ? w0 : w1) >> (8 * (p & 3))) & 0xFFu;
+                int qa = (int)(byte & 0xFu), qb = (int)(byte >> 4);
+                if constexpr (FMT != BQ_UINT4_ASYM) { qa = (qa ^ 8) - 8; qb = (qb ^ 8) - 8; }
+                val[p] = make_float2((float)qa, (float)qb);
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) val[p] = dec_pair<FMT>(((p < 4 ? w0 : w1) >> (8 * (p & 3))) & 0xFFu);
+        }
+    } else {
+        if constexpr (F::is_int) {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const uint32_t word = w[4 * h + (p >> 1)];
+                const int sh = 16 * (p & 1);
+                val[p] = make_float2((float)(int)(int8_t)(word >> sh), (float)(int)(int8_t)(word >> (sh + 8)));
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) val[p] = dec_pair<FMT>((w[4 * h + (p >> 1)] >> (16 * (p & 1))) & 0xFFFFu);
+        }
+    }
+}
+
 // Dequantized fp32 values of chunk c (before any inverse rotation).
 template <int FMT, int SK>
-__device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, float (&xh)[16])
+__device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, const float2 (&val)[8],
+                                              float2 (&xh)[8])
 {
     using F = Fmt<FMT>;
     const uint32_t u = a.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, a.fd_m) + c) >> a.fd_s);
-
-    // element values (integers as exact floats, FP codes decoded)
-    float val[16];
-    if constexpr (F::four) {
-        uint32_t w[2];
-        ld_nc_v2(a.codes + (size_t)c * 8, w);
-        if constexpr (F::is_int) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t nib = (w[i >> 3] >> (4 * (i & 7))) & 0xFu;
-                int q = (int)nib;
-                if constexpr (FMT != BQ_UINT4_ASYM) q = (q ^ 8) - 8;   // sign-extend
-                val[i] = (float)q;
-            }
-        } else {
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const float2 f = dec_pair<FMT>((w[p >> 2] >> (8 * (p & 3))) & 0xFFu);
-                val[2 * p] = f.x;
-                val[2 * p + 1] = f.y;
-            }
-        }
-    } else {
-        uint32_t w[4];
-        ld_nc_v4(a.codes + (size_t)c * 16, w);
-        if constexpr (F::is_int) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) val[i] = (float)(int)(int8_t)(w[i >> 2] >> (8 * (i & 3)));
-        } else {
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const float2 f = dec_pair<FMT>((w[p >> 1] >> (16 * (p & 1))) & 0xFFFFu);
-                val[2 * p] = f.x;
-                val[2 * p + 1] = f.y;
-            }
-        }
-    }
-
     if constexpr (SK == SK_UE8M0) {
         const int e = (int)reinterpret_cast<const uint8_t*>(a.scales)[u] - 127;
-        const float pe = exp2i(e);
+        const float2 pe = splat(exp2i(e));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(val[i], pe);
+        for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], pe);
     } else if constexpr (SK == SK_NV) {
-        const float sbv = e4m3_value(reinterpret_cast<const uint8_t*>(a.scales)[u]);
-        const float S = a.tensor_scale[0];
+        const float2 sbv = splat(e4m3_value(reinterpret_cast<const uint8_t*>(a.scales)[u]));
+        const float2 S = splat(a.tensor_scale[0]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(__fmul_rn(val[i], sbv), S);
+        for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(val[i], sbv), S);
     } else {
         float s, zp = 0.0f;
         if (a.scale_fp16) {
@@ -79,12 +104,14 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
             s = reinterpret_cast<const float*>(a.scales)[u];
             if constexpr (F::asym) zp = reinterpret_cast<const float*>(a.zps)[u];
         }
+        const float2 S = splat(s);
         if constexpr (F::asym) {
+            const float2 nz = splat(-zp);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(s, __fsub_rn(val[i], zp));
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(add2(val[i], nz), S);   // q - zp is exact
         } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(val[i], s);
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], S);
         }
     }
 }
@@ -92,63 +119,89 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
 template <int FMT, int SK, bool HAD, int OUT>
 __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
 {
+    constexpr int NC = SpanCodes<FMT>::n;
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
+    uint32_t t = warp;
+    uint32_t cur[NC];
+    if (t < a.n_dtiles) load_codes<FMT>(a.codes, t * 32 + lane, a.n_chunks, cur);
+    while (t < a.n_dtiles) {
+        const uint32_t tn = t + nwarps;
+        uint32_t nxt[NC];
+        if (tn < a.n_dtiles) load_codes<FMT>(a.codes, tn * 32 + lane, a.n_chunks, nxt);
+        const uint32_t span = t * 32 + lane;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint32_t c = t * 64 + lane + 32 * h;
-            if (c >= a.n_chunks) continue;
-            float xh[16];
-            dequant_chunk<FMT, SK>(a, c, xh);
-            if constexpr (HAD) fwht16(xh);
+            const uint32_t c = 2 * span + h;
+            if (c >= a.n_chunks) break;
+            float2 val[8], xh[8];
+            chunk_values<FMT>(cur, h, val);
+            dequant_chunk<FMT, SK>(a, c, val, xh);
+            if constexpr (HAD) fwht16x2(xh);
             if constexpr (OUT == BQ_DT_BF16) {
                 uint32_t o[8];
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
-                    const __nv_bfloat162 b = __floats2bfloat162_rn(xh[2 * p], xh[2 * p + 1]);
+                    const __nv_bfloat162 b = __floats2bfloat162_rn(xh[p].x, xh[p].y);
                     o[p] = *reinterpret_cast<const uint32_t*>(&b);
                 }
                 st_v8(reinterpret_cast<uint8_t*>(a.out) + (size_t)c * 32, o);
             } else {
                 uint32_t o0[8], o1[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) { o0[i] = __float_as_uint(xh[i]); o1[i] = __float_as_uint(xh[8 + i]); }
+                for (int i = 0; i < 4; ++i) {
+                    o0[2 * i] = __float_as_uint(xh[i].x); o0[2 * i + 1] = __float_as_uint(xh[i].y);
+                    o1[2 * i] = __float_as_uint(xh[4 + i].x); o1[2 * i + 1] = __float_as_uint(xh[4 + i].y);
+                }
                 uint8_t* p = reinterpret_cast<uint8_t*>(a.out) + (size_t)c * 64;
                 st_v8(p, o0);
                 st_v8(p + 32, o1);
             }
         }
+#pragma unroll
+        for (int i = 0; i < NC; ++i) cur[i] = nxt[i];
+        t = tn;
     }
 }
 
 template <int FMT, int SK, bool HAD>
 __global__ void __launch_bounds__(256) k_qsnr(const DequantArgs a)
 {
+    constexpr int NC = SpanCodes<FMT>::n;
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
     Acc acc;
     for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
+        const uint32_t span = t * 32 + lane;
+        uint32_t w[NC];
+        load_codes<FMT>(a.codes, span, a.n_chunks, w);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint32_t c = t * 64 + lane + 32 * h;
-            if (c >= a.n_chunks) continue;
-            float x[16];
-            load16(a.x, c, x);
-            float xh[16];
-            dequant_chunk<FMT, SK>(a, c, xh);
-            if constexpr (HAD) fwht16(xh);
-            float e = 0.0f, s = 0.0f;
+            const uint32_t c = 2 * span + h;
+            if (c >= a.n_chunks) break;
+            uint32_t xw[8];
+            ld_nc_v8(a.x + (size_t)c * 8, xw);
+            float2 x[8], val[8], xh[8];
+            widen16x2(xw, x);
+            chunk_values<FMT>(w, h, val);
+            dequant_chunk<FMT, SK>(a, c, val, xh);
+            if constexpr (HAD) fwht16x2(xh);
+            // sums on values scaled by a power of two fitted to the chunk (no overflow
+            // or underflow in fp32), brought back in double
+            const Pow2 pw = pow2_for(chunk_amax(x, chunk_amax(xh, 0.0f)));
+            float2 e2 = splat(0.0f), x2 = splat(0.0f);
+            const float2 P = splat(pw.p);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float d = __fsub_rn(x[i], xh[i]);
-                e = __fmaf_rn(d, d, e);
-                s = __fmaf_rn(x[i], x[i], s);
+            for (int i = 0; i < 8; ++i) {
+                const float2 d = mul2(sub2(x[i], xh[i]), P);
+                const float2 xp = mul2(x[i], P);
+                e2 = fma2(d, d, e2);
+                x2 = fma2(xp, xp, x2);
             }
-            acc.err2 += (double)e;
-            acc.x2 += (double)s;
+            acc.err2 += (double)__fadd_rn(e2.x, e2.y) * pw.inv_p2;
+            acc.x2 += (double)__fadd_rn(x2.x, x2.y) * pw.inv_p2;
         }
     }
     finish_stats(acc, a.ws, a.stats, false, 0.0f, 0.0, false);

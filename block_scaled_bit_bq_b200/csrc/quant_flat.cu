@@ -2,11 +2,13 @@
 // 16-element chunks: per-tensor (after the range pass), per-group, MX block-32 and
 // NV block-16 granularities; and the per-tensor range pass itself.
 //
-// Layout of the work: a warp takes 64 consecutive chunks (1024 elements, 2 KB of
-// bf16) per step, lane l the chunks 64t + l and 64t + 32 + l, each loaded with one
-// 256-bit load (both loads are issued before either chunk is processed). A scaling
-// unit of G elements spans G/16 adjacent lanes and is reduced with xor shuffles. The
-// grid is a whole number of waves (SM count x resident CTAs) striding over the steps.
+// Layout of the work: lane l of a warp owns a span of two consecutive chunks (32
+// elements, 64 bytes, two 256-bit loads) of the warp's 1024-element tile; the next
+// tile's span is loaded before the current one is processed, so every lane keeps 64
+// bytes in flight while it computes. A scaling unit of G >= 32 elements spans G/32
+// adjacent lanes and is reduced with xor shuffles; 16-element units (NV blocks,
+// groups of 16) are lane-local. The grid is at most one wave (SM count x resident
+// CTAs) striding over the tiles.
 //
 // Steps (source pages): AbsMax scale per unit ("INT vs FP at fine granularity" §2.1,
 // §3.1); MX block 32 with a power-of-two scale, NV block 16 with an E4M3 block scale
@@ -31,40 +33,36 @@ namespace bq {
 // ---------------------------------------------------------------------------
 
 template <bool HAD, bool MINMAX>
+__device__ __forceinline__ void range_chunk(const uint32_t (&w)[8], float& amax, float& mn, float& mx)
+{
+    float2 v[8];
+    widen16x2(w, v);
+    if constexpr (HAD) fwht16x2(v);
+    amax = chunk_amax(v, amax);
+    if constexpr (MINMAX) chunk_minmax(v, mn, mx);
+}
+
+template <bool HAD, bool MINMAX>
 __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, uint32_t n_chunks, uint8_t* ws)
 {
     float amax = 0.0f, mn = 0.0f, mx = 0.0f;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; c + stride < n_chunks; c += 2 * stride) {
-        uint32_t w0[8], w1[8];
-        ld_nc_v8(x + (size_t)c * 8, w0);
-        ld_nc_v8(x + (size_t)(c + stride) * 8, w1);
-        float v[16];
-        widen16(w0, v);
-        if constexpr (HAD) fwht16(v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            amax = fmaxf(amax, fabsf(v[i]));
-            if constexpr (MINMAX) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
-        }
-        widen16(w1, v);
-        if constexpr (HAD) fwht16(v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            amax = fmaxf(amax, fabsf(v[i]));
-            if constexpr (MINMAX) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
-        }
+    for (; c + 3 * stride < n_chunks; c += 4 * stride) {
+        uint32_t w0[8], w1[8], w2[8], w3[8];
+        ld_nc_v8(x + c * 8, w0);
+        ld_nc_v8(x + (c + stride) * 8, w1);
+        ld_nc_v8(x + (c + 2 * stride) * 8, w2);
+        ld_nc_v8(x + (c + 3 * stride) * 8, w3);
+        range_chunk<HAD, MINMAX>(w0, amax, mn, mx);
+        range_chunk<HAD, MINMAX>(w1, amax, mn, mx);
+        range_chunk<HAD, MINMAX>(w2, amax, mn, mx);
+        range_chunk<HAD, MINMAX>(w3, amax, mn, mx);
     }
-    if (c < n_chunks) {
-        float v[16];
-        load16(x, (uint32_t)c, v);
-        if constexpr (HAD) fwht16(v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            amax = fmaxf(amax, fabsf(v[i]));
-            if constexpr (MINMAX) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
-        }
+    for (; c < n_chunks; c += stride) {
+        uint32_t w0[8];
+        ld_nc_v8(x + c * 8, w0);
+        range_chunk<HAD, MINMAX>(w0, amax, mn, mx);
     }
     // min / max start from 0: only min(min, 0) and max(max, 0) are ever used.
     amax = warp_maxf(amax);
@@ -103,43 +101,155 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
 }
 
 // ---------------------------------------------------------------------------
-// One chunk of the flat quantize kernel.
+// Quantize kernel.
 // ---------------------------------------------------------------------------
 
 struct TensorCtx {
     float amax;          // per-tensor / NV: amax of the (rotated) tensor
     PlainScale ps;       // per-tensor plain scale
-    Recip rc;            // per-tensor reciprocal bracket
+    UnitQ u;             // per-tensor unit
+    Pow2 p2;             // per-tensor sum scaling
     float S;             // NV tensor scale
 };
 
+// Accumulate one chunk's QSNR sums (scaled by p) into the lane's doubles.
+__device__ __forceinline__ void add_sums(Acc& acc, const float2 (&y)[8], const float2 (&xh)[8], const Pow2& p,
+                                         float* ss_out)
+{
+    float2 e2 = splat(0.0f), x2 = splat(0.0f);
+    chunk_sums2(y, xh, p.p, e2, x2);
+    const float e = __fadd_rn(e2.x, e2.y), s = __fadd_rn(x2.x, x2.y);
+    acc.err2 += (double)e * p.inv_p2;
+    acc.x2 += (double)s * p.inv_p2;
+    if (ss_out) *ss_out = __fadd_rn(*ss_out, s);
+}
+
+// NV block scale: s_b = E4M3((amax / Qmax) / S), d = s_b * S.
+template <int FMT>
+__device__ __forceinline__ UnitQ nv_unit(float amax, float S, uint32_t& sbc, float& sbv)
+{
+    using F = Fmt<FMT>;
+    sbc = 0;
+    sbv = 0.0f;
+    if (S > 0.0f) {
+        const float sb32 = __fdiv_rn(__fdiv_rn(amax, F::qscale), S);
+        sbc = e4m3_code(sb32);
+        sbv = e4m3_value(sbc);
+    }
+    const float d = __fmul_rn(sbv, S);
+    UnitQ u;
+    u.s = d;
+    u.zpf = 0.0f;
+    u.qmin = -7;
+    u.qmax = 7;
+    u.zero = !(d > 0.0f);
+    const Recip R = make_recip(d, amax);
+    u.rlo = R.rlo;
+    u.rhi = R.rhi;
+    u.fast = R.fast;
+    u.clamp = F::is_int ? needs_clamp(-amax, amax, R, 0.0f, -7, 7) : false;
+    return u;
+}
+
+// Widen (and rotate) one chunk of a span.
+template <bool HAD>
+__device__ __forceinline__ void chunk_in(const uint32_t (&w)[8], float2 (&y)[8])
+{
+    widen16x2(w, y);
+    if constexpr (HAD) fwht16x2(y);
+}
+
+// Quantize one chunk under a known unit, store its codes, add its QSNR sums (and its
+// scaled sum of squares to *ss when ss is given).
+template <int FMT, bool STATS>
+__device__ __forceinline__ void emit_chunk(const float2 (&y)[8], const UnitQ& u, uint8_t* codes, uint32_t c,
+                                           bool valid, const Pow2& pw, Acc& acc, float* ss)
+{
+    constexpr int NW = CodeWords<FMT>::n;
+    uint32_t q[NW];
+    float2 xh[8];
+    quant_unit_chunk<FMT, STATS>(y, u, q, xh);
+    if (valid) {
+        store_codes<FMT>(codes, c, q);
+        if constexpr (STATS) add_sums(acc, y, xh, pw, ss);
+    }
+}
+
 template <int FMT, int GK, bool HAD, bool STATS>
-__device__ __forceinline__ void flat_chunk(const uint32_t (&win)[8], uint32_t c, bool valid, const FlatArgs& a,
-                                           const TensorCtx& tc, Acc& acc, int lane)
+__device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_t (&w1)[8], uint32_t span,
+                                          const FlatArgs& a, const TensorCtx& tc, Acc& acc, int lane)
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
-    float y[16];
-    widen16(win, y);
-    if constexpr (HAD) fwht16(y);
-
-    uint32_t w[NW];
-    float xh[16];
+    const uint32_t c0 = 2 * span;
+    const bool valid[2] = {c0 < a.n_chunks, c0 + 1 < a.n_chunks};
 
     if constexpr (GK == K_TENSOR) {
-        quant_plain_chunk<FMT, STATS>(y, tc.ps, tc.rc, F::qmin, F::qmax, w, xh);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 y[8];
+            chunk_in<HAD>(h ? w1 : w0, y);
+            emit_chunk<FMT, STATS>(y, tc.u, a.codes, c0 + h, valid[h], tc.p2, acc, nullptr);
+        }
+    } else if (GK == K_NV || (GK == K_GROUP && a.lanes_per_group == 0)) {
+        // 16-element units: two per lane, each handled start to finish
+        uint32_t scode[2] = {0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 y[8];
+            chunk_in<HAD>(h ? w1 : w0, y);
+            const float m = chunk_amax(y, 0.0f);
+            const Pow2 pw = pow2_for(m);
+            float ss = 0.0f;
+            if constexpr (GK == K_NV) {
+                uint32_t sbc;
+                float sbv;
+                const UnitQ u = nv_unit<FMT>(m, tc.S, sbc, sbv);
+                scode[h] = sbc;
+                uint32_t q[NW];
+                float2 z[8], xh[8];
+                if constexpr (F::is_int) int_chunk<FMT, STATS>(y, u, q, z);
+                else fp_chunk<FMT, STATS>(y, u, q, z);
+                if (valid[h]) {
+                    store_codes<FMT>(a.codes, c0 + h, q);
+                    if constexpr (STATS) {
+                        const float2 A = splat(sbv), S2 = splat(tc.S);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) xh[i] = u.zero ? splat(0.0f) : mul2(mul2(z[i], A), S2);
+                        add_sums(acc, y, xh, pw, &ss);
+                    }
+                }
+            } else {
+                float mn = 0.0f, mx = 0.0f;
+                if constexpr (F::asym) chunk_minmax(y, mn, mx);
+                const bool f16 = a.scale_fp16 != 0;
+                const PlainScale ps = plain_scale<FMT>(m, mn, mx, f16);
+                const UnitQ u = unit_of_plain<FMT>(ps);
+                emit_chunk<FMT, STATS>(y, u, a.codes, c0 + h, valid[h], pw, acc, &ss);
+                if (valid[h]) store_plain_scale<FMT>(a.scales, a.zps, c0 + h, ps, f16);
+            }
+            if constexpr (STATS) {
+                if (valid[h]) kappa_add(acc, __fmul_rn(m, pw.p), ss, a.inv_unit);
+            }
+        }
+        if constexpr (GK == K_NV) {
+            uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
+            if (valid[1]) *reinterpret_cast<uint16_t*>(sc + c0) = (uint16_t)(scode[0] | (scode[1] << 8));
+            else if (valid[0]) sc[c0] = (uint8_t)scode[0];
+        }
     } else {
-        // range of this lane's 16 values, then of its unit
+        // units of 32 elements or more: one per lane (MX, groups of 32) or T lanes per
+        // unit. Range first (the chunks are widened again for the quantize step, which
+        // keeps register pressure low).
         float amax = 0.0f, mn = 0.0f, mx = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            amax = fmaxf(amax, fabsf(y[i]));
-            if constexpr (F::asym) { mn = fminf(mn, y[i]); mx = fmaxf(mx, y[i]); }
+        for (int h = 0; h < 2; ++h) {
+            float2 y[8];
+            chunk_in<HAD>(h ? w1 : w0, y);
+            amax = chunk_amax(y, amax);
+            if constexpr (F::asym) chunk_minmax(y, mn, mx);
         }
-        int T;
-        if constexpr (GK == K_NV) T = 1;
-        else if constexpr (GK == K_MX) T = 2;
-        else T = a.lanes_per_group;
+        const int T = (GK == K_MX) ? 1 : a.lanes_per_group;
         for (int o = 1; o < T; o <<= 1) {
             amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             if constexpr (F::asym) {
@@ -148,89 +258,68 @@ __device__ __forceinline__ void flat_chunk(const uint32_t (&win)[8], uint32_t c,
             }
         }
         const bool leader = (lane & (T - 1)) == 0;
-
-        if constexpr (GK == K_GROUP) {
-            const PlainScale ps = plain_scale<FMT>(amax, mn, mx, a.scale_fp16 != 0);
-            const Recip R = make_recip(ps.s, ps.bound);
-            quant_plain_chunk<FMT, STATS>(y, ps, R, F::qmin, F::qmax, w, xh);
-            if (valid && leader) store_plain_scale<FMT>(a.scales, a.zps, c >> (__ffs(T) - 1), ps, a.scale_fp16 != 0);
-        } else if constexpr (GK == K_MX) {
+        const Pow2 pw = pow2_for(amax);
+        float ss = 0.0f;
+        if constexpr (GK == K_MX) {
             const int e = ue8m0_exponent<FMT>(amax);
-            const float p2 = exp2i(-e), pe = exp2i(e);
-            if constexpr (F::is_int) {
-                float q[16];
-                quant_int8_chunk_pow2(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&w), q);
-                if constexpr (STATS) {
+            const float p2 = exp2i(-e);
+            const float2 PE = splat(exp2i(e));
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(q[i], pe);
-                }
-            } else {
-                float val[16];
-                quant_fp_chunk_pow2<FMT, STATS>(y, p2, w, val);
-                if constexpr (STATS) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(val[i], pe);
-                }
-            }
-            if (valid && leader) reinterpret_cast<uint8_t*>(a.scales)[c >> 1] = (uint8_t)(e + 127);
-        } else {  // K_NV
-            uint32_t sbc = 0;
-            float sbv = 0.0f;
-            if (tc.S > 0.0f) {
-                const float sb32 = __fdiv_rn(__fdiv_rn(amax, F::qscale), tc.S);
-                sbc = e4m3_code(sb32);
-                sbv = e4m3_value(sbc);
-            }
-            const float d = __fmul_rn(sbv, tc.S);
-            if (valid) reinterpret_cast<uint8_t*>(a.scales)[c] = (uint8_t)sbc;
-            if (d > 0.0f) {
-                const Recip R = make_recip(d, amax);
-                if constexpr (F::is_int) {
-                    float qz[16];
-                    quant_int_chunk<FMT, STATS>(y, R, 0.0f, -7, 7, w, qz);
+            for (int h = 0; h < 2; ++h) {
+                float2 y[8], z[8], xh[8];
+                chunk_in<HAD>(h ? w1 : w0, y);
+                uint32_t q[NW];
+                if constexpr (F::is_int) int8_chunk_pow2<STATS>(y, p2, false, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
+                else fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
+                if (valid[h]) {
+                    store_codes<FMT>(a.codes, c0 + h, q);
                     if constexpr (STATS) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(__fmul_rn(qz[i], sbv), tc.S);
-                    }
-                } else {
-                    float val[16];
-                    quant_fp_chunk<FMT, STATS>(y, R, w, val);
-                    if constexpr (STATS) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(__fmul_rn(val[i], sbv), tc.S);
+                        for (int i = 0; i < 8; ++i) xh[i] = mul2(z[i], PE);
+                        add_sums(acc, y, xh, pw, &ss);
                     }
                 }
-            } else {
-#pragma unroll
-                for (int k = 0; k < NW; ++k) w[k] = 0u;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) xh[i] = 0.0f;
             }
+            if (valid[0]) reinterpret_cast<uint8_t*>(a.scales)[span] = (uint8_t)(e + 127);
+        } else {
+            const bool f16 = a.scale_fp16 != 0;
+            const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+            const UnitQ u = unit_of_plain<FMT>(ps);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float2 y[8];
+                chunk_in<HAD>(h ? w1 : w0, y);
+                emit_chunk<FMT, STATS>(y, u, a.codes, c0 + h, valid[h], pw, acc, &ss);
+            }
+            if (valid[0] && leader) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
         }
-
         if constexpr (STATS) {
-            // crest factor of the unit: amax / sqrt(mean y^2)
-            float ss = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ss = __fmaf_rn(y[i], y[i], ss);
             for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
-            if (valid && leader) kappa_add(acc, amax, ss, a.inv_unit);
-        }
-    }
-
-    if (valid) {
-        store_codes<FMT>(a.codes, c, w);
-        if constexpr (STATS) {
-            float e2, x2;
-            chunk_sums(y, xh, e2, x2);
-            acc.err2 += (double)e2;
-            acc.x2 += (double)x2;
+            if (valid[0] && leader) kappa_add(acc, __fmul_rn(amax, pw.p), ss, a.inv_unit);
         }
     }
 }
 
+__device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint32_t n_chunks,
+                                          uint32_t (&w0)[8], uint32_t (&w1)[8])
+{
+    const uint32_t c0 = 2 * span;
+    if (c0 + 1 < n_chunks) {
+        ld_nc_v8(x + (size_t)c0 * 8, w0);
+        ld_nc_v8(x + (size_t)c0 * 8 + 8, w1);
+    } else {
+        if (c0 < n_chunks) ld_nc_v8(x + (size_t)c0 * 8, w0);
+        else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w0[i] = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w1[i] = 0u;
+    }
+}
+
 template <int FMT, int GK, bool HAD, bool STATS>
-__global__ void __launch_bounds__(256) k_quant_flat(const FlatArgs a)
+__global__ void __launch_bounds__(256, STATS ? 2 : 3) k_quant_flat(const FlatArgs a)
 {
     using F = Fmt<FMT>;
     const int lane = threadIdx.x & 31;
@@ -243,7 +332,8 @@ __global__ void __launch_bounds__(256) k_quant_flat(const FlatArgs a)
         tc.amax = h->amax;
         if constexpr (GK == K_TENSOR) {
             tc.ps = plain_scale<FMT>(h->amax, h->vmin, h->vmax, a.scale_fp16 != 0);
-            tc.rc = make_recip(tc.ps.s, tc.ps.bound);
+            tc.u = unit_of_plain<FMT>(tc.ps);
+            tc.p2 = pow2_for(tc.amax);
             if (blockIdx.x == 0 && threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, 0, tc.ps, a.scale_fp16 != 0);
         } else {
             tc.S = __fdiv_rn(h->amax, F::qscale * 448.0f);
@@ -252,27 +342,22 @@ __global__ void __launch_bounds__(256) k_quant_flat(const FlatArgs a)
     }
 
     Acc acc;
-    for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
-        const uint32_t c0 = t * 64 + lane, c1 = c0 + 32;
-        const bool v0 = c0 < a.n_chunks, v1 = c1 < a.n_chunks;
-        uint32_t w0[8], w1[8];
-        if (v0) ld_nc_v8(a.x + (size_t)c0 * 8, w0);
-        else {
+    // tile t covers spans 32 t .. 32 t + 31 (chunks 64 t .. 64 t + 63)
+    uint32_t t = warp;
+    uint32_t c0[8], c1[8];
+    if (t < a.n_dtiles) load_span(a.x, t * 32 + lane, a.n_chunks, c0, c1);
+    while (t < a.n_dtiles) {
+        const uint32_t tn = t + nwarps;
+        uint32_t n0[8], n1[8];
+        if (tn < a.n_dtiles) load_span(a.x, tn * 32 + lane, a.n_chunks, n0, n1);
+        flat_span<FMT, GK, HAD, STATS>(c0, c1, t * 32 + lane, a, tc, acc, lane);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w0[i] = 0u;
-        }
-        if (v1) ld_nc_v8(a.x + (size_t)c1 * 8, w1);
-        else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w1[i] = 0u;
-        }
-        flat_chunk<FMT, GK, HAD, STATS>(w0, c0, v0, a, tc, acc, lane);
-        flat_chunk<FMT, GK, HAD, STATS>(w1, c1, v1, a, tc, acc, lane);
+        for (int i = 0; i < 8; ++i) { c0[i] = n0[i]; c1[i] = n1[i]; }
+        t = tn;
     }
 
     if constexpr (STATS) {
         // per-tensor kappa comes from the totals: amax / sqrt(sum y^2 / n)
-        acc.ss = acc.x2;
         finish_stats(acc, a.ws, a.stats, GK == K_TENSOR, tc.amax, a.n_elems, true);
     }
 }
@@ -314,7 +399,7 @@ cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
     constexpr int block = 256;
     constexpr auto kern = k_quant_flat<FMT, GK, HAD, STATS>;
-    // one warp step = 64 chunks; a CTA of 8 warps takes 8 steps per sweep
+    // one tile per warp at least (8 tiles per CTA)
     const unsigned grid = grid_for<kern, block>(8, a.n_dtiles);
     kern<<<grid, block, 0, st>>>(a);
     return cudaGetLastError();

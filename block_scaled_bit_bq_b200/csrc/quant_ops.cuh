@@ -1,4 +1,4 @@
-// quant_ops.cuh -- quantize one 16-element chunk given its scale.
+// quant_ops.cuh -- quantize one 16-element chunk given its scale, on fp32 pairs.
 //
 // Code rules ("INT vs FP at fine granularity" §2.1, "INT4/INT8/FP8 quantization"
 // §INT8/§INT4, "Quantization survey" §4.1):
@@ -6,8 +6,10 @@
 //   FP:   code = cvt.rn.satfinite(x / s)
 // with x / s the correctly rounded fp32 quotient, decided through the reciprocal
 // bracket of common.cuh (a correctly rounded division only where the bracket is
-// inconclusive).
+// inconclusive, about one element in 10^4).
 #pragma once
+
+#include <cfloat>
 
 #include "common.cuh"
 
@@ -15,60 +17,99 @@ namespace bq {
 
 template <int FMT> struct CodeWords { static constexpr int n = Fmt<FMT>::four ? 2 : 4; };
 
-// Integer chunk. zpf = zero point as an exact float (0 for symmetric formats);
-// qmin / qmax the code range. On return: w holds the packed codes, qz[i] = q - zp.
+// Everything a chunk needs to know about its unit's scale.
+struct UnitQ {
+    float s;        // scale the codes divide by (stored plain scale, d for NV)
+    float rlo, rhi; // reciprocal bracket
+    float zpf;      // zero point (exact float; 0 for symmetric)
+    int qmin, qmax; // integer code range
+    bool fast;      // bracket usable for this unit
+    bool clamp;     // some element of the unit can fall outside [qmin, qmax]
+    bool zero;      // s == 0 (or d == 0): every code is the zero code
+};
+
+// Is clamping needed? q is monotone in x, so the unit's extreme values bound it.
+__device__ __forceinline__ bool needs_clamp(float lo, float hi, const Recip& R, float zpf, int qmin, int qmax)
+{
+    if (!R.fast) return true;
+    const float top = __fadd_rn(__fmaf_rn(hi, R.rhi, MAGIC), zpf);   // >= MAGIC + q for every x <= hi
+    const float bot = __fadd_rn(__fmaf_rn(lo, R.rhi, MAGIC), zpf);   // <= MAGIC + q for every x >= lo (lo <= 0)
+    return top > MAGIC + (float)qmax || bot < MAGIC + (float)qmin;
+}
+
+// ---------------------------------------------------------------------------
+// Integer chunk. On return: w = packed codes; qz[i] = q - zp (exact floats) when NEED_Q.
+// ---------------------------------------------------------------------------
+
 template <int FMT, bool NEED_Q>
-__device__ __forceinline__ void quant_int_chunk(const float (&y)[16], const Recip& R, float zpf,
-                                                int qmin, int qmax,
-                                                uint32_t (&w)[CodeWords<FMT>::n], float (&qz)[16])
+__device__ __forceinline__ void int_chunk(const float2 (&y)[8], const UnitQ& u,
+                                          uint32_t (&w)[CodeWords<FMT>::n], float2 (&qz)[8])
 {
     using F = Fmt<FMT>;
-    float t[16];
-    bool ok = R.fast;
-    if (ok) {
-        uint32_t mism = 0;
+    float2 t[8];
+    if (u.zero) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = __fmaf_rn(y[i], R.rlo, MAGIC);
-            const float b = __fmaf_rn(y[i], R.rhi, MAGIC);
-            mism |= __float_as_uint(a) ^ __float_as_uint(b);
-            t[i] = a;
+        for (int i = 0; i < 8; ++i) t[i] = splat(__fadd_rn(MAGIC, u.zpf));
+    } else {
+        bool ok = u.fast;
+        if (ok) {
+            uint32_t mism = 0;
+            const float2 lo = splat(u.rlo), hi = splat(u.rhi), m = splat(MAGIC);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 a = fma2(y[i], lo, m);
+                const float2 b = fma2(y[i], hi, m);
+                mism |= (__float_as_uint(a.x) ^ __float_as_uint(b.x)) | (__float_as_uint(a.y) ^ __float_as_uint(b.y));
+                t[i] = a;
+            }
+            ok = (mism == 0);
         }
-        ok = (mism == 0);
-    }
-    if (!ok) {
+        if (!ok) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float q = rintf(__fdiv_rn(y[i], R.s));
-            q = fminf(fmaxf(q, -4194304.0f), 4194304.0f);
-            t[i] = __fadd_rn(q, MAGIC);
+            for (int i = 0; i < 8; ++i) {
+                float qa = rintf(__fdiv_rn(y[i].x, u.s));
+                float qb = rintf(__fdiv_rn(y[i].y, u.s));
+                qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
+                qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
+                t[i] = make_float2(__fadd_rn(qa, MAGIC), __fadd_rn(qb, MAGIC));
+            }
+        }
+        if constexpr (F::asym) {
+            const float2 z = splat(u.zpf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = add2(t[i], z);
+        }
+        if (u.clamp) {
+            const float cmin = MAGIC + (float)u.qmin, cmax = MAGIC + (float)u.qmax;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
         }
     }
-    const float cmin = MAGIC + (float)qmin, cmax = MAGIC + (float)qmax;
-    const float zero_at = __fadd_rn(MAGIC, zpf);
+    if constexpr (NEED_Q) {
+        const float2 z = splat(-__fadd_rn(MAGIC, u.zpf));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        float u = t[i];
-        if constexpr (F::asym) u = __fadd_rn(u, zpf);
-        u = fminf(fmaxf(u, cmin), cmax);
-        t[i] = u;
-        if constexpr (NEED_Q) qz[i] = __fsub_rn(u, zero_at);
+        for (int i = 0; i < 8; ++i) qz[i] = add2(t[i], z);
     }
+    // the low bits of t are the two's complement code
     if constexpr (F::four) {
         uint32_t b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = pack_nibbles(__float_as_uint(t[2 * i]), __float_as_uint(t[2 * i + 1]));
+        for (int i = 0; i < 8; ++i) b[i] = pack_nibbles(__float_as_uint(t[i].x), __float_as_uint(t[i].y));
         w[0] = pack_bytes(b[0], b[1], b[2], b[3]);
         w[1] = pack_bytes(b[4], b[5], b[6], b[7]);
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            w[k] = pack_bytes(__float_as_uint(t[4 * k]), __float_as_uint(t[4 * k + 1]),
-                              __float_as_uint(t[4 * k + 2]), __float_as_uint(t[4 * k + 3]));
+            w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
+                              __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
     }
 }
 
-// Pack eight pair-codes (cvt_pair results, element 2p in the low part) into words.
+// ---------------------------------------------------------------------------
+// FP element chunks.
+// ---------------------------------------------------------------------------
+
 template <int FMT>
 __device__ __forceinline__ void pack_pairs(const uint32_t (&pr)[8], uint32_t (&w)[CodeWords<FMT>::n])
 {
@@ -82,75 +123,88 @@ __device__ __forceinline__ void pack_pairs(const uint32_t (&pr)[8], uint32_t (&w
 }
 
 template <int FMT>
-__device__ __forceinline__ void decode_pairs(const uint32_t (&pr)[8], float (&val)[16])
+__device__ __forceinline__ void decode_pairs(const uint32_t (&pr)[8], float2 (&val)[8])
 {
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const float2 f = dec_pair<FMT>(pr[p]);
-        val[2 * p] = f.x;
-        val[2 * p + 1] = f.y;
-    }
+    for (int p = 0; p < 8; ++p) val[p] = dec_pair<FMT>(pr[p]);
 }
 
-// FP element chunk (E4M3 / E5M2 / E2M1) with a general scale s > 0. On return w holds
-// the packed codes and (NEED_V) val[i] the decoded element values.
+// General scale s > 0: codes of x / s. val = decoded element values when NEED_V.
 template <int FMT, bool NEED_V>
-__device__ __forceinline__ void quant_fp_chunk(const float (&y)[16], const Recip& R,
-                                               uint32_t (&w)[CodeWords<FMT>::n], float (&val)[16])
+__device__ __forceinline__ void fp_chunk(const float2 (&y)[8], const UnitQ& u,
+                                         uint32_t (&w)[CodeWords<FMT>::n], float2 (&val)[8])
 {
     uint32_t pr[8];
-    bool ok = R.fast;
-    if (ok) {
-        uint32_t mism = 0;
+    if (u.zero) {
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const uint32_t lo = cvt_pair<FMT>(__fmul_rn(y[2 * p + 1], R.rlo), __fmul_rn(y[2 * p], R.rlo));
-            const uint32_t hi = cvt_pair<FMT>(__fmul_rn(y[2 * p + 1], R.rhi), __fmul_rn(y[2 * p], R.rhi));
-            mism |= lo ^ hi;
-            pr[p] = lo;
+        for (int p = 0; p < 8; ++p) pr[p] = 0u;
+    } else {
+        bool ok = u.fast;
+        if (ok) {
+            uint32_t mism = 0;
+            const float2 lo = splat(u.rlo), hi = splat(u.rhi);
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const float2 a = mul2(y[p], lo), b = mul2(y[p], hi);
+                const uint32_t cl = cvt_pair<FMT>(a.y, a.x);
+                const uint32_t ch = cvt_pair<FMT>(b.y, b.x);
+                mism |= cl ^ ch;
+                pr[p] = cl;
+            }
+            ok = (mism == 0);
         }
-        ok = (mism == 0);
-    }
-    if (!ok) {
+        if (!ok) {
 #pragma unroll
-        for (int p = 0; p < 8; ++p)
-            pr[p] = cvt_pair<FMT>(__fdiv_rn(y[2 * p + 1], R.s), __fdiv_rn(y[2 * p], R.s));
+            for (int p = 0; p < 8; ++p)
+                pr[p] = cvt_pair<FMT>(__fdiv_rn(y[p].y, u.s), __fdiv_rn(y[p].x, u.s));
+        }
     }
     pack_pairs<FMT>(pr, w);
     if constexpr (NEED_V) decode_pairs<FMT>(pr, val);
 }
 
-// FP element chunk with an exact power-of-two scale: code = cvt(x * 2^-e).
+// Exact power-of-two scale: code = cvt(x * 2^-e) (the product is exact).
 template <int FMT, bool NEED_V>
-__device__ __forceinline__ void quant_fp_chunk_pow2(const float (&y)[16], float p2,
-                                                    uint32_t (&w)[CodeWords<FMT>::n], float (&val)[16])
+__device__ __forceinline__ void fp_chunk_pow2(const float2 (&y)[8], float p2,
+                                              uint32_t (&w)[CodeWords<FMT>::n], float2 (&val)[8])
 {
     uint32_t pr[8];
+    const float2 p = splat(p2);
 #pragma unroll
-    for (int p = 0; p < 8; ++p) pr[p] = cvt_pair<FMT>(__fmul_rn(y[2 * p + 1], p2), __fmul_rn(y[2 * p], p2));
+    for (int i = 0; i < 8; ++i) {
+        const float2 a = mul2(y[i], p);
+        pr[i] = cvt_pair<FMT>(a.y, a.x);
+    }
     pack_pairs<FMT>(pr, w);
     if constexpr (NEED_V) decode_pairs<FMT>(pr, val);
 }
 
-// MXINT8 chunk with an exact power-of-two scale: q = clamp(rne(x * 2^-e), -127, 127).
-__device__ __forceinline__ void quant_int8_chunk_pow2(const float (&y)[16], float p2, uint32_t (&w)[4],
-                                                      float (&q)[16])
+// MXINT8: q = clamp(rne(x * 2^-e), -127, 127); the clamp never binds (amax <= 127 * 2^e)
+// except for the clamped exponent range, which the caller flags.
+template <bool NEED_Q>
+__device__ __forceinline__ void int8_chunk_pow2(const float2 (&y)[8], float p2, bool clamp, uint32_t (&w)[4],
+                                                float2 (&q)[8])
 {
-    const float cmin = MAGIC - 127.0f, cmax = MAGIC + 127.0f;
-    float t[16];
+    float2 t[8];
+    const float2 p = splat(p2), m = splat(MAGIC);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float u = fminf(fmaxf(__fmaf_rn(y[i], p2, MAGIC), cmin), cmax);
-        t[i] = u;
-        q[i] = __fsub_rn(u, MAGIC);
+    for (int i = 0; i < 8; ++i) t[i] = fma2(y[i], p, m);
+    if (clamp) {
+        const float cmin = MAGIC - 127.0f, cmax = MAGIC + 127.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
+    }
+    if constexpr (NEED_Q) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = add2(t[i], splat(-MAGIC));
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        w[k] = pack_bytes(__float_as_uint(t[4 * k]), __float_as_uint(t[4 * k + 1]),
-                          __float_as_uint(t[4 * k + 2]), __float_as_uint(t[4 * k + 3]));
+        w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
+                          __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
 }
 
-// Store one chunk's codes (chunk c of the flat code array).
 template <int FMT>
 __device__ __forceinline__ void store_codes(uint8_t* codes, uint32_t c, const uint32_t (&w)[CodeWords<FMT>::n])
 {
@@ -158,11 +212,14 @@ __device__ __forceinline__ void store_codes(uint8_t* codes, uint32_t c, const ui
     else st_v4(codes + (size_t)c * 16, w);
 }
 
-// Scale of a plain (tensor / row / group) unit from its range.
+// ---------------------------------------------------------------------------
+// Plain (tensor / row / group) scales.
+// ---------------------------------------------------------------------------
+
 struct PlainScale {
     float s;        // stored scale (fp16-rounded when the dtype is fp16)
     float zpf;      // zero point as float (0 for symmetric)
-    float bound;    // max |y| the unit can hold (for the integer magic range)
+    float lo, hi;   // extreme values the unit holds (-amax, amax for symmetric)
 };
 
 template <int FMT>
@@ -172,66 +229,71 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
     PlainScale p;
     if constexpr (F::asym) {
         const float lo = fminf(mn, 0.0f), hi = fmaxf(mx, 0.0f);
-        const float s32 = __fdiv_rn(__fsub_rn(hi, lo), F::qscale);
+        float s32 = __fdiv_rn(__fsub_rn(hi, lo), F::qscale);
+        s32 = fminf(s32, FLT_MAX);                  // a range beyond fp32 saturates
         p.s = fp16 ? round_scale_f16(s32) : s32;
         if (p.s > 0.0f) {
-            float z = __fadd_rn((float)F::qmin, rintf(__fdiv_rn(-lo, p.s)));
-            p.zpf = fminf(fmaxf(z, (float)F::qmin), (float)F::qmax);
+            float z = rintf(__fdiv_rn(-lo, p.s));
+            z = fminf(fmaxf(z, -1.0e9f), 1.0e9f);
+            p.zpf = fminf(fmaxf(__fadd_rn((float)F::qmin, z), (float)F::qmin), (float)F::qmax);
         } else {
             p.zpf = (float)F::qmin;
         }
-        p.bound = fmaxf(-lo, hi);
+        p.lo = lo;
+        p.hi = hi;
     } else {
         const float s32 = __fdiv_rn(amax, F::qscale);
         p.s = fp16 ? round_scale_f16(s32) : s32;
         p.zpf = 0.0f;
-        p.bound = amax;
+        p.lo = -amax;
+        p.hi = amax;
     }
     return p;
 }
 
-// Quantize a chunk under a plain scale; returns codes and, when NEED_X, the dequantized
-// value of each element in xh (rotated domain). A unit with s == 0 gets code "zero"
-// (q = zp for INT, +0 for FP) and xhat = 0.
-template <int FMT, bool NEED_X>
-__device__ __forceinline__ void quant_plain_chunk(const float (&y)[16], const PlainScale& ps, const Recip& R,
-                                                  int qmin, int qmax,
-                                                  uint32_t (&w)[CodeWords<FMT>::n], float (&xh)[16])
+template <int FMT>
+__device__ __forceinline__ UnitQ unit_of_plain(const PlainScale& ps)
 {
     using F = Fmt<FMT>;
-    if (!(ps.s > 0.0f)) {
-        if constexpr (F::is_int) {
-            const uint32_t z = ((uint32_t)(int)ps.zpf) & (F::four ? 0xFu : 0xFFu);
-            const uint32_t b = F::four ? (z | (z << 4)) : z;
-            const uint32_t word = b * 0x01010101u;
-#pragma unroll
-            for (int k = 0; k < CodeWords<FMT>::n; ++k) w[k] = word;
-        } else {
-#pragma unroll
-            for (int k = 0; k < CodeWords<FMT>::n; ++k) w[k] = 0u;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = 0.0f;
-        return;
-    }
+    UnitQ u;
+    u.s = ps.s;
+    u.zpf = ps.zpf;
+    u.qmin = F::qmin;
+    u.qmax = F::qmax;
+    u.zero = !(ps.s > 0.0f);
+    const Recip R = make_recip(ps.s, fmaxf(-ps.lo, ps.hi));
+    u.rlo = R.rlo;
+    u.rhi = R.rhi;
+    u.fast = R.fast;
+    u.clamp = F::is_int ? needs_clamp(ps.lo, ps.hi, R, ps.zpf, F::qmin, F::qmax) : false;
+    return u;
+}
+
+// Quantize a chunk under a unit; xh = dequantized value (rotated domain) when NEED_X.
+template <int FMT, bool NEED_X>
+__device__ __forceinline__ void quant_unit_chunk(const float2 (&y)[8], const UnitQ& u,
+                                                 uint32_t (&w)[CodeWords<FMT>::n], float2 (&xh)[8])
+{
+    using F = Fmt<FMT>;
     if constexpr (F::is_int) {
-        float qz[16];
-        quant_int_chunk<FMT, NEED_X>(y, R, ps.zpf, qmin, qmax, w, qz);
+        float2 qz[8];
+        int_chunk<FMT, NEED_X>(y, u, w, qz);
         if constexpr (NEED_X) {
+            const float2 s = splat(u.s);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(qz[i], ps.s);
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(qz[i], s);
         }
     } else {
-        float val[16];
-        quant_fp_chunk<FMT, NEED_X>(y, R, w, val);
+        float2 val[8];
+        fp_chunk<FMT, NEED_X>(y, u, w, val);
         if constexpr (NEED_X) {
+            const float2 s = splat(u.s);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(val[i], ps.s);
+            for (int i = 0; i < 8; ++i) xh[i] = u.zero ? splat(0.0f) : mul2(val[i], s);
         }
     }
 }
 
-// Store a plain scale (and zero point) at index i.
 template <int FMT>
 __device__ __forceinline__ void store_plain_scale(void* scales, void* zps, size_t i, const PlainScale& ps, bool fp16)
 {
@@ -244,18 +306,39 @@ __device__ __forceinline__ void store_plain_scale(void* scales, void* zps, size_
     }
 }
 
-// Sums for QSNR over one chunk: err2 = sum (y - yhat)^2, x2 = sum y^2.
-__device__ __forceinline__ void chunk_sums(const float (&y)[16], const float (&xh)[16], float& e2, float& x2)
+// ---------------------------------------------------------------------------
+// QSNR sums of one chunk on values scaled by a power of two p:
+// e2 += sum ((y - xh) p)^2, x2 += sum (y p)^2 (pairs accumulate separately).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void chunk_sums2(const float2 (&y)[8], const float2 (&xh)[8], float p,
+                                            float2& e2, float2& x2)
 {
-    float e = 0.0f, s = 0.0f;
+    const float2 P = splat(p), nP = splat(-p);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float d = __fsub_rn(y[i], xh[i]);
-        e = __fmaf_rn(d, d, e);
-        s = __fmaf_rn(y[i], y[i], s);
+    for (int i = 0; i < 8; ++i) {
+        const float2 yp = mul2(y[i], P);
+        const float2 d = fma2(xh[i], nP, yp);    // (y - xh) p: xh * p is exact
+        e2 = fma2(d, d, e2);
+        x2 = fma2(yp, yp, x2);
     }
-    e2 = e;
-    x2 = s;
+}
+
+// range of a chunk
+__device__ __forceinline__ float chunk_amax(const float2 (&y)[8], float m)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = amax3(m, y[i].x, y[i].y);
+    return m;
+}
+
+__device__ __forceinline__ void chunk_minmax(const float2 (&y)[8], float& mn, float& mx)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        mn = min3(mn, y[i].x, y[i].y);
+        mx = max3(mx, y[i].x, y[i].y);
+    }
 }
 
 }  // namespace bq

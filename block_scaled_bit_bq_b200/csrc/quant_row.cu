@@ -7,11 +7,13 @@
 // ("INT vs FP at fine granularity" §2.1); asymmetric rows with a zero point
 // ("INT4/INT8/FP8 quantization" §INT8).
 //
-// A CTA owns a row at a time (persistent over rows). Each thread loads K chunks of 16
-// elements (256-bit loads, all issued before any arithmetic), the row range is reduced
-// with warp shuffles and one barrier through double-buffered shared memory, and the
-// codes are produced from registers: one read of x. Rows longer than K chunks per
-// thread are read twice (range pass, then quantize pass; the second read comes from L2).
+// A CTA owns a row at a time (persistent over rows). Each thread holds K chunks of 16
+// elements of the row (256-bit loads); the next row's chunks are loaded before the
+// current row is reduced and quantized, so the loads of one row overlap the work on
+// the previous one. The row range is reduced with warp shuffles and one barrier
+// through double-buffered shared memory, and the codes come from registers: one read
+// of x. Rows longer than 4 chunks per thread of a 256-thread CTA are read twice
+// (range pass, then quantize pass; the second read comes from L2).
 #include "quant_ops.cuh"
 #include "internal.h"
 
@@ -30,78 +32,80 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
     const bool fp16 = a.scale_fp16 != 0;
     Acc acc;
     int it = 0;
-    for (uint32_t r = blockIdx.x; r < a.rows; r += gridDim.x, ++it) {
-        const uint32_t c_row = r * a.cpr;   // first chunk of the row (flat index)
-        float y[K > 0 ? K : 1][16];
-        float amax = 0.0f, mn = 0.0f, mx = 0.0f, ss = 0.0f;
+    constexpr int KK = K > 0 ? K : 1;
+    uint32_t cur[KK][8];
 
-        auto range_of = [&](const float (&v)[16]) {
+    auto load_row = [&](uint32_t r, uint32_t (&dst)[KK][8]) {
+        const uint32_t c_row = r * a.cpr;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                amax = fmaxf(amax, fabsf(v[i]));
-                if constexpr (F::asym) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
-                if constexpr (STATS) ss = __fmaf_rn(v[i], v[i], ss);
+        for (int k = 0; k < KK; ++k) {
+            const uint32_t c = tid + k * B;
+            if (c < a.cpr) ld_nc_v8(a.x + (size_t)(c_row + c) * 8, dst[k]);
+            else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[k][i] = 0u;
             }
-        };
+        }
+    };
+
+    uint32_t r = blockIdx.x;
+    if constexpr (K > 0) {
+        if (r < a.rows) load_row(r, cur);
+    }
+    for (; r < a.rows; r += gridDim.x, ++it) {
+        const uint32_t c_row = r * a.cpr;
+        float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+        uint32_t nxt[KK][8];
 
         if constexpr (K > 0) {
-            uint32_t win[K][8];
+            const uint32_t rn = r + gridDim.x;
+            if (rn < a.rows) load_row(rn, nxt);
 #pragma unroll
             for (int k = 0; k < K; ++k) {
-                const uint32_t c = tid + k * B;
-                if (c < a.cpr) ld_nc_v8(a.x + (size_t)(c_row + c) * 8, win[k]);
-                else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) win[k][i] = 0u;
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < K; ++k) {
-                widen16(win[k], y[k]);
-                if constexpr (HAD) fwht16(y[k]);
-                range_of(y[k]);
+                float2 v[8];
+                widen16x2(cur[k], v);
+                if constexpr (HAD) fwht16x2(v);
+                amax = chunk_amax(v, amax);
+                if constexpr (F::asym) chunk_minmax(v, mn, mx);
             }
         } else {
             for (uint32_t c = tid; c < a.cpr; c += B) {
-                float v[16];
-                load16(a.x, c_row + c, v);
-                if constexpr (HAD) fwht16(v);
-                range_of(v);
+                uint32_t w[8];
+                float2 v[8];
+                ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
+                widen16x2(w, v);
+                if constexpr (HAD) fwht16x2(v);
+                amax = chunk_amax(v, amax);
+                if constexpr (F::asym) chunk_minmax(v, mn, mx);
             }
         }
 
         amax = warp_maxf(amax);
         if constexpr (F::asym) { mn = warp_minf(mn); mx = warp_maxf(mx); }
-        if constexpr (STATS) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
-        }
         float (*rb)[4] = red[it & 1];
-        if (lane == 0) { rb[warp][0] = amax; rb[warp][1] = mn; rb[warp][2] = mx; rb[warp][3] = ss; }
+        if (lane == 0) { rb[warp][0] = amax; rb[warp][1] = mn; rb[warp][2] = mx; }
         __syncthreads();
-        float A = 0.0f, MN = 0.0f, MX = 0.0f, SS = 0.0f;
-        for (int w = 0; w < nw; ++w) {
-            A = fmaxf(A, rb[w][0]); MN = fminf(MN, rb[w][1]); MX = fmaxf(MX, rb[w][2]);
-            SS = __fadd_rn(SS, rb[w][3]);
-        }
+        float A = 0.0f, MN = 0.0f, MX = 0.0f;
+        for (int w = 0; w < nw; ++w) { A = fmaxf(A, rb[w][0]); MN = fminf(MN, rb[w][1]); MX = fmaxf(MX, rb[w][2]); }
 
         const PlainScale ps = plain_scale<FMT>(A, MN, MX, fp16);
-        const Recip R = make_recip(ps.s, ps.bound);
-        if (tid == 0) {
-            store_plain_scale<FMT>(a.scales, a.zps, r, ps, fp16);
-            if constexpr (STATS) kappa_add(acc, A, SS, a.inv_cols);
-        }
+        const UnitQ u = unit_of_plain<FMT>(ps);
+        if (tid == 0) store_plain_scale<FMT>(a.scales, a.zps, r, ps, fp16);
+        const Pow2 pw = pow2_for(A);
+        float ss = 0.0f;
 
-        auto emit = [&](const float (&v)[16], uint32_t c) {
+        auto emit = [&](const float2 (&v)[8], uint32_t c) {
             uint32_t w[NW];
-            float xh[16];
-            quant_plain_chunk<FMT, STATS>(v, ps, R, F::qmin, F::qmax, w, xh);
+            float2 xh[8];
+            quant_unit_chunk<FMT, STATS>(v, u, w, xh);
             store_codes<FMT>(a.codes, c_row + c, w);
             if constexpr (STATS) {
-                float e2, x2;
-                chunk_sums(v, xh, e2, x2);
-                acc.err2 += (double)e2;
-                acc.x2 += (double)x2;
+                float2 e2 = splat(0.0f), x2 = splat(0.0f);
+                chunk_sums2(v, xh, pw.p, e2, x2);
+                const float s = __fadd_rn(x2.x, x2.y);
+                acc.err2 += (double)__fadd_rn(e2.x, e2.y) * pw.inv_p2;
+                acc.x2 += (double)s * pw.inv_p2;
+                ss = __fadd_rn(ss, s);
             }
         };
 
@@ -109,14 +113,36 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 const uint32_t c = tid + k * B;
-                if (c < a.cpr) emit(y[k], c);
+                float2 v[8];
+                widen16x2(cur[k], v);
+                if constexpr (HAD) fwht16x2(v);
+                if (c < a.cpr) emit(v, c);
             }
+#pragma unroll
+            for (int k = 0; k < K; ++k)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cur[k][i] = nxt[k][i];
         } else {
             for (uint32_t c = tid; c < a.cpr; c += B) {
-                float v[16];
-                load16(a.x, c_row + c, v);
-                if constexpr (HAD) fwht16(v);
+                uint32_t w[8];
+                float2 v[8];
+                ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
+                widen16x2(w, v);
+                if constexpr (HAD) fwht16x2(v);
                 emit(v, c);
+            }
+        }
+
+        if constexpr (STATS) {
+            // crest factor of the row: amax / sqrt(mean of squares), on scaled sums
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+            if (lane == 0) rb[warp][3] = ss;
+            __syncthreads();
+            if (tid == 0) {
+                float SS = 0.0f;
+                for (int w = 0; w < nw; ++w) SS = __fadd_rn(SS, rb[w][3]);
+                kappa_add(acc, __fmul_rn(A, pw.p), SS, a.inv_cols);
             }
         }
     }
@@ -159,19 +185,17 @@ cudaError_t run_row(const RowArgs& a, int block, cudaStream_t st)
 template <int FMT, bool HAD, bool STATS>
 cudaError_t run_row_k(const RowArgs& a, cudaStream_t st)
 {
-    // block: the smallest multiple of 32 (<= 256) that covers the row in <= K chunks
-    // per thread, K in {1, 2, 4}; longer rows stream twice with 256 threads.
+    // two chunks per thread where the row allows it (halves the per-thread scale work),
+    // one for short rows, four for long ones; blocks of 32..256 threads.
     const uint32_t cpr = a.cpr;
-    for (int k : {1, 2, 4}) {
-        const uint32_t threads = (cpr + k - 1) / k;
-        if (threads <= 256) {
-            int block = 32;
-            while ((uint32_t)block < threads) block <<= 1;
-            if (k == 1) return run_row<FMT, HAD, STATS, 1>(a, block, st);
-            if (k == 2) return run_row<FMT, HAD, STATS, 2>(a, block, st);
-            return run_row<FMT, HAD, STATS, 4>(a, block, st);
-        }
-    }
+    auto block_for = [](uint32_t threads) {
+        int b = 32;
+        while ((uint32_t)b < threads) b <<= 1;
+        return b;
+    };
+    if (cpr <= 32) return run_row<FMT, HAD, STATS, 1>(a, block_for(cpr), st);
+    if (cpr <= 512) return run_row<FMT, HAD, STATS, 2>(a, block_for((cpr + 1) / 2), st);
+    if (cpr <= 1024) return run_row<FMT, HAD, STATS, 4>(a, block_for((cpr + 3) / 4), st);
     return run_row<FMT, HAD, STATS, 0>(a, 256, st);
 }
 

@@ -41,7 +41,9 @@
  *  - Hadamard: each run of 16 elements along a row is replaced by H16 x / 4
  *    (Sylvester order, butterfly stages h = 1, 2, 4, 8 of (a+b, a-b), then * 0.25);
  *    the per-tensor range is taken on rotated values; dequantize applies the same
- *    transform again (it is its own inverse).
+ *    transform again (it is its own inverse). Rotated schemes take inputs with
+ *    |x| <= 2^125 (the rotated values then stay finite); larger inputs, and NaN or
+ *    Inf inputs for any scheme, give unspecified codes.
  *
  * Layouts (row-major, rows x cols input):
  *  - codes: 8-bit formats uint8 [rows, cols]; 4-bit formats uint8 [rows, cols/2], element
@@ -54,7 +56,8 @@
  *  - tensor_scale: one fp32 (NV only).
  *
  * Shapes: rows >= 0, cols > 0, cols % 16 == 0 (and cols % block == 0); rows * cols <
- * 2^36. rows == 0 is a valid empty call. Alignment: x, codes and out 32-byte aligned.
+ * 2^36. rows == 0 is a valid empty call. Alignment: x, codes and out 32-byte aligned;
+ * scales, zero points and the tensor scale 4-byte aligned.
  */
 #ifndef BQ_H
 #define BQ_H
@@ -71,7 +74,7 @@ typedef enum bq_status {
     BQ_ERR_INVALID_ARG = 1,   /* null pointer where one is required, bad enum value */
     BQ_ERR_UNSUPPORTED = 2,   /* format x granularity x scale dtype not offered */
     BQ_ERR_SHAPE = 3,         /* negative rows, cols not a multiple of 16 / block, too large */
-    BQ_ERR_ALIGNMENT = 4,     /* x, codes or out not 32-byte aligned */
+    BQ_ERR_ALIGNMENT = 4,     /* x, codes or out not 32-byte aligned, or a scale buffer not 4-byte aligned */
     BQ_ERR_WORKSPACE = 5,     /* workspace missing or smaller than bq_workspace_size() */
     BQ_ERR_CUDA = 6           /* a CUDA call failed (see cudaGetLastError on the caller side) */
 } bq_status;

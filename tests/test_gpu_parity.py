@@ -110,7 +110,7 @@ def check(x: torch.Tensor, s: Scheme, ws: torch.Tensor, what: str = "", full_sta
         ost = o["stats"]
         assert _close(st[1], ost[1]), (what, s, st, ost)
         assert _close(st[0], ost[0], atol=1e-30 + 1e-7 * ost[1]), (what, s, st, ost)
-        if ost[0] > 0 and ost[1] > 0:
+        if ost[0] > 0 and ost[1] > 0 and math.isfinite(ost[0]):
             assert abs(bq.bq_stats_qsnr_db(st) - oracle.qsnr_db(ost[0], ost[1])) < QSNR_TOL_DB
         assert st[4] == ost[4], (what, s, st, ost)
         assert _close(st[2], ost[2]) and _close(st[3], ost[3]), (what, s, st, ost)
@@ -134,12 +134,13 @@ def _valid(s: Scheme, cols: int) -> bool:
         return False
 
 
-def _edge_tensor(rows=8, cols=512, seed=5):
+def _edge_tensor(rows=8, cols=512, seed=5, big=1.5e38):
     g = np.random.default_rng(seed)
     a = (g.standard_t(3, size=(rows, cols)) * 0.5).astype(np.float32)
     a[0] = 0.0                                                   # all-zero row
     a[1] = (g.standard_normal(cols) * 1e-39).astype(np.float32)   # bf16 subnormals
-    a[2] = (g.uniform(-1, 1, cols) * 3.0e38).astype(np.float32)   # near the bf16 maximum
+    a[2] = (g.uniform(-1, 1, cols) * big).astype(np.float32)      # huge values of both signs
+    a[6] = (g.uniform(0.5, 1, cols) * 2.2 * big).astype(np.float32)   # up to the bf16 maximum
     # ties: multiples of 1/2 and 1/4 of a power of two under a power-of-two amax
     a[3] = (g.integers(-64, 65, cols) * 0.5).astype(np.float32)
     a[3, 0] = 64.0
@@ -153,6 +154,8 @@ INPUTS = {
     "weight_37x1024": lambda: synth.weight_outliers(37, 1024, seed=101),
     "t3_16x4096": lambda: synth.activations_t3(16, 4096, seed=102, n_outlier_channels=3),
     "edge_8x512": lambda: _edge_tensor(),
+    # rotated schemes take |x| <= 2^125
+    "edge_rot_8x512": lambda: _edge_tensor(big=1.5e38 / 16),
     "ragged_5x48": lambda: synth.normal(5, 48, seed=103, sigma=3.0),
     "single_1x16": lambda: synth.uniform(1, 16, seed=104),
     "uniform_3x2048": lambda: synth.uniform(3, 2048, seed=105),
@@ -165,6 +168,8 @@ def test_parity_small(s, name, ws):
     x = INPUTS[name]()
     if not _valid(s, x.shape[1]):
         pytest.skip("scheme does not divide this shape")
+    if s.hadamard and name == "edge_8x512":
+        pytest.skip("rotated schemes take |x| <= 2^125 (see edge_rot_8x512)")
     check(x, s, ws, name)
 
 
