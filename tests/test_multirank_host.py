@@ -1,0 +1,70 @@
+"""The multi-GPU host logic of bench.py on CPU: two gloo ranks (no GPU).
+
+Each rank owns an independent tensor (weak scaling, no collective on the data path);
+the harness takes the max of the per-rank step times and reports the whole-job
+throughput from it.
+"""
+
+import datetime
+import multiprocessing as mp
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        ms = 1.0 + 0.5 * rank                     # this rank's step time
+        m = bench.reduce_max(ms)
+        bench.barrier()
+        x = bench.gen_input("tiny_weight", rank)
+        out.put((rank, m, bench.aggregate(1.0e9, world, m), float(x.float().abs().sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_max_time_and_own_distinct_tensors():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, m0, v0, s0), (r1, m1, v1, s1) = res
+    assert m0 == m1 == 1.5                        # max over ranks
+    assert v0 == v1 == pytest.approx(2 * 1.0e9 / 1.5e-3 / 1e9)
+    assert s0 != s1                               # independent inputs per rank
+
+
+def test_single_process_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max(3.0) == 3.0          # no process group: identity
+    q, d = bench.kernel_bytes((1 << 20, 4096, 0, 0), 1024, 2048)
+    assert q == 2 * 1024 * 2048 + (1 << 20) + 4096
+    assert d == (1 << 20) + 4096 + 2 * 1024 * 2048
+    a = bench.gen_input("tiny_weight", 0)
+    b = bench.gen_input("tiny_weight", 0)
+    import torch
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))   # same seed, same bytes
