@@ -321,9 +321,10 @@ __device__ __forceinline__ Recip make_recip(float s, float amax)
     const float inv = rcp_approx(s);
     r.rlo = __fmul_rn(inv, BRACKET_LO);
     r.rhi = __fmul_rn(inv, BRACKET_HI);
-    // s normal and not huge (so 1/s, r_lo, r_hi are normal); |x/s| < 2^22 keeps the
-    // integer magic in range.
-    r.fast = (s >= FP32_MIN_NORMAL) && (s <= 1.0e37f) && (__fmul_rn(amax, r.rhi) < 4194304.0f);
+    // s well inside the normal range (so 1/s, r_lo, r_hi are normal and the residual
+    // x - h s of a tie check is exact when zero); |x/s| < 2^22 keeps the integer magic
+    // in range.
+    r.fast = (s >= 0x1p-100f) && (s <= 1.0e37f) && (__fmul_rn(amax, r.rhi) < 4194304.0f);
     return r;
 }
 

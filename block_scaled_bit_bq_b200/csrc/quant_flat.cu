@@ -112,16 +112,11 @@ struct TensorCtx {
     float S;             // NV tensor scale
 };
 
-// Accumulate one chunk's QSNR sums (scaled by p) into the lane's doubles.
-__device__ __forceinline__ void add_sums(Acc& acc, const float2 (&y)[8], const float2 (&xh)[8], const Pow2& p,
-                                         float* ss_out)
+// Fold a unit's scaled fp32 sums into the lane's doubles.
+__device__ __forceinline__ void add_unit_sums(Acc& acc, float2 e2, float2 x2, const Pow2& p)
 {
-    float2 e2 = splat(0.0f), x2 = splat(0.0f);
-    chunk_sums2(y, xh, p.p, e2, x2);
-    const float e = __fadd_rn(e2.x, e2.y), s = __fadd_rn(x2.x, x2.y);
-    acc.err2 += (double)e * p.inv_p2;
-    acc.x2 += (double)s * p.inv_p2;
-    if (ss_out) *ss_out = __fadd_rn(*ss_out, s);
+    acc.err2 += (double)__fadd_rn(e2.x, e2.y) * p.inv_p2;
+    acc.x2 += (double)__fadd_rn(x2.x, x2.y) * p.inv_p2;
 }
 
 // NV block scale: s_b = E4M3((amax / Qmax) / S), d = s_b * S.
@@ -137,17 +132,17 @@ __device__ __forceinline__ UnitQ nv_unit(float amax, float S, uint32_t& sbc, flo
         sbv = e4m3_value(sbc);
     }
     const float d = __fmul_rn(sbv, S);
+    if constexpr (F::is_int) return int_unit(d, 0.0f, -amax, amax, -7, 7);
     UnitQ u;
     u.s = d;
     u.zpf = 0.0f;
-    u.qmin = -7;
-    u.qmax = 7;
+    u.qmin = u.qmax = 0;
     u.zero = !(d > 0.0f);
     const Recip R = make_recip(d, amax);
     u.rlo = R.rlo;
     u.rhi = R.rhi;
     u.fast = R.fast;
-    u.clamp = F::is_int ? needs_clamp(-amax, amax, R, 0.0f, -7, 7) : false;
+    u.clamp_lo = u.clamp_hi = false;
     return u;
 }
 
@@ -159,19 +154,59 @@ __device__ __forceinline__ void chunk_in(const uint32_t (&w)[8], float2 (&y)[8])
     if constexpr (HAD) fwht16x2(y);
 }
 
-// Quantize one chunk under a known unit, store its codes, add its QSNR sums (and its
-// scaled sum of squares to *ss when ss is given).
-template <int FMT, bool STATS>
-__device__ __forceinline__ void emit_chunk(const float2 (&y)[8], const UnitQ& u, uint8_t* codes, uint32_t c,
-                                           bool valid, const Pow2& pw, Acc& acc, float* ss)
+// Codes of a span (two chunks) stored with one vector store: 32 bytes for 8-bit codes,
+// 16 for 4-bit; a half span (the last chunk of an odd count) stores one chunk.
+template <int FMT>
+__device__ __forceinline__ void store_span(uint8_t* codes, uint32_t span, bool full,
+                                           const uint32_t (&q0)[CodeWords<FMT>::n],
+                                           const uint32_t (&q1)[CodeWords<FMT>::n])
 {
-    constexpr int NW = CodeWords<FMT>::n;
-    uint32_t q[NW];
-    float2 xh[8];
-    quant_unit_chunk<FMT, STATS>(y, u, q, xh);
-    if (valid) {
-        store_codes<FMT>(codes, c, q);
-        if constexpr (STATS) add_sums(acc, y, xh, pw, ss);
+    if constexpr (Fmt<FMT>::four) {
+        uint8_t* p = codes + (size_t)span * 16;
+        if (full) { const uint32_t w[4] = {q0[0], q0[1], q1[0], q1[1]}; st_v4(p, w); }
+        else st_v2(p, q0);
+    } else {
+        uint8_t* p = codes + (size_t)span * 32;
+        if (full) { const uint32_t w[8] = {q0[0], q0[1], q0[2], q0[3], q1[0], q1[1], q1[2], q1[3]}; st_v8(p, w); }
+        else st_v4(p, q0);
+    }
+}
+
+// QSNR sums of one chunk under a unit scaled by p (INT codes): d = (y - q s) p with the
+// product q (s p) rounded once, e2 += d^2, x2 += (y p)^2.
+__device__ __forceinline__ void int_sums(const float2 (&y)[8], const float2 (&qz)[8], float s, float p,
+                                         float2& e2, float2& x2)
+{
+    const float2 P = splat(p), nSP = splat(-__fmul_rn(s, p));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 yp = mul2(y[i], P);
+        const float2 d = fma2(qz[i], nSP, yp);
+        e2 = fma2(d, d, e2);
+        x2 = fma2(yp, yp, x2);
+    }
+}
+
+// QSNR sums of one chunk from dequantized values xh.
+__device__ __forceinline__ void val_sums(const float2 (&y)[8], const float2 (&xh)[8], float p, float2& e2, float2& x2)
+{
+    chunk_sums2(y, xh, p, e2, x2);
+}
+
+// Quantize one chunk under a known unit; codes to q, sums added to e2 / x2.
+template <int FMT, bool STATS>
+__device__ __forceinline__ void unit_chunk(const float2 (&y)[8], const UnitQ& u, float p,
+                                           uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
+{
+    using F = Fmt<FMT>;
+    if constexpr (F::is_int) {
+        float2 qz[8];
+        int_chunk<FMT, STATS>(y, u, q, qz);
+        if constexpr (STATS) int_sums(y, qz, u.s, p, e2, x2);
+    } else {
+        float2 xh[8];
+        quant_unit_chunk<FMT, STATS>(y, u, q, xh);
+        if constexpr (STATS) val_sums(y, xh, p, e2, x2);
     }
 }
 
@@ -182,15 +217,23 @@ __device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     const uint32_t c0 = 2 * span;
-    const bool valid[2] = {c0 < a.n_chunks, c0 + 1 < a.n_chunks};
+    const bool v0 = c0 < a.n_chunks, v1 = c0 + 1 < a.n_chunks;
+    uint32_t q0[NW], q1[NW];
 
     if constexpr (GK == K_TENSOR) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
+        {
             float2 y[8];
-            chunk_in<HAD>(h ? w1 : w0, y);
-            emit_chunk<FMT, STATS>(y, tc.u, a.codes, c0 + h, valid[h], tc.p2, acc, nullptr);
+            chunk_in<HAD>(w0, y);
+            unit_chunk<FMT, STATS>(y, tc.u, tc.p2.p, q0, e2, x2);
         }
+        {
+            float2 y[8];
+            chunk_in<HAD>(w1, y);
+            // a missing second chunk reads as zeros and adds nothing to the sums
+            unit_chunk<FMT, STATS>(y, tc.u, tc.p2.p, q1, e2, x2);
+        }
+        if constexpr (STATS) add_unit_sums(acc, e2, x2, tc.p2);
     } else if (GK == K_NV || (GK == K_GROUP && a.lanes_per_group == 0)) {
         // 16-element units: two per lane, each handled start to finish
         uint32_t scode[2] = {0u, 0u};
@@ -198,25 +241,34 @@ __device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_
         for (int h = 0; h < 2; ++h) {
             float2 y[8];
             chunk_in<HAD>(h ? w1 : w0, y);
+            uint32_t (&q)[NW] = h ? q1 : q0;
             const float m = chunk_amax(y, 0.0f);
             const Pow2 pw = pow2_for(m);
-            float ss = 0.0f;
+            float2 e2 = splat(0.0f), x2 = splat(0.0f);
             if constexpr (GK == K_NV) {
                 uint32_t sbc;
                 float sbv;
                 const UnitQ u = nv_unit<FMT>(m, tc.S, sbc, sbv);
                 scode[h] = sbc;
-                uint32_t q[NW];
-                float2 z[8], xh[8];
-                if constexpr (F::is_int) int_chunk<FMT, STATS>(y, u, q, z);
-                else fp_chunk<FMT, STATS>(y, u, q, z);
-                if (valid[h]) {
-                    store_codes<FMT>(a.codes, c0 + h, q);
+                if constexpr (F::is_int) {
+                    float2 qz[8];
+                    int_chunk<FMT, STATS>(y, u, q, qz);
                     if constexpr (STATS) {
                         const float2 A = splat(sbv), S2 = splat(tc.S);
+                        float2 xh[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(qz[i], A), S2);
+                        val_sums(y, xh, pw.p, e2, x2);
+                    }
+                } else {
+                    float2 z[8];
+                    fp_chunk<FMT, STATS>(y, u, q, z);
+                    if constexpr (STATS) {
+                        const float2 A = splat(sbv), S2 = splat(tc.S);
+                        float2 xh[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) xh[i] = u.zero ? splat(0.0f) : mul2(mul2(z[i], A), S2);
-                        add_sums(acc, y, xh, pw, &ss);
+                        val_sums(y, xh, pw.p, e2, x2);
                     }
                 }
             } else {
@@ -225,17 +277,20 @@ __device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_
                 const bool f16 = a.scale_fp16 != 0;
                 const PlainScale ps = plain_scale<FMT>(m, mn, mx, f16);
                 const UnitQ u = unit_of_plain<FMT>(ps);
-                emit_chunk<FMT, STATS>(y, u, a.codes, c0 + h, valid[h], pw, acc, &ss);
-                if (valid[h]) store_plain_scale<FMT>(a.scales, a.zps, c0 + h, ps, f16);
+                unit_chunk<FMT, STATS>(y, u, pw.p, q, e2, x2);
+                if (h ? v1 : v0) store_plain_scale<FMT>(a.scales, a.zps, c0 + h, ps, f16);
             }
             if constexpr (STATS) {
-                if (valid[h]) kappa_add(acc, __fmul_rn(m, pw.p), ss, a.inv_unit);
+                if (h ? v1 : v0) {
+                    add_unit_sums(acc, e2, x2, pw);
+                    kappa_add(acc, __fmul_rn(m, pw.p), __fadd_rn(x2.x, x2.y), a.inv_unit);
+                }
             }
         }
         if constexpr (GK == K_NV) {
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
-            if (valid[1]) *reinterpret_cast<uint16_t*>(sc + c0) = (uint16_t)(scode[0] | (scode[1] << 8));
-            else if (valid[0]) sc[c0] = (uint8_t)scode[0];
+            if (v1) *reinterpret_cast<uint16_t*>(sc + c0) = (uint16_t)(scode[0] | (scode[1] << 8));
+            else if (v0) sc[c0] = (uint8_t)scode[0];
         }
     } else {
         // units of 32 elements or more: one per lane (MX, groups of 32) or T lanes per
@@ -246,58 +301,71 @@ __device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_
         for (int h = 0; h < 2; ++h) {
             float2 y[8];
             chunk_in<HAD>(h ? w1 : w0, y);
-            amax = chunk_amax(y, amax);
             if constexpr (F::asym) chunk_minmax(y, mn, mx);
+            else amax = chunk_amax(y, amax);
         }
         const int T = (GK == K_MX) ? 1 : a.lanes_per_group;
         for (int o = 1; o < T; o <<= 1) {
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             if constexpr (F::asym) {
                 mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
                 mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+            } else {
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
             }
         }
+        if constexpr (F::asym) amax = fmaxf(-mn, mx);
         const bool leader = (lane & (T - 1)) == 0;
         const Pow2 pw = pow2_for(amax);
-        float ss = 0.0f;
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
         if constexpr (GK == K_MX) {
             const int e = ue8m0_exponent<FMT>(amax);
             const float p2 = exp2i(-e);
-            const float2 PE = splat(exp2i(e));
+            const float pe = exp2i(e);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                float2 y[8], z[8], xh[8];
+                float2 y[8], z[8];
                 chunk_in<HAD>(h ? w1 : w0, y);
-                uint32_t q[NW];
-                if constexpr (F::is_int) int8_chunk_pow2<STATS>(y, p2, false, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
-                else fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
-                if (valid[h]) {
-                    store_codes<FMT>(a.codes, c0 + h, q);
+                uint32_t (&q)[NW] = h ? q1 : q0;
+                if constexpr (F::is_int) {
+                    int8_chunk_pow2<STATS>(y, p2, false, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
+                    if constexpr (STATS) int_sums(y, z, pe, pw.p, e2, x2);
+                } else {
+                    fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
                     if constexpr (STATS) {
+                        float2 xh[8];
+                        const float2 PE = splat(pe);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) xh[i] = mul2(z[i], PE);
-                        add_sums(acc, y, xh, pw, &ss);
+                        val_sums(y, xh, pw.p, e2, x2);
                     }
                 }
             }
-            if (valid[0]) reinterpret_cast<uint8_t*>(a.scales)[span] = (uint8_t)(e + 127);
+            if (v0) reinterpret_cast<uint8_t*>(a.scales)[span] = (uint8_t)(e + 127);
         } else {
             const bool f16 = a.scale_fp16 != 0;
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
             const UnitQ u = unit_of_plain<FMT>(ps);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            {
                 float2 y[8];
-                chunk_in<HAD>(h ? w1 : w0, y);
-                emit_chunk<FMT, STATS>(y, u, a.codes, c0 + h, valid[h], pw, acc, &ss);
+                chunk_in<HAD>(w0, y);
+                unit_chunk<FMT, STATS>(y, u, pw.p, q0, e2, x2);
             }
-            if (valid[0] && leader) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
+            {
+                float2 y[8];
+                chunk_in<HAD>(w1, y);
+                unit_chunk<FMT, STATS>(y, u, pw.p, q1, e2, x2);
+            }
+            if (v0 && leader) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
         }
         if constexpr (STATS) {
+            if (v0) add_unit_sums(acc, e2, x2, pw);
+            float ss = __fadd_rn(x2.x, x2.y);
             for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
-            if (valid[0] && leader) kappa_add(acc, __fmul_rn(amax, pw.p), ss, a.inv_unit);
+            if (v0 && leader) kappa_add(acc, __fmul_rn(amax, pw.p), ss, a.inv_unit);
         }
     }
+
+    if (v0) store_span<FMT>(a.codes, span, v1, q0, q1);
 }
 
 __device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint32_t n_chunks,
@@ -319,7 +387,7 @@ __device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint
 }
 
 template <int FMT, int GK, bool HAD, bool STATS>
-__global__ void __launch_bounds__(256, STATS ? 2 : 3) k_quant_flat(const FlatArgs a)
+__global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
 {
     using F = Fmt<FMT>;
     const int lane = threadIdx.x & 31;

@@ -20,21 +20,65 @@ template <int FMT> struct CodeWords { static constexpr int n = Fmt<FMT>::four ? 
 // Everything a chunk needs to know about its unit's scale.
 struct UnitQ {
     float s;        // scale the codes divide by (stored plain scale, d for NV)
-    float rlo, rhi; // reciprocal bracket
+    float rlo, rhi; // reciprocal bracket (both 0 for an INT unit with s == 0)
     float zpf;      // zero point (exact float; 0 for symmetric)
     int qmin, qmax; // integer code range
     bool fast;      // bracket usable for this unit
-    bool clamp;     // some element of the unit can fall outside [qmin, qmax]
+    bool clamp_lo;  // some element can fall below qmin
+    bool clamp_hi;  // some element can rise above qmax
     bool zero;      // s == 0 (or d == 0): every code is the zero code
 };
 
-// Is clamping needed? q is monotone in x, so the unit's extreme values bound it.
-__device__ __forceinline__ bool needs_clamp(float lo, float hi, const Recip& R, float zpf, int qmin, int qmax)
+// Clamping flags. q is monotone in x, so the unit's extreme values bound it.
+__device__ __forceinline__ void clamp_flags(float lo, float hi, const Recip& R, float zpf, int qmin, int qmax,
+                                            bool& clo, bool& chi)
 {
-    if (!R.fast) return true;
+    if (!R.fast) { clo = chi = true; return; }
     const float top = __fadd_rn(__fmaf_rn(hi, R.rhi, MAGIC), zpf);   // >= MAGIC + q for every x <= hi
     const float bot = __fadd_rn(__fmaf_rn(lo, R.rhi, MAGIC), zpf);   // <= MAGIC + q for every x >= lo (lo <= 0)
-    return top > MAGIC + (float)qmax || bot < MAGIC + (float)qmin;
+    chi = top > MAGIC + (float)qmax;
+    clo = bot < MAGIC + (float)qmin;
+}
+
+// Integer unit from a scale: a unit with s == 0 maps every element to the zero code
+// through the fast path itself (r_lo = r_hi = 0 gives q = 0, plus the zero point).
+__device__ __forceinline__ UnitQ int_unit(float s, float zpf, float lo, float hi, int qmin, int qmax)
+{
+    UnitQ u;
+    u.s = s;
+    u.zpf = zpf;
+    u.qmin = qmin;
+    u.qmax = qmax;
+    u.zero = !(s > 0.0f);
+    if (u.zero) {
+        u.rlo = u.rhi = 0.0f;
+        u.fast = true;
+        u.clamp_lo = u.clamp_hi = false;
+        return u;
+    }
+    const Recip R = make_recip(s, fmaxf(-lo, hi));
+    u.rlo = R.rlo;
+    u.rhi = R.rhi;
+    u.fast = R.fast;
+    clamp_flags(lo, hi, R, zpf, qmin, qmax, u.clamp_lo, u.clamp_hi);
+    return u;
+}
+
+// Settle elements whose bracket ends disagree. The two candidates are adjacent
+// integers; h is the half-integer between them. fma(-h, s, x) is the exactly rounded
+// x - h s, which is zero only when x / s == h exactly: then RN(x/s) = h and the code is
+// the even candidate (the magic sum's low bit is the integer's parity). Any other
+// disagreement returns false and the caller divides.
+__device__ __forceinline__ bool settle_ties(float y, float s, float rhi, float& t)
+{
+    const float a = t;
+    const float b = __fmaf_rn(y, rhi, MAGIC);
+    if (__float_as_uint(a) == __float_as_uint(b)) return true;
+    const float qa = __fsub_rn(a, MAGIC), qb = __fsub_rn(b, MAGIC);   // exact
+    const float h = __fmul_rn(0.5f, __fadd_rn(qa, qb));                // exact: an odd integer / 2
+    if (__fmaf_rn(-h, s, y) != 0.0f) return false;
+    t = (__float_as_uint(a) & 1u) == 0u ? a : b;
+    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -47,44 +91,49 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const UnitQ& u,
 {
     using F = Fmt<FMT>;
     float2 t[8];
-    if (u.zero) {
+    bool ok = u.fast;
+    if (ok) {
+        uint32_t mism = 0;
+        const float2 lo = splat(u.rlo), hi = splat(u.rhi), m = splat(MAGIC);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = splat(__fadd_rn(MAGIC, u.zpf));
-    } else {
-        bool ok = u.fast;
-        if (ok) {
-            uint32_t mism = 0;
-            const float2 lo = splat(u.rlo), hi = splat(u.rhi), m = splat(MAGIC);
+        for (int i = 0; i < 8; ++i) {
+            const float2 a = fma2(y[i], lo, m);
+            const float2 b = fma2(y[i], hi, m);
+            mism |= (__float_as_uint(a.x) ^ __float_as_uint(b.x)) | (__float_as_uint(a.y) ^ __float_as_uint(b.y));
+            t[i] = a;
+        }
+        if (mism) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float2 a = fma2(y[i], lo, m);
-                const float2 b = fma2(y[i], hi, m);
-                mism |= (__float_as_uint(a.x) ^ __float_as_uint(b.x)) | (__float_as_uint(a.y) ^ __float_as_uint(b.y));
-                t[i] = a;
-            }
-            ok = (mism == 0);
-        }
-        if (!ok) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float qa = rintf(__fdiv_rn(y[i].x, u.s));
-                float qb = rintf(__fdiv_rn(y[i].y, u.s));
-                qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
-                qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
-                t[i] = make_float2(__fadd_rn(qa, MAGIC), __fadd_rn(qb, MAGIC));
+                ok &= settle_ties(y[i].x, u.s, u.rhi, t[i].x);
+                ok &= settle_ties(y[i].y, u.s, u.rhi, t[i].y);
             }
         }
-        if constexpr (F::asym) {
-            const float2 z = splat(u.zpf);
+    }
+    if (!ok) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) t[i] = add2(t[i], z);
+        for (int i = 0; i < 8; ++i) {
+            float qa = rintf(__fdiv_rn(y[i].x, u.s));
+            float qb = rintf(__fdiv_rn(y[i].y, u.s));
+            qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
+            qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
+            t[i] = make_float2(__fadd_rn(qa, MAGIC), __fadd_rn(qb, MAGIC));
         }
-        if (u.clamp) {
-            const float cmin = MAGIC + (float)u.qmin, cmax = MAGIC + (float)u.qmax;
+    }
+    if constexpr (F::asym) {
+        const float2 z = splat(u.zpf);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
-        }
+        for (int i = 0; i < 8; ++i) t[i] = add2(t[i], z);
+    }
+    if (u.clamp_hi || !ok) {
+        const float cmax = MAGIC + (float)u.qmax;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = make_float2(fminf(t[i].x, cmax), fminf(t[i].y, cmax));
+    }
+    if (u.clamp_lo || !ok) {
+        const float cmin = MAGIC + (float)u.qmin;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = make_float2(fmaxf(t[i].x, cmin), fmaxf(t[i].y, cmin));
     }
     if constexpr (NEED_Q) {
         const float2 z = splat(-__fadd_rn(MAGIC, u.zpf));
@@ -255,17 +304,17 @@ template <int FMT>
 __device__ __forceinline__ UnitQ unit_of_plain(const PlainScale& ps)
 {
     using F = Fmt<FMT>;
+    if constexpr (F::is_int) return int_unit(ps.s, ps.zpf, ps.lo, ps.hi, F::qmin, F::qmax);
     UnitQ u;
     u.s = ps.s;
-    u.zpf = ps.zpf;
-    u.qmin = F::qmin;
-    u.qmax = F::qmax;
+    u.zpf = 0.0f;
+    u.qmin = u.qmax = 0;
     u.zero = !(ps.s > 0.0f);
     const Recip R = make_recip(ps.s, fmaxf(-ps.lo, ps.hi));
     u.rlo = R.rlo;
     u.rhi = R.rhi;
     u.fast = R.fast;
-    u.clamp = F::is_int ? needs_clamp(ps.lo, ps.hi, R, ps.zpf, F::qmin, F::qmax) : false;
+    u.clamp_lo = u.clamp_hi = false;
     return u;
 }
 
@@ -281,7 +330,7 @@ __device__ __forceinline__ void quant_unit_chunk(const float2 (&y)[8], const Uni
         if constexpr (NEED_X) {
             const float2 s = splat(u.s);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) xh[i] = mul2(qz[i], s);
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(qz[i], s);   // s == 0 gives 0: qz is 0 there
         }
     } else {
         float2 val[8];
