@@ -239,9 +239,11 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
     a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
     a.n_chunks = p.n_chunks;
-    a.n_dtiles = (uint32_t)((p.n_chunks + 63u) / 64u);
-    // units of 16 elements are lane-local (0); larger units span block / 32 lanes
-    a.lanes_per_group = (p.gran == BQ_PER_GROUP && p.block > 16) ? p.block / 32 : (p.gran == BQ_PER_GROUP ? 0 : 1);
+    // a warp tile is 32 lanes x 4 chunks
+    a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
+    // groups: 16 elements -> 0 (four units per lane), 32 -> -1 (two per lane),
+    // 64 and up -> lanes per group (one unit over block / 64 lanes)
+    a.lanes_per_group = p.gran != BQ_PER_GROUP ? 1 : (p.block == 16 ? 0 : (p.block == 32 ? -1 : p.block / 64));
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     a.n_elems = (double)p.n;
     a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;

@@ -233,6 +233,26 @@ __device__ __forceinline__ float min3(float a, float b, float c)
     return r;
 }
 
+// Packed bf16 pairs. min / max pick one of their inputs, so they are exact; the bit
+// patterns of non-negative bf16 values order like unsigned integers, so the largest
+// magnitude of a pair is an unsigned 16-bit max of the sign-cleared halves.
+__device__ __forceinline__ uint32_t bf2_absmax(uint32_t m, uint32_t w) { return __vmaxu2(m, w & 0x7FFF7FFFu); }
+
+__device__ __forceinline__ uint32_t bf2_min(uint32_t a, uint32_t b)
+{
+    const __nv_bfloat162 r = __hmin2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t bf2_max(uint32_t a, uint32_t b)
+{
+    const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 // 16 bf16 -> 8 fp32 pairs (pair i = elements 2i, 2i+1), exactly.
 __device__ __forceinline__ void widen16x2(const uint32_t (&w)[8], float2 (&v)[8])
 {

@@ -44,7 +44,12 @@ __device__ __forceinline__ void load_codes(const uint8_t* codes, uint32_t span, 
     }
 }
 
-// Element values of chunk h (0 or 1) of a span: integers as exact floats, FP codes decoded.
+// Element values of chunk h (0 or 1) of a span: FP codes decoded; integer codes as
+// exact floats offset by MAGIC + bias (the caller subtracts MAGIC + bias + zero point in
+// the same exact addition). An integer code's float is assembled by one byte permute:
+// the (biased, non-negative) code byte becomes the low byte of MAGIC's bit pattern.
+template <int FMT> struct DecodeBias { static constexpr int v = (FMT == BQ_INT8_SYM || FMT == BQ_INT8_ASYM) ? 128 : (FMT == BQ_INT4_SYM ? 8 : 0); };
+
 template <int FMT>
 __device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>::n], int h, float2 (&val)[8])
 {
@@ -52,12 +57,16 @@ __device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>:
     if constexpr (F::four) {
         const uint32_t w0 = w[2 * h], w1 = w[2 * h + 1];
         if constexpr (F::is_int) {
+            constexpr uint32_t flip = DecodeBias<FMT>::v == 8 ? 0x08080808u : 0u;
+            // byte k of lo* holds element 2k, byte k of hi* element 2k + 1
+            const uint32_t lo0 = (w0 & 0x0F0F0F0Fu) ^ flip, hi0 = ((w0 >> 4) & 0x0F0F0F0Fu) ^ flip;
+            const uint32_t lo1 = (w1 & 0x0F0F0F0Fu) ^ flip, hi1 = ((w1 >> 4) & 0x0F0F0F0Fu) ^ flip;
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const uint32_t byte = ((p < 4 ? w0 : w1) >> (8 * (p & 3))) & 0xFFu;
-                int qa = (int)(byte & 0xFu), qb = (int)(byte >> 4);
-                if constexpr (FMT != BQ_UINT4_ASYM) { qa = (qa ^ 8) - 8; qb = (qb ^ 8) - 8; }
-                val[p] = make_float2((float)qa, (float)qb);
+                const uint32_t lo = p < 4 ? lo0 : lo1, hi = p < 4 ? hi0 : hi1;
+                const uint32_t sel = 0x7650u | (uint32_t)(p & 3);
+                val[p] = make_float2(__uint_as_float(__byte_perm(lo, MAGIC_BITS, sel)),
+                                     __uint_as_float(__byte_perm(hi, MAGIC_BITS, sel)));
             }
         } else {
 #pragma unroll
@@ -66,10 +75,12 @@ __device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>:
     } else {
         if constexpr (F::is_int) {
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint32_t word = w[4 * h + (p >> 1)];
-                const int sh = 16 * (p & 1);
-                val[p] = make_float2((float)(int)(int8_t)(word >> sh), (float)(int)(int8_t)(word >> (sh + 8)));
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t word = w[4 * h + k] ^ 0x80808080u;     // two's complement byte + 128
+                val[2 * k] = make_float2(__uint_as_float(__byte_perm(word, MAGIC_BITS, 0x7650u)),
+                                         __uint_as_float(__byte_perm(word, MAGIC_BITS, 0x7651u)));
+                val[2 * k + 1] = make_float2(__uint_as_float(__byte_perm(word, MAGIC_BITS, 0x7652u)),
+                                             __uint_as_float(__byte_perm(word, MAGIC_BITS, 0x7653u)));
             }
         } else {
 #pragma unroll
@@ -84,17 +95,30 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
                                               float2 (&xh)[8])
 {
     using F = Fmt<FMT>;
+    constexpr float off = MAGIC + (float)DecodeBias<FMT>::v;     // integer codes arrive as off + q
     const uint32_t u = a.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, a.fd_m) + c) >> a.fd_s);
     if constexpr (SK == SK_UE8M0) {
         const int e = (int)reinterpret_cast<const uint8_t*>(a.scales)[u] - 127;
         const float2 pe = splat(exp2i(e));
+        if constexpr (F::is_int) {
+            const float2 nz = splat(-off);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], pe);
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(add2(val[i], nz), pe);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], pe);
+        }
     } else if constexpr (SK == SK_NV) {
         const float2 sbv = splat(e4m3_value(reinterpret_cast<const uint8_t*>(a.scales)[u]));
         const float2 S = splat(a.tensor_scale[0]);
+        if constexpr (F::is_int) {
+            const float2 nz = splat(-off);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(val[i], sbv), S);
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(add2(val[i], nz), sbv), S);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(val[i], sbv), S);
+        }
     } else {
         float s, zp = 0.0f;
         if (a.scale_fp16) {
@@ -105,10 +129,11 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
             if constexpr (F::asym) zp = reinterpret_cast<const float*>(a.zps)[u];
         }
         const float2 S = splat(s);
-        if constexpr (F::asym) {
-            const float2 nz = splat(-zp);
+        if constexpr (F::is_int) {
+            // (off + q) - (off + zp) = q - zp, exact
+            const float2 nz = splat(-__fadd_rn(off, zp));
 #pragma unroll
-            for (int i = 0; i < 8; ++i) xh[i] = mul2(add2(val[i], nz), S);   // q - zp is exact
+            for (int i = 0; i < 8; ++i) xh[i] = mul2(add2(val[i], nz), S);
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], S);

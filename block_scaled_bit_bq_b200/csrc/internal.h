@@ -20,8 +20,8 @@ struct FlatArgs {
     bq_stats* stats;
     uint8_t* ws;
     uint32_t n_chunks;          // rows * cols / 16
-    uint32_t n_dtiles;          // ceil(n_chunks / 64): a warp takes 64 chunks per step
-    int32_t lanes_per_group;    // per-group: block / 16 (power of two, <= 32)
+    uint32_t n_dtiles;          // ceil(n_chunks / 128): a warp takes 128 chunks per step
+    int32_t lanes_per_group;    // per-group: 0 (block 16), -1 (block 32), block / 64 (64..512)
     int32_t scale_fp16;         // 1: fp16 scales and zero points
     double n_elems;
     float inv_unit;             // 1 / elements per scaling unit (kappa)

@@ -2,12 +2,10 @@
 // 16-element chunks: per-tensor (after the range pass), per-group, MX block-32 and
 // NV block-16 granularities; and the per-tensor range pass itself.
 //
-// Layout of the work: lane l of a warp owns a span of two consecutive chunks (32
-// elements, 64 bytes, two 256-bit loads) of the warp's 1024-element tile; the next
-// tile's span is loaded before the current one is processed, so every lane keeps 64
-// bytes in flight while it computes. A scaling unit of G >= 32 elements spans G/32
-// adjacent lanes and is reduced with xor shuffles; 16-element units (NV blocks,
-// groups of 16) are lane-local. The grid is at most one wave (SM count x resident
+// Layout of the work: lane l of a warp owns a span of four consecutive chunks (64
+// elements, 128 bytes) of the warp's 2048-element tile. Scaling units of 16, 32 or 64
+// elements are lane-local; a unit of G >= 128 elements spans G/64 adjacent lanes and
+// is reduced with xor shuffles. The grid is at most one wave (SM count x resident
 // CTAs) striding over the tiles.
 //
 // Steps (source pages): AbsMax scale per unit ("INT vs FP at fine granularity" §2.1,
@@ -102,51 +100,22 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
 
 // ---------------------------------------------------------------------------
 // Quantize kernel.
+//
+// Lane l of a warp owns a span of four consecutive chunks (64 elements, 128 bytes,
+// four 256-bit loads, all issued before any arithmetic) of the warp's 2048-element
+// tile; two CTAs of eight warps per SM keep 64 KB of loads in flight.
 // ---------------------------------------------------------------------------
+
+constexpr int SPAN = 4;   // chunks per lane per tile
 
 struct TensorCtx {
     float amax;          // per-tensor / NV: amax of the (rotated) tensor
     PlainScale ps;       // per-tensor plain scale
-    UnitQ u;             // per-tensor unit
-    Pow2 p2;             // per-tensor sum scaling
     float S;             // NV tensor scale
+    float cS;            // ~ 1 / (Qmax * S) for the NV block-scale bracket
 };
 
-// Fold a unit's scaled fp32 sums into the lane's doubles.
-__device__ __forceinline__ void add_unit_sums(Acc& acc, float2 e2, float2 x2, const Pow2& p)
-{
-    acc.err2 += (double)__fadd_rn(e2.x, e2.y) * p.inv_p2;
-    acc.x2 += (double)__fadd_rn(x2.x, x2.y) * p.inv_p2;
-}
-
-// NV block scale: s_b = E4M3((amax / Qmax) / S), d = s_b * S.
-template <int FMT>
-__device__ __forceinline__ UnitQ nv_unit(float amax, float S, uint32_t& sbc, float& sbv)
-{
-    using F = Fmt<FMT>;
-    sbc = 0;
-    sbv = 0.0f;
-    if (S > 0.0f) {
-        const float sb32 = __fdiv_rn(__fdiv_rn(amax, F::qscale), S);
-        sbc = e4m3_code(sb32);
-        sbv = e4m3_value(sbc);
-    }
-    const float d = __fmul_rn(sbv, S);
-    if constexpr (F::is_int) return int_unit(d, 0.0f, -amax, amax, -7, 7);
-    UnitQ u;
-    u.s = d;
-    u.zpf = 0.0f;
-    u.qmin = u.qmax = 0;
-    u.zero = !(d > 0.0f);
-    const Recip R = make_recip(d, amax);
-    u.rlo = R.rlo;
-    u.rhi = R.rhi;
-    u.fast = R.fast;
-    u.clamp_lo = u.clamp_hi = false;
-    return u;
-}
-
-// Widen (and rotate) one chunk of a span.
+// Widen (and rotate) one chunk.
 template <bool HAD>
 __device__ __forceinline__ void chunk_in(const uint32_t (&w)[8], float2 (&y)[8])
 {
@@ -154,235 +123,261 @@ __device__ __forceinline__ void chunk_in(const uint32_t (&w)[8], float2 (&y)[8])
     if constexpr (HAD) fwht16x2(y);
 }
 
-// Codes of a span (two chunks) stored with one vector store: 32 bytes for 8-bit codes,
-// 16 for 4-bit; a half span (the last chunk of an odd count) stores one chunk.
-template <int FMT>
-__device__ __forceinline__ void store_span(uint8_t* codes, uint32_t span, bool full,
-                                           const uint32_t (&q0)[CodeWords<FMT>::n],
-                                           const uint32_t (&q1)[CodeWords<FMT>::n])
+// Range of chunks [c0, c0 + N) of the lane's span: amax, or min and max (asymmetric).
+template <bool HAD, bool ASYM, int N>
+__device__ __forceinline__ void span_range(const uint32_t (&w)[SPAN][8], int c0, float& amax, float& mn, float& mx)
 {
-    if constexpr (Fmt<FMT>::four) {
-        uint8_t* p = codes + (size_t)span * 16;
-        if (full) { const uint32_t w[4] = {q0[0], q0[1], q1[0], q1[1]}; st_v4(p, w); }
-        else st_v2(p, q0);
-    } else {
-        uint8_t* p = codes + (size_t)span * 32;
-        if (full) { const uint32_t w[8] = {q0[0], q0[1], q0[2], q0[3], q1[0], q1[1], q1[2], q1[3]}; st_v8(p, w); }
-        else st_v4(p, q0);
-    }
-}
-
-// QSNR sums of one chunk under a unit scaled by p (INT codes): d = (y - q s) p with the
-// product q (s p) rounded once, e2 += d^2, x2 += (y p)^2.
-__device__ __forceinline__ void int_sums(const float2 (&y)[8], const float2 (&qz)[8], float s, float p,
-                                         float2& e2, float2& x2)
-{
-    const float2 P = splat(p), nSP = splat(-__fmul_rn(s, p));
+    if constexpr (HAD) {
+        amax = 0.0f; mn = 0.0f; mx = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float2 yp = mul2(y[i], P);
-        const float2 d = fma2(qz[i], nSP, yp);
-        e2 = fma2(d, d, e2);
-        x2 = fma2(yp, yp, x2);
+        for (int k = 0; k < N; ++k) {
+            float2 y[8];
+            chunk_in<true>(w[c0 + k], y);
+            if constexpr (ASYM) chunk_minmax(y, mn, mx);
+            else amax = chunk_amax(y, amax);
+        }
+        if constexpr (ASYM) amax = fmaxf(-mn, mx);
+    } else if constexpr (ASYM) {
+        uint32_t lo = 0u, hi = 0u;          // bf16 pair (+0, +0)
+#pragma unroll
+        for (int k = 0; k < N; ++k) words_minmax(w[c0 + k], lo, hi);
+        mn = pair_min(lo);
+        mx = pair_max(hi);
+        amax = fmaxf(-mn, mx);
+    } else {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int k = 0; k < N; ++k) m = words_absmax(w[c0 + k], m);
+        amax = pair_absmax(m);
+        mn = mx = 0.0f;
     }
 }
 
-// QSNR sums of one chunk from dequantized values xh.
-__device__ __forceinline__ void val_sums(const float2 (&y)[8], const float2 (&xh)[8], float p, float2& e2, float2& x2)
-{
-    chunk_sums2(y, xh, p, e2, x2);
-}
-
-// Quantize one chunk under a known unit; codes to q, sums added to e2 / x2.
-template <int FMT, bool STATS>
-__device__ __forceinline__ void unit_chunk(const float2 (&y)[8], const UnitQ& u, float p,
-                                           uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
+// NV block scale: s_b = E4M3((amax / Qmax) / S), d = s_b * S. The E4M3 code is taken
+// from the bracket amax * c (1 -+ 2^-20), c ~ 1 / (Qmax S) within 2^-23, which holds
+// RN(RN(amax / Qmax) / S) strictly inside; where the two codes differ it divides.
+template <int FMT>
+__device__ __forceinline__ uint32_t nv_scale_code(float amax, float S, float cS)
 {
     using F = Fmt<FMT>;
-    if constexpr (F::is_int) {
-        float2 qz[8];
-        int_chunk<FMT, STATS>(y, u, q, qz);
-        if constexpr (STATS) int_sums(y, qz, u.s, p, e2, x2);
+    if (!(S > 0.0f)) return 0u;
+    const float a = __fmul_rn(amax, cS);
+    const uint32_t pair = cvt_pair<BQ_FP8_E4M3>(__fmul_rn(a, BRACKET_HI), __fmul_rn(a, BRACKET_LO));
+    const uint32_t lo = pair & 0xFFu, hi = pair >> 8;
+    if (lo == hi && S >= 0x1p-100f && S <= 1.0e30f) return lo;
+    return e4m3_code(__fdiv_rn(__fdiv_rn(amax, F::qscale), S));
+}
+
+// Codes of chunk k of the lane's span: 4-bit codes are gathered for one 32-byte store
+// per span, 8-bit codes are stored right away (16 bytes per chunk).
+template <int FMT>
+__device__ __forceinline__ void put_codes(uint32_t (&span4)[8], uint8_t* codes, uint32_t c, bool valid, int k,
+                                          const uint32_t (&w)[CodeWords<FMT>::n])
+{
+    if constexpr (Fmt<FMT>::four) {
+        span4[2 * k] = w[0];
+        span4[2 * k + 1] = w[1];
     } else {
-        float2 xh[8];
-        quant_unit_chunk<FMT, STATS>(y, u, q, xh);
-        if constexpr (STATS) val_sums(y, xh, p, e2, x2);
+        if (valid) st_v4(codes + (size_t)c * 16, w);
     }
 }
 
-template <int FMT, int GK, bool HAD, bool STATS>
-__device__ __forceinline__ void flat_span(const uint32_t (&w0)[8], const uint32_t (&w1)[8], uint32_t span,
-                                          const FlatArgs& a, const TensorCtx& tc, Acc& acc, int lane)
+// One lane's span under the per-tensor unit.
+template <int FMT, bool HAD, bool STATS>
+__device__ __forceinline__ void span_tensor(const uint32_t (&w)[SPAN][8], uint32_t span, const FlatArgs& a,
+                                            const PlainUnit<FMT>& u, float p, double inv_p2, bool scaled,
+                                            Acc& acc, uint32_t (&span4)[8])
+{
+    float2 e2 = splat(0.0f), x2 = splat(0.0f);
+    const bool exact_res = !HAD && a.scale_fp16 != 0;
+#pragma unroll
+    for (int k = 0; k < SPAN; ++k) {
+        float2 y[8];
+        uint32_t q[CodeWords<FMT>::n];
+        chunk_in<HAD>(w[k], y);
+        if (scaled) plain_chunk<FMT, STATS, true>(y, u, p, exact_res, q, e2, x2);
+        else plain_chunk<FMT, STATS, false>(y, u, p, exact_res, q, e2, x2);
+        const uint32_t c = SPAN * span + k;
+        put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
+    }
+    if constexpr (STATS) add_unit_sums(acc, e2, x2, scaled ? inv_p2 : 1.0);
+}
+
+// Units of N chunks (N = 1, 2 or 4) inside the lane's span; with N = 4 a unit can
+// also span T lanes (T = 1, 2, 4, 8: groups of 64 .. 512). A one-chunk unit is widened
+// (and rotated) once; larger units take their range from the raw bf16 words (or, when
+// rotated, from a first rotation) and widen again to quantize, which keeps register
+// pressure low.
+template <int FMT, int GK, bool HAD, bool STATS, int N>
+__device__ __forceinline__ void span_units(const uint32_t (&w)[SPAN][8], uint32_t span, const FlatArgs& a,
+                                           const TensorCtx& tc, Acc& acc, int lane, int T,
+                                           uint32_t (&span4)[8], uint8_t (&scode)[SPAN])
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
-    const uint32_t c0 = 2 * span;
-    const bool v0 = c0 < a.n_chunks, v1 = c0 + 1 < a.n_chunks;
-    uint32_t q0[NW], q1[NW];
-
-    if constexpr (GK == K_TENSOR) {
-        float2 e2 = splat(0.0f), x2 = splat(0.0f);
-        {
-            float2 y[8];
-            chunk_in<HAD>(w0, y);
-            unit_chunk<FMT, STATS>(y, tc.u, tc.p2.p, q0, e2, x2);
-        }
-        {
-            float2 y[8];
-            chunk_in<HAD>(w1, y);
-            // a missing second chunk reads as zeros and adds nothing to the sums
-            unit_chunk<FMT, STATS>(y, tc.u, tc.p2.p, q1, e2, x2);
-        }
-        if constexpr (STATS) add_unit_sums(acc, e2, x2, tc.p2);
-    } else if (GK == K_NV || (GK == K_GROUP && a.lanes_per_group == 0)) {
-        // 16-element units: two per lane, each handled start to finish
-        uint32_t scode[2] = {0u, 0u};
+    constexpr bool GASYM = F::asym && GK == K_GROUP;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float2 y[8];
-            chunk_in<HAD>(h ? w1 : w0, y);
-            uint32_t (&q)[NW] = h ? q1 : q0;
-            const float m = chunk_amax(y, 0.0f);
-            const Pow2 pw = pow2_for(m);
-            float2 e2 = splat(0.0f), x2 = splat(0.0f);
-            if constexpr (GK == K_NV) {
-                uint32_t sbc;
-                float sbv;
-                const UnitQ u = nv_unit<FMT>(m, tc.S, sbc, sbv);
-                scode[h] = sbc;
-                if constexpr (F::is_int) {
-                    float2 qz[8];
-                    int_chunk<FMT, STATS>(y, u, q, qz);
-                    if constexpr (STATS) {
-                        const float2 A = splat(sbv), S2 = splat(tc.S);
-                        float2 xh[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(qz[i], A), S2);
-                        val_sums(y, xh, pw.p, e2, x2);
-                    }
-                } else {
-                    float2 z[8];
-                    fp_chunk<FMT, STATS>(y, u, q, z);
-                    if constexpr (STATS) {
-                        const float2 A = splat(sbv), S2 = splat(tc.S);
-                        float2 xh[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) xh[i] = u.zero ? splat(0.0f) : mul2(mul2(z[i], A), S2);
-                        val_sums(y, xh, pw.p, e2, x2);
-                    }
-                }
-            } else {
-                float mn = 0.0f, mx = 0.0f;
-                if constexpr (F::asym) chunk_minmax(y, mn, mx);
-                const bool f16 = a.scale_fp16 != 0;
-                const PlainScale ps = plain_scale<FMT>(m, mn, mx, f16);
-                const UnitQ u = unit_of_plain<FMT>(ps);
-                unit_chunk<FMT, STATS>(y, u, pw.p, q, e2, x2);
-                if (h ? v1 : v0) store_plain_scale<FMT>(a.scales, a.zps, c0 + h, ps, f16);
-            }
-            if constexpr (STATS) {
-                if (h ? v1 : v0) {
-                    add_unit_sums(acc, e2, x2, pw);
-                    kappa_add(acc, __fmul_rn(m, pw.p), __fadd_rn(x2.x, x2.y), a.inv_unit);
-                }
-            }
-        }
-        if constexpr (GK == K_NV) {
-            uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
-            if (v1) *reinterpret_cast<uint16_t*>(sc + c0) = (uint16_t)(scode[0] | (scode[1] << 8));
-            else if (v0) sc[c0] = (uint8_t)scode[0];
-        }
-    } else {
-        // units of 32 elements or more: one per lane (MX, groups of 32) or T lanes per
-        // unit. Range first (the chunks are widened again for the quantize step, which
-        // keeps register pressure low).
+    for (int base = 0; base < SPAN; base += N) {
         float amax = 0.0f, mn = 0.0f, mx = 0.0f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float2 y[8];
-            chunk_in<HAD>(h ? w1 : w0, y);
-            if constexpr (F::asym) chunk_minmax(y, mn, mx);
-            else amax = chunk_amax(y, amax);
+        float2 y1[8];                      // the chunk of a one-chunk unit
+        if constexpr (N == 1) {
+            chunk_in<HAD>(w[base], y1);
+            if constexpr (GASYM) { chunk_minmax(y1, mn, mx); amax = fmaxf(-mn, mx); }
+            else amax = chunk_amax(y1, 0.0f);
+        } else {
+            span_range<HAD, GASYM, N>(w, base, amax, mn, mx);
         }
-        const int T = (GK == K_MX) ? 1 : a.lanes_per_group;
-        for (int o = 1; o < T; o <<= 1) {
-            if constexpr (F::asym) {
-                mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-            } else {
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (N == SPAN && T > 1) {
+            for (int o = 1; o < T; o <<= 1) {
+                if constexpr (GASYM) {
+                    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                } else {
+                    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                }
             }
+            if constexpr (GASYM) amax = fmaxf(-mn, mx);
         }
-        if constexpr (F::asym) amax = fmaxf(-mn, mx);
-        const bool leader = (lane & (T - 1)) == 0;
+        const bool scaled = STATS && __any_sync(0xFFFFFFFFu, !plain_sums_ok(amax));
         const Pow2 pw = pow2_for(amax);
+        const float p = scaled ? pw.p : 1.0f;
         float2 e2 = splat(0.0f), x2 = splat(0.0f);
+
         if constexpr (GK == K_MX) {
             const int e = ue8m0_exponent<FMT>(amax);
-            const float p2 = exp2i(-e);
-            const float pe = exp2i(e);
+            const float p2 = exp2i(-e), pe = exp2i(e);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int k = 0; k < N; ++k) {
                 float2 y[8], z[8];
-                chunk_in<HAD>(h ? w1 : w0, y);
-                uint32_t (&q)[NW] = h ? q1 : q0;
+                uint32_t q[NW];
+                if constexpr (N == 1) { for (int i = 0; i < 8; ++i) y[i] = y1[i]; }
+                else chunk_in<HAD>(w[base + k], y);
                 if constexpr (F::is_int) {
-                    int8_chunk_pow2<STATS>(y, p2, false, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
-                    if constexpr (STATS) int_sums(y, z, pe, pw.p, e2, x2);
+                    int8_chunk_pow2<STATS>(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
+                    if constexpr (STATS) {
+                        if (scaled) int_sums<true>(y, z, pe, p, e2, x2);
+                        else int_sums<false>(y, z, pe, p, e2, x2);
+                    }
                 } else {
                     fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
                     if constexpr (STATS) {
-                        float2 xh[8];
-                        const float2 PE = splat(pe);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) xh[i] = mul2(z[i], PE);
-                        val_sums(y, xh, pw.p, e2, x2);
+                        if (scaled) val_sums<true>(y, z, pe, p, e2, x2);
+                        else val_sums<false>(y, z, pe, p, e2, x2);
                     }
                 }
+                const uint32_t c = SPAN * span + base + k;
+                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base + k, q);
             }
-            if (v0) reinterpret_cast<uint8_t*>(a.scales)[span] = (uint8_t)(e + 127);
-        } else {
+            scode[base] = (uint8_t)(e + 127);
+        } else if constexpr (GK == K_NV) {
+            // N == 1
+            const uint32_t sbc = nv_scale_code<FMT>(amax, tc.S, tc.cS);
+            const float sbv = e4m3_value(sbc);
+            const float d = __fmul_rn(sbv, tc.S);
+            scode[base] = (uint8_t)sbc;
+            uint32_t q[NW];
+            if constexpr (F::is_int) {
+                const IntQ iq = int_unit<FMT>(d, 0.0f, -amax, amax, -7, 7);
+                float2 nq[8];
+                int_chunk<FMT, STATS>(y1, iq, -7, 7, q, nq);
+                if constexpr (STATS) {
+                    // x-hat = (q s_b) S: the first product is exact
+                    float2 val[8];
+                    const float2 nA = splat(-sbv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) val[i] = mul2(nq[i], nA);
+                    if (scaled) val_sums<true>(y1, val, tc.S, p, e2, x2);
+                    else val_sums<false>(y1, val, tc.S, p, e2, x2);
+                }
+            } else {
+                const FpQ fq = fp_unit(d, amax);
+                float2 val[8];
+                fp_chunk<FMT, STATS>(y1, fq, q, val);
+                if constexpr (STATS) {
+                    const float2 A = splat(fq.zero ? 0.0f : sbv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) val[i] = mul2(val[i], A);
+                    if (scaled) val_sums<true>(y1, val, tc.S, p, e2, x2);
+                    else val_sums<false>(y1, val, tc.S, p, e2, x2);
+                }
+            }
+            {
+                const uint32_t c = SPAN * span + base;
+                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base, q);
+            }
+        } else {  // K_GROUP
             const bool f16 = a.scale_fp16 != 0;
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
-            const UnitQ u = unit_of_plain<FMT>(ps);
-            {
+            const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+            const bool exact_res = !HAD && f16;
+#pragma unroll
+            for (int k = 0; k < N; ++k) {
                 float2 y[8];
-                chunk_in<HAD>(w0, y);
-                unit_chunk<FMT, STATS>(y, u, pw.p, q0, e2, x2);
+                uint32_t q[NW];
+                if constexpr (N == 1) { for (int i = 0; i < 8; ++i) y[i] = y1[i]; }
+                else chunk_in<HAD>(w[base + k], y);
+                if (scaled) plain_chunk<FMT, STATS, true>(y, u, p, exact_res, q, e2, x2);
+                else plain_chunk<FMT, STATS, false>(y, u, p, exact_res, q, e2, x2);
+                const uint32_t c = SPAN * span + base + k;
+                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base + k, q);
             }
-            {
-                float2 y[8];
-                chunk_in<HAD>(w1, y);
-                unit_chunk<FMT, STATS>(y, u, pw.p, q1, e2, x2);
+            // the leader of the unit stores its scale
+            const uint32_t c_first = SPAN * span + base;
+            const bool leader = (N < SPAN) || ((lane & (T - 1)) == 0);
+            if (leader && c_first < a.n_chunks) {
+                const uint32_t unit = (N < SPAN) ? c_first / N : span / (uint32_t)T;
+                store_plain_scale<FMT>(a.scales, a.zps, unit, ps, f16);
             }
-            if (v0 && leader) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
         }
+
         if constexpr (STATS) {
-            if (v0) add_unit_sums(acc, e2, x2, pw);
+            const uint32_t c_first = SPAN * span + base;
+            const bool valid = c_first < a.n_chunks;
+            if (valid) add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
             float ss = __fadd_rn(x2.x, x2.y);
-            for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
-            if (v0 && leader) kappa_add(acc, __fmul_rn(amax, pw.p), ss, a.inv_unit);
+            if (N == SPAN && T > 1)
+                for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+            const bool leader = (N < SPAN) || ((lane & (T - 1)) == 0);
+            if (valid && leader) kappa_add(acc, __fmul_rn(amax, p), ss, a.inv_unit);
         }
     }
-
-    if (v0) store_span<FMT>(a.codes, span, v1, q0, q1);
 }
 
-__device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint32_t n_chunks,
-                                          uint32_t (&w0)[8], uint32_t (&w1)[8])
+__device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint32_t n_chunks, uint32_t (&w)[SPAN][8])
 {
-    const uint32_t c0 = 2 * span;
-    if (c0 + 1 < n_chunks) {
-        ld_nc_v8(x + (size_t)c0 * 8, w0);
-        ld_nc_v8(x + (size_t)c0 * 8 + 8, w1);
+    const uint32_t c0 = SPAN * span;
+    if (c0 + SPAN <= n_chunks) {
+#pragma unroll
+        for (int k = 0; k < SPAN; ++k) ld_nc_v8(x + (size_t)(c0 + k) * 8, w[k]);
     } else {
-        if (c0 < n_chunks) ld_nc_v8(x + (size_t)c0 * 8, w0);
-        else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w0[i] = 0u;
+        for (int k = 0; k < SPAN; ++k) {
+            if (c0 + k < n_chunks) ld_nc_v8(x + (size_t)(c0 + k) * 8, w[k]);
+            else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[k][i] = 0u;
+            }
         }
+    }
+}
+
+// Store a span's gathered 4-bit codes: one 32-byte store when the span is whole, chunk
+// by chunk at the ragged end.
+template <int FMT>
+__device__ __forceinline__ void store_span4(uint8_t* codes, uint32_t span, uint32_t n_chunks, const uint32_t (&v)[8])
+{
+    if constexpr (Fmt<FMT>::four) {
+        const uint32_t c0 = SPAN * span;
+        if (c0 + SPAN <= n_chunks) {
+            st_v8(codes + (size_t)span * 32, v);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w1[i] = 0u;
+            for (int k = 0; k < SPAN; ++k)
+                if (c0 + k < n_chunks) {
+                    const uint32_t w2[2] = {v[2 * k], v[2 * k + 1]};
+                    st_v2(codes + (size_t)(c0 + k) * 8, w2);
+                }
+        }
     }
 }
 
@@ -395,33 +390,65 @@ __global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
 
     TensorCtx tc{};
+    PlainUnit<FMT> tu{};
+    Pow2 tp{1.0f, 1.0};
+    bool tscaled = false;
     if constexpr (GK == K_TENSOR || GK == K_NV) {
         const WsHeader* h = ws_header(a.ws);
         tc.amax = h->amax;
         if constexpr (GK == K_TENSOR) {
             tc.ps = plain_scale<FMT>(h->amax, h->vmin, h->vmax, a.scale_fp16 != 0);
-            tc.u = unit_of_plain<FMT>(tc.ps);
-            tc.p2 = pow2_for(tc.amax);
+            tu = plain_unit<FMT>(tc.ps);
+            tp = pow2_for(tc.amax);
+            tscaled = STATS && !plain_sums_ok(tc.amax);
             if (blockIdx.x == 0 && threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, 0, tc.ps, a.scale_fp16 != 0);
         } else {
             tc.S = __fdiv_rn(h->amax, F::qscale * 448.0f);
+            tc.cS = rcp_approx(__fmul_rn(F::qscale, tc.S));
             if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scale[0] = tc.S;
         }
     }
+    // per-group units: 16 elements (N = 1), 32 (N = 2), 64 and up (N = 4, T lanes)
+    const int T = (GK == K_GROUP && a.lanes_per_group > 0) ? a.lanes_per_group : 1;
 
     Acc acc;
-    // tile t covers spans 32 t .. 32 t + 31 (chunks 64 t .. 64 t + 63)
-    uint32_t t = warp;
-    uint32_t c0[8], c1[8];
-    if (t < a.n_dtiles) load_span(a.x, t * 32 + lane, a.n_chunks, c0, c1);
-    while (t < a.n_dtiles) {
-        const uint32_t tn = t + nwarps;
-        uint32_t n0[8], n1[8];
-        if (tn < a.n_dtiles) load_span(a.x, tn * 32 + lane, a.n_chunks, n0, n1);
-        flat_span<FMT, GK, HAD, STATS>(c0, c1, t * 32 + lane, a, tc, acc, lane);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { c0[i] = n0[i]; c1[i] = n1[i]; }
-        t = tn;
+    for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
+        const uint32_t span = t * 32 + lane;
+        uint32_t cur[SPAN][8];
+        load_span(a.x, span, a.n_chunks, cur);
+        uint32_t span4[8];
+        uint8_t scode[SPAN] = {0, 0, 0, 0};
+
+        if constexpr (GK == K_TENSOR) {
+            span_tensor<FMT, HAD, STATS>(cur, span, a, tu, tp.p, tp.inv_p2, tscaled, acc, span4);
+        } else if constexpr (GK == K_NV) {
+            span_units<FMT, GK, HAD, STATS, 1>(cur, span, a, tc, acc, lane, 1, span4, scode);
+        } else if constexpr (GK == K_MX) {
+            span_units<FMT, GK, HAD, STATS, 2>(cur, span, a, tc, acc, lane, 1, span4, scode);
+        } else {
+            if (a.lanes_per_group == 0) span_units<FMT, GK, HAD, STATS, 1>(cur, span, a, tc, acc, lane, 1, span4, scode);
+            else if (a.lanes_per_group < 0) span_units<FMT, GK, HAD, STATS, 2>(cur, span, a, tc, acc, lane, 1, span4, scode);
+            else span_units<FMT, GK, HAD, STATS, SPAN>(cur, span, a, tc, acc, lane, T, span4, scode);
+        }
+
+        store_span4<FMT>(a.codes, span, a.n_chunks, span4);
+        const uint32_t c0 = SPAN * span;
+        if constexpr (GK == K_NV) {
+            // four E4M3 block scales, one per chunk
+            uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
+            if (c0 + SPAN <= a.n_chunks)
+                *reinterpret_cast<uint32_t*>(sc + c0) = (uint32_t)scode[0] | ((uint32_t)scode[1] << 8) |
+                                                        ((uint32_t)scode[2] << 16) | ((uint32_t)scode[3] << 24);
+            else
+                for (int k = 0; k < SPAN; ++k)
+                    if (c0 + k < a.n_chunks) sc[c0 + k] = scode[k];
+        } else if constexpr (GK == K_MX) {
+            uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
+            if (c0 + SPAN <= a.n_chunks)
+                *reinterpret_cast<uint16_t*>(sc + c0 / 2) = (uint16_t)(scode[0] | (scode[2] << 8));
+            else if (c0 < a.n_chunks)
+                sc[c0 / 2] = scode[0];
+        }
     }
 
     if constexpr (STATS) {

@@ -1,12 +1,25 @@
-// quant_ops.cuh -- quantize one 16-element chunk given its scale, on fp32 pairs.
+// quant_ops.cuh -- quantize one 16-element chunk given its unit's scale, on fp32 pairs.
 //
 // Code rules ("INT vs FP at fine granularity" §2.1, "INT4/INT8/FP8 quantization"
 // §INT8/§INT4, "Quantization survey" §4.1):
 //   INT:  q = clamp(rne(x / s) [+ zp], Qmin, Qmax)
 //   FP:   code = cvt.rn.satfinite(x / s)
-// with x / s the correctly rounded fp32 quotient, decided through the reciprocal
-// bracket of common.cuh (a correctly rounded division only where the bracket is
-// inconclusive, about one element in 10^4).
+// with x / s the correctly rounded fp32 quotient.
+//
+// INT codes come from one fused multiply-add per element with r ~ 1/s (within 2^-23):
+// t = RN(x r + M) with M = 1.5 * 2^23 (+ zero point + bias) leaves the integer nearest
+// to x r in t's low bits, and the residual f = x r - q (one more FMA) says how far x r
+// is from a rounding boundary. Whenever |f| < 1/2 - (|x/s| + 2) 2^-21 the quotient
+// RN(x / s) lies strictly inside q's rounding interval, so q is its code. The rest
+// (about 1e-3 of the elements for bf16 inputs over fp16 scales, nearly all of them
+// exact half-integer quotients) are settled exactly: an exact FMA residual recognises
+// x / s == q +- 1/2 (the code is then the even neighbour) and anything else divides.
+// FP codes use a reciprocal bracket: cvt of x r_lo and of x r_hi, r_lo < 1/s < r_hi;
+// where the two differ the element divides.
+//
+// The chunk functions are warp-collective: every lane of a warp calls them together
+// (lanes with nothing to do pass zeros), because their rare-case branches are taken by
+// the whole warp when any lane needs them.
 #pragma once
 
 #include <cfloat>
@@ -17,136 +30,228 @@ namespace bq {
 
 template <int FMT> struct CodeWords { static constexpr int n = Fmt<FMT>::four ? 2 : 4; };
 
-// Everything a chunk needs to know about its unit's scale.
-struct UnitQ {
-    float s;        // scale the codes divide by (stored plain scale, d for NV)
-    float rlo, rhi; // reciprocal bracket (both 0 for an INT unit with s == 0)
-    float zpf;      // zero point (exact float; 0 for symmetric)
-    int qmin, qmax; // integer code range
-    bool fast;      // bracket usable for this unit
-    bool clamp_lo;  // some element can fall below qmin
-    bool clamp_hi;  // some element can rise above qmax
-    bool zero;      // s == 0 (or d == 0): every code is the zero code
+// Offset added to signed 4-bit codes so that the nibbles are non-negative while they
+// are assembled (undone with one XOR per word).
+template <int FMT> struct CodeBias { static constexpr int v = (FMT == BQ_INT4_SYM) ? 8 : 0; };
+
+// ---------------------------------------------------------------------------
+// Integer units.
+// ---------------------------------------------------------------------------
+
+struct IntQ {
+    float s;        // the scale x is divided by (0: every code is the zero point)
+    float r;        // ~ 1/s (0 when s == 0)
+    float mz;       // MAGIC + zero point + bias (exact)
+    float thr;      // |f| below thr: the code is certain
+    bool fast;      // s in the range where the residual test is valid
+    bool clamp;     // some element of the unit can leave [qmin, qmax]
 };
 
-// Clamping flags. q is monotone in x, so the unit's extreme values bound it.
-__device__ __forceinline__ void clamp_flags(float lo, float hi, const Recip& R, float zpf, int qmin, int qmax,
-                                            bool& clo, bool& chi)
+// Unit from its stored scale s, zero point zpf and the extreme values lo <= 0 <= hi it
+// holds; qmin / qmax: the code range.
+template <int FMT>
+__device__ __forceinline__ IntQ int_unit(float s, float zpf, float lo, float hi, int qmin, int qmax)
 {
-    if (!R.fast) { clo = chi = true; return; }
-    const float top = __fadd_rn(__fmaf_rn(hi, R.rhi, MAGIC), zpf);   // >= MAGIC + q for every x <= hi
-    const float bot = __fadd_rn(__fmaf_rn(lo, R.rhi, MAGIC), zpf);   // <= MAGIC + q for every x >= lo (lo <= 0)
-    chi = top > MAGIC + (float)qmax;
-    clo = bot < MAGIC + (float)qmin;
-}
-
-// Integer unit from a scale: a unit with s == 0 maps every element to the zero code
-// through the fast path itself (r_lo = r_hi = 0 gives q = 0, plus the zero point).
-__device__ __forceinline__ UnitQ int_unit(float s, float zpf, float lo, float hi, int qmin, int qmax)
-{
-    UnitQ u;
+    constexpr float bias = (float)CodeBias<FMT>::v;
+    IntQ u;
     u.s = s;
-    u.zpf = zpf;
-    u.qmin = qmin;
-    u.qmax = qmax;
-    u.zero = !(s > 0.0f);
-    if (u.zero) {
-        u.rlo = u.rhi = 0.0f;
+    u.mz = __fadd_rn(__fadd_rn(MAGIC, zpf), bias);
+    if (!(s > 0.0f)) {
+        u.r = 0.0f;
+        u.thr = 1.0f;
         u.fast = true;
-        u.clamp_lo = u.clamp_hi = false;
+        u.clamp = false;
         return u;
     }
-    const Recip R = make_recip(s, fmaxf(-lo, hi));
-    u.rlo = R.rlo;
-    u.rhi = R.rhi;
-    u.fast = R.fast;
-    clamp_flags(lo, hi, R, zpf, qmin, qmax, u.clamp_lo, u.clamp_hi);
+    u.r = rcp_approx(s);
+    const float bound = __fmul_rn(fmaxf(-lo, hi), u.r);          // ~ max |x / s|
+    u.fast = (s >= 0x1p-100f) && (s <= 1.0e37f) && (bound < 4.0e6f);
+    u.thr = __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f));
+    // the code is monotone in x: the extremes bound every code (a quarter step of slack)
+    const float top = __fadd_rn(__fmul_rn(hi, u.r), zpf), bot = __fadd_rn(__fmul_rn(lo, u.r), zpf);
+    u.clamp = !u.fast || top > (float)qmax + 0.25f || bot < (float)qmin - 0.25f;
     return u;
 }
 
-// Settle elements whose bracket ends disagree. The two candidates are adjacent
-// integers; h is the half-integer between them. fma(-h, s, x) is the exactly rounded
-// x - h s, which is zero only when x / s == h exactly: then RN(x/s) = h and the code is
-// the even candidate (the magic sum's low bit is the integer's parity). Any other
-// disagreement returns false and the caller divides.
-__device__ __forceinline__ bool settle_ties(float y, float s, float rhi, float& t)
+// Exact code (magic form, t = mz + q) of one element whose residual test was
+// inconclusive.
+__device__ __forceinline__ float settle(float y, float s, float r, float mz, float t)
 {
-    const float a = t;
-    const float b = __fmaf_rn(y, rhi, MAGIC);
-    if (__float_as_uint(a) == __float_as_uint(b)) return true;
-    const float qa = __fsub_rn(a, MAGIC), qb = __fsub_rn(b, MAGIC);   // exact
-    const float h = __fmul_rn(0.5f, __fadd_rn(qa, qb));                // exact: an odd integer / 2
-    if (__fmaf_rn(-h, s, y) != 0.0f) return false;
-    t = (__float_as_uint(a) & 1u) == 0u ? a : b;
-    return true;
+    const float q = __fsub_rn(t, mz);                        // exact
+    const float f = __fmaf_rn(y, r, -q);
+    const float side = f > 0.0f ? 0.5f : -0.5f;
+    const float h = __fadd_rn(q, side);                      // the half-integer next to q
+    if (__fmaf_rn(-h, s, y) == 0.0f) {
+        // x / s == h exactly: RN(x/s) = h, which rounds half to even
+        const bool q_even = (__float_as_uint(__fadd_rn(q, MAGIC)) & 1u) == 0u;
+        const float qe = q_even ? q : __fadd_rn(q, __fadd_rn(side, side));
+        return __fadd_rn(qe, mz);
+    }
+    float v = rintf(__fdiv_rn(y, s));
+    v = fminf(fmaxf(v, -4194304.0f), 4194304.0f);
+    return __fadd_rn(v, mz);
 }
 
-// ---------------------------------------------------------------------------
-// Integer chunk. On return: w = packed codes; qz[i] = q - zp (exact floats) when NEED_Q.
-// ---------------------------------------------------------------------------
-
+// Integer chunk: codes into w; nq[i] = -(code - zp) (exact) when NEED_Q.
 template <int FMT, bool NEED_Q>
-__device__ __forceinline__ void int_chunk(const float2 (&y)[8], const UnitQ& u,
-                                          uint32_t (&w)[CodeWords<FMT>::n], float2 (&qz)[8])
+__device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, int qmin, int qmax,
+                                          uint32_t (&w)[CodeWords<FMT>::n], float2 (&nq)[8])
 {
     using F = Fmt<FMT>;
-    float2 t[8];
-    bool ok = u.fast;
-    if (ok) {
-        uint32_t mism = 0;
-        const float2 lo = splat(u.rlo), hi = splat(u.rhi), m = splat(MAGIC);
+    constexpr float bias = (float)CodeBias<FMT>::v;
+    float2 t[8], nqq[8];
+    float fm = 0.0f;
+    const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 a = fma2(y[i], lo, m);
-            const float2 b = fma2(y[i], hi, m);
-            mism |= (__float_as_uint(a.x) ^ __float_as_uint(b.x)) | (__float_as_uint(a.y) ^ __float_as_uint(b.y));
-            t[i] = a;
+    for (int i = 0; i < 8; ++i) {
+        t[i] = fma2(y[i], R, MZ);
+        nqq[i] = fma2(t[i], M1, MZ);          // -q, exact
+        const float2 f = fma2(y[i], R, nqq[i]);
+        fm = amax3(fm, f.x, f.y);
+    }
+    const bool rare = !u.fast || !(fm < u.thr);
+    if (__any_sync(0xFFFFFFFFu, rare)) {
+        if (rare) {
+            if (u.fast) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 f = fma2(y[i], R, nqq[i]);
+                    if (!(fabsf(f.x) < u.thr)) t[i].x = settle(y[i].x, u.s, u.r, u.mz, t[i].x);
+                    if (!(fabsf(f.y) < u.thr)) t[i].y = settle(y[i].y, u.s, u.r, u.mz, t[i].y);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float qa = rintf(__fdiv_rn(y[i].x, u.s)), qb = rintf(__fdiv_rn(y[i].y, u.s));
+                    qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
+                    qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
+                    t[i] = make_float2(__fadd_rn(qa, u.mz), __fadd_rn(qb, u.mz));
+                }
+            }
         }
-        if (mism) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                ok &= settle_ties(y[i].x, u.s, u.rhi, t[i].x);
-                ok &= settle_ties(y[i].y, u.s, u.rhi, t[i].y);
+        for (int i = 0; i < 8; ++i) nqq[i] = fma2(t[i], M1, MZ);
+    }
+    if (__any_sync(0xFFFFFFFFu, u.clamp)) {
+        // the bounds hold the code + bias whatever the zero point; clamping is the
+        // identity for units that never leave the range
+        const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) nqq[i] = fma2(t[i], M1, MZ);
+    }
+    if constexpr (NEED_Q) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) nq[i] = nqq[i];
+    }
+    if constexpr (F::four) {
+        // t's low bits hold code + bias in [0, 15]: four codes per multiply-add chain
+        // (MAGIC's bits start at bit 22, so they never reach bits 0..15)
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t a = __float_as_uint(t[2 * k].x), b = __float_as_uint(t[2 * k].y);
+            const uint32_t c = __float_as_uint(t[2 * k + 1].x), d = __float_as_uint(t[2 * k + 1].y);
+            h[k] = a + b * 16u + c * 256u + d * 4096u;
+        }
+        w[0] = __byte_perm(h[0], h[1], 0x5410);
+        w[1] = __byte_perm(h[2], h[3], 0x5410);
+        if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
+                              __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
+    }
+}
+
+// Integer chunk for a scale with at most 11 significant bits (an fp16 scale) and
+// unrotated bf16 inputs. Then every product q s (|q| <= 2^8) and every residual
+// e = x - q s of a candidate q next to the quotient is exact, so the code is decided
+// in the value domain without any approximation: q is right when |e| < s/2, an exact
+// tie when |e| == s/2 (the code is then the even neighbour) and one step off when
+// |e| > s/2 (the reciprocal's error put x r on the far side of a half-integer). Ties
+// are frequent for such inputs (about 1e-3 of the elements). e is returned for the
+// QSNR sums (the error of the final code).
+template <int FMT, bool NEED_E>
+__device__ __forceinline__ void int_chunk_exact(const float2 (&y)[8], const IntQ& u, int qmin, int qmax,
+                                                uint32_t (&w)[CodeWords<FMT>::n], float2 (&e)[8])
+{
+    using F = Fmt<FMT>;
+    constexpr float bias = (float)CodeBias<FMT>::v;
+    float2 t[8], ee[8];
+    float em = 0.0f;
+    const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f), S = splat(u.s);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        t[i] = fma2(y[i], R, MZ);
+        const float2 nq = fma2(t[i], M1, MZ);          // -q, exact
+        ee[i] = fma2(nq, S, y[i]);                      // x - q s, exact
+        em = amax3(em, ee[i].x, ee[i].y);
+    }
+    const float hs = __fmul_rn(0.5f, u.s);
+    // (a zero scale has only zero elements: every code is the zero point)
+    const bool rare = !u.fast || (!(em < hs) && hs > 0.0f);
+    if (__any_sync(0xFFFFFFFFu, rare)) {
+        if (rare) {
+            if (u.fast) {
+                // parity of q from t's bits: t = MAGIC + zp + bias + q
+                const uint32_t zb = (uint32_t)(int)__fsub_rn(u.mz, MAGIC) & 1u;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float ax = fabsf(ee[i].x), ay = fabsf(ee[i].y);
+                    if (ax > hs || (ax == hs && ((__float_as_uint(t[i].x) ^ zb) & 1u)))
+                        t[i].x = __fadd_rn(t[i].x, copysignf(1.0f, ee[i].x));
+                    if (ay > hs || (ay == hs && ((__float_as_uint(t[i].y) ^ zb) & 1u)))
+                        t[i].y = __fadd_rn(t[i].y, copysignf(1.0f, ee[i].y));
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float qa = rintf(__fdiv_rn(y[i].x, u.s)), qb = rintf(__fdiv_rn(y[i].y, u.s));
+                    qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
+                    qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
+                    t[i] = make_float2(__fadd_rn(qa, u.mz), __fadd_rn(qb, u.mz));
+                }
+            }
+        }
+        if constexpr (NEED_E) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
+        }
+    }
+    if (__any_sync(0xFFFFFFFFu, u.clamp)) {
+        const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
+        float tmx = cmin, tmn = cmax;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { tmx = max3(tmx, t[i].x, t[i].y); tmn = min3(tmn, t[i].x, t[i].y); }
+        if (__any_sync(0xFFFFFFFFu, tmx > cmax || tmn < cmin)) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
+            if constexpr (NEED_E) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
             }
         }
     }
-    if (!ok) {
+    if constexpr (NEED_E) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float qa = rintf(__fdiv_rn(y[i].x, u.s));
-            float qb = rintf(__fdiv_rn(y[i].y, u.s));
-            qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
-            qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
-            t[i] = make_float2(__fadd_rn(qa, MAGIC), __fadd_rn(qb, MAGIC));
-        }
+        for (int i = 0; i < 8; ++i) e[i] = ee[i];
     }
-    if constexpr (F::asym) {
-        const float2 z = splat(u.zpf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = add2(t[i], z);
-    }
-    if (u.clamp_hi || !ok) {
-        const float cmax = MAGIC + (float)u.qmax;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = make_float2(fminf(t[i].x, cmax), fminf(t[i].y, cmax));
-    }
-    if (u.clamp_lo || !ok) {
-        const float cmin = MAGIC + (float)u.qmin;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = make_float2(fmaxf(t[i].x, cmin), fmaxf(t[i].y, cmin));
-    }
-    if constexpr (NEED_Q) {
-        const float2 z = splat(-__fadd_rn(MAGIC, u.zpf));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qz[i] = add2(t[i], z);
-    }
-    // the low bits of t are the two's complement code
     if constexpr (F::four) {
-        uint32_t b[8];
+        uint32_t h[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = pack_nibbles(__float_as_uint(t[i].x), __float_as_uint(t[i].y));
-        w[0] = pack_bytes(b[0], b[1], b[2], b[3]);
-        w[1] = pack_bytes(b[4], b[5], b[6], b[7]);
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t a = __float_as_uint(t[2 * k].x), b = __float_as_uint(t[2 * k].y);
+            const uint32_t c = __float_as_uint(t[2 * k + 1].x), d = __float_as_uint(t[2 * k + 1].y);
+            h[k] = a + b * 16u + c * 256u + d * 4096u;
+        }
+        w[0] = __byte_perm(h[0], h[1], 0x5410);
+        w[1] = __byte_perm(h[2], h[3], 0x5410);
+        if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -158,6 +263,25 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const UnitQ& u,
 // ---------------------------------------------------------------------------
 // FP element chunks.
 // ---------------------------------------------------------------------------
+
+struct FpQ {
+    float s;        // the scale x is divided by
+    float rlo, rhi; // reciprocal bracket
+    bool fast;
+    bool zero;      // s == 0: every code is +0
+};
+
+__device__ __forceinline__ FpQ fp_unit(float s, float amax)
+{
+    FpQ u;
+    u.s = s;
+    u.zero = !(s > 0.0f);
+    const Recip R = make_recip(s, amax);
+    u.rlo = u.zero ? 0.0f : R.rlo;
+    u.rhi = u.zero ? 0.0f : R.rhi;
+    u.fast = R.fast && !u.zero;
+    return u;
+}
 
 template <int FMT>
 __device__ __forceinline__ void pack_pairs(const uint32_t (&pr)[8], uint32_t (&w)[CodeWords<FMT>::n])
@@ -178,34 +302,36 @@ __device__ __forceinline__ void decode_pairs(const uint32_t (&pr)[8], float2 (&v
     for (int p = 0; p < 8; ++p) val[p] = dec_pair<FMT>(pr[p]);
 }
 
-// General scale s > 0: codes of x / s. val = decoded element values when NEED_V.
+// Codes of x / s (s > 0) or +0 codes (s == 0); val = decoded element values (NEED_V).
 template <int FMT, bool NEED_V>
-__device__ __forceinline__ void fp_chunk(const float2 (&y)[8], const UnitQ& u,
+__device__ __forceinline__ void fp_chunk(const float2 (&y)[8], const FpQ& u,
                                          uint32_t (&w)[CodeWords<FMT>::n], float2 (&val)[8])
 {
     uint32_t pr[8];
-    if (u.zero) {
+    uint32_t mism = 0;
+    const float2 lo = splat(u.rlo), hi = splat(u.rhi);
 #pragma unroll
-        for (int p = 0; p < 8; ++p) pr[p] = 0u;
-    } else {
-        bool ok = u.fast;
-        if (ok) {
-            uint32_t mism = 0;
-            const float2 lo = splat(u.rlo), hi = splat(u.rhi);
+    for (int p = 0; p < 8; ++p) {
+        const float2 a = mul2(y[p], lo), b = mul2(y[p], hi);
+        const uint32_t cl = cvt_pair<FMT>(a.y, a.x);
+        const uint32_t ch = cvt_pair<FMT>(b.y, b.x);
+        mism |= cl ^ ch;
+        pr[p] = cl;
+    }
+    const bool rare = u.zero || !u.fast || mism != 0u;
+    if (__any_sync(0xFFFFFFFFu, rare)) {
+        if (rare) {
+            if (u.zero) {
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const float2 a = mul2(y[p], lo), b = mul2(y[p], hi);
-                const uint32_t cl = cvt_pair<FMT>(a.y, a.x);
-                const uint32_t ch = cvt_pair<FMT>(b.y, b.x);
-                mism |= cl ^ ch;
-                pr[p] = cl;
+                for (int p = 0; p < 8; ++p) pr[p] = 0u;
+            } else {
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const float2 a = mul2(y[p], lo), b = mul2(y[p], hi);
+                    const bool bad = !u.fast || (cvt_pair<FMT>(a.y, a.x) != cvt_pair<FMT>(b.y, b.x));
+                    if (bad) pr[p] = cvt_pair<FMT>(__fdiv_rn(y[p].y, u.s), __fdiv_rn(y[p].x, u.s));
+                }
             }
-            ok = (mism == 0);
-        }
-        if (!ok) {
-#pragma unroll
-            for (int p = 0; p < 8; ++p)
-                pr[p] = cvt_pair<FMT>(__fdiv_rn(y[p].y, u.s), __fdiv_rn(y[p].x, u.s));
         }
     }
     pack_pairs<FMT>(pr, w);
@@ -228,37 +354,21 @@ __device__ __forceinline__ void fp_chunk_pow2(const float2 (&y)[8], float p2,
     if constexpr (NEED_V) decode_pairs<FMT>(pr, val);
 }
 
-// MXINT8: q = clamp(rne(x * 2^-e), -127, 127); the clamp never binds (amax <= 127 * 2^e)
-// except for the clamped exponent range, which the caller flags.
+// MXINT8: q = rne(x * 2^-e) (exact product, |q| <= 127 by the choice of e); nq = -q.
 template <bool NEED_Q>
-__device__ __forceinline__ void int8_chunk_pow2(const float2 (&y)[8], float p2, bool clamp, uint32_t (&w)[4],
-                                                float2 (&q)[8])
+__device__ __forceinline__ void int8_chunk_pow2(const float2 (&y)[8], float p2, uint32_t (&w)[4], float2 (&nq)[8])
 {
     float2 t[8];
-    const float2 p = splat(p2), m = splat(MAGIC);
+    const float2 p = splat(p2), m = splat(MAGIC), M1 = splat(-1.0f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = fma2(y[i], p, m);
-    if (clamp) {
-        const float cmin = MAGIC - 127.0f, cmax = MAGIC + 127.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
-    }
-    if constexpr (NEED_Q) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = add2(t[i], splat(-MAGIC));
+    for (int i = 0; i < 8; ++i) {
+        t[i] = fma2(y[i], p, m);
+        if constexpr (NEED_Q) nq[i] = fma2(t[i], M1, m);
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k)
         w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
                           __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
-}
-
-template <int FMT>
-__device__ __forceinline__ void store_codes(uint8_t* codes, uint32_t c, const uint32_t (&w)[CodeWords<FMT>::n])
-{
-    if constexpr (Fmt<FMT>::four) st_v2(codes + (size_t)c * 8, w);
-    else st_v4(codes + (size_t)c * 16, w);
 }
 
 // ---------------------------------------------------------------------------
@@ -282,8 +392,16 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
         s32 = fminf(s32, FLT_MAX);                  // a range beyond fp32 saturates
         p.s = fp16 ? round_scale_f16(s32) : s32;
         if (p.s > 0.0f) {
-            float z = rintf(__fdiv_rn(-lo, p.s));
-            z = fminf(fmaxf(z, -1.0e9f), 1.0e9f);
+            // zp = Qmin + rne(RN(-lo / s)), decided like a code: residual test, else exact
+            const float r = rcp_approx(p.s);
+            const float q = __fsub_rn(__fmaf_rn(-lo, r, MAGIC), MAGIC);
+            const float f = __fmaf_rn(-lo, r, -q);
+            const float bound = __fmul_rn(-lo, r);
+            float z;
+            if (p.s >= 0x1p-100f && bound < 4.0e6f && fabsf(f) < __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f)))
+                z = q;
+            else
+                z = fminf(fmaxf(rintf(__fdiv_rn(-lo, p.s)), -1.0e9f), 1.0e9f);
             p.zpf = fminf(fmaxf(__fadd_rn((float)F::qmin, z), (float)F::qmin), (float)F::qmax);
         } else {
             p.zpf = (float)F::qmin;
@@ -301,49 +419,6 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
 }
 
 template <int FMT>
-__device__ __forceinline__ UnitQ unit_of_plain(const PlainScale& ps)
-{
-    using F = Fmt<FMT>;
-    if constexpr (F::is_int) return int_unit(ps.s, ps.zpf, ps.lo, ps.hi, F::qmin, F::qmax);
-    UnitQ u;
-    u.s = ps.s;
-    u.zpf = 0.0f;
-    u.qmin = u.qmax = 0;
-    u.zero = !(ps.s > 0.0f);
-    const Recip R = make_recip(ps.s, fmaxf(-ps.lo, ps.hi));
-    u.rlo = R.rlo;
-    u.rhi = R.rhi;
-    u.fast = R.fast;
-    u.clamp_lo = u.clamp_hi = false;
-    return u;
-}
-
-// Quantize a chunk under a unit; xh = dequantized value (rotated domain) when NEED_X.
-template <int FMT, bool NEED_X>
-__device__ __forceinline__ void quant_unit_chunk(const float2 (&y)[8], const UnitQ& u,
-                                                 uint32_t (&w)[CodeWords<FMT>::n], float2 (&xh)[8])
-{
-    using F = Fmt<FMT>;
-    if constexpr (F::is_int) {
-        float2 qz[8];
-        int_chunk<FMT, NEED_X>(y, u, w, qz);
-        if constexpr (NEED_X) {
-            const float2 s = splat(u.s);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xh[i] = mul2(qz[i], s);   // s == 0 gives 0: qz is 0 there
-        }
-    } else {
-        float2 val[8];
-        fp_chunk<FMT, NEED_X>(y, u, w, val);
-        if constexpr (NEED_X) {
-            const float2 s = splat(u.s);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xh[i] = u.zero ? splat(0.0f) : mul2(val[i], s);
-        }
-    }
-}
-
-template <int FMT>
 __device__ __forceinline__ void store_plain_scale(void* scales, void* zps, size_t i, const PlainScale& ps, bool fp16)
 {
     if (fp16) {
@@ -355,25 +430,143 @@ __device__ __forceinline__ void store_plain_scale(void* scales, void* zps, size_
     }
 }
 
-// ---------------------------------------------------------------------------
-// QSNR sums of one chunk on values scaled by a power of two p:
-// e2 += sum ((y - xh) p)^2, x2 += sum (y p)^2 (pairs accumulate separately).
-// ---------------------------------------------------------------------------
+// A plain unit, INT or FP.
+template <int FMT>
+struct PlainUnit {
+    IntQ iq;
+    FpQ fq;
+    float s;
+};
 
-__device__ __forceinline__ void chunk_sums2(const float2 (&y)[8], const float2 (&xh)[8], float p,
-                                            float2& e2, float2& x2)
+template <int FMT>
+__device__ __forceinline__ PlainUnit<FMT> plain_unit(const PlainScale& ps)
 {
-    const float2 P = splat(p), nP = splat(-p);
+    PlainUnit<FMT> u;
+    u.s = ps.s;
+    if constexpr (Fmt<FMT>::is_int) u.iq = int_unit<FMT>(ps.s, ps.zpf, ps.lo, ps.hi, Fmt<FMT>::qmin, Fmt<FMT>::qmax);
+    else u.fq = fp_unit(ps.s, fmaxf(-ps.lo, ps.hi));
+    return u;
+}
+
+// QSNR sums. Plain form (units whose values lie in [2^-40, 2^40]): e2 += (y - q s)^2
+// and x2 += y^2 in fp32. Scaled form (any other unit): x-hat is formed in fp32 first
+// (so an x-hat past the fp32 range is inf, as it is for the dequantized tensor), then
+// the difference and y are scaled by the power of two p before squaring.
+template <bool SCALED>
+__device__ __forceinline__ void int_sums(const float2 (&y)[8], const float2 (&nq)[8], float s, float p,
+                                         float2& e2, float2& x2)
+{
+    if constexpr (SCALED) {
+        const float2 P = splat(p), nP = splat(-p), nS = splat(-s);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float2 yp = mul2(y[i], P);
-        const float2 d = fma2(xh[i], nP, yp);    // (y - xh) p: xh * p is exact
-        e2 = fma2(d, d, e2);
-        x2 = fma2(yp, yp, x2);
+        for (int i = 0; i < 8; ++i) {
+            const float2 xh = mul2(nq[i], nS);
+            const float2 yp = mul2(y[i], P);
+            const float2 d = fma2(xh, nP, yp);
+            e2 = fma2(d, d, e2);
+            x2 = fma2(yp, yp, x2);
+        }
+    } else {
+        const float2 S = splat(s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = fma2(nq[i], S, y[i]);
+            e2 = fma2(d, d, e2);
+            x2 = fma2(y[i], y[i], x2);
+        }
     }
 }
 
-// range of a chunk
+// Sums from exact residuals e = x - x-hat.
+template <bool SCALED>
+__device__ __forceinline__ void res_sums(const float2 (&y)[8], const float2 (&e)[8], float p, float2& e2, float2& x2)
+{
+    if constexpr (SCALED) {
+        const float2 P = splat(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = mul2(e[i], P), yp = mul2(y[i], P);
+            e2 = fma2(d, d, e2);
+            x2 = fma2(yp, yp, x2);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            e2 = fma2(e[i], e[i], e2);
+            x2 = fma2(y[i], y[i], x2);
+        }
+    }
+}
+
+// Sums from element values val with x-hat = val * s.
+template <bool SCALED>
+__device__ __forceinline__ void val_sums(const float2 (&y)[8], const float2 (&val)[8], float s, float p,
+                                         float2& e2, float2& x2)
+{
+    if constexpr (SCALED) {
+        const float2 P = splat(p), nP = splat(-p), S = splat(s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 xh = mul2(val[i], S);
+            const float2 yp = mul2(y[i], P);
+            const float2 d = fma2(xh, nP, yp);
+            e2 = fma2(d, d, e2);
+            x2 = fma2(yp, yp, x2);
+        }
+    } else {
+        const float2 nS = splat(-s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = fma2(val[i], nS, y[i]);
+            e2 = fma2(d, d, e2);
+            x2 = fma2(y[i], y[i], x2);
+        }
+    }
+}
+
+// Quantize one chunk of a plain unit; STATS adds its sums (scaled form when SCALED).
+// exact_res: the unit's scale has at most 11 significant bits (fp16) and y is unrotated
+// bf16 (uniform over the launch).
+template <int FMT, bool STATS, bool SCALED>
+__device__ __forceinline__ void plain_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, float p, bool exact_res,
+                                            uint32_t (&w)[CodeWords<FMT>::n], float2& e2, float2& x2)
+{
+    using F = Fmt<FMT>;
+    if constexpr (F::is_int) {
+        if (exact_res) {
+            float2 e[8];
+            int_chunk_exact<FMT, STATS>(y, u.iq, F::qmin, F::qmax, w, e);
+            if constexpr (STATS) res_sums<SCALED>(y, e, p, e2, x2);
+        } else {
+            float2 nq[8];
+            int_chunk<FMT, STATS>(y, u.iq, F::qmin, F::qmax, w, nq);
+            if constexpr (STATS) int_sums<SCALED>(y, nq, u.s, p, e2, x2);
+        }
+    } else {
+        float2 val[8];
+        fp_chunk<FMT, STATS>(y, u.fq, w, val);
+        if constexpr (STATS) val_sums<SCALED>(y, val, u.s, p, e2, x2);
+    }
+}
+
+// Fold a unit's fp32 sums into the lane's doubles (inv_p2 = 1 / p^2).
+__device__ __forceinline__ void add_unit_sums(Acc& acc, float2 e2, float2 x2, double inv_p2)
+{
+    acc.err2 += (double)__fadd_rn(e2.x, e2.y) * inv_p2;
+    acc.x2 += (double)__fadd_rn(x2.x, x2.y) * inv_p2;
+}
+
+template <int FMT>
+__device__ __forceinline__ void store_codes(uint8_t* codes, uint32_t c, const uint32_t (&w)[CodeWords<FMT>::n])
+{
+    if constexpr (Fmt<FMT>::four) st_v2(codes + (size_t)c * 8, w);
+    else st_v4(codes + (size_t)c * 16, w);
+}
+
+// ---------------------------------------------------------------------------
+// Ranges.
+// ---------------------------------------------------------------------------
+
 __device__ __forceinline__ float chunk_amax(const float2 (&y)[8], float m)
 {
 #pragma unroll
@@ -389,5 +582,30 @@ __device__ __forceinline__ void chunk_minmax(const float2 (&y)[8], float& mn, fl
         mx = max3(mx, y[i].x, y[i].y);
     }
 }
+
+// on raw bf16 words (no widening)
+__device__ __forceinline__ uint32_t words_absmax(const uint32_t (&w)[8], uint32_t m)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = bf2_absmax(m, w[i]);
+    return m;
+}
+
+__device__ __forceinline__ void words_minmax(const uint32_t (&w)[8], uint32_t& mn, uint32_t& mx)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        mn = bf2_min(mn, w[i]);
+        mx = bf2_max(mx, w[i]);
+    }
+}
+
+__device__ __forceinline__ float pair_absmax(uint32_t m) { return fmaxf(bf_lo(m), bf_hi(m)); }
+__device__ __forceinline__ float pair_min(uint32_t m) { return fminf(bf_lo(m), bf_hi(m)); }
+__device__ __forceinline__ float pair_max(uint32_t m) { return fmaxf(bf_lo(m), bf_hi(m)); }
+
+// Plain fp32 QSNR sums are safe (no overflow, no underflow that matters) for units whose
+// largest magnitude lies in [2^-40, 2^40] (or is zero).
+__device__ __forceinline__ bool plain_sums_ok(float amax) { return amax <= 0x1p40f && (amax >= 0x1p-40f || amax == 0.0f); }
 
 }  // namespace bq

@@ -57,16 +57,30 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
         float amax = 0.0f, mn = 0.0f, mx = 0.0f;
         uint32_t nxt[KK][8];
 
+        // range of this thread's part of the row: raw bf16 words, or rotated values
         if constexpr (K > 0) {
             const uint32_t rn = r + gridDim.x;
             if (rn < a.rows) load_row(rn, nxt);
+            if constexpr (HAD) {
 #pragma unroll
-            for (int k = 0; k < K; ++k) {
-                float2 v[8];
-                widen16x2(cur[k], v);
-                if constexpr (HAD) fwht16x2(v);
-                amax = chunk_amax(v, amax);
-                if constexpr (F::asym) chunk_minmax(v, mn, mx);
+                for (int k = 0; k < K; ++k) {
+                    float2 v[8];
+                    widen16x2(cur[k], v);
+                    fwht16x2(v);
+                    if constexpr (F::asym) chunk_minmax(v, mn, mx);
+                    else amax = chunk_amax(v, amax);
+                }
+            } else if constexpr (F::asym) {
+                uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+                for (int k = 0; k < K; ++k) words_minmax(cur[k], lo, hi);
+                mn = pair_min(lo);
+                mx = pair_max(hi);
+            } else {
+                uint32_t m = 0u;
+#pragma unroll
+                for (int k = 0; k < K; ++k) m = words_absmax(cur[k], m);
+                amax = pair_absmax(m);
             }
         } else {
             for (uint32_t c = tid; c < a.cpr; c += B) {
@@ -75,66 +89,70 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
                 ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
                 widen16x2(w, v);
                 if constexpr (HAD) fwht16x2(v);
-                amax = chunk_amax(v, amax);
                 if constexpr (F::asym) chunk_minmax(v, mn, mx);
+                else amax = chunk_amax(v, amax);
             }
         }
 
-        amax = warp_maxf(amax);
         if constexpr (F::asym) { mn = warp_minf(mn); mx = warp_maxf(mx); }
+        else amax = warp_maxf(amax);
         float (*rb)[4] = red[it & 1];
         if (lane == 0) { rb[warp][0] = amax; rb[warp][1] = mn; rb[warp][2] = mx; }
         __syncthreads();
         float A = 0.0f, MN = 0.0f, MX = 0.0f;
         for (int w = 0; w < nw; ++w) { A = fmaxf(A, rb[w][0]); MN = fminf(MN, rb[w][1]); MX = fmaxf(MX, rb[w][2]); }
+        if constexpr (F::asym) A = fmaxf(-MN, MX);
 
         const PlainScale ps = plain_scale<FMT>(A, MN, MX, fp16);
-        const UnitQ u = unit_of_plain<FMT>(ps);
+        const PlainUnit<FMT> u = plain_unit<FMT>(ps);
         if (tid == 0) store_plain_scale<FMT>(a.scales, a.zps, r, ps, fp16);
         const Pow2 pw = pow2_for(A);
-        float ss = 0.0f;
+        const bool scaled = STATS && !plain_sums_ok(A);      // uniform over the CTA
+        const bool exact_res = !HAD && fp16;
+        const float p = scaled ? pw.p : 1.0f;
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
 
-        auto emit = [&](const float2 (&v)[8], uint32_t c) {
-            uint32_t w[NW];
-            float2 xh[8];
-            quant_unit_chunk<FMT, STATS>(v, u, w, xh);
-            store_codes<FMT>(a.codes, c_row + c, w);
-            if constexpr (STATS) {
-                float2 e2 = splat(0.0f), x2 = splat(0.0f);
-                chunk_sums2(v, xh, pw.p, e2, x2);
-                const float s = __fadd_rn(x2.x, x2.y);
-                acc.err2 += (double)__fadd_rn(e2.x, e2.y) * pw.inv_p2;
-                acc.x2 += (double)s * pw.inv_p2;
-                ss = __fadd_rn(ss, s);
-            }
+        // every lane of a warp quantizes (lanes past the row's end pass zeros and store
+        // nothing): the chunk functions are warp-collective
+        auto emit = [&](const uint32_t (&wi)[8], uint32_t c, bool valid) {
+            float2 v[8];
+            uint32_t q[NW];
+            widen16x2(wi, v);
+            if constexpr (HAD) fwht16x2(v);
+            if (scaled) plain_chunk<FMT, STATS, true>(v, u, p, exact_res, q, e2, x2);
+            else plain_chunk<FMT, STATS, false>(v, u, p, exact_res, q, e2, x2);
+            if (valid) store_codes<FMT>(a.codes, c_row + c, q);
         };
 
         if constexpr (K > 0) {
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 const uint32_t c = tid + k * B;
-                float2 v[8];
-                widen16x2(cur[k], v);
-                if constexpr (HAD) fwht16x2(v);
-                if (c < a.cpr) emit(v, c);
+                emit(cur[k], c, c < a.cpr);
             }
 #pragma unroll
             for (int k = 0; k < K; ++k)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) cur[k][i] = nxt[k][i];
         } else {
-            for (uint32_t c = tid; c < a.cpr; c += B) {
+            // all lanes run the same trip count (those past the end pass zeros)
+            const uint32_t trips = (a.cpr + B - 1) / B;
+            for (uint32_t j = 0; j < trips; ++j) {
+                const uint32_t c = tid + j * B;
                 uint32_t w[8];
-                float2 v[8];
-                ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
-                widen16x2(w, v);
-                if constexpr (HAD) fwht16x2(v);
-                emit(v, c);
+                if (c < a.cpr) ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
+                else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = 0u;
+                }
+                emit(w, c, c < a.cpr);
             }
         }
 
         if constexpr (STATS) {
-            // crest factor of the row: amax / sqrt(mean of squares), on scaled sums
+            add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
+            // crest factor of the row: amax / sqrt(mean of squares), on the same scaling
+            float ss = __fadd_rn(x2.x, x2.y);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
             if (lane == 0) rb[warp][3] = ss;
@@ -142,7 +160,7 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
             if (tid == 0) {
                 float SS = 0.0f;
                 for (int w = 0; w < nw; ++w) SS = __fadd_rn(SS, rb[w][3]);
-                kappa_add(acc, __fmul_rn(A, pw.p), SS, a.inv_cols);
+                kappa_add(acc, __fmul_rn(A, p), SS, a.inv_cols);
             }
         }
     }
