@@ -74,6 +74,8 @@ def _lib() -> ctypes.CDLL:
         L.bq_dequantize.argtypes = [vp, vp, vp, vp, i64, i64, sp, vp, i32, vp]
         L.bq_qsnr.restype = ctypes.c_int
         L.bq_qsnr.argtypes = [vp, i32, vp, vp, vp, vp, i64, i64, sp, vp, vp, sz, vp]
+        L.bq_quantize_noalloc.restype = ctypes.c_int
+        L.bq_quantize_noalloc.argtypes = [vp, i32, i64, i64, sp, vp, vp, vp, vp, vp, vp]
         L.bq_stats_qsnr_db.restype = ctypes.c_double
         L.bq_stats_qsnr_db.argtypes = [ctypes.POINTER(BqStats)]
         _L = L
@@ -164,6 +166,18 @@ def bq_quantize(x: torch.Tensor, scheme: Scheme, codes: torch.Tensor, scales: to
     _check(_lib().bq_quantize(_ptr(x), DT["bf16"], rows, cols, ctypes.byref(sc), _ptr(codes), _ptr(scales),
                               _ptr(zero_points), _ptr(tensor_scale), _ptr(stats), _ptr(workspace), ws_bytes,
                               _stream(stream)), "bq_quantize")
+
+
+def bq_quantize_noalloc(x: torch.Tensor, scheme: Scheme, codes: torch.Tensor, scales: torch.Tensor,
+                        zero_points: torch.Tensor | None, tensor_scale: torch.Tensor | None,
+                        stats: torch.Tensor | None, stream=None) -> None:
+    """bq_quantize with the library's own static device scratch instead of a workspace
+    (for callers that cannot allocate device memory; calls must not overlap)."""
+    rows, cols = x.shape
+    sc = scheme.c()
+    _check(_lib().bq_quantize_noalloc(_ptr(x), DT["bf16"], rows, cols, ctypes.byref(sc), _ptr(codes), _ptr(scales),
+                                      _ptr(zero_points), _ptr(tensor_scale), _ptr(stats), _stream(stream)),
+           "bq_quantize_noalloc")
 
 
 def bq_dequantize(codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor | None,

@@ -185,6 +185,26 @@ bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void*
                   int64_t rows, int64_t cols, const bq_scheme* scheme,
                   bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * bq_quantize without a caller-provided workspace, for callers that cannot allocate
+ * device memory: code running under another component's allocator (a framework or
+ * serving runtime that owns all device memory), code that must not call cudaMalloc
+ * in the middle of an asynchronous pipeline, or code with a fixed memory budget.
+ * The paper has no counterpart of this call (it serves such callers, not the method).
+ * Arguments and results are those of bq_quantize. The scratch is a file-scope device
+ * array of 131328 bytes (the workspace size of every scheme and shape); every GPU that
+ * loads the library holds one copy until the process exits. A call whose scheme would
+ * need more returns BQ_ERR_WORKSPACE. The first call on a device looks the array's
+ * device address up (cudaGetSymbolAddress); make that first call before any stream
+ * capture. Every call shares the one array and zeroes its counters on the stream
+ * first: calls that may overlap on the GPU (other streams, other threads) race, and
+ * must be serialized by the caller. No cudaMalloc or cudaFree is made.
+ */
+bq_status bq_quantize_noalloc(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                              const bq_scheme* scheme,
+                              void* codes, void* scales, void* zero_points, float* tensor_scale,
+                              bq_stats* stats, void* stream);
+
 /* -10 log10(err2 / x2) from a host copy of the stats (+inf when err2 = 0). */
 double bq_stats_qsnr_db(const bq_stats* host_stats);
 
