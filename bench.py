@@ -255,39 +255,40 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ws = bq.new_workspace(device)
     stream = torch.cuda.current_stream(device)
 
-    def step(i, evs=None, st=None):
-        st = st or stream
+    def launch(j, kind, i, st):
+        """Kernel `kind` ("quantize" / "dequantize") of scheme j on buffer set i."""
         xi, outs, deqs = sets[i % n_sets]
-        k = 0
-        for (lab, s), q, dq in zip(schemes, outs, deqs):
-            if evs is not None:
-                evs[k].record(st)
+        s, q = schemes[j][1], outs[j]
+        if kind == "quantize":
             bq.bq_quantize(xi, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, st)
-            if evs is not None:
-                evs[k + 1].record(st)
-            bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, dq, st)
-            k += 2
-        if evs is not None:
-            evs[k].record(st)
+        else:
+            bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, deqs[j], st)
+
+    def step(i, st=None):
+        st = st or stream
+        for j in range(len(schemes)):
+            launch(j, "quantize", i, st)
+            launch(j, "dequantize", i, st)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(device)
 
-    n_k = 2 * len(schemes)
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_k + 1)] for _ in range(args.steps)]
-    # The K timed steps are captured once into a CUDA graph (the kernel launches and the
-    # per-kernel timing events) and replayed once inside the timed region, so host-side
-    # launch overhead does not enter the device time.
-    graph = None
-    if not args.eager:
-        graph = torch.cuda.CUDAGraph()
+    def capture(fn):
+        """A CUDA graph of fn(stream) (captured on a side stream, replayed on `stream`)."""
+        g = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream(device)
         cap.wait_stream(stream)
-        with torch.cuda.graph(graph, stream=cap):
-            for i in range(args.steps):
-                step(args.warmup + i, evs[i], cap)
+        with torch.cuda.graph(g, stream=cap):
+            fn(cap)
         torch.cuda.synchronize(device)
+        return g
+
+    # The K timed steps are captured once into a CUDA graph and replayed once inside the
+    # timed region, so host-side launch overhead does not enter the device time.
+    graph = None
+    if not args.eager:
+        graph = capture(lambda st: [step(args.warmup + i, st) for i in range(args.steps)])
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     sampler = ClockSampler(vis.split(",")[local_rank].strip() if vis else device.index)
     if rank == 0:
@@ -302,7 +303,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         graph.replay()
     else:
         for i in range(args.steps):
-            step(args.warmup + i, evs[i])
+            step(args.warmup + i)
     t1.record(stream)
     torch.cuda.synchronize(device)
     sampler.mark_off()
@@ -311,14 +312,34 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = reduce_max(ms, device)
 
-    # per-kernel mean durations (events between consecutive launches on this stream)
-    per_k = [statistics.fmean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) for k in range(n_k)]
+    # Per-kernel launch durations: each kernel of the step alone, K launches back to back
+    # over the same rotating buffer sets (a graph of them, or eager), between two events
+    # on the launching stream. (Events between the kernels of one graph would add their
+    # own gaps to every interval.)
+    n_k = 2 * len(schemes)
+    n_per = max(8, min(args.steps, 64))
     kernels = []
     for j, (lab, s) in enumerate(schemes):
         qb, db = per_scheme_bytes[j]
-        for kind, nbytes, kms in (("quantize", qb, per_k[2 * j]), ("dequantize", db, per_k[2 * j + 1])):
+        for kind, nbytes in (("quantize", qb), ("dequantize", db)):
+            def seq(st, j=j, kind=kind):
+                for i in range(n_per):
+                    launch(j, kind, args.warmup + i, st)
+            seq(stream)                                  # warm
+            g = None if args.eager else capture(seq)
+            k0 = torch.cuda.Event(enable_timing=True)
+            k1 = torch.cuda.Event(enable_timing=True)
+            k0.record(stream)
+            if g is not None:
+                g.replay()
+            else:
+                seq(stream)
+            k1.record(stream)
+            torch.cuda.synchronize(device)
+            kms = reduce_max(k0.elapsed_time(k1) / n_per, device)
             kernels.append({"kernel": f"{kind}:{lab}", "bytes": nbytes, "ms": kms,
                             "gbs": nbytes / (kms * 1e-3) / 1e9})
+            del g
     dom = max(kernels, key=lambda k: k["ms"])
     peak, peak_kind = measured_peaks()
 
@@ -404,6 +425,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "l2": f"inputs larger than L2: {n_sets} rotating buffer sets of {set_bytes / 2**20:.1f} MiB",
             "parallelism": f"dp{world} (one independent tensor per GPU, no collective on the data path)",
             "launch": "eager" if graph is None else "CUDA graph of the K timed steps",
+            "kernel_timing": f"each kernel alone, {n_per} launches back to back over the rotating sets",
         },
         "pct_hbm_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(dom["gbs"], 1),
@@ -411,7 +433,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "traffic": traffic, "algorithmic_bytes": dom["bytes"], "peak_source": peak_kind},
         "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kernels],
         "qsnr": qsnr,
-        "gpu_launches": args.steps * n_k,
+        # quantize: one kernel, plus the range pass for per-tensor and NV scales; dequantize: one
+        "gpu_launches": args.steps * sum((2 if s.gran in ("tensor", "nv") else 1) + 1 for _, s in schemes),
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,

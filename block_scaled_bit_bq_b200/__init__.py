@@ -78,6 +78,8 @@ def _lib() -> ctypes.CDLL:
         L.bq_quantize_noalloc.argtypes = [vp, i32, i64, i64, sp, vp, vp, vp, vp, vp, vp]
         L.bq_stats_qsnr_db.restype = ctypes.c_double
         L.bq_stats_qsnr_db.argtypes = [ctypes.POINTER(BqStats)]
+        L.bq_wait_timeouts.restype = ctypes.c_int
+        L.bq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         _L = L
     return _L
 
@@ -198,6 +200,14 @@ def bq_qsnr(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zero_poi
     _check(_lib().bq_qsnr(_ptr(x), DT["bf16"], _ptr(codes), _ptr(scales), _ptr(zero_points), _ptr(tensor_scale),
                           rows, cols, ctypes.byref(sc), _ptr(stats), _ptr(workspace), ws_bytes, _stream(stream)),
            "bq_qsnr")
+
+
+def bq_wait_timeouts(reset: bool = False) -> int:
+    """Tile waits of the quantize kernels that gave up on the current device (each
+    leaves its call's outputs incomplete); synchronizes with the device."""
+    c = ctypes.c_uint32(0)
+    _check(_lib().bq_wait_timeouts(ctypes.byref(c), 1 if reset else 0), "bq_wait_timeouts")
+    return int(c.value)
 
 
 def bq_stats_qsnr_db(stats_host) -> float:

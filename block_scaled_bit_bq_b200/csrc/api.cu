@@ -298,6 +298,15 @@ bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void*
     return cuda_status(launch_qsnr(p.fmt, scale_kind(p), p.had != 0, a, s));
 }
 
+bq_status bq_wait_timeouts(uint32_t* count, int32_t reset)
+{
+    if (!count) return BQ_ERR_INVALID_ARG;
+    unsigned int c = 0;
+    if (bq::flat_wait_timeouts(&c, reset != 0) != cudaSuccess) return BQ_ERR_CUDA;
+    *count = c;
+    return BQ_OK;
+}
+
 double bq_stats_qsnr_db(const bq_stats* host_stats)
 {
     if (!host_stats) return NAN;

@@ -20,7 +20,7 @@ struct FlatArgs {
     bq_stats* stats;
     uint8_t* ws;
     uint32_t n_chunks;          // rows * cols / 16
-    uint32_t n_dtiles;          // ceil(n_chunks / 128): a warp takes 128 chunks per step
+    uint32_t n_dtiles;          // ceil(n_chunks / 128): a warp takes 128 chunks (one tile) per step
     int32_t lanes_per_group;    // per-group: 0 (block 16), -1 (block 32), block / 64 (64..512)
     int32_t scale_fp16;         // 1: fp16 scales and zero points
     double n_elems;
@@ -71,5 +71,9 @@ cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& 
 cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
                            cudaStream_t st);
 cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);
+
+// Tile waits of the quantize kernels that gave up (each leaves that call's results
+// incomplete); reset: set the count back to zero. Synchronous.
+cudaError_t flat_wait_timeouts(unsigned int* count, bool reset);
 
 }  // namespace bq

@@ -19,6 +19,7 @@
 // real arithmetic; this saves the inverse transform (bq_qsnr and bq_dequantize
 // work in the original domain).
 #include "quant_ops.cuh"
+#include "tma.cuh"
 #include "internal.h"
 
 #include <atomic>
@@ -101,12 +102,53 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
 // ---------------------------------------------------------------------------
 // Quantize kernel.
 //
-// Lane l of a warp owns a span of four consecutive chunks (64 elements, 128 bytes,
-// four 256-bit loads, all issued before any arithmetic) of the warp's 2048-element
-// tile; two CTAs of eight warps per SM keep 64 KB of loads in flight.
+// A warp owns a 2048-element tile at a time (grid-stride over the tiles): 32 rows of
+// 64 elements, lane l taking row l, a span of four consecutive 16-element chunks. The
+// tiles reach shared memory through the tensor-memory-access unit (a 2-D tensor map
+// over x seen as rows of 64 bf16, boxes of 32 rows, 128-byte swizzle), NST tiles ahead
+// of the one being quantized, each completed on the warp's own mbarrier; the warps of
+// a CTA never wait on each other. The 128-byte swizzle stores 16-byte unit u of row r
+// at unit u ^ (r & 7), so the 32 lanes' 16-byte reads hit distinct banks.
 // ---------------------------------------------------------------------------
 
-constexpr int SPAN = 4;   // chunks per lane per tile
+#ifndef BQ_FLAT_WARPS
+#define BQ_FLAT_WARPS 8
+#endif
+#ifndef BQ_FLAT_NST
+#define BQ_FLAT_NST 3
+#endif
+#ifndef BQ_FLAT_MINB
+#define BQ_FLAT_MINB 2
+#endif
+
+constexpr int SPAN = 4;                                    // chunks per lane per tile
+constexpr int FLAT_WARPS = BQ_FLAT_WARPS;                  // warps per CTA
+constexpr int NST = BQ_FLAT_NST;                           // tile buffers per warp
+constexpr uint32_t ROW_BYTES = SPAN * 32;                  // 128
+constexpr uint32_t TILE_BYTES = 32 * ROW_BYTES;            // 4 KiB
+constexpr uint32_t FLAT_SMEM = FLAT_WARPS * NST * TILE_BYTES + 1024;
+
+__device__ unsigned int g_flat_wait_timeouts = 0;
+
+// A lane's row of the current tile buffer.
+struct Row {
+    uint32_t addr;      // shared address of the row
+    uint32_t sw;        // row & 7 (the swizzle)
+};
+
+__device__ __forceinline__ void row_chunk(const Row& r, int k, uint32_t (&w)[8])
+{
+    const uint32_t u0 = (uint32_t)(2 * k) ^ r.sw, u1 = (uint32_t)(2 * k + 1) ^ r.sw;
+    lds_v4(r.addr + (u0 << 4), w[0], w[1], w[2], w[3]);
+    lds_v4(r.addr + (u1 << 4), w[4], w[5], w[6], w[7]);
+}
+
+__device__ __forceinline__ void row_put_chunk(const Row& r, int k, const uint32_t (&w)[8])
+{
+    const uint32_t u0 = (uint32_t)(2 * k) ^ r.sw, u1 = (uint32_t)(2 * k + 1) ^ r.sw;
+    sts_v4(r.addr + (u0 << 4), w[0], w[1], w[2], w[3]);
+    sts_v4(r.addr + (u1 << 4), w[4], w[5], w[6], w[7]);
+}
 
 struct TensorCtx {
     float amax;          // per-tensor / NV: amax of the (rotated) tensor
@@ -123,36 +165,6 @@ __device__ __forceinline__ void chunk_in(const uint32_t (&w)[8], float2 (&y)[8])
     if constexpr (HAD) fwht16x2(y);
 }
 
-// Range of chunks [c0, c0 + N) of the lane's span: amax, or min and max (asymmetric).
-template <bool HAD, bool ASYM, int N>
-__device__ __forceinline__ void span_range(const uint32_t (&w)[SPAN][8], int c0, float& amax, float& mn, float& mx)
-{
-    if constexpr (HAD) {
-        amax = 0.0f; mn = 0.0f; mx = 0.0f;
-#pragma unroll
-        for (int k = 0; k < N; ++k) {
-            float2 y[8];
-            chunk_in<true>(w[c0 + k], y);
-            if constexpr (ASYM) chunk_minmax(y, mn, mx);
-            else amax = chunk_amax(y, amax);
-        }
-        if constexpr (ASYM) amax = fmaxf(-mn, mx);
-    } else if constexpr (ASYM) {
-        uint32_t lo = 0u, hi = 0u;          // bf16 pair (+0, +0)
-#pragma unroll
-        for (int k = 0; k < N; ++k) words_minmax(w[c0 + k], lo, hi);
-        mn = pair_min(lo);
-        mx = pair_max(hi);
-        amax = fmaxf(-mn, mx);
-    } else {
-        uint32_t m = 0u;
-#pragma unroll
-        for (int k = 0; k < N; ++k) m = words_absmax(w[c0 + k], m);
-        amax = pair_absmax(m);
-        mn = mx = 0.0f;
-    }
-}
-
 // NV block scale: s_b = E4M3((amax / Qmax) / S), d = s_b * S. The E4M3 code is taken
 // from the bracket amax * c (1 -+ 2^-20), c ~ 1 / (Qmax S) within 2^-23, which holds
 // RN(RN(amax / Qmax) / S) strictly inside; where the two codes differ it divides.
@@ -165,199 +177,285 @@ __device__ __forceinline__ uint32_t nv_scale_code(float amax, float S, float cS)
     const uint32_t pair = cvt_pair<BQ_FP8_E4M3>(__fmul_rn(a, BRACKET_HI), __fmul_rn(a, BRACKET_LO));
     const uint32_t lo = pair & 0xFFu, hi = pair >> 8;
     if (lo == hi && S >= 0x1p-100f && S <= 1.0e30f) return lo;
-    return e4m3_code(__fdiv_rn(__fdiv_rn(amax, F::qscale), S));
+    return e4m3_code(div_rn_call(div_rn_call(amax, F::qscale), S));
 }
 
-// Codes of chunk k of the lane's span: 4-bit codes are gathered for one 32-byte store
-// per span, 8-bit codes are stored right away (16 bytes per chunk).
+// Codes of chunk k (0..3, not a compile-time constant) of the lane's span: 4-bit codes
+// are gathered for one 32-byte store per span, 8-bit codes are stored right away.
 template <int FMT>
 __device__ __forceinline__ void put_codes(uint32_t (&span4)[8], uint8_t* codes, uint32_t c, bool valid, int k,
                                           const uint32_t (&w)[CodeWords<FMT>::n])
 {
     if constexpr (Fmt<FMT>::four) {
-        span4[2 * k] = w[0];
-        span4[2 * k + 1] = w[1];
+#pragma unroll
+        for (int j = 0; j < SPAN; ++j) {
+            span4[2 * j] = (j == k) ? w[0] : span4[2 * j];
+            span4[2 * j + 1] = (j == k) ? w[1] : span4[2 * j + 1];
+        }
     } else {
         if (valid) st_v4(codes + (size_t)c * 16, w);
     }
 }
 
-// One lane's span under the per-tensor unit.
-template <int FMT, bool HAD, bool STATS>
-__device__ __forceinline__ void span_tensor(const uint32_t (&w)[SPAN][8], uint32_t span, const FlatArgs& a,
-                                            const PlainUnit<FMT>& u, float p, double inv_p2, bool scaled,
-                                            Acc& acc, uint32_t (&span4)[8])
+// Chunk sums of a unit into the lane's accumulators.
+__device__ __forceinline__ void unit_done(Acc& acc, float2 e2, float2 x2, bool scaled, const Pow2& pw)
 {
-    float2 e2 = splat(0.0f), x2 = splat(0.0f);
-    const bool exact_res = !HAD && a.scale_fp16 != 0;
-#pragma unroll
-    for (int k = 0; k < SPAN; ++k) {
-        float2 y[8];
-        uint32_t q[CodeWords<FMT>::n];
-        chunk_in<HAD>(w[k], y);
-        if (scaled) plain_chunk<FMT, STATS, true>(y, u, p, exact_res, q, e2, x2);
-        else plain_chunk<FMT, STATS, false>(y, u, p, exact_res, q, e2, x2);
-        const uint32_t c = SPAN * span + k;
-        put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
-    }
-    if constexpr (STATS) add_unit_sums(acc, e2, x2, scaled ? inv_p2 : 1.0);
+    add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
 }
 
-// Units of N chunks (N = 1, 2 or 4) inside the lane's span; with N = 4 a unit can
-// also span T lanes (T = 1, 2, 4, 8: groups of 64 .. 512). A one-chunk unit is widened
-// (and rotated) once; larger units take their range from the raw bf16 words (or, when
-// rotated, from a first rotation) and widen again to quantize, which keeps register
-// pressure low.
-template <int FMT, int GK, bool HAD, bool STATS, int N>
-__device__ __forceinline__ void span_units(const uint32_t (&w)[SPAN][8], uint32_t span, const FlatArgs& a,
-                                           const TensorCtx& tc, Acc& acc, int lane, int T,
-                                           uint32_t (&span4)[8], uint8_t (&scode)[SPAN])
+// ---- per-tensor unit -------------------------------------------------------
+
+template <int FMT, bool HAD, bool STATS>
+__device__ __forceinline__ void span_tensor(const Row& row, uint32_t span, const FlatArgs& a,
+                                            const PlainUnit<FMT>& u, const Pow2& tp, bool scaled, Acc& acc,
+                                            uint32_t (&span4)[8])
+{
+    constexpr int NW = CodeWords<FMT>::n;
+    const bool exact_res = !HAD && a.scale_fp16 != 0;
+    const float p = scaled ? tp.p : 1.0f;
+    float2 e2 = splat(0.0f), x2 = splat(0.0f);
+    with_chunk_flags<FMT>(exact_res, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
+#pragma unroll 1
+        for (int k = 0; k < SPAN; ++k) {
+            uint32_t w[8], q[NW];
+            float2 y[8];
+            row_chunk(row, k, w);
+            chunk_in<HAD>(w, y);
+            plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
+            const uint32_t c = SPAN * span + k;
+            put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
+        }
+    });
+    if constexpr (STATS) unit_done(acc, e2, x2, scaled, tp);
+}
+
+// ---- one-chunk units: NV block 16, groups of 16 ------------------------------
+
+template <int FMT, int GK, bool HAD, bool STATS>
+__device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const FlatArgs& a, const TensorCtx& tc,
+                                        Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     constexpr bool GASYM = F::asym && GK == K_GROUP;
-#pragma unroll
-    for (int base = 0; base < SPAN; base += N) {
-        float amax = 0.0f, mn = 0.0f, mx = 0.0f;
-        float2 y1[8];                      // the chunk of a one-chunk unit
-        if constexpr (N == 1) {
-            chunk_in<HAD>(w[base], y1);
-            if constexpr (GASYM) { chunk_minmax(y1, mn, mx); amax = fmaxf(-mn, mx); }
-            else amax = chunk_amax(y1, 0.0f);
-        } else {
-            span_range<HAD, GASYM, N>(w, base, amax, mn, mx);
-        }
-        if (N == SPAN && T > 1) {
-            for (int o = 1; o < T; o <<= 1) {
-                if constexpr (GASYM) {
-                    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-                } else {
-                    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-                }
-            }
-            if constexpr (GASYM) amax = fmaxf(-mn, mx);
-        }
+    const bool f16 = a.scale_fp16 != 0;
+#pragma unroll 1
+    for (int k = 0; k < SPAN; ++k) {
+        uint32_t w[8], q[NW];
+        float2 y[8];
+        row_chunk(row, k, w);
+        chunk_in<HAD>(w, y);
+        float amax, mn = 0.0f, mx = 0.0f;
+        if constexpr (GASYM) { chunk_minmax(y, mn, mx); amax = fmaxf(-mn, mx); }
+        else amax = chunk_amax(y, 0.0f);
         const bool scaled = STATS && __any_sync(0xFFFFFFFFu, !plain_sums_ok(amax));
         const Pow2 pw = pow2_for(amax);
         const float p = scaled ? pw.p : 1.0f;
         float2 e2 = splat(0.0f), x2 = splat(0.0f);
+        const uint32_t c = SPAN * span + k;
+        const bool valid = c < a.n_chunks;
 
-        if constexpr (GK == K_MX) {
-            const int e = ue8m0_exponent<FMT>(amax);
-            const float p2 = exp2i(-e), pe = exp2i(e);
-#pragma unroll
-            for (int k = 0; k < N; ++k) {
-                float2 y[8], z[8];
-                uint32_t q[NW];
-                if constexpr (N == 1) { for (int i = 0; i < 8; ++i) y[i] = y1[i]; }
-                else chunk_in<HAD>(w[base + k], y);
-                if constexpr (F::is_int) {
-                    int8_chunk_pow2<STATS>(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
-                    if constexpr (STATS) {
-                        if (scaled) int_sums<true>(y, z, pe, p, e2, x2);
-                        else int_sums<false>(y, z, pe, p, e2, x2);
-                    }
-                } else {
-                    fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
-                    if constexpr (STATS) {
-                        if (scaled) val_sums<true>(y, z, pe, p, e2, x2);
-                        else val_sums<false>(y, z, pe, p, e2, x2);
-                    }
-                }
-                const uint32_t c = SPAN * span + base + k;
-                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base + k, q);
-            }
-            scode[base] = (uint8_t)(e + 127);
-        } else if constexpr (GK == K_NV) {
-            // N == 1
+        if constexpr (GK == K_NV) {
             const uint32_t sbc = nv_scale_code<FMT>(amax, tc.S, tc.cS);
             const float sbv = e4m3_value(sbc);
             const float d = __fmul_rn(sbv, tc.S);
-            scode[base] = (uint8_t)sbc;
-            uint32_t q[NW];
+            scodes |= sbc << (8 * k);
             if constexpr (F::is_int) {
                 const IntQ iq = int_unit<FMT>(d, 0.0f, -amax, amax, -7, 7);
                 float2 nq[8];
-                int_chunk<FMT, STATS>(y1, iq, -7, 7, q, nq);
+                int_chunk<FMT, STATS>(y, iq, -7, 7, q, nq);
                 if constexpr (STATS) {
                     // x-hat = (q s_b) S: the first product is exact
                     float2 val[8];
                     const float2 nA = splat(-sbv);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) val[i] = mul2(nq[i], nA);
-                    if (scaled) val_sums<true>(y1, val, tc.S, p, e2, x2);
-                    else val_sums<false>(y1, val, tc.S, p, e2, x2);
+                    if (scaled) val_sums<true>(y, val, tc.S, p, e2, x2);
+                    else val_sums<false>(y, val, tc.S, p, e2, x2);
                 }
             } else {
                 const FpQ fq = fp_unit(d, amax);
                 float2 val[8];
-                fp_chunk<FMT, STATS>(y1, fq, q, val);
+                fp_chunk<FMT, STATS>(y, fq, q, val);
                 if constexpr (STATS) {
                     const float2 A = splat(fq.zero ? 0.0f : sbv);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) val[i] = mul2(val[i], A);
-                    if (scaled) val_sums<true>(y1, val, tc.S, p, e2, x2);
-                    else val_sums<false>(y1, val, tc.S, p, e2, x2);
+                    if (scaled) val_sums<true>(y, val, tc.S, p, e2, x2);
+                    else val_sums<false>(y, val, tc.S, p, e2, x2);
                 }
             }
-            {
-                const uint32_t c = SPAN * span + base;
-                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base, q);
-            }
-        } else {  // K_GROUP
-            const bool f16 = a.scale_fp16 != 0;
+        } else {
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
             const PlainUnit<FMT> u = plain_unit<FMT>(ps);
-            const bool exact_res = !HAD && f16;
-#pragma unroll
-            for (int k = 0; k < N; ++k) {
-                float2 y[8];
-                uint32_t q[NW];
-                if constexpr (N == 1) { for (int i = 0; i < 8; ++i) y[i] = y1[i]; }
-                else chunk_in<HAD>(w[base + k], y);
-                if (scaled) plain_chunk<FMT, STATS, true>(y, u, p, exact_res, q, e2, x2);
-                else plain_chunk<FMT, STATS, false>(y, u, p, exact_res, q, e2, x2);
-                const uint32_t c = SPAN * span + base + k;
-                put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, base + k, q);
-            }
-            // the leader of the unit stores its scale
-            const uint32_t c_first = SPAN * span + base;
-            const bool leader = (N < SPAN) || ((lane & (T - 1)) == 0);
-            if (leader && c_first < a.n_chunks) {
-                const uint32_t unit = (N < SPAN) ? c_first / N : span / (uint32_t)T;
-                store_plain_scale<FMT>(a.scales, a.zps, unit, ps, f16);
-            }
+            with_chunk_flags<FMT>(!HAD && f16, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
+                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
+            });
+            if (valid) store_plain_scale<FMT>(a.scales, a.zps, c, ps, f16);
         }
-
+        put_codes<FMT>(span4, a.codes, c, valid, k, q);
         if constexpr (STATS) {
-            const uint32_t c_first = SPAN * span + base;
-            const bool valid = c_first < a.n_chunks;
-            if (valid) add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
-            float ss = __fadd_rn(x2.x, x2.y);
-            if (N == SPAN && T > 1)
-                for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
-            const bool leader = (N < SPAN) || ((lane & (T - 1)) == 0);
-            if (valid && leader) kappa_add(acc, __fmul_rn(amax, p), ss, a.inv_unit);
+            if (valid) {
+                unit_done(acc, e2, x2, scaled, pw);
+                kappa_add(acc, __fmul_rn(amax, p), __fadd_rn(x2.x, x2.y), a.inv_unit);
+            }
         }
     }
 }
 
-__device__ __forceinline__ void load_span(const uint32_t* x, uint32_t span, uint32_t n_chunks, uint32_t (&w)[SPAN][8])
+// ---- two-chunk units: MX block 32, groups of 32 -------------------------------
+
+template <int FMT, int GK, bool STATS>
+__device__ __forceinline__ void mx_chunk(const float2 (&y)[8], float p2, float pe, bool scaled, float p,
+                                         uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
 {
-    const uint32_t c0 = SPAN * span;
-    if (c0 + SPAN <= n_chunks) {
-#pragma unroll
-        for (int k = 0; k < SPAN; ++k) ld_nc_v8(x + (size_t)(c0 + k) * 8, w[k]);
+    using F = Fmt<FMT>;
+    float2 z[8];
+    if constexpr (F::is_int) {
+        int8_chunk_pow2<STATS>(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
+        if constexpr (STATS) {
+            if (scaled) int_sums<true>(y, z, pe, p, e2, x2);
+            else int_sums<false>(y, z, pe, p, e2, x2);
+        }
     } else {
-#pragma unroll
-        for (int k = 0; k < SPAN; ++k) {
-            if (c0 + k < n_chunks) ld_nc_v8(x + (size_t)(c0 + k) * 8, w[k]);
-            else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[k][i] = 0u;
+        fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
+        if constexpr (STATS) {
+            if (scaled) val_sums<true>(y, z, pe, p, e2, x2);
+            else val_sums<false>(y, z, pe, p, e2, x2);
+        }
+    }
+}
+
+template <int FMT, int GK, bool HAD, bool STATS>
+__device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const FlatArgs& a, Acc& acc,
+                                        uint32_t (&span4)[8], uint32_t& scodes)
+{
+    using F = Fmt<FMT>;
+    constexpr int NW = CodeWords<FMT>::n;
+    constexpr bool GASYM = F::asym && GK == K_GROUP;
+    const bool f16 = a.scale_fp16 != 0;
+#pragma unroll 1
+    for (int b = 0; b < SPAN; b += 2) {
+        uint32_t w0[8], w1[8], q0[NW], q1[NW];
+        float2 y0[8], y1[8];
+        row_chunk(row, b, w0);
+        row_chunk(row, b + 1, w1);
+        chunk_in<HAD>(w0, y0);
+        chunk_in<HAD>(w1, y1);
+        float amax, mn = 0.0f, mx = 0.0f;
+        if constexpr (GASYM) { chunk_minmax(y0, mn, mx); chunk_minmax(y1, mn, mx); amax = fmaxf(-mn, mx); }
+        else amax = chunk_amax(y1, chunk_amax(y0, 0.0f));
+        const bool scaled = STATS && __any_sync(0xFFFFFFFFu, !plain_sums_ok(amax));
+        const Pow2 pw = pow2_for(amax);
+        const float p = scaled ? pw.p : 1.0f;
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
+        const uint32_t c = SPAN * span + b;
+        const bool valid = c < a.n_chunks;
+
+        if constexpr (GK == K_MX) {
+            const int e = ue8m0_exponent<FMT>(amax);
+            const float p2 = exp2i(-e), pe = exp2i(e);
+            mx_chunk<FMT, GK, STATS>(y0, p2, pe, scaled, p, q0, e2, x2);
+            mx_chunk<FMT, GK, STATS>(y1, p2, pe, scaled, p, q1, e2, x2);
+            scodes |= (uint32_t)(e + 127) << (4 * b);
+        } else {
+            const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+            const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+            with_chunk_flags<FMT>(!HAD && f16, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
+                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y0, u, scaled, p, q0, e2, x2);
+                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y1, u, scaled, p, q1, e2, x2);
+            });
+            if (valid) store_plain_scale<FMT>(a.scales, a.zps, c / 2, ps, f16);
+        }
+        put_codes<FMT>(span4, a.codes, c, valid, b, q0);
+        put_codes<FMT>(span4, a.codes, c + 1, c + 1 < a.n_chunks, b + 1, q1);
+        if constexpr (STATS) {
+            if (valid) {
+                unit_done(acc, e2, x2, scaled, pw);
+                kappa_add(acc, __fmul_rn(amax, p), __fadd_rn(x2.x, x2.y), a.inv_unit);
             }
         }
+    }
+}
+
+// ---- groups of 64 .. 512: the span, or T = G / 64 adjacent lanes ---------------
+
+template <int FMT, bool HAD, bool STATS>
+__device__ __forceinline__ void span_n4(const Row& row, uint32_t span, const FlatArgs& a, Acc& acc, int lane, int T,
+                                        uint32_t (&span4)[8])
+{
+    using F = Fmt<FMT>;
+    constexpr int NW = CodeWords<FMT>::n;
+    const bool f16 = a.scale_fp16 != 0;
+    float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+    // range: from the raw bf16 words, or (rotated) from a first rotation
+    if constexpr (HAD) {
+#pragma unroll
+        for (int k = 0; k < SPAN; ++k) {
+            uint32_t w[8];
+            float2 y[8];
+            row_chunk(row, k, w);
+            chunk_in<true>(w, y);
+            if constexpr (F::asym) chunk_minmax(y, mn, mx);
+            else amax = chunk_amax(y, amax);
+        }
+    } else if constexpr (F::asym) {
+        uint32_t lo = 0u, hi = 0u;          // bf16 pair (+0, +0)
+#pragma unroll
+        for (int k = 0; k < SPAN; ++k) {
+            uint32_t w[8];
+            row_chunk(row, k, w);
+            words_minmax(w, lo, hi);
+        }
+        mn = pair_min(lo);
+        mx = pair_max(hi);
+    } else {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int k = 0; k < SPAN; ++k) {
+            uint32_t w[8];
+            row_chunk(row, k, w);
+            m = words_absmax(w, m);
+        }
+        amax = pair_absmax(m);
+    }
+    for (int o = 1; o < T; o <<= 1) {
+        if constexpr (F::asym) {
+            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        } else {
+            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        }
+    }
+    if constexpr (F::asym) amax = fmaxf(-mn, mx);
+
+    const bool scaled = STATS && __any_sync(0xFFFFFFFFu, !plain_sums_ok(amax));
+    const Pow2 pw = pow2_for(amax);
+    const float p = scaled ? pw.p : 1.0f;
+    const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+    const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+    const bool exact_res = !HAD && f16;
+    float2 e2 = splat(0.0f), x2 = splat(0.0f);
+    with_chunk_flags<FMT>(exact_res, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
+#pragma unroll 1
+        for (int k = 0; k < SPAN; ++k) {
+            uint32_t w[8], q[NW];
+            float2 y[8];
+            row_chunk(row, k, w);
+            chunk_in<HAD>(w, y);
+            plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
+            const uint32_t c = SPAN * span + k;
+            put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
+        }
+    });
+    const bool valid = SPAN * span < a.n_chunks;
+    const bool leader = (lane & (T - 1)) == 0;
+    if (leader && valid) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
+    if constexpr (STATS) {
+        if (valid) unit_done(acc, e2, x2, scaled, pw);
+        float ss = __fadd_rn(x2.x, x2.y);
+        for (int o = 1; o < T; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+        if (valid && leader) kappa_add(acc, __fmul_rn(amax, p), ss, a.inv_unit);
     }
 }
 
@@ -382,12 +480,37 @@ __device__ __forceinline__ void store_span4(uint8_t* codes, uint32_t span, uint3
 }
 
 template <int FMT, int GK, bool HAD, bool STATS>
-__global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
+__global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(const __grid_constant__ CUtensorMap xmap,
+                                                                  const FlatArgs a)
 {
     using F = Fmt<FMT>;
-    const int lane = threadIdx.x & 31;
-    const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    extern __shared__ uint8_t flat_smem[];
+    __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const uint32_t warp = blockIdx.x * FLAT_WARPS + wib;
+    const uint32_t nwarps = gridDim.x * FLAT_WARPS;
+    const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
+    const uint32_t bar0 = smem_addr(&bars[wib][0]);
+    const uint32_t rows_mapped = a.n_chunks / SPAN;     // whole rows the tensor map covers
+
+    if (lane == 0) {
+        for (int s = 0; s < NST; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    uint32_t inflight = 0, parity = 0;                  // per stage bits (warp-uniform)
+    auto issue = [&](uint32_t t, int s) {
+        if (t < a.n_dtiles && t * 32 < rows_mapped) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar0 + 8 * s, TILE_BYTES);
+                tma_load_2d(buf0 + s * TILE_BYTES, &xmap, bar0 + 8 * s, 0, (int)(t * 32));
+            }
+            inflight |= 1u << s;
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < NST; ++s) issue(warp + s * nwarps, s);
 
     TensorCtx tc{};
     PlainUnit<FMT> tu{};
@@ -403,33 +526,59 @@ __global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
             tscaled = STATS && !plain_sums_ok(tc.amax);
             if (blockIdx.x == 0 && threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, 0, tc.ps, a.scale_fp16 != 0);
         } else {
-            tc.S = __fdiv_rn(h->amax, F::qscale * 448.0f);
+            tc.S = div_rn_call(h->amax, F::qscale * 448.0f);
             tc.cS = rcp_approx(__fmul_rn(F::qscale, tc.S));
             if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scale[0] = tc.S;
         }
     }
-    // per-group units: 16 elements (N = 1), 32 (N = 2), 64 and up (N = 4, T lanes)
+    // per-group units: 16 elements (one chunk), 32 (two), 64 and up (the span, T lanes)
     const int T = (GK == K_GROUP && a.lanes_per_group > 0) ? a.lanes_per_group : 1;
 
     Acc acc;
+    bool ok = true;
+    int s = 0;
     for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
+        const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
         const uint32_t span = t * 32 + lane;
-        uint32_t cur[SPAN][8];
-        load_span(a.x, span, a.n_chunks, cur);
-        uint32_t span4[8];
-        uint8_t scode[SPAN] = {0, 0, 0, 0};
-
-        if constexpr (GK == K_TENSOR) {
-            span_tensor<FMT, HAD, STATS>(cur, span, a, tu, tp.p, tp.inv_p2, tscaled, acc, span4);
-        } else if constexpr (GK == K_NV) {
-            span_units<FMT, GK, HAD, STATS, 1>(cur, span, a, tc, acc, lane, 1, span4, scode);
-        } else if constexpr (GK == K_MX) {
-            span_units<FMT, GK, HAD, STATS, 2>(cur, span, a, tc, acc, lane, 1, span4, scode);
+        if (inflight >> s & 1u) {
+            const bool got = mbar_wait(bar0 + 8 * s, parity >> s & 1u);
+            parity ^= 1u << s;
+            inflight &= ~(1u << s);
+            if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
         } else {
-            if (a.lanes_per_group == 0) span_units<FMT, GK, HAD, STATS, 1>(cur, span, a, tc, acc, lane, 1, span4, scode);
-            else if (a.lanes_per_group < 0) span_units<FMT, GK, HAD, STATS, 2>(cur, span, a, tc, acc, lane, 1, span4, scode);
-            else span_units<FMT, GK, HAD, STATS, SPAN>(cur, span, a, tc, acc, lane, T, span4, scode);
+            // no row of this tile is covered by the tensor map
+            const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int k = 0; k < SPAN; ++k) row_put_chunk(row, k, z);
         }
+        if (span == rows_mapped && rows_mapped * SPAN < a.n_chunks) {
+            // the ragged end: chunks past the last whole row come from global memory
+            for (int k = 0; k < SPAN; ++k) {
+                uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                const uint32_t c = SPAN * span + k;
+                if (c < a.n_chunks) ld_nc_v8(a.x + (size_t)c * 8, w);
+                row_put_chunk(row, k, w);
+            }
+        }
+        fence_proxy_async();
+        __syncwarp();
+
+        uint32_t span4[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        uint32_t scodes = 0u;
+        if constexpr (GK == K_TENSOR) {
+            span_tensor<FMT, HAD, STATS>(row, span, a, tu, tp, tscaled, acc, span4);
+        } else if constexpr (GK == K_NV) {
+            span_n1<FMT, GK, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
+        } else if constexpr (GK == K_MX) {
+            span_n2<FMT, GK, HAD, STATS>(row, span, a, acc, span4, scodes);
+        } else {
+            if (a.lanes_per_group == 0) span_n1<FMT, GK, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
+            else if (a.lanes_per_group < 0) span_n2<FMT, GK, HAD, STATS>(row, span, a, acc, span4, scodes);
+            else span_n4<FMT, HAD, STATS>(row, span, a, acc, lane, T, span4);
+        }
+        __syncwarp();                       // every lane is done with the buffer
+        issue(t + NST * nwarps, s);
+        s = (s + 1 == NST) ? 0 : s + 1;
 
         store_span4<FMT>(a.codes, span, a.n_chunks, span4);
         const uint32_t c0 = SPAN * span;
@@ -437,18 +586,24 @@ __global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
             // four E4M3 block scales, one per chunk
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
             if (c0 + SPAN <= a.n_chunks)
-                *reinterpret_cast<uint32_t*>(sc + c0) = (uint32_t)scode[0] | ((uint32_t)scode[1] << 8) |
-                                                        ((uint32_t)scode[2] << 16) | ((uint32_t)scode[3] << 24);
+                *reinterpret_cast<uint32_t*>(sc + c0) = scodes;
             else
                 for (int k = 0; k < SPAN; ++k)
-                    if (c0 + k < a.n_chunks) sc[c0 + k] = scode[k];
+                    if (c0 + k < a.n_chunks) sc[c0 + k] = (uint8_t)(scodes >> (8 * k));
         } else if constexpr (GK == K_MX) {
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
             if (c0 + SPAN <= a.n_chunks)
-                *reinterpret_cast<uint16_t*>(sc + c0 / 2) = (uint16_t)(scode[0] | (scode[2] << 8));
+                *reinterpret_cast<uint16_t*>(sc + c0 / 2) = (uint16_t)scodes;
             else if (c0 < a.n_chunks)
-                sc[c0 / 2] = scode[0];
+                sc[c0 / 2] = (uint8_t)scodes;
         }
+    }
+    if (!ok) {
+        // a tile never arrived: record it, give the other loads in flight their chance
+        // to land (bounded) and stop; the results of this call are incomplete
+        if (lane == 0) atomicAdd(&g_flat_wait_timeouts, 1u);
+        for (int k = 0; k < NST; ++k)
+            if (inflight >> k & 1u) (void)mbar_wait(bar0 + 8 * k, parity >> k & 1u);
     }
 
     if constexpr (STATS) {
@@ -463,14 +618,16 @@ __global__ void __launch_bounds__(256, 2) k_quant_flat(const FlatArgs a)
 
 namespace {
 
-// Resident CTAs per SM of one kernel at one block size (cached per instantiation).
-template <auto KERN, int BLOCK>
+// Resident CTAs per SM of one kernel at one block size and dynamic shared memory size
+// (cached per instantiation; raises the kernel's dynamic shared memory limit first).
+template <auto KERN, int BLOCK, uint32_t SMEM>
 int resident_ctas()
 {
     static std::atomic<int> cached{-1};
     int v = cached.load(std::memory_order_relaxed);
     if (v < 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, KERN, BLOCK, 0) != cudaSuccess || v < 1) v = 1;
+        if (SMEM > 48u * 1024u) cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, KERN, BLOCK, SMEM) != cudaSuccess || v < 1) v = 1;
         cached.store(v, std::memory_order_relaxed);
     }
     return v;
@@ -478,10 +635,10 @@ int resident_ctas()
 
 // Grid of at most one wave (SM count x resident CTAs), at least enough CTAs to give
 // each min_items_per_cta items, capped at the workspace slot count.
-template <auto KERN, int BLOCK>
+template <auto KERN, int BLOCK, uint32_t SMEM>
 unsigned grid_for(uint64_t min_items_per_cta, uint64_t total_items)
 {
-    const uint64_t waves = (uint64_t)device_sm_count() * (uint64_t)resident_ctas<KERN, BLOCK>();
+    const uint64_t waves = (uint64_t)device_sm_count() * (uint64_t)resident_ctas<KERN, BLOCK, SMEM>();
     uint64_t need = (total_items + min_items_per_cta - 1) / min_items_per_cta;
     if (need < 1) need = 1;
     uint64_t g = need < waves ? need : waves;
@@ -489,14 +646,54 @@ unsigned grid_for(uint64_t min_items_per_cta, uint64_t total_items)
     return (unsigned)g;
 }
 
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
+EncodeTiled encode_tiled()
+{
+    static std::atomic<void*> fn{nullptr};
+    void* f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<EncodeTiled>(f);
+}
+
+// x seen as rows of 64 bf16 (128 bytes): boxes of 32 rows, 128-byte swizzle, zero fill
+// past the last row. rows = 0: a zeroed map that no launch reads.
+cudaError_t x_rows_map(const uint32_t* x, uint32_t rows, CUtensorMap* map)
+{
+    *map = CUtensorMap{};
+    if (rows == 0) return cudaSuccess;
+    const EncodeTiled enc = encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {64, rows};
+    const cuuint64_t strides[1] = {ROW_BYTES};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint32_t*>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int FMT, int GK, bool HAD, bool STATS>
 cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
-    constexpr int block = 256;
+    constexpr int block = FLAT_WARPS * 32;
     constexpr auto kern = k_quant_flat<FMT, GK, HAD, STATS>;
-    // one tile per warp at least (8 tiles per CTA)
-    const unsigned grid = grid_for<kern, block>(8, a.n_dtiles);
-    kern<<<grid, block, 0, st>>>(a);
+    CUtensorMap map;
+    const cudaError_t e = x_rows_map(a.x, a.n_chunks / SPAN, &map);
+    if (e != cudaSuccess) return e;
+    // one tile per warp at least
+    const unsigned grid = grid_for<kern, block, FLAT_SMEM>(FLAT_WARPS, a.n_dtiles);
+    kern<<<grid, block, FLAT_SMEM, st>>>(map, a);
     return cudaGetLastError();
 }
 
@@ -512,12 +709,22 @@ cudaError_t run_range(const uint32_t* x, uint32_t n_chunks, uint8_t* ws, cudaStr
 {
     constexpr int block = 256;
     constexpr auto kern = k_range<HAD, MINMAX>;
-    const unsigned grid = grid_for<kern, block>((uint64_t)block * 4, n_chunks);
+    const unsigned grid = grid_for<kern, block, 0>((uint64_t)block * 4, n_chunks);
     kern<<<grid, block, 0, st>>>(x, n_chunks, ws);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t flat_wait_timeouts(unsigned int* count, bool reset)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(count, g_flat_wait_timeouts, sizeof(unsigned int));
+    if (e == cudaSuccess && reset) {
+        const unsigned int zero = 0u;
+        e = cudaMemcpyToSymbol(g_flat_wait_timeouts, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
 
 cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool had, bool minmax, uint8_t* ws, cudaStream_t st)
 {

@@ -23,6 +23,7 @@
 #pragma once
 
 #include <cfloat>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -33,6 +34,81 @@ template <int FMT> struct CodeWords { static constexpr int n = Fmt<FMT>::four ? 
 // Offset added to signed 4-bit codes so that the nibbles are non-negative while they
 // are assembled (undone with one XOR per word).
 template <int FMT> struct CodeBias { static constexpr int v = (FMT == BQ_INT4_SYM) ? 8 : 0; };
+
+// ---------------------------------------------------------------------------
+// Ranges.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float chunk_amax(const float2 (&y)[8], float m)
+{
+    // a tree of three-input maxima (depth 3) instead of a chain of eight
+    const float a0 = amax3(fabsf(y[0].x), y[0].y, y[1].x);
+    const float a1 = amax3(fabsf(y[1].y), y[2].x, y[2].y);
+    const float a2 = amax3(fabsf(y[3].x), y[3].y, y[4].x);
+    const float a3 = amax3(fabsf(y[4].y), y[5].x, y[5].y);
+    const float a4 = amax3(fabsf(y[6].x), y[6].y, y[7].x);
+    const float b0 = amax3(a0, a1, a2), b1 = amax3(a3, a4, y[7].y);
+    return max3(m, b0, b1);
+}
+
+__device__ __forceinline__ void chunk_minmax(const float2 (&y)[8], float& mn, float& mx)
+{
+    float lo[3], hi[3];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float2 a = y[3 * j], b = y[3 * j + 1], c = y[3 * j + 2];
+        lo[j] = min3(min3(a.x, a.y, b.x), b.y, fminf(c.x, c.y));
+        hi[j] = max3(max3(a.x, a.y, b.x), b.y, fmaxf(c.x, c.y));
+    }
+    lo[2] = min3(y[6].x, y[6].y, fminf(y[7].x, y[7].y));
+    hi[2] = max3(y[6].x, y[6].y, fmaxf(y[7].x, y[7].y));
+    mn = min3(mn, min3(lo[0], lo[1], lo[2]), mn);
+    mx = max3(mx, max3(hi[0], hi[1], hi[2]), mx);
+}
+
+// on raw bf16 words (no widening); pairwise trees
+__device__ __forceinline__ uint32_t words_absmax(const uint32_t (&w)[8], uint32_t m)
+{
+    uint32_t a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = bf2_absmax(w[2 * i] & 0x7FFF7FFFu, w[2 * i + 1]);
+    return bf2_absmax(m, __vmaxu2(__vmaxu2(a[0], a[1]), __vmaxu2(a[2], a[3])));
+}
+
+__device__ __forceinline__ void words_minmax(const uint32_t (&w)[8], uint32_t& mn, uint32_t& mx)
+{
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lo[i] = bf2_min(w[2 * i], w[2 * i + 1]);
+        hi[i] = bf2_max(w[2 * i], w[2 * i + 1]);
+    }
+    mn = bf2_min(mn, bf2_min(bf2_min(lo[0], lo[1]), bf2_min(lo[2], lo[3])));
+    mx = bf2_max(mx, bf2_max(bf2_max(hi[0], hi[1]), bf2_max(hi[2], hi[3])));
+}
+
+// ---------------------------------------------------------------------------
+// Out-of-line slow paths. They run for a small fraction of the elements (or of the
+// units); keeping them out of line keeps the hot loops small for the instruction
+// cache.
+// ---------------------------------------------------------------------------
+
+// rne(RN(y / s)) as a float, clamped to +-2^22 (far outside every code range).
+static __device__ __noinline__ float div_rne_clamped(float y, float s)
+{
+    const float v = rintf(__fdiv_rn(y, s));
+    return fminf(fmaxf(v, -4194304.0f), 4194304.0f);
+}
+
+// The correctly rounded quotient a / b.
+static __device__ __noinline__ float div_rn_call(float a, float b) { return __fdiv_rn(a, b); }
+
+// FP codes of RN(hi / s) (upper byte) and RN(lo / s) (lower byte).
+template <int FMT>
+static __device__ __noinline__ uint32_t fp_div_pair(float hi, float lo, float s)
+{
+    return cvt_pair<FMT>(__fdiv_rn(hi, s), __fdiv_rn(lo, s));
+}
 
 // ---------------------------------------------------------------------------
 // Integer units.
@@ -75,7 +151,7 @@ __device__ __forceinline__ IntQ int_unit(float s, float zpf, float lo, float hi,
 
 // Exact code (magic form, t = mz + q) of one element whose residual test was
 // inconclusive.
-__device__ __forceinline__ float settle(float y, float s, float r, float mz, float t)
+static __device__ __noinline__ float settle(float y, float s, float r, float mz, float t)
 {
     const float q = __fsub_rn(t, mz);                        // exact
     const float f = __fmaf_rn(y, r, -q);
@@ -87,28 +163,27 @@ __device__ __forceinline__ float settle(float y, float s, float r, float mz, flo
         const float qe = q_even ? q : __fadd_rn(q, __fadd_rn(side, side));
         return __fadd_rn(qe, mz);
     }
-    float v = rintf(__fdiv_rn(y, s));
-    v = fminf(fmaxf(v, -4194304.0f), 4194304.0f);
-    return __fadd_rn(v, mz);
+    return __fadd_rn(div_rne_clamped(y, s), mz);
 }
 
-// Integer chunk: codes into w; nq[i] = -(code - zp) (exact) when NEED_Q.
-template <int FMT, bool NEED_Q>
+// Integer chunk: codes into w; nq[i] = -(code - zp) (exact) when NEED_Q. CHECK: test
+// for codes outside [qmin, qmax] (a caller passes false only for units whose clamp
+// flag is clear in every lane of the warp).
+template <int FMT, bool NEED_Q, bool CHECK = true>
 __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, int qmin, int qmax,
                                           uint32_t (&w)[CodeWords<FMT>::n], float2 (&nq)[8])
 {
     using F = Fmt<FMT>;
     constexpr float bias = (float)CodeBias<FMT>::v;
-    float2 t[8], nqq[8];
-    float fm = 0.0f;
+    float2 t[8], nqq[8], f[8];
     const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         t[i] = fma2(y[i], R, MZ);
         nqq[i] = fma2(t[i], M1, MZ);          // -q, exact
-        const float2 f = fma2(y[i], R, nqq[i]);
-        fm = amax3(fm, f.x, f.y);
+        f[i] = fma2(y[i], R, nqq[i]);
     }
+    const float fm = chunk_amax(f, 0.0f);
     const bool rare = !u.fast || !(fm < u.thr);
     if (__any_sync(0xFFFFFFFFu, rare)) {
         if (rare) {
@@ -121,18 +196,15 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, i
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float qa = rintf(__fdiv_rn(y[i].x, u.s)), qb = rintf(__fdiv_rn(y[i].y, u.s));
-                    qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
-                    qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
-                    t[i] = make_float2(__fadd_rn(qa, u.mz), __fadd_rn(qb, u.mz));
-                }
+                for (int i = 0; i < 8; ++i)
+                    t[i] = make_float2(__fadd_rn(div_rne_clamped(y[i].x, u.s), u.mz),
+                                       __fadd_rn(div_rne_clamped(y[i].y, u.s), u.mz));
             }
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) nqq[i] = fma2(t[i], M1, MZ);
     }
-    if (__any_sync(0xFFFFFFFFu, u.clamp)) {
+    if (CHECK && __any_sync(0xFFFFFFFFu, u.clamp)) {
         // the bounds hold the code + bias whatever the zero point; clamping is the
         // identity for units that never leave the range
         const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
@@ -175,54 +247,55 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, i
 // |e| > s/2 (the reciprocal's error put x r on the far side of a half-integer). Ties
 // are frequent for such inputs (about 1e-3 of the elements). e is returned for the
 // QSNR sums (the error of the final code).
-template <int FMT, bool NEED_E>
+template <int FMT, bool NEED_E, bool CHECK = true>
 __device__ __forceinline__ void int_chunk_exact(const float2 (&y)[8], const IntQ& u, int qmin, int qmax,
                                                 uint32_t (&w)[CodeWords<FMT>::n], float2 (&e)[8])
 {
     using F = Fmt<FMT>;
     constexpr float bias = (float)CodeBias<FMT>::v;
     float2 t[8], ee[8];
-    float em = 0.0f;
     const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f), S = splat(u.s);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         t[i] = fma2(y[i], R, MZ);
         const float2 nq = fma2(t[i], M1, MZ);          // -q, exact
         ee[i] = fma2(nq, S, y[i]);                      // x - q s, exact
-        em = amax3(em, ee[i].x, ee[i].y);
     }
+    const float em = chunk_amax(ee, 0.0f);
     const float hs = __fmul_rn(0.5f, u.s);
     // (a zero scale has only zero elements: every code is the zero point)
     const bool rare = !u.fast || (!(em < hs) && hs > 0.0f);
     if (__any_sync(0xFFFFFFFFu, rare)) {
         if (rare) {
             if (u.fast) {
-                // parity of q from t's bits: t = MAGIC + zp + bias + q
+                // d = |e| - s/2 is exact. The code moves one step towards e when d > 0, or
+                // when d == 0 (an exact tie) and q is odd: as integers, d's bits + odd(q) > 0
+                // (d = +0 has bits 0; a negative d has negative bits).
                 const uint32_t zb = (uint32_t)(int)__fsub_rn(u.mz, MAGIC) & 1u;
+                auto fix = [&](float& tv, float& ev) {
+                    const int d = __float_as_int(__fsub_rn(fabsf(ev), hs));
+                    const int odd = (int)((__float_as_uint(tv) ^ zb) & 1u);
+                    if (d + odd > 0) {
+                        tv = __fadd_rn(tv, copysignf(1.0f, ev));
+                        ev = __fsub_rn(ev, copysignf(u.s, ev));      // exact
+                    }
+                };
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float ax = fabsf(ee[i].x), ay = fabsf(ee[i].y);
-                    if (ax > hs || (ax == hs && ((__float_as_uint(t[i].x) ^ zb) & 1u)))
-                        t[i].x = __fadd_rn(t[i].x, copysignf(1.0f, ee[i].x));
-                    if (ay > hs || (ay == hs && ((__float_as_uint(t[i].y) ^ zb) & 1u)))
-                        t[i].y = __fadd_rn(t[i].y, copysignf(1.0f, ee[i].y));
+                    fix(t[i].x, ee[i].x);
+                    fix(t[i].y, ee[i].y);
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float qa = rintf(__fdiv_rn(y[i].x, u.s)), qb = rintf(__fdiv_rn(y[i].y, u.s));
-                    qa = fminf(fmaxf(qa, -4194304.0f), 4194304.0f);
-                    qb = fminf(fmaxf(qb, -4194304.0f), 4194304.0f);
-                    t[i] = make_float2(__fadd_rn(qa, u.mz), __fadd_rn(qb, u.mz));
+                    t[i] = make_float2(__fadd_rn(div_rne_clamped(y[i].x, u.s), u.mz),
+                                       __fadd_rn(div_rne_clamped(y[i].y, u.s), u.mz));
+                    if constexpr (NEED_E) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
                 }
             }
         }
-        if constexpr (NEED_E) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
-        }
     }
-    if (__any_sync(0xFFFFFFFFu, u.clamp)) {
+    if (CHECK && __any_sync(0xFFFFFFFFu, u.clamp)) {
         const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
         float tmx = cmin, tmn = cmax;
 #pragma unroll
@@ -329,7 +402,7 @@ __device__ __forceinline__ void fp_chunk(const float2 (&y)[8], const FpQ& u,
                 for (int p = 0; p < 8; ++p) {
                     const float2 a = mul2(y[p], lo), b = mul2(y[p], hi);
                     const bool bad = !u.fast || (cvt_pair<FMT>(a.y, a.x) != cvt_pair<FMT>(b.y, b.x));
-                    if (bad) pr[p] = cvt_pair<FMT>(__fdiv_rn(y[p].y, u.s), __fdiv_rn(y[p].x, u.s));
+                    if (bad) pr[p] = fp_div_pair<FMT>(y[p].y, y[p].x, u.s);
                 }
             }
         }
@@ -388,7 +461,7 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
     PlainScale p;
     if constexpr (F::asym) {
         const float lo = fminf(mn, 0.0f), hi = fmaxf(mx, 0.0f);
-        float s32 = __fdiv_rn(__fsub_rn(hi, lo), F::qscale);
+        float s32 = div_rn_call(__fsub_rn(hi, lo), F::qscale);
         s32 = fminf(s32, FLT_MAX);                  // a range beyond fp32 saturates
         p.s = fp16 ? round_scale_f16(s32) : s32;
         if (p.s > 0.0f) {
@@ -401,7 +474,7 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
             if (p.s >= 0x1p-100f && bound < 4.0e6f && fabsf(f) < __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f)))
                 z = q;
             else
-                z = fminf(fmaxf(rintf(__fdiv_rn(-lo, p.s)), -1.0e9f), 1.0e9f);
+                z = div_rne_clamped(-lo, p.s);
             p.zpf = fminf(fmaxf(__fadd_rn((float)F::qmin, z), (float)F::qmin), (float)F::qmax);
         } else {
             p.zpf = (float)F::qmin;
@@ -409,7 +482,7 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
         p.lo = lo;
         p.hi = hi;
     } else {
-        const float s32 = __fdiv_rn(amax, F::qscale);
+        const float s32 = div_rn_call(amax, F::qscale);
         p.s = fp16 ? round_scale_f16(s32) : s32;
         p.zpf = 0.0f;
         p.lo = -amax;
@@ -524,28 +597,63 @@ __device__ __forceinline__ void val_sums(const float2 (&y)[8], const float2 (&va
     }
 }
 
-// Quantize one chunk of a plain unit; STATS adds its sums (scaled form when SCALED).
-// exact_res: the unit's scale has at most 11 significant bits (fp16) and y is unrotated
-// bf16 (uniform over the launch).
-template <int FMT, bool STATS, bool SCALED>
-__device__ __forceinline__ void plain_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, float p, bool exact_res,
+// Quantize one chunk of a plain unit; STATS adds its sums. EXACT: the unit's scale has
+// at most 11 significant bits (fp16) and y is unrotated bf16 (the value-domain residual
+// decides the codes). GENERAL: clamping is tested and the sums take the scaled form when
+// `scaled`; without it (a unit whose clamp flag is clear in every lane of the warp and
+// whose sums are plain) neither is looked at.
+template <int FMT, bool STATS, bool EXACT, bool GENERAL>
+__device__ __forceinline__ void plain_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, bool scaled, float p,
                                             uint32_t (&w)[CodeWords<FMT>::n], float2& e2, float2& x2)
 {
     using F = Fmt<FMT>;
     if constexpr (F::is_int) {
-        if (exact_res) {
+        if constexpr (EXACT) {
             float2 e[8];
-            int_chunk_exact<FMT, STATS>(y, u.iq, F::qmin, F::qmax, w, e);
-            if constexpr (STATS) res_sums<SCALED>(y, e, p, e2, x2);
+            int_chunk_exact<FMT, STATS, GENERAL>(y, u.iq, F::qmin, F::qmax, w, e);
+            if constexpr (STATS) {
+                if (GENERAL && scaled) res_sums<true>(y, e, p, e2, x2);
+                else res_sums<false>(y, e, p, e2, x2);
+            }
         } else {
             float2 nq[8];
-            int_chunk<FMT, STATS>(y, u.iq, F::qmin, F::qmax, w, nq);
-            if constexpr (STATS) int_sums<SCALED>(y, nq, u.s, p, e2, x2);
+            int_chunk<FMT, STATS, GENERAL>(y, u.iq, F::qmin, F::qmax, w, nq);
+            if constexpr (STATS) {
+                if (GENERAL && scaled) int_sums<true>(y, nq, u.s, p, e2, x2);
+                else int_sums<false>(y, nq, u.s, p, e2, x2);
+            }
         }
     } else {
         float2 val[8];
         fp_chunk<FMT, STATS>(y, u.fq, w, val);
-        if constexpr (STATS) val_sums<SCALED>(y, val, u.s, p, e2, x2);
+        if constexpr (STATS) {
+            if (GENERAL && scaled) val_sums<true>(y, val, u.s, p, e2, x2);
+            else val_sums<false>(y, val, u.s, p, e2, x2);
+        }
+    }
+}
+
+// Whether a plain unit needs the general chunk path (warp-uniform: clamping in some lane,
+// or scaled sums).
+template <int FMT>
+__device__ __forceinline__ bool unit_general(const PlainUnit<FMT>& u, bool scaled)
+{
+    if constexpr (Fmt<FMT>::is_int) return scaled || __any_sync(0xFFFFFFFFu, u.iq.clamp);
+    else return scaled;
+}
+
+// Call f(std::integral_constant<bool, EXACT>, std::integral_constant<bool, GENERAL>) with
+// the runtime flags as compile-time constants (the integer formats only use EXACT).
+template <int FMT, typename Fn>
+__device__ __forceinline__ void with_chunk_flags(bool exact, bool general, Fn&& f)
+{
+    using T = std::true_type;
+    using N = std::false_type;
+    if constexpr (Fmt<FMT>::is_int) {
+        if (exact) { if (general) f(T{}, T{}); else f(T{}, N{}); }
+        else { if (general) f(N{}, T{}); else f(N{}, N{}); }
+    } else {
+        if (general) f(N{}, T{}); else f(N{}, N{});
     }
 }
 
@@ -561,43 +669,6 @@ __device__ __forceinline__ void store_codes(uint8_t* codes, uint32_t c, const ui
 {
     if constexpr (Fmt<FMT>::four) st_v2(codes + (size_t)c * 8, w);
     else st_v4(codes + (size_t)c * 16, w);
-}
-
-// ---------------------------------------------------------------------------
-// Ranges.
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ float chunk_amax(const float2 (&y)[8], float m)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = amax3(m, y[i].x, y[i].y);
-    return m;
-}
-
-__device__ __forceinline__ void chunk_minmax(const float2 (&y)[8], float& mn, float& mx)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        mn = min3(mn, y[i].x, y[i].y);
-        mx = max3(mx, y[i].x, y[i].y);
-    }
-}
-
-// on raw bf16 words (no widening)
-__device__ __forceinline__ uint32_t words_absmax(const uint32_t (&w)[8], uint32_t m)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = bf2_absmax(m, w[i]);
-    return m;
-}
-
-__device__ __forceinline__ void words_minmax(const uint32_t (&w)[8], uint32_t& mn, uint32_t& mx)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        mn = bf2_min(mn, w[i]);
-        mx = bf2_max(mx, w[i]);
-    }
 }
 
 __device__ __forceinline__ float pair_absmax(uint32_t m) { return fmaxf(bf_lo(m), bf_hi(m)); }

@@ -114,39 +114,41 @@ __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
 
         // every lane of a warp quantizes (lanes past the row's end pass zeros and store
         // nothing): the chunk functions are warp-collective
-        auto emit = [&](const uint32_t (&wi)[8], uint32_t c, bool valid) {
-            float2 v[8];
-            uint32_t q[NW];
-            widen16x2(wi, v);
-            if constexpr (HAD) fwht16x2(v);
-            if (scaled) plain_chunk<FMT, STATS, true>(v, u, p, exact_res, q, e2, x2);
-            else plain_chunk<FMT, STATS, false>(v, u, p, exact_res, q, e2, x2);
-            if (valid) store_codes<FMT>(a.codes, c_row + c, q);
-        };
-
-        if constexpr (K > 0) {
+        with_chunk_flags<FMT>(exact_res, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
+            auto emit = [&](const uint32_t (&wi)[8], uint32_t c, bool valid) {
+                float2 v[8];
+                uint32_t q[NW];
+                widen16x2(wi, v);
+                if constexpr (HAD) fwht16x2(v);
+                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(v, u, scaled, p, q, e2, x2);
+                if (valid) store_codes<FMT>(a.codes, c_row + c, q);
+            };
+            if constexpr (K > 0) {
 #pragma unroll
-            for (int k = 0; k < K; ++k) {
-                const uint32_t c = tid + k * B;
-                emit(cur[k], c, c < a.cpr);
+                for (int k = 0; k < K; ++k) {
+                    const uint32_t c = tid + k * B;
+                    emit(cur[k], c, c < a.cpr);
+                }
+            } else {
+                // all lanes run the same trip count (those past the end pass zeros)
+                const uint32_t trips = (a.cpr + B - 1) / B;
+                for (uint32_t j = 0; j < trips; ++j) {
+                    const uint32_t c = tid + j * B;
+                    uint32_t w[8];
+                    if (c < a.cpr) ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
+                    else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) w[i] = 0u;
+                    }
+                    emit(w, c, c < a.cpr);
+                }
             }
+        });
+        if constexpr (K > 0) {
 #pragma unroll
             for (int k = 0; k < K; ++k)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) cur[k][i] = nxt[k][i];
-        } else {
-            // all lanes run the same trip count (those past the end pass zeros)
-            const uint32_t trips = (a.cpr + B - 1) / B;
-            for (uint32_t j = 0; j < trips; ++j) {
-                const uint32_t c = tid + j * B;
-                uint32_t w[8];
-                if (c < a.cpr) ld_nc_v8(a.x + (size_t)(c_row + c) * 8, w);
-                else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) w[i] = 0u;
-                }
-                emit(w, c, c < a.cpr);
-            }
         }
 
         if constexpr (STATS) {

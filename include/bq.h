@@ -205,6 +205,21 @@ bq_status bq_quantize_noalloc(const void* x, int32_t x_dtype, int64_t rows, int6
                               void* codes, void* scales, void* zero_points, float* tensor_scale,
                               bq_stats* stats, void* stream);
 
+/*
+ * Bounded waits. The quantize kernels stage their input tiles in shared memory with
+ * tensor-map bulk copies and wait for each on an mbarrier; a wait that has not
+ * completed after about one second gives up instead of hanging. The kernel then stops
+ * early and the call's outputs are incomplete. This is a failure of the device or
+ * driver, not of the arguments.
+ *
+ * bq_wait_timeouts writes to *count how many such waits gave up on the current device
+ * since the library was loaded or last reset (reset != 0 sets the count back to zero).
+ * It synchronizes with the device (a blocking copy). count: host pointer.
+ * Returns BQ_ERR_INVALID_ARG for a NULL count, BQ_ERR_CUDA if the copy fails.
+ * (The source pages have no counterpart: this only reports the library's own waits.)
+ */
+bq_status bq_wait_timeouts(uint32_t* count, int32_t reset);
+
 /* -10 log10(err2 / x2) from a host copy of the stats (+inf when err2 = 0). */
 double bq_stats_qsnr_db(const bq_stats* host_stats);
 

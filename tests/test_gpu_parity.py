@@ -159,6 +159,9 @@ INPUTS = {
     # rotated schemes take |x| <= 2^125
     "edge_rot_8x512": lambda: _edge_tensor(big=1.5e38 / 16),
     "ragged_5x48": lambda: synth.normal(5, 48, seed=103, sigma=3.0),
+    # 129 and 387 chunks: the last warp tile holds only the ragged end (no whole row)
+    "tail_1x2064": lambda: synth.normal(1, 2064, seed=106, sigma=2.0),
+    "tail_3x2064": lambda: synth.weight_outliers(3, 2064, seed=107),
     "single_1x16": lambda: synth.uniform(1, 16, seed=104),
     "uniform_3x2048": lambda: synth.uniform(3, 2048, seed=105),
 }
@@ -259,3 +262,8 @@ def test_weight_x50_full(ws):
         st = q.stats.cpu().numpy()
         assert abs(bq.bq_stats_qsnr_db(st) - oracle.qsnr_db(o["stats"][0], o["stats"][1])) < QSNR_TOL_DB
         assert st[4] == o["stats"][4] and _close(st[2], o["stats"][2])
+
+
+def test_no_tile_wait_gave_up(cuda_device):
+    # every staged tile of every call above arrived (bounded waits never ran out)
+    assert bq.bq_wait_timeouts() == 0
