@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
-KERNEL_SOURCES = ["common.cuh", "quant_ops.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu"]
+KERNEL_SOURCES = ("common.cuh", "quant_ops.cuh", "tma.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu")
 
 # workload -> (generator kwargs, list of (label, scheme args))
 WORKLOADS = {
