@@ -224,6 +224,32 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
         const cudaError_t e = launch_range(xw, p.n_chunks, p.had != 0, p.gran == BQ_PER_TENSOR && p.asym, ws, s);
         if (e != cudaSuccess) return BQ_ERR_CUDA;
     }
+    const bool pow2_segments = cols % 64 == 0 && ((cols / 64) & (cols / 64 - 1)) == 0;
+    if (p.gran == BQ_PER_ROW && pow2_segments && cols <= 2048) {
+        // a row is a group of cols elements inside one warp tile (cols / 64 lanes)
+        FlatArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.n_chunks = p.n_chunks;
+        a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
+        a.lanes_per_group = (int32_t)(cols / 64);
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.n_elems = (double)p.n;
+        a.inv_unit = 1.0f / (float)cols;
+        return cuda_status(launch_quant_flat(p.fmt, K_GROUP, p.had != 0, want_stats, a, s));
+    }
+    if (p.gran == BQ_PER_ROW && cols % 64 == 0) {
+        RowsArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols; a.cpr = (uint32_t)(cols / 16);
+        a.nseg = (uint32_t)(cols / 64); a.tiles = (a.nseg + 31u) / 32u;
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.inv_cols = 1.0f / (float)cols;
+        return cuda_status(launch_quant_rows(p.fmt, p.had != 0, want_stats, a, s));
+    }
     if (p.gran == BQ_PER_ROW) {
         RowArgs a;
         std::memset(&a, 0, sizeof a);

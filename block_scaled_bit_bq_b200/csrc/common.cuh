@@ -454,42 +454,64 @@ __device__ __forceinline__ float warp_minf(float v)
     return v;
 }
 
-// Block-wide reduction of an Acc into thread 0 (fixed order: warp tree, then warps
-// in index order). blockDim.x must be a multiple of 32 and at most 1024.
-// Block totals in double (fixed order: warp tree, then warps in index order).
+// Block totals in double.
 struct AccD {
     double err2 = 0.0, x2 = 0.0, ksum = 0.0, kmax = 0.0, nunits = 0.0;
 };
 
+// Sum (max for kmax) over the 32 lanes of a warp: a fixed xor tree, the same in every
+// lane, so the result does not depend on timing.
+__device__ __forceinline__ AccD warp_reduce_acc(AccD a)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a.err2 += __shfl_xor_sync(0xFFFFFFFFu, a.err2, o);
+        a.x2 += __shfl_xor_sync(0xFFFFFFFFu, a.x2, o);
+        a.ksum += __shfl_xor_sync(0xFFFFFFFFu, a.ksum, o);
+        a.kmax = fmax(a.kmax, __shfl_xor_sync(0xFFFFFFFFu, a.kmax, o));
+        a.nunits += __shfl_xor_sync(0xFFFFFFFFu, a.nunits, o);
+    }
+    return a;
+}
+
+// Block-wide reduction (every thread calls it; blockDim.x a multiple of 32, at most
+// 1024): warps reduce, then warp 0 reduces the warps' totals. The result is valid in
+// warp 0.
 __device__ __forceinline__ AccD block_reduce_acc(AccD a)
 {
     __shared__ double sh[32][5];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    a.err2 = warp_sum(a.err2);
-    a.x2 = warp_sum(a.x2);
-    a.ksum = warp_sum(a.ksum);
-    a.kmax = warp_max(a.kmax);
-    a.nunits = warp_sum(a.nunits);
-    __syncthreads();
+    a = warp_reduce_acc(a);
+    __syncthreads();                 // sh may still be read by a previous call
     if (lane == 0) {
         sh[warp][0] = a.err2; sh[warp][1] = a.x2; sh[warp][2] = a.ksum;
         sh[warp][3] = a.kmax; sh[warp][4] = a.nunits;
     }
     __syncthreads();
     AccD t;
-    if (threadIdx.x == 0) {
-        for (int w = 0; w < nw; ++w) {
-            t.err2 += sh[w][0]; t.x2 += sh[w][1]; t.ksum += sh[w][2];
-            t.kmax = fmax(t.kmax, sh[w][3]); t.nunits += sh[w][4];
+    if (warp == 0) {
+        if (lane < nw) {
+            t.err2 = sh[lane][0]; t.x2 = sh[lane][1]; t.ksum = sh[lane][2];
+            t.kmax = sh[lane][3]; t.nunits = sh[lane][4];
         }
+        t = warp_reduce_acc(t);
     }
     return t;
 }
 
+// Add one to a counter with release (this thread's earlier writes are visible to whoever
+// observes the new value) and acquire (later reads see what the earlier adders released).
+__device__ __forceinline__ unsigned int atomic_add_acq_rel(unsigned int* p, unsigned int v)
+{
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Called by every thread of every CTA at kernel end. Each CTA leaves its partial in
-// a workspace slot; the CTA that arrives last sums the slots in index order and
-// writes the result. tensor_kappa: the unit is the whole tensor; kappa = amax /
-// sqrt(x2 / n_elems) is formed from the totals.
+// a workspace slot; the CTA that arrives last sums the slots (in a fixed order: slot by
+// slot per thread, then the xor trees) and writes the result. tensor_kappa: the unit is
+// the whole tensor; kappa = amax / sqrt(x2 / n_elems) is formed from the totals.
 __device__ __forceinline__ void finish_stats(Acc mine, uint8_t* ws, bq_stats* out,
                                              bool tensor_kappa, float tensor_amax,
                                              double n_elems, bool write_kappa)
@@ -497,26 +519,22 @@ __device__ __forceinline__ void finish_stats(Acc mine, uint8_t* ws, bq_stats* ou
     __shared__ bool is_last;
     AccD m;
     m.err2 = mine.err2; m.x2 = mine.x2; m.ksum = mine.ksum; m.kmax = (double)mine.kmax; m.nunits = (double)mine.nunits;
-    AccD t = block_reduce_acc(m);
+    const AccD t = block_reduce_acc(m);
     StatSlot* slots = ws_stats(ws);
     WsHeader* h = ws_header(ws);
     if (threadIdx.x == 0) {
-        StatSlot s{t.err2, t.x2, t.ksum, t.kmax, t.nunits, 0.0};
-        slots[blockIdx.x] = s;
-        __threadfence();
-        const unsigned ticket = atomicAdd(&h->counter_stats, 1u);
-        is_last = (ticket == gridDim.x - 1);
+        slots[blockIdx.x] = StatSlot{t.err2, t.x2, t.ksum, t.kmax, t.nunits, 0.0};
+        is_last = (atomic_add_acq_rel(&h->counter_stats, 1u) == gridDim.x - 1);
     }
     __syncthreads();
     if (!is_last) return;
-    __threadfence();
     AccD a;
     for (unsigned i = threadIdx.x; i < gridDim.x; i += blockDim.x) {
         const double* p = reinterpret_cast<const double*>(&slots[i]);
         a.err2 += __ldcg(p + 0); a.x2 += __ldcg(p + 1); a.ksum += __ldcg(p + 2);
         a.kmax = fmax(a.kmax, __ldcg(p + 3)); a.nunits += __ldcg(p + 4);
     }
-    AccD tot = block_reduce_acc(a);
+    const AccD tot = block_reduce_acc(a);
     if (threadIdx.x == 0) {
         bq_stats r;
         r.err2 = tot.err2;

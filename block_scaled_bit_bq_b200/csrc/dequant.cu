@@ -89,17 +89,43 @@ __device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>:
     }
 }
 
-// Dequantized fp32 values of chunk c (before any inverse rotation).
+// The scale factors of chunk c's unit, as loaded (a, b): plain scales (s, zero point),
+// MX (2^e, unused), NV (s_b, the tensor scale). Loaded ahead of the chunk's codes' use.
+struct UnitScale {
+    float a, b;
+};
+
 template <int FMT, int SK>
-__device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, const float2 (&val)[8],
-                                              float2 (&xh)[8])
+__device__ __forceinline__ UnitScale load_unit_scale(const DequantArgs& d, uint32_t c)
+{
+    const uint32_t u = d.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, d.fd_m) + c) >> d.fd_s);
+    UnitScale r{0.0f, 0.0f};
+    if constexpr (SK == SK_UE8M0) {
+        r.a = exp2i((int)__ldg(reinterpret_cast<const uint8_t*>(d.scales) + u) - 127);
+    } else if constexpr (SK == SK_NV) {
+        r.a = e4m3_value(__ldg(reinterpret_cast<const uint8_t*>(d.scales) + u));
+        r.b = __ldg(d.tensor_scale);
+    } else {
+        if (d.scale_fp16) {
+            r.a = __half2float(__ldg(reinterpret_cast<const __half*>(d.scales) + u));
+            if constexpr (Fmt<FMT>::asym) r.b = __half2float(__ldg(reinterpret_cast<const __half*>(d.zps) + u));
+        } else {
+            r.a = __ldg(reinterpret_cast<const float*>(d.scales) + u);
+            if constexpr (Fmt<FMT>::asym) r.b = __ldg(reinterpret_cast<const float*>(d.zps) + u);
+        }
+    }
+    return r;
+}
+
+// Dequantized fp32 values of a chunk (before any inverse rotation) from its element
+// values and its unit's scale factors.
+template <int FMT, int SK>
+__device__ __forceinline__ void dequant_chunk(const UnitScale& us, const float2 (&val)[8], float2 (&xh)[8])
 {
     using F = Fmt<FMT>;
     constexpr float off = MAGIC + (float)DecodeBias<FMT>::v;     // integer codes arrive as off + q
-    const uint32_t u = a.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, a.fd_m) + c) >> a.fd_s);
     if constexpr (SK == SK_UE8M0) {
-        const int e = (int)reinterpret_cast<const uint8_t*>(a.scales)[u] - 127;
-        const float2 pe = splat(exp2i(e));
+        const float2 pe = splat(us.a);
         if constexpr (F::is_int) {
             const float2 nz = splat(-off);
 #pragma unroll
@@ -109,8 +135,7 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
             for (int i = 0; i < 8; ++i) xh[i] = mul2(val[i], pe);
         }
     } else if constexpr (SK == SK_NV) {
-        const float2 sbv = splat(e4m3_value(reinterpret_cast<const uint8_t*>(a.scales)[u]));
-        const float2 S = splat(a.tensor_scale[0]);
+        const float2 sbv = splat(us.a), S = splat(us.b);
         if constexpr (F::is_int) {
             const float2 nz = splat(-off);
 #pragma unroll
@@ -120,18 +145,10 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs& a, uint32_t c, 
             for (int i = 0; i < 8; ++i) xh[i] = mul2(mul2(val[i], sbv), S);
         }
     } else {
-        float s, zp = 0.0f;
-        if (a.scale_fp16) {
-            s = __half2float(reinterpret_cast<const __half*>(a.scales)[u]);
-            if constexpr (F::asym) zp = __half2float(reinterpret_cast<const __half*>(a.zps)[u]);
-        } else {
-            s = reinterpret_cast<const float*>(a.scales)[u];
-            if constexpr (F::asym) zp = reinterpret_cast<const float*>(a.zps)[u];
-        }
-        const float2 S = splat(s);
+        const float2 S = splat(us.a);
         if constexpr (F::is_int) {
             // (off + q) - (off + zp) = q - zp, exact
-            const float2 nz = splat(-__fadd_rn(off, zp));
+            const float2 nz = splat(-__fadd_rn(off, us.b));
 #pragma unroll
             for (int i = 0; i < 8; ++i) xh[i] = mul2(add2(val[i], nz), S);
         } else {
@@ -150,11 +167,23 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
     uint32_t t = warp;
     uint32_t cur[NC];
-    if (t < a.n_dtiles) load_codes<FMT>(a.codes, t * 32 + lane, a.n_chunks, cur);
+    UnitScale cs[2];
+    // a chunk index past the end reads the last unit's scale (in bounds, unused)
+    auto clampc = [&](uint32_t c) { return c < a.n_chunks ? c : a.n_chunks - 1; };
+    if (t < a.n_dtiles) {
+        load_codes<FMT>(a.codes, t * 32 + lane, a.n_chunks, cur);
+        cs[0] = load_unit_scale<FMT, SK>(a, clampc(2 * (t * 32 + lane)));
+        cs[1] = load_unit_scale<FMT, SK>(a, clampc(2 * (t * 32 + lane) + 1));
+    }
     while (t < a.n_dtiles) {
         const uint32_t tn = t + nwarps;
         uint32_t nxt[NC];
-        if (tn < a.n_dtiles) load_codes<FMT>(a.codes, tn * 32 + lane, a.n_chunks, nxt);
+        UnitScale ns[2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+        if (tn < a.n_dtiles) {
+            load_codes<FMT>(a.codes, tn * 32 + lane, a.n_chunks, nxt);
+            ns[0] = load_unit_scale<FMT, SK>(a, clampc(2 * (tn * 32 + lane)));
+            ns[1] = load_unit_scale<FMT, SK>(a, clampc(2 * (tn * 32 + lane) + 1));
+        }
         const uint32_t span = t * 32 + lane;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -162,7 +191,7 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
             if (c >= a.n_chunks) break;
             float2 val[8], xh[8];
             chunk_values<FMT>(cur, h, val);
-            dequant_chunk<FMT, SK>(a, c, val, xh);
+            dequant_chunk<FMT, SK>(cs[h], val, xh);
             if constexpr (HAD) fwht16x2(xh);
             if constexpr (OUT == BQ_DT_BF16) {
                 uint32_t o[8];
@@ -186,6 +215,8 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
         }
 #pragma unroll
         for (int i = 0; i < NC; ++i) cur[i] = nxt[i];
+        cs[0] = ns[0];
+        cs[1] = ns[1];
         t = tn;
     }
 }
@@ -211,7 +242,7 @@ __global__ void __launch_bounds__(256) k_qsnr(const DequantArgs a)
             float2 x[8], val[8], xh[8];
             widen16x2(xw, x);
             chunk_values<FMT>(w, h, val);
-            dequant_chunk<FMT, SK>(a, c, val, xh);
+            dequant_chunk<FMT, SK>(load_unit_scale<FMT, SK>(a, c), val, xh);
             if constexpr (HAD) fwht16x2(xh);
             // sums on values scaled by a power of two fitted to the chunk (no overflow
             // or underflow in fp32), brought back in double

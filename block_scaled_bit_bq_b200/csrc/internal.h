@@ -41,6 +41,24 @@ struct RowArgs {
     float inv_cols;
 };
 
+// Per-row quantize of rows of cols % 64 == 0 elements, a warp per row (the row passes
+// through the warp's tile ring twice: range, then codes).
+struct RowsArgs {
+    const uint32_t* x;
+    uint8_t* codes;
+    void* scales;
+    void* zps;
+    bq_stats* stats;
+    uint8_t* ws;
+    uint32_t rows;
+    uint32_t cols;
+    uint32_t cpr;               // chunks per row = cols / 16
+    uint32_t nseg;              // 64-element segments per row = cols / 64
+    uint32_t tiles;             // tiles per row = ceil(nseg / 32)
+    int32_t scale_fp16;
+    float inv_cols;
+};
+
 struct DequantArgs {
     const uint8_t* codes;
     const void* scales;
@@ -68,6 +86,7 @@ cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool hadamard, bo
 cudaError_t launch_quant_flat(int fmt, int kind, bool hadamard, bool stats, const FlatArgs& a,
                               cudaStream_t st);
 cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& a, cudaStream_t st);
+cudaError_t launch_quant_rows(int fmt, bool hadamard, bool stats, const RowsArgs& a, cudaStream_t st);
 cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
                            cudaStream_t st);
 cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);

@@ -183,7 +183,7 @@ __device__ __forceinline__ uint32_t nv_scale_code(float amax, float S, float cS)
 // Codes of chunk k (0..3, not a compile-time constant) of the lane's span: 4-bit codes
 // are gathered for one 32-byte store per span, 8-bit codes are stored right away.
 template <int FMT>
-__device__ __forceinline__ void put_codes(uint32_t (&span4)[8], uint8_t* codes, uint32_t c, bool valid, int k,
+__device__ __forceinline__ void put_codes(uint32_t (&span4)[8], uint8_t* codes, size_t c, bool valid, int k,
                                           const uint32_t (&w)[CodeWords<FMT>::n])
 {
     if constexpr (Fmt<FMT>::four) {
@@ -193,8 +193,106 @@ __device__ __forceinline__ void put_codes(uint32_t (&span4)[8], uint8_t* codes, 
             span4[2 * j + 1] = (j == k) ? w[1] : span4[2 * j + 1];
         }
     } else {
-        if (valid) st_v4(codes + (size_t)c * 16, w);
+        if (valid) st_v4(codes + c * 16, w);
     }
+}
+
+// The chunks of a lane's span whose bit is set in `mask` through the general chunk path
+// (clamping, scaled sums, exact settling of the elements the fast path could not
+// decide); their sums are added to o.e2 / o.x2 and their codes stored (8-bit, chunks
+// k < n_valid) or gathered into o.span4 (4-bit). Chunk k is chunk c_first + k of the
+// tensor. Out of line and called once per span at most: the hot loops stay small.
+// Warp-collective (every lane calls it, mask 0 for lanes with nothing to redo).
+struct SpanOut {
+    float2 e2, x2;
+    uint32_t span4[8];
+};
+
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__device__ __noinline__ SpanOut general_chunks(uint32_t row_addr, uint32_t sw, PlainUnit<FMT> u, bool scaled, float p,
+                                               uint8_t* codes, size_t c_first, uint32_t mask, int n_valid, SpanOut o)
+{
+    const Row row{row_addr, sw};
+    for (int k = 0; k < SPAN; ++k) {
+        const bool mine = (mask >> k) & 1u;
+        if (!__any_sync(0xFFFFFFFFu, mine)) continue;
+        uint32_t w[8], q[CodeWords<FMT>::n];
+        float2 y[8];
+        float2 ce2 = splat(0.0f), cx2 = splat(0.0f);
+        row_chunk(row, k, w);
+        chunk_in<HAD>(w, y);
+        plain_chunk<FMT, STATS, EXACT, true>(y, u, scaled, p, q, ce2, cx2);
+        if (mine) {
+            o.e2 = add2(o.e2, ce2);
+            o.x2 = add2(o.x2, cx2);
+            put_codes<FMT>(o.span4, codes, c_first + k, k < n_valid, k, q);
+        }
+    }
+    return o;
+}
+
+// Hand a span's running sums and gathered codes to general_chunks and take them back.
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__device__ __forceinline__ void run_general(const Row& row, const PlainUnit<FMT>& u, bool scaled, float p,
+                                            uint8_t* codes, size_t c_first, uint32_t mask, int n_valid,
+                                            float2& e2, float2& x2, uint32_t (&span4)[8])
+{
+    SpanOut o;
+    o.e2 = e2;
+    o.x2 = x2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o.span4[i] = span4[i];
+    o = general_chunks<FMT, HAD, STATS, EXACT>(row.addr, row.sw, u, scaled, p, codes, c_first, mask, n_valid, o);
+    e2 = o.e2;
+    x2 = o.x2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) span4[i] = o.span4[i];
+}
+
+// Chunks [k0, k0 + n) of the lane's span through the fast path (codes placed, sums
+// added; it decides every element). With `general` (the unit needs the general path as
+// a whole) it does nothing and returns the mask of all n chunks; else 0.
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__device__ __forceinline__ uint32_t fast_chunks(const Row& row, const PlainUnit<FMT>& u, bool general, uint8_t* codes,
+                                                size_t c_first, int k0, int n, int n_valid,
+                                                float2& e2, float2& x2, uint32_t (&span4)[8])
+{
+    constexpr int NW = CodeWords<FMT>::n;
+    if (general) return ((1u << n) - 1u) << k0;
+#pragma unroll 1
+    for (int k = k0; k < k0 + n; ++k) {
+        uint32_t w[8], q[NW];
+        float2 y[8], ce2, cx2;
+        row_chunk(row, k, w);
+        chunk_in<HAD>(w, y);
+        (void)plain_chunk_fast<FMT, STATS, EXACT>(y, u, q, ce2, cx2);
+        if constexpr (STATS) {
+            e2 = add2(e2, ce2);
+            x2 = add2(x2, cx2);
+        }
+        put_codes<FMT>(span4, codes, c_first + k, k < n_valid, k, q);
+    }
+    return 0u;
+}
+
+// A plain unit over chunks [k0, k0 + n) of the lane's span: fast path, then the
+// general path for whatever it could not do.
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__device__ __forceinline__ void plain_unit_chunks(const Row& row, const PlainUnit<FMT>& u, bool scaled, float p,
+                                                  uint8_t* codes, size_t c_first, int k0, int n, int n_valid,
+                                                  float2& e2, float2& x2, uint32_t (&span4)[8])
+{
+    const bool general = unit_general_fast<FMT, EXACT>(u, scaled);
+    const uint32_t redo = fast_chunks<FMT, HAD, STATS, EXACT>(row, u, general, codes, c_first, k0, n, n_valid,
+                                                              e2, x2, span4);
+    if (general) run_general<FMT, HAD, STATS, EXACT>(row, u, scaled, p, codes, c_first, redo, n_valid, e2, x2, span4);
+}
+
+// Leading chunks of span `span` inside the tensor (0..4).
+__device__ __forceinline__ int span_valid(uint32_t span, uint32_t n_chunks)
+{
+    const uint32_t c0 = SPAN * span;
+    return c0 >= n_chunks ? 0 : (n_chunks - c0 >= (uint32_t)SPAN ? SPAN : (int)(n_chunks - c0));
 }
 
 // Chunk sums of a unit into the lane's accumulators.
@@ -205,33 +303,20 @@ __device__ __forceinline__ void unit_done(Acc& acc, float2 e2, float2 x2, bool s
 
 // ---- per-tensor unit -------------------------------------------------------
 
-template <int FMT, bool HAD, bool STATS>
+template <int FMT, bool HAD, bool STATS, bool EXACT>
 __device__ __forceinline__ void span_tensor(const Row& row, uint32_t span, const FlatArgs& a,
                                             const PlainUnit<FMT>& u, const Pow2& tp, bool scaled, Acc& acc,
                                             uint32_t (&span4)[8])
 {
-    constexpr int NW = CodeWords<FMT>::n;
-    const bool exact_res = !HAD && a.scale_fp16 != 0;
-    const float p = scaled ? tp.p : 1.0f;
     float2 e2 = splat(0.0f), x2 = splat(0.0f);
-    with_chunk_flags<FMT>(exact_res, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
-#pragma unroll 1
-        for (int k = 0; k < SPAN; ++k) {
-            uint32_t w[8], q[NW];
-            float2 y[8];
-            row_chunk(row, k, w);
-            chunk_in<HAD>(w, y);
-            plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
-            const uint32_t c = SPAN * span + k;
-            put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
-        }
-    });
+    plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, scaled ? tp.p : 1.0f, a.codes, (size_t)SPAN * span, 0,
+                                              SPAN, span_valid(span, a.n_chunks), e2, x2, span4);
     if constexpr (STATS) unit_done(acc, e2, x2, scaled, tp);
 }
 
 // ---- one-chunk units: NV block 16, groups of 16 ------------------------------
 
-template <int FMT, int GK, bool HAD, bool STATS>
+template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 __device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const FlatArgs& a, const TensorCtx& tc,
                                         Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
 {
@@ -253,7 +338,7 @@ __device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const Fla
         const float p = scaled ? pw.p : 1.0f;
         float2 e2 = splat(0.0f), x2 = splat(0.0f);
         const uint32_t c = SPAN * span + k;
-        const bool valid = c < a.n_chunks;
+        bool valid = c < a.n_chunks;
 
         if constexpr (GK == K_NV) {
             const uint32_t sbc = nv_scale_code<FMT>(amax, tc.S, tc.cS);
@@ -288,14 +373,16 @@ __device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const Fla
         } else {
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
             const PlainUnit<FMT> u = plain_unit<FMT>(ps);
-            with_chunk_flags<FMT>(!HAD && f16, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
-                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
-            });
-            if (valid) store_plain_scale<FMT>(a.scales, a.zps, c, ps, f16);
+            // codes go straight to span4 / memory (valid = false below skips put_codes)
+            plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, p, a.codes, (size_t)SPAN * span, k, 1,
+                                                      span_valid(span, a.n_chunks), e2, x2, span4);
+            if constexpr (Fmt<FMT>::four) { q[0] = span4[2 * k]; q[1] = span4[2 * k + 1]; }
+            else { valid = false; }
+            if (c < a.n_chunks) store_plain_scale<FMT>(a.scales, a.zps, c, ps, f16);
         }
         put_codes<FMT>(span4, a.codes, c, valid, k, q);
         if constexpr (STATS) {
-            if (valid) {
+            if (c < a.n_chunks) {
                 unit_done(acc, e2, x2, scaled, pw);
                 kappa_add(acc, __fmul_rn(amax, p), __fadd_rn(x2.x, x2.y), a.inv_unit);
             }
@@ -326,7 +413,7 @@ __device__ __forceinline__ void mx_chunk(const float2 (&y)[8], float p2, float p
     }
 }
 
-template <int FMT, int GK, bool HAD, bool STATS>
+template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 __device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const FlatArgs& a, Acc& acc,
                                         uint32_t (&span4)[8], uint32_t& scodes)
 {
@@ -351,6 +438,7 @@ __device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const Fla
         float2 e2 = splat(0.0f), x2 = splat(0.0f);
         const uint32_t c = SPAN * span + b;
         const bool valid = c < a.n_chunks;
+        bool gen = false;                 // codes already placed by the general path
 
         if constexpr (GK == K_MX) {
             const int e = ue8m0_exponent<FMT>(amax);
@@ -361,14 +449,15 @@ __device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const Fla
         } else {
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
             const PlainUnit<FMT> u = plain_unit<FMT>(ps);
-            with_chunk_flags<FMT>(!HAD && f16, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
-                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y0, u, scaled, p, q0, e2, x2);
-                plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y1, u, scaled, p, q1, e2, x2);
-            });
+            plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, p, a.codes, (size_t)SPAN * span, b, 2,
+                                                      span_valid(span, a.n_chunks), e2, x2, span4);
+            gen = true;
             if (valid) store_plain_scale<FMT>(a.scales, a.zps, c / 2, ps, f16);
         }
-        put_codes<FMT>(span4, a.codes, c, valid, b, q0);
-        put_codes<FMT>(span4, a.codes, c + 1, c + 1 < a.n_chunks, b + 1, q1);
+        if (!gen) {
+            put_codes<FMT>(span4, a.codes, c, valid, b, q0);
+            put_codes<FMT>(span4, a.codes, c + 1, c + 1 < a.n_chunks, b + 1, q1);
+        }
         if constexpr (STATS) {
             if (valid) {
                 unit_done(acc, e2, x2, scaled, pw);
@@ -380,7 +469,7 @@ __device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const Fla
 
 // ---- groups of 64 .. 512: the span, or T = G / 64 adjacent lanes ---------------
 
-template <int FMT, bool HAD, bool STATS>
+template <int FMT, bool HAD, bool STATS, bool EXACT>
 __device__ __forceinline__ void span_n4(const Row& row, uint32_t span, const FlatArgs& a, Acc& acc, int lane, int T,
                                         uint32_t (&span4)[8])
 {
@@ -434,20 +523,9 @@ __device__ __forceinline__ void span_n4(const Row& row, uint32_t span, const Fla
     const float p = scaled ? pw.p : 1.0f;
     const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
     const PlainUnit<FMT> u = plain_unit<FMT>(ps);
-    const bool exact_res = !HAD && f16;
     float2 e2 = splat(0.0f), x2 = splat(0.0f);
-    with_chunk_flags<FMT>(exact_res, unit_general<FMT>(u, scaled), [&](auto ex, auto ge) {
-#pragma unroll 1
-        for (int k = 0; k < SPAN; ++k) {
-            uint32_t w[8], q[NW];
-            float2 y[8];
-            row_chunk(row, k, w);
-            chunk_in<HAD>(w, y);
-            plain_chunk<FMT, STATS, decltype(ex)::value, decltype(ge)::value>(y, u, scaled, p, q, e2, x2);
-            const uint32_t c = SPAN * span + k;
-            put_codes<FMT>(span4, a.codes, c, c < a.n_chunks, k, q);
-        }
-    });
+    plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, p, a.codes, (size_t)SPAN * span, 0, SPAN,
+                                              span_valid(span, a.n_chunks), e2, x2, span4);
     const bool valid = SPAN * span < a.n_chunks;
     const bool leader = (lane & (T - 1)) == 0;
     if (leader && valid) store_plain_scale<FMT>(a.scales, a.zps, span / (uint32_t)T, ps, f16);
@@ -479,7 +557,7 @@ __device__ __forceinline__ void store_span4(uint8_t* codes, uint32_t span, uint3
     }
 }
 
-template <int FMT, int GK, bool HAD, bool STATS>
+template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(const __grid_constant__ CUtensorMap xmap,
                                                                   const FlatArgs a)
 {
@@ -566,15 +644,15 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         uint32_t span4[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         uint32_t scodes = 0u;
         if constexpr (GK == K_TENSOR) {
-            span_tensor<FMT, HAD, STATS>(row, span, a, tu, tp, tscaled, acc, span4);
+            span_tensor<FMT, HAD, STATS, EXACT>(row, span, a, tu, tp, tscaled, acc, span4);
         } else if constexpr (GK == K_NV) {
-            span_n1<FMT, GK, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
+            span_n1<FMT, GK, HAD, STATS, false>(row, span, a, tc, acc, span4, scodes);
         } else if constexpr (GK == K_MX) {
-            span_n2<FMT, GK, HAD, STATS>(row, span, a, acc, span4, scodes);
+            span_n2<FMT, GK, HAD, STATS, false>(row, span, a, acc, span4, scodes);
         } else {
-            if (a.lanes_per_group == 0) span_n1<FMT, GK, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
-            else if (a.lanes_per_group < 0) span_n2<FMT, GK, HAD, STATS>(row, span, a, acc, span4, scodes);
-            else span_n4<FMT, HAD, STATS>(row, span, a, acc, lane, T, span4);
+            if (a.lanes_per_group == 0) span_n1<FMT, GK, HAD, STATS, EXACT>(row, span, a, tc, acc, span4, scodes);
+            else if (a.lanes_per_group < 0) span_n2<FMT, GK, HAD, STATS, EXACT>(row, span, a, acc, span4, scodes);
+            else span_n4<FMT, HAD, STATS, EXACT>(row, span, a, acc, lane, T, span4);
         }
         __syncwarp();                       // every lane is done with the buffer
         issue(t + NST * nwarps, s);
@@ -610,6 +688,143 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         // per-tensor kappa comes from the totals: amax / sqrt(sum y^2 / n)
         finish_stats(acc, a.ws, a.stats, GK == K_TENSOR, tc.amax, a.n_elems, true);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Per-row quantize, a warp per row (rows of cols % 64 == 0 elements).
+//
+// The row reaches shared memory as M = ceil(cols / 2048) tiles of a 3-D tensor map (x
+// as [rows][cols / 64][64]; a box is 32 segments of 64 elements of one row, zero past
+// the row's end), lane l taking segment l of each tile (four chunks, as in the flat
+// kernel). The tiles pass through the warp's ring twice: for the row's range, then
+// (from L2) for the codes, so the ring needs no room for a whole row. One scale per
+// row, computed by every lane from the warp's reduced range.
+// ---------------------------------------------------------------------------
+
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_rows(const __grid_constant__ CUtensorMap xmap,
+                                                                            const RowsArgs a)
+{
+    using F = Fmt<FMT>;
+    constexpr int NW = CodeWords<FMT>::n;
+    extern __shared__ uint8_t flat_smem[];
+    __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const uint32_t warp = blockIdx.x * FLAT_WARPS + wib;
+    const uint32_t nwarps = gridDim.x * FLAT_WARPS;
+    const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
+    const uint32_t bar0 = smem_addr(&bars[wib][0]);
+    const uint32_t M = a.tiles, L = 2 * a.tiles;         // tiles per row, loads per row
+
+    if (lane == 0) {
+        for (int s = 0; s < NST; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    uint32_t inflight = 0, parity = 0;                   // per stage bits (warp-uniform)
+    // load k of this warp: row warp + (k / L) nwarps, tile (k % L) % M
+    auto issue = [&](uint32_t k, int s) {
+        const uint32_t r = warp + (k / L) * nwarps;
+        if (r < a.rows) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar0 + 8 * s, TILE_BYTES);
+                tma_load_3d(buf0 + s * TILE_BYTES, &xmap, bar0 + 8 * s, 0, (int)(((k % L) % M) * 32), (int)r);
+            }
+            inflight |= 1u << s;
+        }
+    };
+    auto wait_stage = [&](int s) -> bool {
+        if (!(inflight >> s & 1u)) return true;
+        const bool got = mbar_wait(bar0 + 8 * s, parity >> s & 1u);
+        parity ^= 1u << s;
+        inflight &= ~(1u << s);
+        return __all_sync(0xFFFFFFFFu, got);
+    };
+#pragma unroll
+    for (int s = 0; s < NST; ++s) issue((uint32_t)s, s);
+
+    const bool f16 = a.scale_fp16 != 0;
+    Acc acc;
+    bool ok = true;
+    uint32_t k = 0;
+    int s = 0;
+    for (uint32_t r = warp; r < a.rows && ok; r += nwarps) {
+        // pass 1: the lane's part of the row's range
+        float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+        uint32_t plo = 0u, phi = 0u, pm = 0u;            // packed bf16 pairs
+        for (uint32_t j = 0; j < M; ++j) {
+            if (!wait_stage(s)) { ok = false; break; }
+            const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
+#pragma unroll
+            for (int kk = 0; kk < SPAN; ++kk) {
+                uint32_t w[8];
+                row_chunk(row, kk, w);
+                if constexpr (HAD) {
+                    float2 y[8];
+                    chunk_in<true>(w, y);
+                    if constexpr (F::asym) chunk_minmax(y, mn, mx);
+                    else amax = chunk_amax(y, amax);
+                } else if constexpr (F::asym) {
+                    words_minmax(w, plo, phi);
+                } else {
+                    pm = words_absmax(w, pm);
+                }
+            }
+            __syncwarp();
+            issue(k + NST, s);
+            ++k;
+            s = (s + 1 == NST) ? 0 : s + 1;
+        }
+        if (!ok) break;
+        if constexpr (!HAD) {
+            if constexpr (F::asym) { mn = pair_min(plo); mx = pair_max(phi); }
+            else amax = pair_absmax(pm);
+        }
+        if constexpr (F::asym) { mn = warp_minf(mn); mx = warp_maxf(mx); amax = fmaxf(-mn, mx); }
+        else amax = warp_maxf(amax);
+
+        const bool scaled = STATS && !plain_sums_ok(amax);   // uniform over the warp
+        const Pow2 pw = pow2_for(amax);
+        const float p = scaled ? pw.p : 1.0f;
+        const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+        const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
+
+        // pass 2: codes
+        for (uint32_t j = 0; j < M; ++j) {
+            if (!wait_stage(s)) { ok = false; break; }
+            const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
+            const uint32_t g = j * 32 + lane;                    // the lane's segment
+            const bool seg_ok = g < a.nseg;
+            const size_t c0 = (size_t)r * a.cpr + 4u * g;        // its first chunk
+            uint32_t span4[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, p, a.codes, c0, 0, SPAN, seg_ok ? SPAN : 0,
+                                                      e2, x2, span4);
+            if constexpr (F::four) {
+                if (seg_ok) st_v8(a.codes + c0 * 8, span4);
+            }
+            __syncwarp();
+            issue(k + NST, s);
+            ++k;
+            s = (s + 1 == NST) ? 0 : s + 1;
+        }
+        if (!ok) break;
+        if (lane == 0) store_plain_scale<FMT>(a.scales, a.zps, r, ps, f16);
+        if constexpr (STATS) {
+            add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
+            float ss = __fadd_rn(x2.x, x2.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+            if (lane == 0) kappa_add(acc, __fmul_rn(amax, p), ss, a.inv_cols);
+        }
+    }
+    if (!ok) {
+        if (lane == 0) atomicAdd(&g_flat_wait_timeouts, 1u);
+        for (int kk = 0; kk < NST; ++kk)
+            if (inflight >> kk & 1u) (void)mbar_wait(bar0 + 8 * kk, parity >> kk & 1u);
+    }
+    if constexpr (STATS) finish_stats(acc, a.ws, a.stats, false, 0.0f, 0.0, true);
 }
 
 // ---------------------------------------------------------------------------
@@ -683,11 +898,56 @@ cudaError_t x_rows_map(const uint32_t* x, uint32_t rows, CUtensorMap* map)
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int FMT, int GK, bool HAD, bool STATS>
+// x seen as [rows][cols / 64][64]: boxes of 32 segments of one row, 128-byte swizzle,
+// zero fill past a row's end.
+cudaError_t x_segments_map(const uint32_t* x, uint32_t rows, uint32_t cols, CUtensorMap* map)
+{
+    *map = CUtensorMap{};
+    const EncodeTiled enc = encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {64, cols / 64, rows};
+    const cuuint64_t strides[2] = {ROW_BYTES, (cuuint64_t)cols * 2};
+    const cuuint32_t box[3] = {64, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint32_t*>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+cudaError_t run_rows(const RowsArgs& a, cudaStream_t st)
+{
+    constexpr int block = FLAT_WARPS * 32;
+    constexpr auto kern = k_quant_rows<FMT, HAD, STATS, EXACT>;
+    CUtensorMap map;
+    const cudaError_t e = x_segments_map(a.x, a.rows, a.cols, &map);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = grid_for<kern, block, FLAT_SMEM>(FLAT_WARPS, a.rows);
+    kern<<<grid, block, FLAT_SMEM, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+// The exact (value-domain) integer path: integer formats, fp16 scales, unrotated input.
+template <int FMT>
+constexpr bool can_exact() { return Fmt<FMT>::is_int; }
+
+template <int FMT>
+cudaError_t run_rows_hs(bool had, bool stats, const RowsArgs& a, cudaStream_t st)
+{
+    if (had) return stats ? run_rows<FMT, true, true, false>(a, st) : run_rows<FMT, true, false, false>(a, st);
+    if constexpr (can_exact<FMT>()) {
+        if (a.scale_fp16)
+            return stats ? run_rows<FMT, false, true, true>(a, st) : run_rows<FMT, false, false, true>(a, st);
+    }
+    return stats ? run_rows<FMT, false, true, false>(a, st) : run_rows<FMT, false, false, false>(a, st);
+}
+
+template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
     constexpr int block = FLAT_WARPS * 32;
-    constexpr auto kern = k_quant_flat<FMT, GK, HAD, STATS>;
+    constexpr auto kern = k_quant_flat<FMT, GK, HAD, STATS, EXACT>;
     CUtensorMap map;
     const cudaError_t e = x_rows_map(a.x, a.n_chunks / SPAN, &map);
     if (e != cudaSuccess) return e;
@@ -700,8 +960,12 @@ cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 template <int FMT, int GK>
 cudaError_t run_flat_hs(bool had, bool stats, const FlatArgs& a, cudaStream_t st)
 {
-    if (had) return stats ? run_flat<FMT, GK, true, true>(a, st) : run_flat<FMT, GK, true, false>(a, st);
-    return stats ? run_flat<FMT, GK, false, true>(a, st) : run_flat<FMT, GK, false, false>(a, st);
+    if (had) return stats ? run_flat<FMT, GK, true, true, false>(a, st) : run_flat<FMT, GK, true, false, false>(a, st);
+    if constexpr (can_exact<FMT>() && (GK == K_TENSOR || GK == K_GROUP)) {
+        if (a.scale_fp16)
+            return stats ? run_flat<FMT, GK, false, true, true>(a, st) : run_flat<FMT, GK, false, false, true>(a, st);
+    }
+    return stats ? run_flat<FMT, GK, false, true, false>(a, st) : run_flat<FMT, GK, false, false, false>(a, st);
 }
 
 template <bool HAD, bool MINMAX>
@@ -730,6 +994,19 @@ cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool had, bool mi
 {
     if (had) return minmax ? run_range<true, true>(x, n_chunks, ws, st) : run_range<true, false>(x, n_chunks, ws, st);
     return minmax ? run_range<false, true>(x, n_chunks, ws, st) : run_range<false, false>(x, n_chunks, ws, st);
+}
+
+cudaError_t launch_quant_rows(int fmt, bool had, bool stats, const RowsArgs& a, cudaStream_t st)
+{
+    switch (fmt) {
+    case BQ_INT8_SYM:   return run_rows_hs<BQ_INT8_SYM>(had, stats, a, st);
+    case BQ_INT8_ASYM:  return run_rows_hs<BQ_INT8_ASYM>(had, stats, a, st);
+    case BQ_INT4_SYM:   return run_rows_hs<BQ_INT4_SYM>(had, stats, a, st);
+    case BQ_UINT4_ASYM: return run_rows_hs<BQ_UINT4_ASYM>(had, stats, a, st);
+    case BQ_FP8_E4M3:   return run_rows_hs<BQ_FP8_E4M3>(had, stats, a, st);
+    case BQ_FP8_E5M2:   return run_rows_hs<BQ_FP8_E5M2>(had, stats, a, st);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_quant_flat(int fmt, int kind, bool had, bool stats, const FlatArgs& a, cudaStream_t st)

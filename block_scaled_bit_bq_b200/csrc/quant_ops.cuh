@@ -117,10 +117,15 @@ static __device__ __noinline__ uint32_t fp_div_pair(float hi, float lo, float s)
 struct IntQ {
     float s;        // the scale x is divided by (0: every code is the zero point)
     float r;        // ~ 1/s (0 when s == 0)
+    float rlo, rhi; // r (1 -+ 2^-22): strictly below and above 1/s (0 when s == 0)
     float mz;       // MAGIC + zero point + bias (exact)
     float thr;      // |f| below thr: the code is certain
+    float xc;       // asymmetric: inputs above xc take the code qmax (+inf: none do)
+    float rn;       // RN(1/s), the correctly rounded reciprocal (0 when s == 0)
+    bool mk;        // the fast paths' exact quotient holds for every element of the unit
     bool fast;      // s in the range where the residual test is valid
-    bool clamp;     // some element of the unit can leave [qmin, qmax]
+    bool br;        // the bracket decides every code of the unit (fp16 scales, see int_chunk_exact)
+    bool clamp;     // codes must be clamped (beyond what xc does)
 };
 
 // Unit from its stored scale s, zero point zpf and the extreme values lo <= 0 <= hi it
@@ -132,20 +137,43 @@ __device__ __forceinline__ IntQ int_unit(float s, float zpf, float lo, float hi,
     IntQ u;
     u.s = s;
     u.mz = __fadd_rn(__fadd_rn(MAGIC, zpf), bias);
+    u.xc = __int_as_float(0x7F800000);
     if (!(s > 0.0f)) {
-        u.r = 0.0f;
+        u.r = u.rlo = u.rhi = u.rn = 0.0f;
         u.thr = 1.0f;
-        u.fast = true;
+        u.fast = u.br = u.mk = true;
         u.clamp = false;
         return u;
     }
     u.r = rcp_approx(s);
+    u.rlo = __fmul_rn(u.r, 0x1.fffff8p-1f);                        // 1 - 2^-22
+    u.rhi = __fmul_rn(u.r, 0x1.000004p+0f);                        // 1 + 2^-22
     const float bound = __fmul_rn(fmaxf(-lo, hi), u.r);          // ~ max |x / s|
     u.fast = (s >= 0x1p-100f) && (s <= 1.0e37f) && (bound < 4.0e6f);
+    u.br = u.fast && bound < 400.0f;
+    u.rn = __frcp_rn(s);
+    u.mk = (s >= 0x1p-60f) && (s <= 0x1p100f) && (bound < 0x1p20f);
     u.thr = __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f));
-    // the code is monotone in x: the extremes bound every code (a quarter step of slack)
-    const float top = __fadd_rn(__fmul_rn(hi, u.r), zpf), bot = __fadd_rn(__fmul_rn(lo, u.r), zpf);
-    u.clamp = !u.fast || top > (float)qmax + 0.25f || bot < (float)qmin - 0.25f;
+    if constexpr (Fmt<FMT>::asym) {
+        // The code is monotone in x, so the extremes bound every code: rne(hi r_hi) + zp
+        // bounds the top one, rne(lo r_hi) + zp the bottom one. With zp = qmin +
+        // rne(-lo / s) the bottom code is qmin (round-half-even is odd-symmetric), and the
+        // top one can exceed qmax by one, when both -lo/s and hi/s lie near half-integers.
+        // Then inputs are capped at xc = (qmax - zp) s, whose quotient is exactly
+        // qmax - zp: the capped inputs take the code qmax, the others keep theirs.
+        bool under = false;
+        if (u.fast) {
+            const float qt = __fsub_rn(__fmaf_rn(hi, u.rhi, MAGIC), MAGIC);
+            const float qb = __fsub_rn(__fmaf_rn(lo, u.rhi, MAGIC), MAGIC);
+            if (__fadd_rn(qt, zpf) > (float)qmax) u.xc = __fmul_rn(__fsub_rn((float)qmax, zpf), s);
+            under = __fadd_rn(qb, zpf) < (float)qmin;
+        }
+        u.clamp = !u.fast || under;
+    } else {
+        // |x / s| <= Qmax (1 + 2^-10) for an AbsMax scale: a quarter step of slack
+        const float top = __fadd_rn(__fmul_rn(hi, u.r), zpf), bot = __fadd_rn(__fmul_rn(lo, u.r), zpf);
+        u.clamp = !u.fast || top > (float)qmax + 0.25f || bot < (float)qmin - 0.25f;
+    }
     return u;
 }
 
@@ -175,13 +203,15 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, i
 {
     using F = Fmt<FMT>;
     constexpr float bias = (float)CodeBias<FMT>::v;
-    float2 t[8], nqq[8], f[8];
+    float2 t[8], nqq[8], f[8], yq[8];
     const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        t[i] = fma2(y[i], R, MZ);
+        // asymmetric: inputs capped at xc for the code (the sums use y itself)
+        yq[i] = F::asym ? make_float2(fminf(y[i].x, u.xc), fminf(y[i].y, u.xc)) : y[i];
+        t[i] = fma2(yq[i], R, MZ);
         nqq[i] = fma2(t[i], M1, MZ);          // -q, exact
-        f[i] = fma2(y[i], R, nqq[i]);
+        f[i] = fma2(yq[i], R, nqq[i]);
     }
     const float fm = chunk_amax(f, 0.0f);
     const bool rare = !u.fast || !(fm < u.thr);
@@ -190,15 +220,14 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, i
             if (u.fast) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float2 f = fma2(y[i], R, nqq[i]);
-                    if (!(fabsf(f.x) < u.thr)) t[i].x = settle(y[i].x, u.s, u.r, u.mz, t[i].x);
-                    if (!(fabsf(f.y) < u.thr)) t[i].y = settle(y[i].y, u.s, u.r, u.mz, t[i].y);
+                    if (!(fabsf(f[i].x) < u.thr)) t[i].x = settle(yq[i].x, u.s, u.r, u.mz, t[i].x);
+                    if (!(fabsf(f[i].y) < u.thr)) t[i].y = settle(yq[i].y, u.s, u.r, u.mz, t[i].y);
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    t[i] = make_float2(__fadd_rn(div_rne_clamped(y[i].x, u.s), u.mz),
-                                       __fadd_rn(div_rne_clamped(y[i].y, u.s), u.mz));
+                    t[i] = make_float2(__fadd_rn(div_rne_clamped(yq[i].x, u.s), u.mz),
+                                       __fadd_rn(div_rne_clamped(yq[i].y, u.s), u.mz));
             }
         }
 #pragma unroll
@@ -240,96 +269,107 @@ __device__ __forceinline__ void int_chunk(const float2 (&y)[8], const IntQ& u, i
 }
 
 // Integer chunk for a scale with at most 11 significant bits (an fp16 scale) and
-// unrotated bf16 inputs. Then every product q s (|q| <= 2^8) and every residual
-// e = x - q s of a candidate q next to the quotient is exact, so the code is decided
-// in the value domain without any approximation: q is right when |e| < s/2, an exact
-// tie when |e| == s/2 (the code is then the even neighbour) and one step off when
-// |e| > s/2 (the reciprocal's error put x r on the far side of a half-integer). Ties
-// are frequent for such inputs (about 1e-3 of the elements). e is returned for the
-// QSNR sums (the error of the final code).
-template <int FMT, bool NEED_E, bool CHECK = true>
+// unrotated bf16 inputs (x has 8 significant bits).
+//
+// Then x / s is either an exact half-integer (a tie) or at least 2^-12 away from every
+// half-integer: 2x - (2k+1) s is a multiple of min(2 ulp(x), ulp(s)), and dividing by 2s
+// leaves at least 2^-12 (ulp(s) > s 2^-11; and 2 ulp(x) > |x| 2^-7 >= s 2^-8 whenever
+// |x/s| >= 1/2). The codes rne(x r_lo) and rne(x r_hi) of the bracket
+// r_lo < 1/s < r_hi are within |x/s| 1.25 2^-21 of it, less than 2^-12 for |x/s| < 400,
+// so they agree with rne(x/s) off ties. On a tie they are the two neighbours k, k+1,
+// and round-half-even takes the even one. So the code is the bracket code whose q is
+// even, and no element divides or branches.
+//
+// e[i] = x - q_lo s (exact) for the QSNR sums: off ties q_lo is the code, on a tie both
+// neighbours are s/2 away, so e^2 is the final code's either way.
+// GENERAL: clamp to [qmin, qmax] (e then follows the clamped code).
+template <int FMT, bool NEED_E, bool GENERAL>
 __device__ __forceinline__ void int_chunk_exact(const float2 (&y)[8], const IntQ& u, int qmin, int qmax,
                                                 uint32_t (&w)[CodeWords<FMT>::n], float2 (&e)[8])
 {
     using F = Fmt<FMT>;
     constexpr float bias = (float)CodeBias<FMT>::v;
-    float2 t[8], ee[8];
-    const float2 R = splat(u.r), MZ = splat(u.mz), M1 = splat(-1.0f), S = splat(u.s);
+    float2 tl[8], th[8], yq[8];
+    const float2 RL = splat(u.rlo), RH = splat(u.rhi), MZ = splat(u.mz), M1 = splat(-1.0f), S = splat(u.s);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        t[i] = fma2(y[i], R, MZ);
-        const float2 nq = fma2(t[i], M1, MZ);          // -q, exact
-        ee[i] = fma2(nq, S, y[i]);                      // x - q s, exact
+        // asymmetric: inputs capped at xc for the code (the residuals use y itself)
+        yq[i] = F::asym ? make_float2(fminf(y[i].x, u.xc), fminf(y[i].y, u.xc)) : y[i];
+        tl[i] = fma2(yq[i], RL, MZ);
+        th[i] = fma2(yq[i], RH, MZ);
     }
-    const float em = chunk_amax(ee, 0.0f);
-    const float hs = __fmul_rn(0.5f, u.s);
-    // (a zero scale has only zero elements: every code is the zero point)
-    const bool rare = !u.fast || (!(em < hs) && hs > 0.0f);
-    if (__any_sync(0xFFFFFFFFu, rare)) {
-        if (rare) {
-            if (u.fast) {
-                // d = |e| - s/2 is exact. The code moves one step towards e when d > 0, or
-                // when d == 0 (an exact tie) and q is odd: as integers, d's bits + odd(q) > 0
-                // (d = +0 has bits 0; a negative d has negative bits).
-                const uint32_t zb = (uint32_t)(int)__fsub_rn(u.mz, MAGIC) & 1u;
-                auto fix = [&](float& tv, float& ev) {
-                    const int d = __float_as_int(__fsub_rn(fabsf(ev), hs));
-                    const int odd = (int)((__float_as_uint(tv) ^ zb) & 1u);
-                    if (d + odd > 0) {
-                        tv = __fadd_rn(tv, copysignf(1.0f, ev));
-                        ev = __fsub_rn(ev, copysignf(u.s, ev));      // exact
-                    }
-                };
+    if (GENERAL && __any_sync(0xFFFFFFFFu, !u.br)) {
+        // units outside the bracket's range (huge quotients): correctly rounded quotients
+        // (without GENERAL the caller guarantees br)
+        if (!u.br) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    fix(t[i].x, ee[i].x);
-                    fix(t[i].y, ee[i].y);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    t[i] = make_float2(__fadd_rn(div_rne_clamped(y[i].x, u.s), u.mz),
-                                       __fadd_rn(div_rne_clamped(y[i].y, u.s), u.mz));
-                    if constexpr (NEED_E) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
-                }
+            for (int i = 0; i < 8; ++i) {
+                tl[i] = make_float2(__fadd_rn(div_rne_clamped(yq[i].x, u.s), u.mz),
+                                    __fadd_rn(div_rne_clamped(yq[i].y, u.s), u.mz));
+                th[i] = tl[i];
             }
         }
     }
-    if (CHECK && __any_sync(0xFFFFFFFFu, u.clamp)) {
-        const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
-        float tmx = cmin, tmn = cmax;
+    // parity of q = t - mz from t's bits: t = MAGIC + zp + bias + q and MAGIC is even
+    const uint32_t zb = (uint32_t)(int)__fsub_rn(u.mz, MAGIC) & 1u;
+    if constexpr (!GENERAL) {
+        // every code is in range: select per packed code (nibble or byte) with one LOP3
+        if constexpr (F::four) {
+            uint32_t hl[4], hh[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { tmx = max3(tmx, t[i].x, t[i].y); tmn = min3(tmn, t[i].x, t[i].y); }
-        if (__any_sync(0xFFFFFFFFu, tmx > cmax || tmn < cmin)) {
+            for (int k = 0; k < 4; ++k) {
+                hl[k] = __float_as_uint(tl[2 * k].x) + __float_as_uint(tl[2 * k].y) * 16u +
+                        __float_as_uint(tl[2 * k + 1].x) * 256u + __float_as_uint(tl[2 * k + 1].y) * 4096u;
+                hh[k] = __float_as_uint(th[2 * k].x) + __float_as_uint(th[2 * k].y) * 16u +
+                        __float_as_uint(th[2 * k + 1].x) * 256u + __float_as_uint(th[2 * k + 1].y) * 4096u;
+                const uint32_t odd = (hl[k] ^ (zb * 0x1111u)) & 0x1111u;
+                const uint32_t m = odd * 15u;
+                hl[k] = (hl[k] & ~m) | (hh[k] & m);
+            }
+            w[0] = __byte_perm(hl[0], hl[1], 0x5410);
+            w[1] = __byte_perm(hl[2], hl[3], 0x5410);
+            if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
+        } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                t[i] = make_float2(fminf(fmaxf(t[i].x, cmin), cmax), fminf(fmaxf(t[i].y, cmin), cmax));
-            if constexpr (NEED_E) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ee[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t bl = pack_bytes(__float_as_uint(tl[2 * k].x), __float_as_uint(tl[2 * k].y),
+                                               __float_as_uint(tl[2 * k + 1].x), __float_as_uint(tl[2 * k + 1].y));
+                const uint32_t bh = pack_bytes(__float_as_uint(th[2 * k].x), __float_as_uint(th[2 * k].y),
+                                               __float_as_uint(th[2 * k + 1].x), __float_as_uint(th[2 * k + 1].y));
+                const uint32_t odd = (bl ^ (zb * 0x01010101u)) & 0x01010101u;
+                const uint32_t m = odd * 255u;
+                w[k] = (bl & ~m) | (bh & m);
             }
         }
-    }
-    if constexpr (NEED_E) {
+        if constexpr (NEED_E) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) e[i] = ee[i];
-    }
-    if constexpr (F::four) {
-        uint32_t h[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t a = __float_as_uint(t[2 * k].x), b = __float_as_uint(t[2 * k].y);
-            const uint32_t c = __float_as_uint(t[2 * k + 1].x), d = __float_as_uint(t[2 * k + 1].y);
-            h[k] = a + b * 16u + c * 256u + d * 4096u;
+            for (int i = 0; i < 8; ++i) e[i] = fma2(fma2(tl[i], M1, MZ), S, y[i]);
         }
-        w[0] = __byte_perm(h[0], h[1], 0x5410);
-        w[1] = __byte_perm(h[2], h[3], 0x5410);
-        if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
     } else {
+        const float cmin = MAGIC + (float)qmin + bias, cmax = MAGIC + (float)qmax + bias;
+        float2 t[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
-                              __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
+        for (int i = 0; i < 8; ++i) {
+            const float a = ((__float_as_uint(tl[i].x) ^ zb) & 1u) ? th[i].x : tl[i].x;
+            const float b = ((__float_as_uint(tl[i].y) ^ zb) & 1u) ? th[i].y : tl[i].y;
+            t[i] = make_float2(fminf(fmaxf(a, cmin), cmax), fminf(fmaxf(b, cmin), cmax));
+            if constexpr (NEED_E) e[i] = fma2(fma2(t[i], M1, MZ), S, y[i]);
+        }
+        if constexpr (F::four) {
+            uint32_t h[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                h[k] = __float_as_uint(t[2 * k].x) + __float_as_uint(t[2 * k].y) * 16u +
+                       __float_as_uint(t[2 * k + 1].x) * 256u + __float_as_uint(t[2 * k + 1].y) * 4096u;
+            w[0] = __byte_perm(h[0], h[1], 0x5410);
+            w[1] = __byte_perm(h[2], h[3], 0x5410);
+            if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
+                                  __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
+        }
     }
 }
 
@@ -340,8 +380,10 @@ __device__ __forceinline__ void int_chunk_exact(const float2 (&y)[8], const IntQ
 struct FpQ {
     float s;        // the scale x is divided by
     float rlo, rhi; // reciprocal bracket
+    float rn;       // RN(1/s) (0 when s == 0)
     bool fast;
     bool zero;      // s == 0: every code is +0
+    bool mk;        // the exact reciprocal-correction quotient holds for every element
 };
 
 __device__ __forceinline__ FpQ fp_unit(float s, float amax)
@@ -353,6 +395,8 @@ __device__ __forceinline__ FpQ fp_unit(float s, float amax)
     u.rlo = u.zero ? 0.0f : R.rlo;
     u.rhi = u.zero ? 0.0f : R.rhi;
     u.fast = R.fast && !u.zero;
+    u.rn = u.zero ? 0.0f : __frcp_rn(s);
+    u.mk = u.zero || ((s >= 0x1p-60f) && (s <= 0x1p100f) && __fmul_rn(amax, u.rn) < 0x1p20f);
     return u;
 }
 
@@ -654,6 +698,145 @@ __device__ __forceinline__ void with_chunk_flags(bool exact, bool general, Fn&& 
         else { if (general) f(N{}, T{}); else f(N{}, N{}); }
     } else {
         if (general) f(N{}, T{}); else f(N{}, N{});
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fast chunk paths, for units that need neither clamping (beyond the asymmetric cap at
+// xc) nor scaled sums nor a divide. No branches, no votes, no calls: the hot loops stay
+// small. They decide every element of a unit whose flags admit them; ce2 / cx2 are the
+// chunk's plain sums. (The bool result, always false, is kept for the callers' shape.)
+// ---------------------------------------------------------------------------
+
+// Integer codes from the magic form t = MAGIC + zero point + bias + q.
+template <int FMT>
+__device__ __forceinline__ void pack_int(const float2 (&t)[8], uint32_t (&w)[CodeWords<FMT>::n])
+{
+    if constexpr (Fmt<FMT>::four) {
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            h[k] = __float_as_uint(t[2 * k].x) + __float_as_uint(t[2 * k].y) * 16u +
+                   __float_as_uint(t[2 * k + 1].x) * 256u + __float_as_uint(t[2 * k + 1].y) * 4096u;
+        w[0] = __byte_perm(h[0], h[1], 0x5410);
+        w[1] = __byte_perm(h[2], h[3], 0x5410);
+        if constexpr (CodeBias<FMT>::v == 8) { w[0] ^= 0x88888888u; w[1] ^= 0x88888888u; }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = pack_bytes(__float_as_uint(t[2 * k].x), __float_as_uint(t[2 * k].y),
+                              __float_as_uint(t[2 * k + 1].x), __float_as_uint(t[2 * k + 1].y));
+    }
+}
+
+// The fast paths take the correctly rounded quotient RN(x / s) without a divide: with
+// rn = RN(1/s), q0 = RN(x rn) is within an ulp of x / s, the remainder x - q0 s is
+// exact (one FMA), and RN(q0 + rem rn) = RN(x / s) (Markstein's theorem on division
+// with a correctly rounded reciprocal). It holds for every element a unit's mk flag
+// admits: s in [2^-60, 2^100] and |x / s| < 2^20; a quotient below 2^-40 (where the
+// remainder may underflow) can be off by a few of its ulps, but every format codes it
+// as zero. (Checked against IEEE division for every bf16 x and every scale
+// RN(amax / Q) of a bf16 amax, Q each format's Qmax, and on 10^9 random fp32 pairs.)
+
+// Integer codes, any scale (unit flags fast, mk and no clamp): t = RN(q + 2^23 1.5)
+// rounds the exact quotient half to even, then zero point and bias are added exactly.
+// Decides every element.
+template <int FMT, bool STATS>
+__device__ __forceinline__ bool int_chunk_fast(const float2 (&y)[8], const IntQ& u, uint32_t (&w)[CodeWords<FMT>::n],
+                                               float2& ce2, float2& cx2)
+{
+    using F = Fmt<FMT>;
+    float2 t[8], nq[8];
+    const float2 RN = splat(u.rn), S = splat(u.s), NS = splat(-u.s), M = splat(MAGIC), M1 = splat(-1.0f);
+    const float2 ZB = splat(__fsub_rn(u.mz, MAGIC));           // zero point + bias (exact)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 yq = F::asym ? make_float2(fminf(y[i].x, u.xc), fminf(y[i].y, u.xc)) : y[i];
+        const float2 q0 = mul2(yq, RN);
+        const float2 q1 = fma2(fma2(q0, NS, yq), RN, q0);       // RN(x / s)
+        const float2 t0 = add2(q1, M);                          // MAGIC + rne(q)
+        nq[i] = fma2(t0, M1, M);                                // -q, exact
+        t[i] = add2(t0, ZB);
+    }
+    pack_int<FMT>(t, w);
+    if constexpr (STATS) {
+        ce2 = cx2 = splat(0.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = fma2(nq[i], S, y[i]);
+            ce2 = fma2(d, d, ce2);
+            cx2 = fma2(y[i], y[i], cx2);
+        }
+    }
+    return false;
+}
+
+// Integer codes, fp16 scale, unrotated bf16 input: the bracket select of
+// int_chunk_exact (its unit must have br set). Decides every element.
+template <int FMT, bool STATS>
+__device__ __forceinline__ bool int_chunk_exact_fast(const float2 (&y)[8], const IntQ& u,
+                                                     uint32_t (&w)[CodeWords<FMT>::n], float2& ce2, float2& cx2)
+{
+    float2 e[8];
+    int_chunk_exact<FMT, STATS, false>(y, u, 0, 0, w, e);
+    if constexpr (STATS) {
+        ce2 = cx2 = splat(0.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            ce2 = fma2(e[i], e[i], ce2);
+            cx2 = fma2(y[i], y[i], cx2);
+        }
+    }
+    return false;
+}
+
+// FP codes (unit flag mk): cvt of the exact quotient. Decides every element.
+template <int FMT, bool STATS>
+__device__ __forceinline__ bool fp_chunk_fast(const float2 (&y)[8], const FpQ& u, uint32_t (&w)[CodeWords<FMT>::n],
+                                              float2& ce2, float2& cx2)
+{
+    uint32_t pr[8];
+    const float2 RN = splat(u.rn), NS = splat(-u.s);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const float2 q0 = mul2(y[p], RN);
+        const float2 q1 = fma2(fma2(q0, NS, y[p]), RN, q0);       // RN(x / s)
+        pr[p] = cvt_pair<FMT>(q1.y, q1.x);
+    }
+    pack_pairs<FMT>(pr, w);
+    if constexpr (STATS) {
+        float2 val[8];
+        decode_pairs<FMT>(pr, val);
+        ce2 = cx2 = splat(0.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = fma2(val[i], NS, y[i]);
+            ce2 = fma2(d, d, ce2);
+            cx2 = fma2(y[i], y[i], cx2);
+        }
+    }
+    return false;
+}
+
+template <int FMT, bool STATS, bool EXACT>
+__device__ __forceinline__ bool plain_chunk_fast(const float2 (&y)[8], const PlainUnit<FMT>& u,
+                                                 uint32_t (&w)[CodeWords<FMT>::n], float2& ce2, float2& cx2)
+{
+    if constexpr (!Fmt<FMT>::is_int) return fp_chunk_fast<FMT, STATS>(y, u.fq, w, ce2, cx2);
+    else if constexpr (EXACT) return int_chunk_exact_fast<FMT, STATS>(y, u.iq, w, ce2, cx2);
+    else return int_chunk_fast<FMT, STATS>(y, u.iq, w, ce2, cx2);
+}
+
+// Whether a plain unit must take the general path as a whole (warp-uniform): scaled
+// sums, clamping, or a scale outside the fast paths' range.
+template <int FMT, bool EXACT>
+__device__ __forceinline__ bool unit_general_fast(const PlainUnit<FMT>& u, bool scaled)
+{
+    if constexpr (Fmt<FMT>::is_int) {
+        const bool g = u.iq.clamp || !u.iq.fast || (EXACT ? !u.iq.br : !u.iq.mk);
+        return scaled || __any_sync(0xFFFFFFFFu, g);
+    } else {
+        return scaled || __any_sync(0xFFFFFFFFu, !u.fq.mk);
     }
 }
 
