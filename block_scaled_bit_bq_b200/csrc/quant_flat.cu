@@ -346,7 +346,7 @@ __device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const Fla
             const float d = __fmul_rn(sbv, tc.S);
             scodes |= sbc << (8 * k);
             if constexpr (F::is_int) {
-                const IntQ iq = int_unit<FMT>(d, 0.0f, -amax, amax, -7, 7);
+                const IntQ iq = int_unit<FMT>(d, rcp_approx(d), false, 0.0f, -amax, amax, -7, 7);
                 float2 nq[8];
                 int_chunk<FMT, STATS>(y, iq, -7, 7, q, nq);
                 if constexpr (STATS) {

@@ -128,10 +128,11 @@ struct IntQ {
     bool clamp;     // codes must be clamped (beyond what xc does)
 };
 
-// Unit from its stored scale s, zero point zpf and the extreme values lo <= 0 <= hi it
-// holds; qmin / qmax: the code range.
+// Unit from its stored scale s, a reciprocal r of it (exact: r = RN(1/s); else within
+// an ulp), its zero point zpf and the extreme values lo <= 0 <= hi it holds; qmin / qmax:
+// the code range.
 template <int FMT>
-__device__ __forceinline__ IntQ int_unit(float s, float zpf, float lo, float hi, int qmin, int qmax)
+__device__ __forceinline__ IntQ int_unit(float s, float r, bool r_exact, float zpf, float lo, float hi, int qmin, int qmax)
 {
     constexpr float bias = (float)CodeBias<FMT>::v;
     IntQ u;
@@ -145,14 +146,14 @@ __device__ __forceinline__ IntQ int_unit(float s, float zpf, float lo, float hi,
         u.clamp = false;
         return u;
     }
-    u.r = rcp_approx(s);
+    u.r = r;
+    u.rn = r;
     u.rlo = __fmul_rn(u.r, 0x1.fffff8p-1f);                        // 1 - 2^-22
     u.rhi = __fmul_rn(u.r, 0x1.000004p+0f);                        // 1 + 2^-22
     const float bound = __fmul_rn(fmaxf(-lo, hi), u.r);          // ~ max |x / s|
     u.fast = (s >= 0x1p-100f) && (s <= 1.0e37f) && (bound < 4.0e6f);
     u.br = u.fast && bound < 400.0f;
-    u.rn = __frcp_rn(s);
-    u.mk = (s >= 0x1p-60f) && (s <= 0x1p100f) && (bound < 0x1p20f);
+    u.mk = r_exact && (s >= 0x1p-60f) && (s <= 0x1p100f) && (bound < 0x1p20f);
     u.thr = __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f));
     if constexpr (Fmt<FMT>::asym) {
         // The code is monotone in x, so the extremes bound every code: rne(hi r_hi) + zp
@@ -386,7 +387,8 @@ struct FpQ {
     bool mk;        // the exact reciprocal-correction quotient holds for every element
 };
 
-__device__ __forceinline__ FpQ fp_unit(float s, float amax)
+// rn: RN(1/s) (exact), or 0 when the caller has none (then mk is false).
+__device__ __forceinline__ FpQ fp_unit(float s, float amax, float rn = 0.0f)
 {
     FpQ u;
     u.s = s;
@@ -395,8 +397,8 @@ __device__ __forceinline__ FpQ fp_unit(float s, float amax)
     u.rlo = u.zero ? 0.0f : R.rlo;
     u.rhi = u.zero ? 0.0f : R.rhi;
     u.fast = R.fast && !u.zero;
-    u.rn = u.zero ? 0.0f : __frcp_rn(s);
-    u.mk = u.zero || ((s >= 0x1p-60f) && (s <= 0x1p100f) && __fmul_rn(amax, u.rn) < 0x1p20f);
+    u.rn = u.zero ? 0.0f : rn;
+    u.mk = u.zero || (rn > 0.0f && (s >= 0x1p-60f) && (s <= 0x1p100f) && __fmul_rn(amax, rn) < 0x1p20f);
     return u;
 }
 
@@ -494,9 +496,25 @@ __device__ __forceinline__ void int8_chunk_pow2(const float2 (&y)[8], float p2, 
 
 struct PlainScale {
     float s;        // stored scale (fp16-rounded when the dtype is fp16)
+    float rn;       // RN(1/s) (0 when s == 0)
     float zpf;      // zero point as float (0 for symmetric)
     float lo, hi;   // extreme values the unit holds (-amax, amax for symmetric)
 };
+
+// RN(a / Qmax) for a >= 0: the reciprocal correction with the compile-time RN(1/Qmax)
+// where it is exact (quotients in [2^-40, 2^20]: checked for every fp32 a and every
+// Qmax), else a division.
+template <int FMT>
+__device__ __forceinline__ float div_by_qscale(float a)
+{
+    constexpr float Q = Fmt<FMT>::qscale;
+    constexpr float RQ = 1.0f / Q;
+    if (a >= 0x1p-40f * Q && a <= 0x1p20f * Q) {
+        const float q0 = __fmul_rn(a, RQ);
+        return __fmaf_rn(__fmaf_rn(-q0, Q, a), RQ, q0);
+    }
+    return a == 0.0f ? 0.0f : div_rn_call(a, Q);
+}
 
 template <int FMT>
 __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx, bool fp16)
@@ -505,20 +523,22 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
     PlainScale p;
     if constexpr (F::asym) {
         const float lo = fminf(mn, 0.0f), hi = fmaxf(mx, 0.0f);
-        float s32 = div_rn_call(__fsub_rn(hi, lo), F::qscale);
-        s32 = fminf(s32, FLT_MAX);                  // a range beyond fp32 saturates
+        const float range = __fsub_rn(hi, lo);
+        float s32 = range <= FLT_MAX ? div_by_qscale<FMT>(range) : FLT_MAX;   // a range beyond fp32 saturates
+        s32 = fminf(s32, FLT_MAX);
         p.s = fp16 ? round_scale_f16(s32) : s32;
+        p.rn = p.s > 0.0f ? __frcp_rn(p.s) : 0.0f;
         if (p.s > 0.0f) {
-            // zp = Qmin + rne(RN(-lo / s)), decided like a code: residual test, else exact
-            const float r = rcp_approx(p.s);
-            const float q = __fsub_rn(__fmaf_rn(-lo, r, MAGIC), MAGIC);
-            const float f = __fmaf_rn(-lo, r, -q);
-            const float bound = __fmul_rn(-lo, r);
+            // zp = Qmin + rne(RN(-lo / s)): the exact quotient by the reciprocal correction
+            // where it holds, else a division
             float z;
-            if (p.s >= 0x1p-100f && bound < 4.0e6f && fabsf(f) < __fsub_rn(0.5f, __fmul_rn(__fadd_rn(bound, 2.0f), 0x1p-21f)))
-                z = q;
-            else
+            if (p.s >= 0x1p-60f && p.s <= 0x1p100f && __fmul_rn(-lo, p.rn) < 0x1p20f) {
+                const float q0 = __fmul_rn(-lo, p.rn);
+                const float q1 = __fmaf_rn(__fmaf_rn(-q0, p.s, -lo), p.rn, q0);
+                z = __fsub_rn(__fadd_rn(q1, MAGIC), MAGIC);
+            } else {
                 z = div_rne_clamped(-lo, p.s);
+            }
             p.zpf = fminf(fmaxf(__fadd_rn((float)F::qmin, z), (float)F::qmin), (float)F::qmax);
         } else {
             p.zpf = (float)F::qmin;
@@ -526,8 +546,9 @@ __device__ __forceinline__ PlainScale plain_scale(float amax, float mn, float mx
         p.lo = lo;
         p.hi = hi;
     } else {
-        const float s32 = div_rn_call(amax, F::qscale);
+        const float s32 = div_by_qscale<FMT>(amax);
         p.s = fp16 ? round_scale_f16(s32) : s32;
+        p.rn = p.s > 0.0f ? __frcp_rn(p.s) : 0.0f;
         p.zpf = 0.0f;
         p.lo = -amax;
         p.hi = amax;
@@ -560,8 +581,8 @@ __device__ __forceinline__ PlainUnit<FMT> plain_unit(const PlainScale& ps)
 {
     PlainUnit<FMT> u;
     u.s = ps.s;
-    if constexpr (Fmt<FMT>::is_int) u.iq = int_unit<FMT>(ps.s, ps.zpf, ps.lo, ps.hi, Fmt<FMT>::qmin, Fmt<FMT>::qmax);
-    else u.fq = fp_unit(ps.s, fmaxf(-ps.lo, ps.hi));
+    if constexpr (Fmt<FMT>::is_int) u.iq = int_unit<FMT>(ps.s, ps.rn, true, ps.zpf, ps.lo, ps.hi, Fmt<FMT>::qmin, Fmt<FMT>::qmax);
+    else u.fq = fp_unit(ps.s, fmaxf(-ps.lo, ps.hi), ps.rn);
     return u;
 }
 

@@ -6,10 +6,12 @@
  * s in [2^-60, 2^100] and quotients |x / s| in [2^-40, 2^20] (smaller quotients code as
  * zero in every format). Built with hardware FMA and no contraction.
  *
- *   markstein_check A_STEP NRAND
+ *   markstein_check A_STEP NRAND Q_STEP
  *     - scales RN(amax / Q) for every A_STEP-th positive normal bf16 amax and each Q
  *       (the formats' Qmax and the NV products), against every bf16 x;
- *     - NRAND random fp32 scales against 256 random fp32 x each.
+ *     - NRAND random fp32 scales against 256 random fp32 x each;
+ *     - division by each Qmax itself (the scale computation): every Q_STEP-th fp32
+ *       dividend with quotient in [2^-40, 2^20], with the reciprocal RN(1/Qmax).
  * Prints the counts; exits 1 on any mismatch.
  */
 #include <math.h>
@@ -66,6 +68,19 @@ int main(int argc, char** argv)
             if (!(x > 0.0f) || isinf(x)) continue;
             ++n;
             if (!same(quot(x, s, rn), x / s)) ++bad;
+        }
+    }
+    const long qstep = argc > 3 ? atol(argv[3]) : 0;
+    for (int qi = 0; qstep > 0 && qi < 7; ++qi) {
+        const float q = Q[qi], rq = 1.0f / q, flo = 0x1p-40f * q, fhi = 0x1p20f * q;
+        uint32_t lo, hi;
+        memcpy(&lo, &flo, 4);
+        memcpy(&hi, &fhi, 4);
+        for (uint32_t u = lo; u <= hi; u += (uint32_t)qstep) {
+            float a;
+            memcpy(&a, &u, 4);
+            ++n;
+            if (!same(quot(a, q, rq), a / q)) ++bad;
         }
     }
     printf("checked %lld mismatches %lld\n", n, bad);

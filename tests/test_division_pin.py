@@ -3,7 +3,8 @@ use the reciprocal correction q0 = RN(x rn), rem = fma(-q0, s, x), RN(q0 + rem r
 rn = RN(1/s) (Markstein's theorem). This test checks that identity against IEEE
 division on the CPU, on the domain the kernels use it for: every bf16 x against
 scales RN(amax / Q) derived from bf16 amax values (a sample of them; the full sweep
-was run when the kernels were written), and random fp32 pairs.
+was run when the kernels were written), random fp32 pairs, and the scale computation
+itself (fp32 dividends over each format's Qmax, with the compile-time RN(1/Qmax)).
 """
 
 import os
@@ -31,6 +32,6 @@ def checker(tmp_path_factory):
 
 
 def test_reciprocal_correction_is_the_ieee_quotient(checker):
-    r = subprocess.run([checker, "3", "40000"], capture_output=True, text=True, timeout=600)
+    r = subprocess.run([checker, "3", "40000", "5"], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "mismatches 0" in r.stdout
