@@ -18,28 +18,37 @@
 
 namespace bq {
 
-template <int FMT>
+// Codes of a lane's span of CPL consecutive chunks (CPL = 2 or 4), as 32-bit words.
+template <int FMT, int CPL = 2>
 struct SpanCodes {
-    // 8-bit codes: 8 words (two chunks); 4-bit codes: 4 words
-    static constexpr int n = Fmt<FMT>::four ? 4 : 8;
+    static constexpr int n = (Fmt<FMT>::four ? 2 : 4) * CPL;
 };
 
-template <int FMT>
+template <int FMT, int CPL = 2>
 __device__ __forceinline__ void load_codes(const uint8_t* codes, uint32_t span, uint32_t n_chunks,
-                                           uint32_t (&w)[SpanCodes<FMT>::n])
+                                           uint32_t (&w)[SpanCodes<FMT, CPL>::n])
 {
-    constexpr int NB = Fmt<FMT>::four ? 16 : 32;   // bytes per span
-    const uint32_t c0 = 2 * span;
-    if (c0 + 1 < n_chunks) {
-        if constexpr (Fmt<FMT>::four) ld_nc_v4(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[4]>(&w));
-        else ld_nc_v8(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[8]>(&w));
+    constexpr int CB = Fmt<FMT>::four ? 8 : 16;     // code bytes per chunk
+    constexpr int NB = CB * CPL;                    // per span
+    const uint32_t c0 = CPL * span;
+    const uint8_t* p = codes + (size_t)span * NB;
+    if (c0 + CPL <= n_chunks) {
+        if constexpr (NB == 16) ld_nc_v4(p, *reinterpret_cast<uint32_t(*)[4]>(&w));
+        else if constexpr (NB == 32) ld_nc_v8(p, *reinterpret_cast<uint32_t(*)[8]>(&w));
+        else {
+            ld_nc_v8(p, *reinterpret_cast<uint32_t(*)[8]>(&w));
+            ld_nc_v8(p + 32, *reinterpret_cast<uint32_t(*)[8]>(&w[8]));
+        }
     } else {
 #pragma unroll
-        for (int i = 0; i < SpanCodes<FMT>::n; ++i) w[i] = 0u;
-        if (c0 < n_chunks) {
-            // half span: one chunk's codes
-            if constexpr (Fmt<FMT>::four) ld_nc_v2(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[2]>(&w));
-            else ld_nc_v4(codes + (size_t)span * NB, *reinterpret_cast<uint32_t(*)[4]>(&w));
+        for (int i = 0; i < SpanCodes<FMT, CPL>::n; ++i) w[i] = 0u;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            if (c0 + k < n_chunks) {
+                // one chunk's codes
+                if constexpr (CB == 8) ld_nc_v2(p + k * CB, *reinterpret_cast<uint32_t(*)[2]>(&w[2 * k]));
+                else ld_nc_v4(p + k * CB, *reinterpret_cast<uint32_t(*)[4]>(&w[4 * k]));
+            }
         }
     }
 }
@@ -50,8 +59,8 @@ __device__ __forceinline__ void load_codes(const uint8_t* codes, uint32_t span, 
 // the (biased, non-negative) code byte becomes the low byte of MAGIC's bit pattern.
 template <int FMT> struct DecodeBias { static constexpr int v = (FMT == BQ_INT8_SYM || FMT == BQ_INT8_ASYM) ? 128 : (FMT == BQ_INT4_SYM ? 8 : 0); };
 
-template <int FMT>
-__device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT>::n], int h, float2 (&val)[8])
+template <int FMT, int CPL = 2>
+__device__ __forceinline__ void chunk_values(const uint32_t (&w)[SpanCodes<FMT, CPL>::n], int h, float2 (&val)[8])
 {
     using F = Fmt<FMT>;
     if constexpr (F::four) {
@@ -158,39 +167,48 @@ __device__ __forceinline__ void dequant_chunk(const UnitScale& us, const float2 
     }
 }
 
+// Dequantize: lane l of a warp owns a span of DQ_CPL consecutive chunks of the warp's
+// tile; the next tile's codes and unit scales are loaded before the current tile is
+// decoded. (Two chunks per lane measured faster than four.)
+constexpr int DQ_CPL = 2;
+
 template <int FMT, int SK, bool HAD, int OUT>
 __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
 {
-    constexpr int NC = SpanCodes<FMT>::n;
+    constexpr int NC = SpanCodes<FMT, DQ_CPL>::n;
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    uint32_t t = warp;
-    uint32_t cur[NC];
-    UnitScale cs[2];
+    const uint32_t ntiles = (a.n_chunks + 32u * DQ_CPL - 1u) / (32u * DQ_CPL);
     // a chunk index past the end reads the last unit's scale (in bounds, unused)
     auto clampc = [&](uint32_t c) { return c < a.n_chunks ? c : a.n_chunks - 1; };
-    if (t < a.n_dtiles) {
-        load_codes<FMT>(a.codes, t * 32 + lane, a.n_chunks, cur);
-        cs[0] = load_unit_scale<FMT, SK>(a, clampc(2 * (t * 32 + lane)));
-        cs[1] = load_unit_scale<FMT, SK>(a, clampc(2 * (t * 32 + lane) + 1));
+    uint32_t t = warp;
+    uint32_t cur[NC];
+    UnitScale cs[DQ_CPL];
+    if (t < ntiles) {
+        load_codes<FMT, DQ_CPL>(a.codes, t * 32 + lane, a.n_chunks, cur);
+#pragma unroll
+        for (int h = 0; h < DQ_CPL; ++h) cs[h] = load_unit_scale<FMT, SK>(a, clampc(DQ_CPL * (t * 32 + lane) + h));
     }
-    while (t < a.n_dtiles) {
+    while (t < ntiles) {
         const uint32_t tn = t + nwarps;
         uint32_t nxt[NC];
-        UnitScale ns[2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
-        if (tn < a.n_dtiles) {
-            load_codes<FMT>(a.codes, tn * 32 + lane, a.n_chunks, nxt);
-            ns[0] = load_unit_scale<FMT, SK>(a, clampc(2 * (tn * 32 + lane)));
-            ns[1] = load_unit_scale<FMT, SK>(a, clampc(2 * (tn * 32 + lane) + 1));
+        UnitScale ns[DQ_CPL];
+        if (tn < ntiles) {
+            load_codes<FMT, DQ_CPL>(a.codes, tn * 32 + lane, a.n_chunks, nxt);
+#pragma unroll
+            for (int h = 0; h < DQ_CPL; ++h) ns[h] = load_unit_scale<FMT, SK>(a, clampc(DQ_CPL * (tn * 32 + lane) + h));
+        } else {
+#pragma unroll
+            for (int h = 0; h < DQ_CPL; ++h) ns[h] = UnitScale{0.0f, 0.0f};
         }
         const uint32_t span = t * 32 + lane;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t c = 2 * span + h;
+        for (int h = 0; h < DQ_CPL; ++h) {
+            const uint32_t c = DQ_CPL * span + h;
             if (c >= a.n_chunks) break;
             float2 val[8], xh[8];
-            chunk_values<FMT>(cur, h, val);
+            chunk_values<FMT, DQ_CPL>(cur, h, val);
             dequant_chunk<FMT, SK>(cs[h], val, xh);
             if constexpr (HAD) fwht16x2(xh);
             if constexpr (OUT == BQ_DT_BF16) {
@@ -215,8 +233,8 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
         }
 #pragma unroll
         for (int i = 0; i < NC; ++i) cur[i] = nxt[i];
-        cs[0] = ns[0];
-        cs[1] = ns[1];
+#pragma unroll
+        for (int h = 0; h < DQ_CPL; ++h) cs[h] = ns[h];
         t = tn;
     }
 }
@@ -291,8 +309,10 @@ cudaError_t launch_flat_kernel(const DequantArgs& a, cudaStream_t st)
 }
 
 template <int FMT, int SK>
-cudaError_t run_dq(bool had, int out, const DequantArgs& a, cudaStream_t st)
+cudaError_t run_dq(bool had, int out, const DequantArgs& a0, cudaStream_t st)
 {
+    DequantArgs a = a0;                 // the dequantize tile is 32 lanes x DQ_CPL chunks
+    a.n_dtiles = (a0.n_chunks + 32u * DQ_CPL - 1u) / (32u * DQ_CPL);
     if (had) {
         return out == BQ_DT_BF16 ? launch_flat_kernel<k_dequant<FMT, SK, true, BQ_DT_BF16>>(a, st)
                                  : launch_flat_kernel<k_dequant<FMT, SK, true, BQ_DT_FP32>>(a, st);
