@@ -390,6 +390,151 @@ __device__ __forceinline__ void span_n1(const Row& row, uint32_t span, const Fla
     }
 }
 
+// ---- NV block 16 ---------------------------------------------------------------
+
+// One NV block through the general path (scaled sums, or a block scale outside the fast
+// path's range): the residual-test integer codes with exact settling, or the bracketed
+// FP codes with exact division where the bracket is inconclusive. Out of line.
+struct NvOut {
+    uint32_t w[2];
+    float2 e2, x2;
+};
+
+template <int FMT, bool STATS>
+__device__ __noinline__ NvOut nv_general(float2 y0, float2 y1, float2 y2, float2 y3, float2 y4, float2 y5, float2 y6,
+                                         float2 y7, float amax, float sbv, float S, bool scaled, float p)
+{
+    using F = Fmt<FMT>;
+    const float2 y[8] = {y0, y1, y2, y3, y4, y5, y6, y7};
+    NvOut o;
+    o.e2 = o.x2 = splat(0.0f);
+    const float d = __fmul_rn(sbv, S);
+    float2 val[8];
+    if constexpr (F::is_int) {
+        const IntQ iq = int_unit<FMT>(d, rcp_approx(d), false, 0.0f, -amax, amax, -7, 7);
+        float2 nq[8];
+        int_chunk<FMT, STATS>(y, iq, -7, 7, o.w, nq);
+        // x-hat = (q s_b) S: the first product is exact
+#pragma unroll
+        for (int i = 0; i < 8; ++i) val[i] = mul2(nq[i], splat(-sbv));
+    } else {
+        const FpQ fq = fp_unit(d, amax);
+        fp_chunk<FMT, STATS>(y, fq, o.w, val);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) val[i] = mul2(val[i], splat(fq.zero ? 0.0f : sbv));
+    }
+    if constexpr (STATS) {
+        if (scaled) val_sums<true>(y, val, S, p, o.e2, o.x2);
+        else val_sums<false>(y, val, S, p, o.e2, o.x2);
+    }
+    return o;
+}
+
+// A lane's four NV blocks. Fast path per block: the exact quotient RN(x / d), d = s_b S,
+// by the reciprocal correction with rn = RN(1/d); FP codes by cvt, INT4 codes rounded
+// half to even and clamped to [-7, 7]. x-hat = (code value * s_b) * S (the first
+// product is exact). The span's plain sums and crest factors are gathered in fp32 and
+// folded into the lane's doubles once per span.
+template <int FMT, bool HAD, bool STATS>
+__device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const FlatArgs& a, const TensorCtx& tc,
+                                        Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
+{
+    using F = Fmt<FMT>;
+    float2 se2 = splat(0.0f), sx2 = splat(0.0f);
+    float ksum = 0.0f, kmax = 0.0f;
+    uint32_t kn = 0u;
+    const float S = tc.S;
+    const float2 SS = splat(S), M = splat(MAGIC), M1 = splat(-1.0f);
+#pragma unroll 1
+    for (int k = 0; k < SPAN; ++k) {
+        uint32_t w[8], q[2];
+        float2 y[8];
+        row_chunk(row, k, w);
+        chunk_in<HAD>(w, y);
+        const float amax = chunk_amax(y, 0.0f);
+        const uint32_t sbc = nv_scale_code<FMT>(amax, S, tc.cS);
+        const float sbv = e4m3_value(sbc);
+        const float d = __fmul_rn(sbv, S);
+        scodes |= sbc << (8 * k);
+        const float rn = d > 0.0f ? __frcp_rn(d) : 0.0f;
+        // d = 0 codes every element as +0: INT4 gets that from the fast path, FP (where -0
+        // would keep its sign) from the general path
+        const bool mk = (F::is_int && !(d > 0.0f)) || (d >= 0x1p-60f && d <= 0x1p100f && __fmul_rn(amax, rn) < 0x1p20f);
+        const bool scaled = STATS && !plain_sums_ok(amax);
+        if (!__any_sync(0xFFFFFFFFu, !mk || scaled)) {
+            const float2 RN = splat(rn), ND = splat(-d), NB = splat(-sbv);
+            float2 val[8];
+            if constexpr (F::is_int) {
+                float2 t[8];
+                const float cmin = MAGIC - 7.0f, cmax = MAGIC + 7.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 q0 = mul2(y[i], RN);
+                    const float2 q1 = fma2(fma2(q0, ND, y[i]), RN, q0);      // RN(x / d)
+                    float2 t0 = add2(q1, M);                                  // MAGIC + rne(q)
+                    t0 = make_float2(fminf(fmaxf(t0.x, cmin), cmax), fminf(fmaxf(t0.y, cmin), cmax));
+                    val[i] = mul2(fma2(t0, M1, M), NB);                       // q s_b, exact
+                    t[i] = add2(t0, splat(8.0f));                             // + bias
+                }
+                pack_int<FMT>(t, q);
+            } else {
+                uint32_t pr[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 q0 = mul2(y[i], RN);
+                    const float2 q1 = fma2(fma2(q0, ND, y[i]), RN, q0);      // RN(x / d)
+                    pr[i] = cvt_pair<FMT>(q1.y, q1.x);
+                }
+                pack_pairs<FMT>(pr, q);
+                if constexpr (STATS) {
+                    decode_pairs<FMT>(pr, val);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) val[i] = mul2(val[i], splat(sbv));
+                }
+            }
+            if constexpr (STATS) {
+                float2 ce2 = splat(0.0f), cx2 = splat(0.0f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 dd = fma2(val[i], splat(-S), y[i]);
+                    ce2 = fma2(dd, dd, ce2);
+                    cx2 = fma2(y[i], y[i], cx2);
+                }
+                se2 = add2(se2, ce2);
+                sx2 = add2(sx2, cx2);
+                const float ss = __fadd_rn(cx2.x, cx2.y);
+                if (ss > 0.0f) {
+                    const float kk = __fmul_rn(amax, rsqrtf(__fmul_rn(ss, a.inv_unit)));
+                    ksum = __fadd_rn(ksum, kk);
+                    kmax = fmaxf(kmax, kk);
+                    ++kn;
+                }
+            }
+        } else {
+            const Pow2 pw = pow2_for(amax);
+            const float p = scaled ? pw.p : 1.0f;
+            const NvOut o = nv_general<FMT, STATS>(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7], amax, sbv, S,
+                                                   scaled, p);
+            q[0] = o.w[0];
+            q[1] = o.w[1];
+            if constexpr (STATS) {
+                if (SPAN * span + k < a.n_chunks) {
+                    unit_done(acc, o.e2, o.x2, scaled, pw);
+                    kappa_add(acc, __fmul_rn(amax, p), __fadd_rn(o.x2.x, o.x2.y), a.inv_unit);
+                }
+            }
+        }
+        put_codes<FMT>(span4, a.codes, SPAN * span + k, true, k, q);
+    }
+    if constexpr (STATS) {
+        // chunks past the tensor's end are zeros: they add nothing
+        add_unit_sums(acc, se2, sx2, 1.0);
+        acc.ksum += (double)ksum;
+        acc.kmax = fmaxf(acc.kmax, kmax);
+        acc.nunits += kn;
+    }
+}
+
 // ---- two-chunk units: MX block 32, groups of 32 -------------------------------
 
 template <int FMT, int GK, bool STATS>
@@ -646,7 +791,7 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         if constexpr (GK == K_TENSOR) {
             span_tensor<FMT, HAD, STATS, EXACT>(row, span, a, tu, tp, tscaled, acc, span4);
         } else if constexpr (GK == K_NV) {
-            span_n1<FMT, GK, HAD, STATS, false>(row, span, a, tc, acc, span4, scodes);
+            span_nv<FMT, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
         } else if constexpr (GK == K_MX) {
             span_n2<FMT, GK, HAD, STATS, false>(row, span, a, acc, span4, scodes);
         } else {
