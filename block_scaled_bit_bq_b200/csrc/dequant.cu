@@ -33,7 +33,8 @@ __device__ __forceinline__ void load_codes(const uint8_t* codes, uint32_t span, 
     const uint32_t c0 = CPL * span;
     const uint8_t* p = codes + (size_t)span * NB;
     if (c0 + CPL <= n_chunks) {
-        if constexpr (NB == 16) ld_nc_v4(p, *reinterpret_cast<uint32_t(*)[4]>(&w));
+        if constexpr (NB == 8) ld_nc_v2(p, *reinterpret_cast<uint32_t(*)[2]>(&w));
+        else if constexpr (NB == 16) ld_nc_v4(p, *reinterpret_cast<uint32_t(*)[4]>(&w));
         else if constexpr (NB == 32) ld_nc_v8(p, *reinterpret_cast<uint32_t(*)[8]>(&w));
         else {
             ld_nc_v8(p, *reinterpret_cast<uint32_t(*)[8]>(&w));

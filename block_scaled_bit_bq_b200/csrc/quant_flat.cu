@@ -259,7 +259,7 @@ __device__ __forceinline__ uint32_t fast_chunks(const Row& row, const PlainUnit<
 {
     constexpr int NW = CodeWords<FMT>::n;
     if (general) return ((1u << n) - 1u) << k0;
-#pragma unroll 1
+#pragma unroll
     for (int k = k0; k < k0 + n; ++k) {
         uint32_t w[8], q[NW];
         float2 y[8], ce2, cx2;
@@ -431,13 +431,14 @@ __device__ __noinline__ NvOut nv_general(float2 y0, float2 y1, float2 y2, float2
 }
 
 // A lane's four NV blocks. Fast path per block: the exact quotient RN(x / d), d = s_b S,
-// by the reciprocal correction with rn = RN(1/d); FP codes by cvt, INT4 codes rounded
+// by the reciprocal correction with rn = RN(1/d) (s_b, d and rn from the CTA's table
+// over the 127 block-scale codes); FP codes by cvt, INT4 codes rounded
 // half to even and clamped to [-7, 7]. x-hat = (code value * s_b) * S (the first
 // product is exact). The span's plain sums and crest factors are gathered in fp32 and
 // folded into the lane's doubles once per span.
 template <int FMT, bool HAD, bool STATS>
 __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const FlatArgs& a, const TensorCtx& tc,
-                                        Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
+                                        const float4* nvtab, Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
 {
     using F = Fmt<FMT>;
     float2 se2 = splat(0.0f), sx2 = splat(0.0f);
@@ -453,10 +454,9 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
         chunk_in<HAD>(w, y);
         const float amax = chunk_amax(y, 0.0f);
         const uint32_t sbc = nv_scale_code<FMT>(amax, S, tc.cS);
-        const float sbv = e4m3_value(sbc);
-        const float d = __fmul_rn(sbv, S);
+        const float4 tb = nvtab[sbc];                  // s_b, d = s_b S, RN(1/d)
+        const float sbv = tb.x, d = tb.y, rn = tb.z;
         scodes |= sbc << (8 * k);
-        const float rn = d > 0.0f ? __frcp_rn(d) : 0.0f;
         // d = 0 codes every element as +0: INT4 gets that from the fast path, FP (where -0
         // would keep its sign) from the general path
         const bool mk = (F::is_int && !(d > 0.0f)) || (d >= 0x1p-60f && d <= 0x1p100f && __fmul_rn(amax, rn) < 0x1p20f);
@@ -493,13 +493,16 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
                 }
             }
             if constexpr (STATS) {
-                float2 ce2 = splat(0.0f), cx2 = splat(0.0f);
+                float2 ea = splat(0.0f), eb = splat(0.0f), xa = splat(0.0f), xb = splat(0.0f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float2 dd = fma2(val[i], splat(-S), y[i]);
-                    ce2 = fma2(dd, dd, ce2);
-                    cx2 = fma2(y[i], y[i], cx2);
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 d0 = fma2(val[i], splat(-S), y[i]), d1 = fma2(val[i + 1], splat(-S), y[i + 1]);
+                    ea = fma2(d0, d0, ea);
+                    eb = fma2(d1, d1, eb);
+                    xa = fma2(y[i], y[i], xa);
+                    xb = fma2(y[i + 1], y[i + 1], xb);
                 }
+                const float2 ce2 = add2(ea, eb), cx2 = add2(xa, xb);
                 se2 = add2(se2, ce2);
                 sx2 = add2(sx2, cx2);
                 const float ss = __fadd_rn(cx2.x, cx2.y);
@@ -664,8 +667,8 @@ __device__ __forceinline__ void span_n4(const Row& row, uint32_t span, const Fla
     if constexpr (F::asym) amax = fmaxf(-mn, mx);
 
     const bool scaled = STATS && __any_sync(0xFFFFFFFFu, !plain_sums_ok(amax));
-    const Pow2 pw = pow2_for(amax);
-    const float p = scaled ? pw.p : 1.0f;
+    const Pow2 pw = scaled ? pow2_for(amax) : Pow2{1.0f, 1.0};
+    const float p = pw.p;
     const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
     const PlainUnit<FMT> u = plain_unit<FMT>(ps);
     float2 e2 = splat(0.0f), x2 = splat(0.0f);
@@ -754,6 +757,17 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
             if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scale[0] = tc.S;
         }
     }
+    // NV: per block-scale code c (0..126; satfinite never gives the NaN code 127): s_b,
+    // d = s_b S and RN(1/d), computed once per CTA
+    __shared__ float4 nvtab[GK == K_NV ? 128 : 1];
+    if constexpr (GK == K_NV) {
+        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+            const float sb = e4m3_value((uint32_t)c);
+            const float d = __fmul_rn(sb, tc.S);
+            nvtab[c] = make_float4(sb, d, d > 0.0f ? __frcp_rn(d) : 0.0f, 0.0f);
+        }
+        __syncthreads();
+    }
     // per-group units: 16 elements (one chunk), 32 (two), 64 and up (the span, T lanes)
     const int T = (GK == K_GROUP && a.lanes_per_group > 0) ? a.lanes_per_group : 1;
 
@@ -791,7 +805,7 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         if constexpr (GK == K_TENSOR) {
             span_tensor<FMT, HAD, STATS, EXACT>(row, span, a, tu, tp, tscaled, acc, span4);
         } else if constexpr (GK == K_NV) {
-            span_nv<FMT, HAD, STATS>(row, span, a, tc, acc, span4, scodes);
+            span_nv<FMT, HAD, STATS>(row, span, a, tc, nvtab, acc, span4, scodes);
         } else if constexpr (GK == K_MX) {
             span_n2<FMT, GK, HAD, STATS, false>(row, span, a, acc, span4, scodes);
         } else {

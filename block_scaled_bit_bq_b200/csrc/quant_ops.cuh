@@ -781,13 +781,18 @@ __device__ __forceinline__ bool int_chunk_fast(const float2 (&y)[8], const IntQ&
     }
     pack_int<FMT>(t, w);
     if constexpr (STATS) {
-        ce2 = cx2 = splat(0.0f);
+        // two accumulators each: shorter dependency chains
+        float2 ea = splat(0.0f), eb = splat(0.0f), xa = splat(0.0f), xb = splat(0.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 d = fma2(nq[i], S, y[i]);
-            ce2 = fma2(d, d, ce2);
-            cx2 = fma2(y[i], y[i], cx2);
+        for (int i = 0; i < 8; i += 2) {
+            const float2 d0 = fma2(nq[i], S, y[i]), d1 = fma2(nq[i + 1], S, y[i + 1]);
+            ea = fma2(d0, d0, ea);
+            eb = fma2(d1, d1, eb);
+            xa = fma2(y[i], y[i], xa);
+            xb = fma2(y[i + 1], y[i + 1], xb);
         }
+        ce2 = add2(ea, eb);
+        cx2 = add2(xa, xb);
     }
     return false;
 }
@@ -801,12 +806,16 @@ __device__ __forceinline__ bool int_chunk_exact_fast(const float2 (&y)[8], const
     float2 e[8];
     int_chunk_exact<FMT, STATS, false>(y, u, 0, 0, w, e);
     if constexpr (STATS) {
-        ce2 = cx2 = splat(0.0f);
+        float2 ea = splat(0.0f), eb = splat(0.0f), xa = splat(0.0f), xb = splat(0.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            ce2 = fma2(e[i], e[i], ce2);
-            cx2 = fma2(y[i], y[i], cx2);
+        for (int i = 0; i < 8; i += 2) {
+            ea = fma2(e[i], e[i], ea);
+            eb = fma2(e[i + 1], e[i + 1], eb);
+            xa = fma2(y[i], y[i], xa);
+            xb = fma2(y[i + 1], y[i + 1], xb);
         }
+        ce2 = add2(ea, eb);
+        cx2 = add2(xa, xb);
     }
     return false;
 }
@@ -828,13 +837,17 @@ __device__ __forceinline__ bool fp_chunk_fast(const float2 (&y)[8], const FpQ& u
     if constexpr (STATS) {
         float2 val[8];
         decode_pairs<FMT>(pr, val);
-        ce2 = cx2 = splat(0.0f);
+        float2 ea = splat(0.0f), eb = splat(0.0f), xa = splat(0.0f), xb = splat(0.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 d = fma2(val[i], NS, y[i]);
-            ce2 = fma2(d, d, ce2);
-            cx2 = fma2(y[i], y[i], cx2);
+        for (int i = 0; i < 8; i += 2) {
+            const float2 d0 = fma2(val[i], NS, y[i]), d1 = fma2(val[i + 1], NS, y[i + 1]);
+            ea = fma2(d0, d0, ea);
+            eb = fma2(d1, d1, eb);
+            xa = fma2(y[i], y[i], xa);
+            xb = fma2(y[i + 1], y[i + 1], xb);
         }
+        ce2 = add2(ea, eb);
+        cx2 = add2(xa, xb);
     }
     return false;
 }
