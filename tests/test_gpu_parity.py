@@ -178,11 +178,12 @@ def test_parity_small(s, name, ws):
     check(x, s, ws, name)
 
 
-@pytest.mark.parametrize("cols", [16, 96, 640, 4096, 8192, 12288, 16384, 20480])
+@pytest.mark.parametrize("cols", [16, 96, 640, 2112, 3136, 4096, 8192, 12288, 16384, 20480])
 @pytest.mark.parametrize("s", [Scheme("int8_sym", "row"), Scheme("uint4_asym", "row", scale_dtype="fp16"),
                                Scheme("e5m2", "row", hadamard=True)], ids=str)
 def test_row_kernel_shapes(s, cols, ws):
-    # covers 1, 2 and 4 chunks per thread, blocks of 32..256 threads, and the two-pass path
+    # cols % 64 != 0 (16, 96): a CTA per row; other widths: a warp per row through the
+    # segment tensor map, with a partly filled last tile (640, 2112, 3136) or whole tiles
     x = synth.activations_t3(9, cols, seed=200 + cols, n_outlier_channels=1)
     check(x, s, ws, f"rows9x{cols}")
 
