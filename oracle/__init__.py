@@ -8,7 +8,8 @@ The arithmetic lives in ``bq_oracle.c`` (plain C loops, no SIMD, ``-ffp-contract
 no fast-math), which cites the pages each step follows. This module only builds the
 shared library, marshals numpy arrays, and names schemes by string:
 
-  fmt:         int8_sym | int8_asym | int4_sym | uint4_asym | e4m3 | e5m2 | e2m1
+  fmt:         int8_sym | int8_asym | int4_sym | uint4_asym | e4m3 | e5m2 | e2m1 | e2m3 | e3m2
+               (e2m3, e3m2: FP6, MX granularity only, one code per byte)
   gran:        tensor | row | group | mx | nv
   scale_dtype: fp32 | fp16 | ue8m0 | e4m3   (default: ue8m0 for mx, e4m3 for nv, else fp32)
 """
@@ -27,7 +28,7 @@ _SRC = os.path.join(_HERE, "bq_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 FMTS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3,
-        "e4m3": 4, "e5m2": 5, "e2m1": 6}
+        "e4m3": 4, "e5m2": 5, "e2m1": 6, "e2m3": 7, "e3m2": 8}
 GRANS = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4}
 SDTS = {"fp32": 0, "fp16": 1, "ue8m0": 2, "e4m3": 3}
 FOUR_BIT = {"int4_sym", "uint4_asym", "e2m1"}

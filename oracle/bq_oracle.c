@@ -62,7 +62,7 @@
 /* ------------------------------------------------------------------------- */
 
 enum { F_INT8_SYM = 0, F_INT8_ASYM = 1, F_INT4_SYM = 2, F_UINT4_ASYM = 3,
-       F_E4M3 = 4, F_E5M2 = 5, F_E2M1 = 6 };
+       F_E4M3 = 4, F_E5M2 = 5, F_E2M1 = 6, F_E2M3 = 7, F_E3M2 = 8 };
 enum { G_TENSOR = 0, G_ROW = 1, G_GROUP = 2, G_MX = 3, G_NV = 4 };
 enum { SD_FP32 = 0, SD_FP16 = 1, SD_UE8M0 = 2, SD_E4M3 = 3 };
 
@@ -71,9 +71,13 @@ enum { SD_FP32 = 0, SD_FP16 = 1, SD_UE8M0 = 2, SD_E4M3 = 3 };
 /* ------------------------------------------------------------------------- */
 
 /* E4M3 ("FN" variant: the top exponent holds normals, only S.1111.111 is NaN),
- * E5M2 (IEEE-like: the top exponent is inf/NaN), E2M1 (no specials).
+ * E5M2 (IEEE-like: the top exponent is inf/NaN), E2M1, E2M3, E3M2 (no specials).
  * The biases 7, 15, 1 are the ones that give the pages' smallest positive values
- * 2^-9 ~ 0.00195, 2^-16 ~ 1.5e-5 and 0.5. */
+ * 2^-9 ~ 0.00195, 2^-16 ~ 1.5e-5 and 0.5 ("Quantization survey" §4.1 table).
+ * FP6: that table gives E2M3 range +-7.5 and E3M2 range +-28, which fix the biases at
+ * 1 and 3; its smallest positive values (0.0625, ~0.0156) belong to other biases and
+ * contradict the ranges. The ranges are kept: the smallest positive values are then
+ * 0.125 (E2M3) and 0.0625 (E3M2). */
 typedef struct { int ebits, mbits, bias, kind; } fpspec;
 enum { KIND_FN = 0, KIND_IEEE = 1, KIND_PLAIN = 2 };
 
@@ -83,6 +87,8 @@ static int spec_of(int fp, fpspec* s)
     case F_E4M3: s->ebits = 4; s->mbits = 3; s->bias = 7;  s->kind = KIND_FN;    return 0;
     case F_E5M2: s->ebits = 5; s->mbits = 2; s->bias = 15; s->kind = KIND_IEEE;  return 0;
     case F_E2M1: s->ebits = 2; s->mbits = 1; s->bias = 1;  s->kind = KIND_PLAIN; return 0;
+    case F_E2M3: s->ebits = 2; s->mbits = 3; s->bias = 1;  s->kind = KIND_PLAIN; return 0;
+    case F_E3M2: s->ebits = 3; s->mbits = 2; s->bias = 3;  s->kind = KIND_PLAIN; return 0;
     default: return -1;
     }
 }
@@ -128,10 +134,14 @@ static void build_table(int fp, fptable* t)
 
 static const fptable* table_of(int fp)
 {
-    static fptable t4, t5, t2;
+    static fptable t4, t5, t2, t6a, t6b;
     static int ready = 0;
-    if (!ready) { build_table(F_E4M3, &t4); build_table(F_E5M2, &t5); build_table(F_E2M1, &t2); ready = 1; }
-    return fp == F_E4M3 ? &t4 : fp == F_E5M2 ? &t5 : &t2;
+    if (!ready) {
+        build_table(F_E4M3, &t4); build_table(F_E5M2, &t5); build_table(F_E2M1, &t2);
+        build_table(F_E2M3, &t6a); build_table(F_E3M2, &t6b);
+        ready = 1;
+    }
+    return fp == F_E4M3 ? &t4 : fp == F_E5M2 ? &t5 : fp == F_E2M1 ? &t2 : fp == F_E2M3 ? &t6a : &t6b;
 }
 
 /* Nearest table value to v; ties go to the code whose mantissa LSB is 0 (even);
@@ -250,6 +260,8 @@ static int make_scheme(int fmt, int gran, int block, int sdt, int had, int64_t c
     case F_E4M3: s->qscale = 448.0f; break;
     case F_E5M2: s->qscale = 57344.0f; break;
     case F_E2M1: s->bits4 = 1; s->qscale = 6.0f; break;
+    case F_E2M3: s->qscale = 7.5f; break;          /* FP6, one code per byte */
+    case F_E3M2: s->qscale = 28.0f; break;
     default: return -1;
     }
     if (cols <= 0 || cols % 16) return -2;
@@ -257,19 +269,20 @@ static int make_scheme(int fmt, int gran, int block, int sdt, int had, int64_t c
     switch (gran) {
     case G_TENSOR:
     case G_ROW:
-        if (fmt == F_E2M1) return -1;
+        if (fmt == F_E2M1 || fmt == F_E2M3 || fmt == F_E3M2) return -1;
         if (sdt != SD_FP32 && sdt != SD_FP16) return -1;
         s->unit = gran == G_ROW ? cols : 0;
         break;
     case G_GROUP:
-        if (fmt == F_E2M1) return -1;
+        if (fmt == F_E2M1 || fmt == F_E2M3 || fmt == F_E3M2) return -1;
         if (sdt != SD_FP32 && sdt != SD_FP16) return -1;
         if (block != 16 && block != 32 && block != 64 && block != 128 && block != 256 && block != 512) return -1;
         if (cols % block) return -2;
         s->unit = block;
         break;
     case G_MX:
-        if (!(fmt == F_INT8_SYM || fmt == F_E4M3 || fmt == F_E5M2 || fmt == F_E2M1)) return -1;
+        if (!(fmt == F_INT8_SYM || fmt == F_E4M3 || fmt == F_E5M2 || fmt == F_E2M1 ||
+              fmt == F_E2M3 || fmt == F_E3M2)) return -1;
         if (block != 32 || sdt != SD_UE8M0) return -1;
         if (cols % 32) return -2;
         s->unit = 32;

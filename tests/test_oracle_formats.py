@@ -183,3 +183,46 @@ def test_fwht16_matches_hadamard_matrix_and_is_an_involution():
     two = np.zeros(16, np.float32)
     two[:2] = 1.0
     assert np.array_equal(oracle.fwht16(two), np.tile(np.array([0.5, 0.0], np.float32), 8))
+
+
+# --- FP6 (MXFP6 element formats) -------------------------------------------------
+
+@pytest.mark.parametrize("fmt", ["e2m3", "e3m2"])
+def test_fp6_page_range_and_code_count(fmt):
+    g = _formats()[fmt]
+    vals = [oracle.fp_decode(fmt, c) for c in range(64)]
+    assert all(math.isfinite(v) for v in vals)          # no inf / NaN codes
+    assert max(vals) == g["max"] and min(vals) == -g["max"]
+    # the page's smallest positive value contradicts its range; the range's bias wins
+    assert min(v for v in vals if v > 0) == g["min_positive_of_the_range"]
+    assert min(v for v in vals if v > 0) != g["page_min_positive"]
+
+
+@pytest.mark.parametrize("fmt,mltype", [("e2m3", "float6_e2m3fn"), ("e3m2", "float6_e3m2fn")])
+def test_fp6_decode_and_encode_against_ml_dtypes(fmt, mltype):
+    ml = pytest.importorskip("ml_dtypes")
+    t = getattr(ml, mltype)
+    codes = np.arange(64, dtype=np.uint8)
+    lib_vals = codes.view(t).astype(np.float32)
+    assert [oracle.fp_decode(fmt, int(c)) for c in codes] == [float(v) for v in lib_vals]
+    # every midpoint between neighbours, its fp32 neighbours, values past the range, and
+    # random values: the library's round-to-nearest-even cast (saturating) must agree
+    pos = sorted(set(float(v) for v in lib_vals if v >= 0))
+    cand = []
+    for a, b in zip(pos[:-1], pos[1:]):
+        m = np.float32((a + b) / 2)
+        cand += [m, np.nextafter(m, np.float32(np.inf)), np.nextafter(m, np.float32(-np.inf))]
+    g = np.random.default_rng(11)
+    cand += list(g.uniform(-1.2 * pos[-1], 1.2 * pos[-1], 4000).astype(np.float32))
+    cand += [np.float32(pos[-1] * 4), np.float32(1e30), np.float32(-0.0)]
+    cand = np.array(cand, dtype=np.float32)
+    cand = np.concatenate([cand, -cand])
+    want = cand.astype(t).view(np.uint8)
+    got = np.array([oracle.fp_encode(fmt, float(v)) for v in cand], dtype=np.uint8)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("fmt", ["e2m3", "e3m2"])
+def test_fp6_exhaustive_round_trip(fmt):
+    for c in range(64):
+        assert oracle.fp_encode(fmt, oracle.fp_decode(fmt, c)) == c, (fmt, hex(c))

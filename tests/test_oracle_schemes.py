@@ -348,3 +348,52 @@ def test_asymmetric_range_beyond_fp32_saturates():
     zp = int(r["zps"][0])
     q = r["codes"].view(np.int8).reshape(-1).astype(int)
     assert -128 <= zp <= 127 and q.min() >= -128 and q.max() <= 127
+
+
+# --------------------------------------------------------------------------
+# MXFP6 (E2M3 / E3M2 elements, block 32, UE8M0 scale)
+# --------------------------------------------------------------------------
+
+def _ue8m0(amax, qmax):
+    """Smallest e with amax <= qmax 2^e, clamped to [-127, 127] (brute force)."""
+    if not amax > 0:
+        return -127
+    for e in range(-300, 300):
+        if float(amax) <= float(qmax) * math.ldexp(1.0, e):
+            return max(-127, min(127, e))
+    raise AssertionError
+
+
+@pytest.mark.parametrize("fmt,mltype,qmax", [("e2m3", "float6_e2m3fn", 7.5), ("e3m2", "float6_e3m2fn", 28.0)])
+def test_mxfp6_blocks_against_ml_dtypes(fmt, mltype, qmax):
+    # each block of 32: scale 2^e by the brute-force exponent rule, then the element codes
+    # are the library's saturating round-to-nearest-even cast of x / 2^e (an exact scaling)
+    ml = pytest.importorskip("ml_dtypes")
+    t = getattr(ml, mltype)
+    x = synth.bf16_bits(synth.ffn_lognormal(0, rows=16, cols=256))
+    vals = np.array([oracle.bf16_to_f32(int(b)) for b in x.reshape(-1)], dtype=np.float32).reshape(x.shape)
+    r = oracle.quantize(x, Scheme(fmt, "mx"))
+    codes = np.asarray(r["codes"]).reshape(16, 256)
+    scales = np.asarray(r["scales"]).reshape(16, 8)
+    for i in range(16):
+        for b in range(8):
+            blk = vals[i, 32 * b:32 * b + 32]
+            e = _ue8m0(np.abs(blk).max(), qmax)
+            assert int(scales[i, b]) == e + 127
+            want = (blk.astype(np.float64) * 2.0 ** (-e)).astype(np.float32).astype(t).view(np.uint8)
+            assert np.array_equal(codes[i, 32 * b:32 * b + 32], want), (i, b)
+
+
+def test_mxfp6_sits_between_mxfp4_and_mxfp8_on_gaussian_blocks():
+    # more element mantissa bits, less block error: E2M1 (1 bit) < E2M3 (3 bits) and
+    # E3M2 (2 bits) < E2M3; E4M3 (3 bits, wider range) >= E2M3
+    x = synth.bf16_bits(synth.ffn_lognormal(0, rows=128, cols=2048))
+    db = {f: oracle.qsnr_db(*oracle.quantize(x, Scheme(f, "mx"))["stats"][:2]) for f in ("e2m1", "e3m2", "e2m3", "e4m3")}
+    assert db["e2m1"] < db["e3m2"] < db["e2m3"] <= db["e4m3"] + 0.5
+
+
+def test_fp6_only_with_mx_blocks():
+    x = np.zeros((2, 32), np.uint16)
+    for s in [Scheme("e2m3", "row"), Scheme("e3m2", "tensor"), Scheme("e2m3", "group", 32), Scheme("e3m2", "nv")]:
+        with pytest.raises(ValueError):
+            oracle.quantize(x, s)
