@@ -1,7 +1,7 @@
 """Benchmark of the block-scaled quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|weight_x50]
+                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_x50]
 
 A step is one pass of the whole path over one synthetic tensor of the workload:
 quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
@@ -56,6 +56,10 @@ WORKLOADS = {
                        ("e5m2_token", ("e5m2", "row", 0, "fp32", False))],
     "ffn_lognormal": [("mxint8", ("int8_sym", "mx", 32, "ue8m0", False)),
                       ("mxfp8_e4m3", ("e4m3", "mx", 32, "ue8m0", False))],
+    # the rest of the MX family on the same FFN tensor (MXFP4 and MXFP6)
+    "ffn_mx_family": [("mxfp4", ("e2m1", "mx", 32, "ue8m0", False)),
+                      ("mxfp6_e2m3", ("e2m3", "mx", 32, "ue8m0", False)),
+                      ("mxfp6_e3m2", ("e3m2", "mx", 32, "ue8m0", False))],
     "weight_x50": [("nvfp4", ("e2m1", "nv", 16, "e4m3", False)),
                    ("nvint4", ("int4_sym", "nv", 16, "e4m3", False)),
                    ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
@@ -64,7 +68,7 @@ WORKLOADS = {
 
 def gen_input(workload: str, rank: int) -> torch.Tensor:
     """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
-    if workload == "ffn_lognormal":
+    if workload in ("ffn_lognormal", "ffn_mx_family"):
         return synth.ffn_lognormal(rank)
     gen, _, _ = synth.WORKLOADS[workload]
     base = {"tiny_weight": 0, "weight_outliers": 1, "activations_t3": 2, "weight_x50": 4}[workload]

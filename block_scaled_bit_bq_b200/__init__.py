@@ -23,7 +23,8 @@ LIB_PATH = os.path.join(_HERE, "libbq.so")
 
 # enums of include/bq.h
 DT = {"bf16": 0, "fp16": 1, "fp32": 2, "ue8m0": 3, "e4m3": 4}
-FORMATS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3, "e4m3": 4, "e5m2": 5, "e2m1": 6}
+FORMATS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3, "e4m3": 4, "e5m2": 5, "e2m1": 6,
+           "e2m3": 7, "e3m2": 8}
 GRANULARITIES = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4}
 FOUR_BIT = {"int4_sym", "uint4_asym", "e2m1"}
 ASYMMETRIC = {"int8_asym", "uint4_asym"}

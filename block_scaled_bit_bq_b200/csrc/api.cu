@@ -33,29 +33,30 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
 {
     if (!s) return BQ_ERR_INVALID_ARG;
     if (s->reserved != 0 || (s->hadamard != 0 && s->hadamard != 1)) return BQ_ERR_INVALID_ARG;
-    if (s->format < BQ_INT8_SYM || s->format > BQ_FP4_E2M1) return BQ_ERR_INVALID_ARG;
+    if (s->format < BQ_INT8_SYM || s->format > BQ_FP6_E3M2) return BQ_ERR_INVALID_ARG;
     if (s->granularity < BQ_PER_TENSOR || s->granularity > BQ_NV_BLOCK) return BQ_ERR_INVALID_ARG;
     if (s->scale_dtype < BQ_DT_BF16 || s->scale_dtype > BQ_DT_E4M3) return BQ_ERR_INVALID_ARG;
     std::memset(p, 0, sizeof *p);
     p->fmt = s->format; p->gran = s->granularity; p->sdt = s->scale_dtype; p->had = s->hadamard;
     p->four = fmt_four(p->fmt); p->asym = fmt_asym(p->fmt); p->is_int = fmt_is_int(p->fmt);
 
+    const bool fp6 = p->fmt == BQ_FP6_E2M3 || p->fmt == BQ_FP6_E3M2;
     switch (p->gran) {
     case BQ_PER_TENSOR:
     case BQ_PER_ROW:
-        if (p->fmt == BQ_FP4_E2M1) return BQ_ERR_UNSUPPORTED;
+        if (p->fmt == BQ_FP4_E2M1 || fp6) return BQ_ERR_UNSUPPORTED;
         if (p->sdt != BQ_DT_FP32 && p->sdt != BQ_DT_FP16) return BQ_ERR_UNSUPPORTED;
         p->block = 0;
         break;
     case BQ_PER_GROUP:
-        if (p->fmt == BQ_FP4_E2M1) return BQ_ERR_UNSUPPORTED;
+        if (p->fmt == BQ_FP4_E2M1 || fp6) return BQ_ERR_UNSUPPORTED;
         if (p->sdt != BQ_DT_FP32 && p->sdt != BQ_DT_FP16) return BQ_ERR_UNSUPPORTED;
         if (!(s->block == 16 || s->block == 32 || s->block == 64 || s->block == 128 ||
               s->block == 256 || s->block == 512)) return BQ_ERR_UNSUPPORTED;
         p->block = s->block;
         break;
     case BQ_MX_BLOCK:
-        if (!(p->fmt == BQ_INT8_SYM || p->fmt == BQ_FP8_E4M3 || p->fmt == BQ_FP8_E5M2 || p->fmt == BQ_FP4_E2M1))
+        if (!(p->fmt == BQ_INT8_SYM || p->fmt == BQ_FP8_E4M3 || p->fmt == BQ_FP8_E5M2 || p->fmt == BQ_FP4_E2M1 || fp6))
             return BQ_ERR_UNSUPPORTED;
         if (!(s->block == 32 || s->block == 0) || p->sdt != BQ_DT_UE8M0) return BQ_ERR_UNSUPPORTED;
         p->block = 32;

@@ -26,6 +26,9 @@ template <> struct Fmt<BQ_UINT4_ASYM> { static constexpr bool is_int = true,  as
 template <> struct Fmt<BQ_FP8_E4M3>   { static constexpr bool is_int = false, asym = false, four = false; static constexpr int qmin = 0,    qmax = 0;   static constexpr float qscale = 448.0f; };
 template <> struct Fmt<BQ_FP8_E5M2>   { static constexpr bool is_int = false, asym = false, four = false; static constexpr int qmin = 0,    qmax = 0;   static constexpr float qscale = 57344.0f; };
 template <> struct Fmt<BQ_FP4_E2M1>   { static constexpr bool is_int = false, asym = false, four = true;  static constexpr int qmin = 0,    qmax = 0;   static constexpr float qscale = 6.0f; };
+// FP6, one code per byte (the low six bits), as the cvt instructions leave them
+template <> struct Fmt<BQ_FP6_E2M3>   { static constexpr bool is_int = false, asym = false, four = false; static constexpr int qmin = 0,    qmax = 0;   static constexpr float qscale = 7.5f; };
+template <> struct Fmt<BQ_FP6_E3M2>   { static constexpr bool is_int = false, asym = false, four = false; static constexpr int qmin = 0,    qmax = 0;   static constexpr float qscale = 28.0f; };
 
 // Granularity kinds as the kernels see them.
 enum { K_TENSOR = 0, K_GROUP = 1, K_MX = 2, K_NV = 3 };
@@ -139,6 +142,14 @@ __device__ __forceinline__ uint32_t cvt_pair(float hi, float lo)
         uint16_t h;
         asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
         r = h;
+    } else if constexpr (FMT == BQ_FP6_E2M3) {
+        uint16_t h;
+        asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+        r = h;
+    } else if constexpr (FMT == BQ_FP6_E3M2) {
+        uint16_t h;
+        asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+        r = h;
     } else {
         asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
             : "=r"(r) : "f"(hi), "f"(lo));
@@ -147,7 +158,7 @@ __device__ __forceinline__ uint32_t cvt_pair(float hi, float lo)
 }
 
 // Decode a pair of FP codes (packed as cvt_pair produces them) to two fp32 values,
-// exactly (every E4M3 / E5M2 / E2M1 value is an fp16 value).
+// exactly (every E4M3 / E5M2 / E2M1 / E2M3 / E3M2 value is an fp16 value).
 template <int FMT>
 __device__ __forceinline__ float2 dec_pair(uint32_t pair)
 {
@@ -156,6 +167,10 @@ __device__ __forceinline__ float2 dec_pair(uint32_t pair)
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pair));
     } else if constexpr (FMT == BQ_FP8_E5M2) {
         asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pair));
+    } else if constexpr (FMT == BQ_FP6_E2M3) {
+        asm("cvt.rn.f16x2.e2m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pair));
+    } else if constexpr (FMT == BQ_FP6_E3M2) {
+        asm("cvt.rn.f16x2.e3m2x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pair));
     } else {
         asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h) : "r"(pair));
     }

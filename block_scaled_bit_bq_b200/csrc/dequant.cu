@@ -351,6 +351,8 @@ cudaError_t dispatch(int fmt, int sk, Fn&& fn)
         case BQ_FP8_E4M3: return fn.template operator()<BQ_FP8_E4M3, SK_UE8M0>();
         case BQ_FP8_E5M2: return fn.template operator()<BQ_FP8_E5M2, SK_UE8M0>();
         case BQ_FP4_E2M1: return fn.template operator()<BQ_FP4_E2M1, SK_UE8M0>();
+        case BQ_FP6_E2M3: return fn.template operator()<BQ_FP6_E2M3, SK_UE8M0>();
+        case BQ_FP6_E3M2: return fn.template operator()<BQ_FP6_E3M2, SK_UE8M0>();
         default: return cudaErrorInvalidValue;
         }
     }

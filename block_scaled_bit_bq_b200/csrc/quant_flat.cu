@@ -1188,6 +1188,8 @@ cudaError_t launch_quant_flat(int fmt, int kind, bool had, bool stats, const Fla
         case BQ_FP8_E4M3: return run_flat_hs<BQ_FP8_E4M3, K_MX>(had, stats, a, st);
         case BQ_FP8_E5M2: return run_flat_hs<BQ_FP8_E5M2, K_MX>(had, stats, a, st);
         case BQ_FP4_E2M1: return run_flat_hs<BQ_FP4_E2M1, K_MX>(had, stats, a, st);
+        case BQ_FP6_E2M3: return run_flat_hs<BQ_FP6_E2M3, K_MX>(had, stats, a, st);
+        case BQ_FP6_E3M2: return run_flat_hs<BQ_FP6_E3M2, K_MX>(had, stats, a, st);
         default: return cudaErrorInvalidValue;
         }
     case K_NV:

@@ -16,8 +16,10 @@
  *  - Affine INT: q = round(w/scale) + zero_point, w = scale * (q - zero_point):
  *    "INT4/INT8/FP8 quantization" §INT8; INT4 [-8, 7] groups, two codes per byte:
  *    same page §INT4; E4M3 +-448, E5M2 +-57344: same page §FP8.
- *  - FP element formats E2M1 / E4M3 / E5M2 and their bit layouts: "Quantization
- *    survey" §4.1; MX (block 32, power-of-two E8M0 scale) and NV (block 16, E4M3
+ *  - FP element formats E2M1 / E4M3 / E5M2 / FP6 E2M3 / FP6 E3M2 and their bit layouts:
+ *    "Quantization survey" §4.1 (FP6 biases 1 and 3 follow that table's ranges +-7.5
+ *    and +-28; its printed smallest values contradict them); the MX family, MXFP6
+ *    included: same page §4.3; MX (block 32, power-of-two E8M0 scale) and NV (block 16, E4M3
  *    block scale plus an FP32 tensor scale, x = x_q * s_block * S_tensor): same page
  *    §4.3.1 and §4.3.2.
  *  - Hadamard rotation before quantizing: "INT vs FP at fine granularity" §4.2 and
@@ -47,7 +49,8 @@
  *
  * Layouts (row-major, rows x cols input):
  *  - codes: 8-bit formats uint8 [rows, cols]; 4-bit formats uint8 [rows, cols/2], element
- *    2j in the low nibble of byte j; INT codes are two's complement (UINT4 unsigned);
+ *    2j in the low nibble of byte j; FP6 formats one code per byte [rows, cols] (the low
+ *    six bits, sign at bit 5); INT codes are two's complement (UINT4 unsigned);
  *  - scales: per tensor 1 value; per row [rows]; per group [rows, cols/block]; MX uint8
  *    [rows, cols/32] (UE8M0 codes); NV uint8 [rows, cols/16] (E4M3 codes);
  *    fp32 or fp16 as scheme.scale_dtype says for the first three;
@@ -90,7 +93,9 @@ enum {
     BQ_UINT4_ASYM = 3,   /* [0, 15] with zero point, 15 levels                 */
     BQ_FP8_E4M3 = 4,     /* +-448                                              */
     BQ_FP8_E5M2 = 5,     /* +-57344                                            */
-    BQ_FP4_E2M1 = 6      /* +-6 (MX or NV granularity only)                    */
+    BQ_FP4_E2M1 = 6,     /* +-6 (MX or NV granularity only)                    */
+    BQ_FP6_E2M3 = 7,     /* FP6 +-7.5, exponent bias 1 (MX granularity only)   */
+    BQ_FP6_E3M2 = 8      /* FP6 +-28, exponent bias 3 (MX granularity only)    */
 };
 
 /* scaling granularity */
@@ -98,7 +103,7 @@ enum {
     BQ_PER_TENSOR = 0,   /* one scale; per-tensor range pass first (needs a workspace) */
     BQ_PER_ROW = 1,      /* one scale per row (output channel of a weight, or token)   */
     BQ_PER_GROUP = 2,    /* block in {16, 32, 64, 128, 256, 512} contiguous along a row */
-    BQ_MX_BLOCK = 3,     /* block 32, UE8M0 scale: INT8_SYM, E4M3, E5M2, E2M1          */
+    BQ_MX_BLOCK = 3,     /* block 32, UE8M0 scale: INT8_SYM, E4M3, E5M2, E2M1, E2M3, E3M2 */
     BQ_NV_BLOCK = 4      /* block 16, E4M3 scale + fp32 tensor scale: E2M1, INT4_SYM    */
 };
 

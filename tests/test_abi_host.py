@@ -41,6 +41,7 @@ SCHEMES = [
     Scheme("int8_asym", "group", 128, "fp16"), Scheme("int4_sym", "group", 64),
     Scheme("uint4_asym", "group", 128, "fp16"), Scheme("e4m3", "tensor"), Scheme("e5m2", "row"),
     Scheme("int8_sym", "mx"), Scheme("e4m3", "mx"), Scheme("e5m2", "mx"), Scheme("e2m1", "mx"),
+    Scheme("e2m3", "mx"), Scheme("e3m2", "mx"),
     Scheme("e2m1", "nv"), Scheme("int4_sym", "nv"), Scheme("int4_sym", "nv", hadamard=True),
     Scheme("int8_sym", "group", 512), Scheme("e4m3", "group", 16, "fp16"),
 ]
@@ -73,6 +74,9 @@ def _status(fn, *args):
 @pytest.mark.parametrize("s,shape,want", [
     (Scheme("e2m1", "row"), (4, 64), 2),
     (Scheme("e2m1", "tensor"), (4, 64), 2),
+    (Scheme("e2m3", "row"), (4, 64), 2),
+    (Scheme("e3m2", "group", 32), (4, 64), 2),
+    (Scheme("e3m2", "nv"), (4, 64), 2),
     (Scheme("int8_asym", "mx"), (4, 64), 2),
     (Scheme("e4m3", "nv"), (4, 64), 2),
     (Scheme("int8_sym", "group", 48), (4, 96), 2),

@@ -39,6 +39,7 @@ ALL_SCHEMES = [
     Scheme("int4_sym", "nv", hadamard=True), Scheme("e2m1", "nv", hadamard=True),
     Scheme("int8_sym", "row", hadamard=True), Scheme("e4m3", "tensor", hadamard=True),
     Scheme("uint4_asym", "group", 128, "fp16", hadamard=True), Scheme("int8_sym", "mx", hadamard=True),
+    Scheme("e2m3", "mx"), Scheme("e3m2", "mx"), Scheme("e2m3", "mx", hadamard=True),
 ]
 
 
