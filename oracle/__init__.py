@@ -10,7 +10,7 @@ shared library, marshals numpy arrays, and names schemes by string:
 
   fmt:         int8_sym | int8_asym | int4_sym | uint4_asym | e4m3 | e5m2 | e2m1 | e2m3 | e3m2
                (e2m3, e3m2: FP6, MX granularity only, one code per byte)
-  gran:        tensor | row | group | mx | nv
+  gran:        tensor | row | group | mx | nv | tile2d (one scale per 128 x 128 tile)
   scale_dtype: fp32 | fp16 | ue8m0 | e4m3   (default: ue8m0 for mx, e4m3 for nv, else fp32)
 """
 
@@ -29,7 +29,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 FMTS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3,
         "e4m3": 4, "e5m2": 5, "e2m1": 6, "e2m3": 7, "e3m2": 8}
-GRANS = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4}
+GRANS = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4, "tile2d": 5}
 SDTS = {"fp32": 0, "fp16": 1, "ue8m0": 2, "e4m3": 3}
 FOUR_BIT = {"int4_sym", "uint4_asym", "e2m1"}
 ASYM = {"int8_asym", "uint4_asym"}
@@ -103,7 +103,7 @@ class Scheme:
             sd = {"mx": "ue8m0", "nv": "e4m3"}.get(self.gran, "fp32")
         blk = self.block
         if blk == 0:
-            blk = {"mx": 32, "nv": 16}.get(self.gran, 0)
+            blk = {"mx": 32, "nv": 16, "tile2d": 128}.get(self.gran, 0)
         return Scheme(self.fmt, self.gran, blk, sd, bool(self.hadamard))
 
     def args(self):

@@ -63,7 +63,12 @@
 
 enum { F_INT8_SYM = 0, F_INT8_ASYM = 1, F_INT4_SYM = 2, F_UINT4_ASYM = 3,
        F_E4M3 = 4, F_E5M2 = 5, F_E2M1 = 6, F_E2M3 = 7, F_E3M2 = 8 };
-enum { G_TENSOR = 0, G_ROW = 1, G_GROUP = 2, G_MX = 3, G_NV = 4 };
+enum { G_TENSOR = 0, G_ROW = 1, G_GROUP = 2, G_MX = 3, G_NV = 4, G_TILE2D = 5 };
+
+/* 2-D tiles: one scale per TILE_ROWS x block (= 128 x 128) tile, the weight scaling of
+ * DeepSeek-V3's FP8 training ("Quantization survey" (walkerchi) §4.4: 1x128 activation
+ * tiles, 128x128 weight tiles, E4M3 throughout). */
+#define TILE_ROWS 128
 enum { SD_FP32 = 0, SD_FP16 = 1, SD_UE8M0 = 2, SD_E4M3 = 3 };
 
 /* ------------------------------------------------------------------------- */
@@ -287,6 +292,13 @@ static int make_scheme(int fmt, int gran, int block, int sdt, int had, int64_t c
         if (cols % 32) return -2;
         s->unit = 32;
         break;
+    case G_TILE2D:
+        if (fmt == F_E2M1 || fmt == F_E2M3 || fmt == F_E3M2) return -1;
+        if (sdt != SD_FP32 && sdt != SD_FP16) return -1;
+        if (block != 128) return -1;
+        if (cols % 128) return -2;
+        s->unit = 128;
+        break;
     case G_NV:
         if (!(fmt == F_E2M1 || fmt == F_INT4_SYM)) return -1;
         if (block != 16 || sdt != SD_E4M3) return -1;
@@ -297,6 +309,14 @@ static int make_scheme(int fmt, int gran, int block, int sdt, int had, int64_t c
         return -1;
     }
     return 0;
+}
+
+/* Index of the scale of row r, unit u (u = column / unit). */
+static int64_t scale_index(int gran, int64_t r, int64_t u, int64_t upr)
+{
+    if (gran == G_TENSOR) return 0;
+    if (gran == G_TILE2D) return (r / TILE_ROWS) * upr + u;
+    return r * upr + u;
 }
 
 /* Round a computed fp32 scale to its storage dtype and back (fp16 saturates). */
@@ -509,13 +529,78 @@ static void kappa_add(double* st, float amax, const float* y, int64_t n)
     }
 }
 
+/* 2-D tiles: the range of each TILE_ROWS x 128 tile (rows of the last tile row may be
+ * fewer), then every element of the tile quantized with the tile's scale, exactly as a
+ * unit of the other granularities; kappa per tile over all its elements. */
+static int quantize_tile2d(const scheme* s, const uint16_t* x, int64_t rows, int64_t cols,
+                           uint8_t* codes, void* scales, void* zps, double* stats)
+{
+    const int64_t tpr = cols / 128;
+    float* y = (float*)malloc(sizeof(float) * (size_t)cols);
+    float* yh = (float*)malloc(sizeof(float) * (size_t)cols);
+    unsigned* cd = (unsigned*)malloc(sizeof(unsigned) * (size_t)cols);
+    unit_range* ur = (unit_range*)malloc(sizeof(unit_range) * (size_t)tpr);
+    double* ss = (double*)malloc(sizeof(double) * (size_t)tpr);
+    if (!y || !yh || !cd || !ur || !ss) { free(y); free(yh); free(cd); free(ur); free(ss); return -3; }
+    for (int64_t r0 = 0; r0 < rows; r0 += TILE_ROWS) {
+        const int64_t r1 = r0 + TILE_ROWS < rows ? r0 + TILE_ROWS : rows;
+        for (int64_t u = 0; u < tpr; u++) { ss[u] = 0.0; ur[u].S = 0.0f; }
+        for (int64_t r = r0; r < r1; r++) {
+            load_row(x, r, cols, s->had, y);
+            for (int64_t u = 0; u < tpr; u++) {
+                unit_range t;
+                range_of(y + u * 128, 128, &t);
+                if (r == r0) ur[u] = t;
+                else {
+                    if (t.amax > ur[u].amax) ur[u].amax = t.amax;
+                    if (t.mn < ur[u].mn) ur[u].mn = t.mn;
+                    if (t.mx > ur[u].mx) ur[u].mx = t.mx;
+                }
+                for (int64_t j = 0; j < 128; j++) ss[u] += (double)y[u * 128 + j] * (double)y[u * 128 + j];
+            }
+        }
+        for (int64_t r = r0; r < r1; r++) {
+            load_row(x, r, cols, s->had, y);
+            for (int64_t u = 0; u < tpr; u++) {
+                float sc = 0.0f, zp = 0.0f;
+                uint8_t scode = 0;
+                quant_unit(s, y + u * 128, 128, ur[u], cd + u * 128, &sc, &zp, &scode, yh + u * 128);
+                const int64_t si = (r0 / TILE_ROWS) * tpr + u;
+                write_scale(scales, si, sc, s->sdt);
+                if (s->is_asym && zps) write_scale(zps, si, zp, s->sdt);
+            }
+            for (int64_t j = 0; j < cols; j++) put_code(codes, r, cols, j, cd[j], s->bits4);
+            if (s->had)
+                for (int64_t j = 0; j < cols; j += 16) orc_fwht16(yh + j);
+            if (stats)
+                for (int64_t j = 0; j < cols; j++) {
+                    double xv = (double)orc_bf16_to_f32(x[r * cols + j]);
+                    double e = xv - (double)yh[j];
+                    stats[0] += e * e;
+                    stats[1] += xv * xv;
+                }
+        }
+        if (stats)
+            for (int64_t u = 0; u < tpr; u++)
+                if (ss[u] > 0.0) {
+                    double k = (double)ur[u].amax / sqrt(ss[u] / (double)((r1 - r0) * 128));
+                    stats[2] += k;
+                    if (k > stats[3]) stats[3] = k;
+                    stats[4] += 1.0;
+                }
+    }
+    free(y); free(yh); free(cd); free(ur); free(ss);
+    return 0;
+}
+
 /*
  * Quantize x [rows, cols] (bf16 bits, row-major).
  * tensor_range: NULL, or {amax, min, max} of the whole (rotated) tensor when the
  * given rows are only part of it (per-tensor and NV schemes need it).
  * Outputs follow the library's layout: 8-bit codes [rows, cols]; 4-bit codes
  * [rows, cols/2] with element 2j in the low nibble; scales and zero points
- * row-major [rows, cols/unit] (one value for per-tensor); tensor_scale[0] for NV.
+ * row-major [rows, cols/unit] (one value for per-tensor; [ceil(rows/128), cols/128] for
+ * 2-D tiles); tensor_scale[0] for NV.
  * Returns 0, or a negative value for an invalid scheme or shape.
  */
 int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols,
@@ -530,6 +615,7 @@ int orc_quantize(const uint16_t* x, int64_t rows, int64_t cols,
     if (rows < 0) return -2;
     if (stats) for (int i = 0; i < 5; i++) stats[i] = 0.0;
     if (rows == 0) return 0;
+    if (gran == G_TILE2D) return quantize_tile2d(&s, x, rows, cols, codes, scales, zps, stats);
 
     float* y = (float*)malloc(sizeof(float) * (size_t)cols);
     float* yh = (float*)malloc(sizeof(float) * (size_t)cols);
@@ -614,7 +700,7 @@ int orc_dequantize(const uint8_t* codes, const void* scales, const void* zps,
         float* o = out + r * cols;
         for (int64_t j = 0; j < cols; j++) {
             int64_t u = j / unit;
-            int64_t si = gran == G_TENSOR ? 0 : r * upr + u;
+            int64_t si = scale_index(gran, r, u, upr);
             unsigned c = get_code(codes, r, cols, j, s.bits4);
             float v;
             if (gran == G_MX) {
@@ -667,8 +753,11 @@ int orc_qsnr_sums(const uint16_t* x, const uint8_t* codes, const void* scales, c
     size_t sz = (gran == G_MX || gran == G_NV) ? 1 : (scale_dtype == SD_FP16 ? 2 : 4);
     for (int64_t r = 0; r < rows; r++) {
         const uint8_t* cr = codes + r * cb;
-        const char* sr = gran == G_TENSOR ? (const char*)scales : (const char*)scales + (size_t)(r * upr) * sz;
-        const char* zr = !zps ? NULL : gran == G_TENSOR ? (const char*)zps : (const char*)zps + (size_t)(r * upr) * sz;
+        /* the row's scales: dequantize sees a one-row tensor (a 2-D tile row's scales
+         * serve every row of that tile row) */
+        const int64_t off = gran == G_TENSOR ? 0 : gran == G_TILE2D ? (r / TILE_ROWS) * upr : r * upr;
+        const char* sr = (const char*)scales + (size_t)off * sz;
+        const char* zr = !zps ? NULL : (const char*)zps + (size_t)off * sz;
         rc = orc_dequantize(cr, sr, zr, tensor_scale, 1, cols, fmt, gran, block, scale_dtype, hadamard, o);
         if (rc) { free(o); return rc; }
         for (int64_t j = 0; j < cols; j++) {
@@ -696,7 +785,8 @@ int orc_buffer_sizes(int fmt, int gran, int block, int scale_dtype, int hadamard
     int rc = make_scheme(fmt, gran, block, scale_dtype, hadamard, cols, &s);
     if (rc) return rc;
     int64_t n = rows * cols;
-    int64_t nscale = gran == G_TENSOR ? 1 : rows * (cols / s.unit);
+    int64_t nscale = gran == G_TENSOR ? 1 : gran == G_TILE2D ? ((rows + TILE_ROWS - 1) / TILE_ROWS) * (cols / s.unit)
+                                                               : rows * (cols / s.unit);
     int64_t ssz = (gran == G_MX || gran == G_NV) ? 1 : (scale_dtype == SD_FP16 ? 2 : 4);
     out4[0] = s.bits4 ? n / 2 : n;
     out4[1] = nscale * ssz;

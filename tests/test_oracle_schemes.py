@@ -88,6 +88,7 @@ ALL_SCHEMES = [
     Scheme("int8_sym", "mx"), Scheme("e4m3", "mx"), Scheme("e5m2", "mx"), Scheme("e2m1", "mx"),
     Scheme("e2m1", "nv"), Scheme("int4_sym", "nv"), Scheme("int4_sym", "nv", hadamard=True),
     Scheme("e2m1", "nv", hadamard=True), Scheme("int8_sym", "row", hadamard=True),
+    Scheme("int8_sym", "tile2d"), Scheme("e4m3", "tile2d"), Scheme("uint4_asym", "tile2d", scale_dtype="fp16"),
 ]
 
 SYM = [s for s in ALL_SCHEMES if s.fmt not in oracle.ASYM]
@@ -397,3 +398,132 @@ def test_fp6_only_with_mx_blocks():
     for s in [Scheme("e2m3", "row"), Scheme("e3m2", "tensor"), Scheme("e2m3", "group", 32), Scheme("e3m2", "nv")]:
         with pytest.raises(ValueError):
             oracle.quantize(x, s)
+
+
+# --------------------------------------------------------------------------
+# 2-D tiles: one scale per 128 x 128 tile ("Quantization survey" §4.4, the DeepSeek-V3
+# weight tiles)
+# --------------------------------------------------------------------------
+
+TILE2D = [Scheme("int8_sym", "tile2d"), Scheme("e4m3", "tile2d"), Scheme("e5m2", "tile2d", scale_dtype="fp16"),
+          Scheme("int8_asym", "tile2d", scale_dtype="fp16"), Scheme("int4_sym", "tile2d"),
+          Scheme("uint4_asym", "tile2d", scale_dtype="fp16"), Scheme("e4m3", "tile2d", hadamard=True)]
+
+
+def _tile_codes(codes, s, r0, r1, c0):
+    """Codes of the tile rows r0:r1, columns c0:c0+128 (4-bit codes: 64 bytes)."""
+    if s.fmt in oracle.FOUR_BIT:
+        return codes[r0:r1, c0 // 2:c0 // 2 + 64]
+    return codes[r0:r1, c0:c0 + 128]
+
+
+@pytest.mark.parametrize("s", TILE2D, ids=str)
+def test_tile2d_is_per_tensor_on_each_tile(s):
+    # a tile's scale covers exactly its 128 x 128 elements (fewer rows in the last tile
+    # row): each tile quantizes as a per-tensor call on that tile alone, whose scheme the
+    # hand cases and invariants pin; kappa is the tile's own
+    rows, cols = 300, 384                          # tile rows of 128, 128, 44; 3 tile columns
+    x = synth.bf16_bits(synth.weight_outliers(rows, cols, seed=71))
+    r = oracle.quantize(x, s)
+    sdt = r["scales"].dtype
+    sc = r["scales"].reshape(3, 3)
+    zp = None if r["zps"] is None else r["zps"].reshape(3, 3)
+    kap = []
+    err2 = 0.0
+    for ti, (r0, r1) in enumerate([(0, 128), (128, 256), (256, 300)]):
+        for tj in range(3):
+            t = np.ascontiguousarray(x[r0:r1, 128 * tj:128 * tj + 128])
+            p = oracle.quantize(t, Scheme(s.fmt, "tensor", 0, s.scale_dtype, s.hadamard))
+            assert p["scales"].dtype == sdt
+            assert p["scales"][0] == sc[ti, tj], (ti, tj)
+            if zp is not None:
+                assert p["zps"][0] == zp[ti, tj]
+            assert np.array_equal(_tile_codes(r["codes"], s, r0, r1, 128 * tj), p["codes"]), (ti, tj)
+            kap.append(p["stats"][2])
+            err2 += p["stats"][0]
+    st = r["stats"]
+    assert st[4] == 9
+    assert st[3] == pytest.approx(max(kap), rel=1e-12)
+    assert st[2] == pytest.approx(sum(kap), rel=1e-12)
+    assert st[0] == pytest.approx(err2, rel=1e-9)
+
+
+def test_tile2d_int8_brute_force():
+    # scale = amax / 127 over the 128 x 128 tile in fp32; code = clip(RNE(x / s), +-127)
+    rows, cols = 200, 256
+    x = synth.bf16_bits(synth.activations_t3(rows, cols, seed=72, n_outlier_channels=3))
+    xv = np.array([oracle.bf16_to_f32(int(b)) for b in x.reshape(-1)], np.float32).reshape(rows, cols)
+    r = oracle.quantize(x, Scheme("int8_sym", "tile2d"))
+    sc = r["scales"].reshape(2, 2)
+    q = r["codes"].view(np.int8).reshape(rows, cols).astype(np.int64)
+    for ti in range(2):
+        for tj in range(2):
+            blk = xv[128 * ti:128 * ti + 128, 128 * tj:128 * tj + 128]
+            want_s = np.float32(np.abs(blk).max()) / np.float32(127.0)
+            assert sc[ti, tj] == want_s
+            want_q = np.clip(np.rint(blk / want_s), -127, 127).astype(np.int64)
+            assert np.array_equal(q[128 * ti:128 * ti + 128, 128 * tj:128 * tj + 128], want_q)
+
+
+def test_tile2d_e4m3_against_ml_dtypes():
+    # E4M3 elements: the fp32 quotient x / s, then the library's round-to-nearest-even cast
+    ml = pytest.importorskip("ml_dtypes")
+    rows, cols = 130, 128
+    x = synth.bf16_bits(synth.ffn_lognormal(0, rows=rows, cols=cols))
+    xv = np.array([oracle.bf16_to_f32(int(b)) for b in x.reshape(-1)], np.float32).reshape(rows, cols)
+    r = oracle.quantize(x, Scheme("e4m3", "tile2d"))
+    assert r["scales"].shape == (2,)
+    for ti, (r0, r1) in enumerate([(0, 128), (128, 130)]):
+        blk = xv[r0:r1]
+        s = np.float32(np.abs(blk).max()) / np.float32(448.0)
+        assert r["scales"][ti] == s
+        want = (blk / s).astype(ml.float8_e4m3fn).view(np.uint8)
+        assert np.array_equal(r["codes"][r0:r1], want)
+
+
+def test_tile2d_scale_follows_its_own_tile():
+    # multiplying one tile by 2 (exact) doubles its scale and leaves every code and the
+    # other tiles' scales unchanged
+    rows, cols = 256, 256
+    x = synth.bf16_bits(synth.normal(rows, cols, seed=73, sigma=0.5))
+    s = Scheme("int8_sym", "tile2d")
+    a = oracle.quantize(x, s)
+    xv = (x.astype(np.uint32) << 16).view(np.float32)          # bf16 bits to fp32, exact
+    xv[128:, :128] *= 2.0                                        # still exact in bf16
+    y = (xv.view(np.uint32) >> 16).astype(np.uint16)
+    b = oracle.quantize(y, s)
+    assert np.array_equal(a["codes"], b["codes"])
+    want = a["scales"].copy()
+    want[2] *= 2
+    assert np.array_equal(b["scales"], want)
+
+
+def test_tile2d_buffer_sizes_and_dequantize_index():
+    s = Scheme("uint4_asym", "tile2d", scale_dtype="fp16")
+    c, sb, zb, tb = oracle.buffer_sizes(s, 257, 512)
+    assert (c, sb, zb, tb) == (257 * 256, 3 * 4 * 2, 3 * 4 * 2, 0)
+    # dequantize: element (r, j) takes the scale and zero point of tile (r // 128, j // 128)
+    x = synth.bf16_bits(synth.weight_outliers(257, 512, seed=74))
+    r = oracle.quantize(x, s)
+    xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], None, 257, 512, s)
+    q = np.empty((257, 512), np.int64)
+    q[:, 0::2] = r["codes"] & 0xF
+    q[:, 1::2] = r["codes"] >> 4
+    sc = np.array([oracle.f16_to_f32(int(v)) for v in r["scales"]], np.float32).reshape(3, 4)
+    zp = np.array([oracle.f16_to_f32(int(v)) for v in r["zps"]], np.float32).reshape(3, 4)
+    ti = np.arange(257)[:, None] // 128
+    tj = np.arange(512)[None, :] // 128
+    want = sc[ti, tj] * (q - zp[ti, tj]).astype(np.float32)
+    assert np.array_equal(want.astype(np.float32), xh)
+    st = oracle.qsnr_sums(x, r["codes"], r["scales"], r["zps"], None, s)
+    assert st[0] == r["stats"][0] and st[1] == r["stats"][1]
+
+
+def test_tile2d_rejects_other_shapes():
+    x = np.zeros((2, 256), np.uint16)
+    for s in [Scheme("e2m1", "tile2d"), Scheme("e2m3", "tile2d"), Scheme("int8_sym", "tile2d", 64),
+              Scheme("int8_sym", "tile2d", scale_dtype="ue8m0")]:
+        with pytest.raises(ValueError):
+            oracle.quantize(x, s)
+    with pytest.raises(ValueError):
+        oracle.quantize(np.zeros((2, 192), np.uint16), Scheme("int8_sym", "tile2d"))
