@@ -1,7 +1,7 @@
 """Benchmark of the block-scaled quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_x50]
+                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_tiles_fp8|weight_x50]
 
 A step is one pass of the whole path over one synthetic tensor of the workload:
 quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
@@ -60,6 +60,10 @@ WORKLOADS = {
     "ffn_mx_family": [("mxfp4", ("e2m1", "mx", 32, "ue8m0", False)),
                       ("mxfp6_e2m3", ("e2m3", "mx", 32, "ue8m0", False)),
                       ("mxfp6_e3m2", ("e3m2", "mx", 32, "ue8m0", False))],
+    # the DeepSeek-V3 FP8 recipe on the 4096 x 4096 outlier weight: E4M3 with one fp32
+    # scale per 128 x 128 tile (weights), and per 1 x 128 tile (the activation tiling)
+    "weight_tiles_fp8": [("e4m3_tile128x128", ("e4m3", "tile2d", 128, "fp32", False)),
+                         ("e4m3_tile1x128", ("e4m3", "group", 128, "fp32", False))],
     "weight_x50": [("nvfp4", ("e2m1", "nv", 16, "e4m3", False)),
                    ("nvint4", ("int4_sym", "nv", 16, "e4m3", False)),
                    ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
@@ -70,6 +74,8 @@ def gen_input(workload: str, rank: int) -> torch.Tensor:
     """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
     if workload in ("ffn_lognormal", "ffn_mx_family"):
         return synth.ffn_lognormal(rank)
+    if workload == "weight_tiles_fp8":
+        return synth.weight_outliers(seed=1 + 1000 * rank)
     gen, _, _ = synth.WORKLOADS[workload]
     base = {"tiny_weight": 0, "weight_outliers": 1, "activations_t3": 2, "weight_x50": 4}[workload]
     return gen(seed=base + 1000 * rank)

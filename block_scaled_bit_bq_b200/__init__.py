@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libbq.so")
 DT = {"bf16": 0, "fp16": 1, "fp32": 2, "ue8m0": 3, "e4m3": 4}
 FORMATS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3, "e4m3": 4, "e5m2": 5, "e2m1": 6,
            "e2m3": 7, "e3m2": 8}
-GRANULARITIES = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4}
+GRANULARITIES = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4, "tile2d": 5}
 FOUR_BIT = {"int4_sym", "uint4_asym", "e2m1"}
 ASYMMETRIC = {"int8_asym", "uint4_asym"}
 
@@ -94,7 +94,8 @@ def lib() -> ctypes.CDLL:
 class Scheme:
     """A quantization scheme: element format, scaling granularity, group size, scale
     dtype and the Hadamard flag. block / scale_dtype default to the granularity's own
-    (32 / ue8m0 for mx, 16 / e4m3 for nv, fp32 otherwise)."""
+    (32 / ue8m0 for mx, 16 / e4m3 for nv, 128 / fp32 for tile2d (128 x 128 tiles),
+    fp32 otherwise)."""
     fmt: str
     gran: str
     block: int = 0
@@ -103,7 +104,7 @@ class Scheme:
 
     def resolved(self) -> "Scheme":
         sd = self.scale_dtype or {"mx": "ue8m0", "nv": "e4m3"}.get(self.gran, "fp32")
-        blk = self.block or {"mx": 32, "nv": 16}.get(self.gran, 0)
+        blk = self.block or {"mx": 32, "nv": 16, "tile2d": 128}.get(self.gran, 0)
         return Scheme(self.fmt, self.gran, blk, sd, bool(self.hadamard))
 
     def c(self) -> BqScheme:

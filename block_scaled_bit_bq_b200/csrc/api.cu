@@ -34,7 +34,7 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
     if (!s) return BQ_ERR_INVALID_ARG;
     if (s->reserved != 0 || (s->hadamard != 0 && s->hadamard != 1)) return BQ_ERR_INVALID_ARG;
     if (s->format < BQ_INT8_SYM || s->format > BQ_FP6_E3M2) return BQ_ERR_INVALID_ARG;
-    if (s->granularity < BQ_PER_TENSOR || s->granularity > BQ_NV_BLOCK) return BQ_ERR_INVALID_ARG;
+    if (s->granularity < BQ_PER_TENSOR || s->granularity > BQ_TILE_2D) return BQ_ERR_INVALID_ARG;
     if (s->scale_dtype < BQ_DT_BF16 || s->scale_dtype > BQ_DT_E4M3) return BQ_ERR_INVALID_ARG;
     std::memset(p, 0, sizeof *p);
     p->fmt = s->format; p->gran = s->granularity; p->sdt = s->scale_dtype; p->had = s->hadamard;
@@ -66,6 +66,12 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
         if (!(s->block == 16 || s->block == 0) || p->sdt != BQ_DT_E4M3) return BQ_ERR_UNSUPPORTED;
         p->block = 16;
         break;
+    case BQ_TILE_2D:
+        if (p->fmt == BQ_FP4_E2M1 || fp6) return BQ_ERR_UNSUPPORTED;
+        if (p->sdt != BQ_DT_FP32 && p->sdt != BQ_DT_FP16) return BQ_ERR_UNSUPPORTED;
+        if (!(s->block == 128 || s->block == 0)) return BQ_ERR_UNSUPPORTED;
+        p->block = TILE;
+        break;
     }
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return BQ_ERR_SHAPE;
     if (p->block && cols % p->block != 0) return BQ_ERR_SHAPE;
@@ -77,6 +83,7 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
     switch (p->gran) {
     case BQ_PER_TENSOR: p->n_scales = 1; break;
     case BQ_PER_ROW: p->n_scales = (uint64_t)rows; break;
+    case BQ_TILE_2D: p->n_scales = (((uint64_t)rows + TILE - 1) / TILE) * ((uint64_t)cols / TILE); break;
     default: p->n_scales = p->n / (uint64_t)p->block; break;
     }
     const size_t se = (p->sdt == BQ_DT_FP32) ? 4 : (p->sdt == BQ_DT_FP16) ? 2 : 1;
@@ -120,6 +127,7 @@ DequantArgs dequant_args(const Plan& p, int64_t cols)
     switch (p.gran) {
     case BQ_PER_TENSOR: cpu = 0; break;
     case BQ_PER_ROW: cpu = (uint32_t)(cols / 16); break;
+    case BQ_TILE_2D: cpu = (uint32_t)(cols / 16); break;     // divides a chunk index into its row
     default: cpu = (uint32_t)(p.block / 16); break;
     }
     a.chunks_per_unit = cpu;
@@ -128,6 +136,7 @@ DequantArgs dequant_args(const Plan& p, int64_t cols)
         a.fd_m = f.m;
         a.fd_s = f.s;
     }
+    a.tile_cols = p.gran == BQ_TILE_2D ? (uint32_t)(cols / TILE) : 0u;
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     return a;
 }
@@ -224,6 +233,17 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     if (p.needs_range) {
         const cudaError_t e = launch_range(xw, p.n_chunks, p.had != 0, p.gran == BQ_PER_TENSOR && p.asym, ws, s);
         if (e != cudaSuccess) return BQ_ERR_CUDA;
+    }
+    if (p.gran == BQ_TILE_2D) {
+        Tile2dArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols;
+        a.tpr = (uint32_t)(cols / TILE);
+        a.ntiles = (uint32_t)p.n_scales;
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        return cuda_status(launch_quant_tile2d(p.fmt, p.had != 0, want_stats, a, s));
     }
     const bool pow2_segments = cols % 64 == 0 && ((cols / 64) & (cols / 64 - 1)) == 0;
     if (p.gran == BQ_PER_ROW && pow2_segments && cols <= 2048) {

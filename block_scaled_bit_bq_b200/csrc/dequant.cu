@@ -108,7 +108,14 @@ struct UnitScale {
 template <int FMT, int SK>
 __device__ __forceinline__ UnitScale load_unit_scale(const DequantArgs& d, uint32_t c)
 {
-    const uint32_t u = d.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, d.fd_m) + c) >> d.fd_s);
+    uint32_t u = d.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, d.fd_m) + c) >> d.fd_s);
+    if constexpr (SK == SK_F32 || SK == SK_F16) {
+        if (d.tile_cols) {
+            // u is the chunk's row: tile (row / 128, column / 128), 8 chunks per tile column
+            const uint32_t cc = c - u * d.chunks_per_unit;
+            u = (u / TILE) * d.tile_cols + cc / (TILE / 16);
+        }
+    }
     UnitScale r{0.0f, 0.0f};
     if constexpr (SK == SK_UE8M0) {
         r.a = exp2i((int)__ldg(reinterpret_cast<const uint8_t*>(d.scales) + u) - 127);
@@ -170,7 +177,8 @@ __device__ __forceinline__ void dequant_chunk(const UnitScale& us, const float2 
 
 // Dequantize: lane l of a warp owns a span of DQ_CPL consecutive chunks of the warp's
 // tile; the next tile's codes and unit scales are loaded before the current tile is
-// decoded. (Two chunks per lane measured faster than four.)
+// decoded. (Two chunks per lane measured faster than four.) A 2-D tile's scale is found
+// from the chunk's row and column.
 constexpr int DQ_CPL = 2;
 
 template <int FMT, int SK, bool HAD, int OUT>

@@ -59,6 +59,23 @@ struct RowsArgs {
     float inv_cols;
 };
 
+// 2-D tiles: one scale per TILE x TILE tile, a CTA per tile at a time.
+constexpr uint32_t TILE = 128;
+
+struct Tile2dArgs {
+    const uint32_t* x;
+    uint8_t* codes;
+    void* scales;
+    void* zps;
+    bq_stats* stats;
+    uint8_t* ws;
+    uint32_t rows;
+    uint32_t cols;
+    uint32_t tpr;               // tiles per tile row = cols / TILE
+    uint32_t ntiles;            // ceil(rows / TILE) * tpr
+    int32_t scale_fp16;
+};
+
 struct DequantArgs {
     const uint8_t* codes;
     const void* scales;
@@ -70,8 +87,10 @@ struct DequantArgs {
     uint8_t* ws;                // QSNR only
     uint32_t n_chunks;
     uint32_t n_dtiles;
-    uint32_t chunks_per_unit;   // chunks sharing one scale (0: one scale for the tensor)
+    uint32_t chunks_per_unit;   // chunks sharing one scale (0: one scale for the tensor);
+                                // 2-D tiles: chunks per row
     uint32_t fd_m, fd_s;        // fast division by chunks_per_unit
+    uint32_t tile_cols;         // 2-D tiles: tiles per tile row (cols / TILE); else 0
     int32_t scale_fp16;
 };
 
@@ -87,6 +106,7 @@ cudaError_t launch_quant_flat(int fmt, int kind, bool hadamard, bool stats, cons
                               cudaStream_t st);
 cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& a, cudaStream_t st);
 cudaError_t launch_quant_rows(int fmt, bool hadamard, bool stats, const RowsArgs& a, cudaStream_t st);
+cudaError_t launch_quant_tile2d(int fmt, bool hadamard, bool stats, const Tile2dArgs& a, cudaStream_t st);
 cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
                            cudaStream_t st);
 cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);

@@ -987,6 +987,174 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_rows(co
 }
 
 // ---------------------------------------------------------------------------
+// 2-D tiles: one scale per 128 x 128 tile (the DeepSeek-V3 weight tiles, "Quantization
+// survey" §4.4).
+//
+// A CTA of 8 warps owns a tile at a time (grid-stride over the tiles in row-major
+// order). The tile reaches shared memory as two boxes of a 2-D tensor map over x (128
+// rows x 64 columns each, 128-byte swizzle, zero past the last row), TILE_NST tiles
+// ahead, completed on one mbarrier per stage. Thread t takes row t & 127 of box t >> 7
+// (warps 0-3 the left half, 4-7 the right), a 64-element span as in the flat kernel.
+// The warps' partial ranges meet in shared memory at one barrier per tile; passing it
+// also means every thread is done with the previous tile, so its stage is refilled
+// right there, and that tile's kappa is formed from the warps' sums of squares.
+// ---------------------------------------------------------------------------
+
+constexpr int TILE_NST = 3;                                 // tile buffers per CTA
+constexpr uint32_t TBOX_BYTES = TILE * ROW_BYTES;           // 128 rows x 64 bf16 = 16 KiB
+constexpr uint32_t TSTAGE_BYTES = 2 * TBOX_BYTES;           // a whole tile, 32 KiB
+constexpr uint32_t TILE2D_SMEM = TILE_NST * TSTAGE_BYTES + 1024;
+
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+__global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__ CUtensorMap xmap,
+                                                         const Tile2dArgs a)
+{
+    using F = Fmt<FMT>;
+    extern __shared__ uint8_t tile_smem[];
+    __shared__ __align__(8) uint64_t bars[TILE_NST];
+    __shared__ float4 red[2][8];          // per warp: amax, min, max (by tile parity)
+    __shared__ float red_ss[2][8];        // per warp: sum of squares of the scaled values
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const uint32_t trow = threadIdx.x & (TILE - 1), half = threadIdx.x / TILE;
+    const uint32_t buf0 = (smem_addr(tile_smem) + 1023u) & ~1023u;
+    const uint32_t bar0 = smem_addr(&bars[0]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TILE_NST; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // thread 0: stages with a load in flight, and each stage's next phase
+    uint32_t inflight = 0, phase = 0;
+    auto issue = [&](uint32_t j, uint32_t s) {           // the CTA's tile j into stage s
+        const uint32_t t = blockIdx.x + j * gridDim.x;
+        if (t < a.ntiles) {
+            const uint32_t tr = t / a.tpr, tc = t - tr * a.tpr;
+            const uint32_t dst = buf0 + s * TSTAGE_BYTES, bar = bar0 + 8 * s;
+            mbar_arrive_expect_tx(bar, TSTAGE_BYTES);
+            tma_load_2d(dst, &xmap, bar, (int)(tc * TILE), (int)(tr * TILE));
+            tma_load_2d(dst + TBOX_BYTES, &xmap, bar, (int)(tc * TILE + 64), (int)(tr * TILE));
+            inflight |= 1u << s;
+        }
+    };
+    if (threadIdx.x == 0)
+        for (uint32_t s = 0; s < (uint32_t)TILE_NST; ++s) issue(s, s);
+
+    const bool f16 = a.scale_fp16 != 0;
+    Acc acc;
+    float kap_amax = 0.0f, kap_inv_n = 0.0f;              // thread 0: the last tile's kappa inputs
+    bool ok = true;
+    uint32_t j = 0;
+    for (uint32_t t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++j) {
+        const uint32_t s = j % TILE_NST;
+        const bool got = mbar_wait(bar0 + 8 * s, (j / TILE_NST) & 1u);
+        if (threadIdx.x == 0 && got) { inflight &= ~(1u << s); phase ^= 1u << s; }
+        const Row row{buf0 + s * TSTAGE_BYTES + half * TBOX_BYTES + trow * ROW_BYTES, trow & 7u};
+
+        // pass 1: the thread's part of the tile's range, then the warp's
+        float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+        if constexpr (HAD) {
+#pragma unroll
+            for (int k = 0; k < SPAN; ++k) {
+                uint32_t w[8];
+                float2 y[8];
+                row_chunk(row, k, w);
+                chunk_in<true>(w, y);
+                if constexpr (F::asym) chunk_minmax(y, mn, mx);
+                else amax = chunk_amax(y, amax);
+            }
+        } else {
+            uint32_t plo = 0u, phi = 0u, pm = 0u;         // packed bf16 pairs
+#pragma unroll
+            for (int k = 0; k < SPAN; ++k) {
+                uint32_t w[8];
+                row_chunk(row, k, w);
+                if constexpr (F::asym) words_minmax(w, plo, phi);
+                else pm = words_absmax(w, pm);
+            }
+            if constexpr (F::asym) { mn = pair_min(plo); mx = pair_max(phi); }
+            else amax = pair_absmax(pm);
+        }
+        if constexpr (F::asym) { mn = warp_minf(mn); mx = warp_maxf(mx); }
+        else amax = warp_maxf(amax);
+        if (lane == 0) red[j & 1][wib] = make_float4(amax, mn, mx, 0.0f);
+        if (__syncthreads_or(!got)) { ok = false; break; }
+
+        if (threadIdx.x == 0 && j > 0) {
+            const uint32_t jp = j - 1;
+            if constexpr (STATS) {
+                float ss = red_ss[jp & 1][0];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) ss = __fadd_rn(ss, red_ss[jp & 1][w]);
+                kappa_add(acc, kap_amax, ss, kap_inv_n);
+            }
+            issue(jp + TILE_NST, jp % TILE_NST);
+        }
+
+        // the tile's range and scale (the same in every thread)
+        {
+            const float4 v0 = red[j & 1][0];
+            amax = v0.x; mn = v0.y; mx = v0.z;
+#pragma unroll
+            for (int w = 1; w < 8; ++w) {
+                const float4 v = red[j & 1][w];
+                amax = fmaxf(amax, v.x); mn = fminf(mn, v.y); mx = fmaxf(mx, v.z);
+            }
+            if constexpr (F::asym) amax = fmaxf(-mn, mx);
+        }
+        const bool scaled = STATS && !plain_sums_ok(amax);
+        const Pow2 pw = pow2_for(amax);
+        const float p = scaled ? pw.p : 1.0f;
+        const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+        const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+
+        // pass 2: codes of the thread's span
+        const uint32_t tr = t / a.tpr, tc = t - tr * a.tpr;
+        const uint32_t r = tr * TILE + trow;
+        const bool row_ok = r < a.rows;
+        const size_t c0 = ((size_t)r * a.cols + tc * TILE + half * 64u) / 16u;   // its first chunk
+        float2 e2 = splat(0.0f), x2 = splat(0.0f);
+        uint32_t span4[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        plain_unit_chunks<FMT, HAD, STATS, EXACT>(row, u, scaled, p, a.codes, c0, 0, SPAN, row_ok ? SPAN : 0,
+                                                  e2, x2, span4);
+        if constexpr (F::four) {
+            if (row_ok) st_v8(a.codes + c0 * 8, span4);
+        }
+        if (threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, t, ps, f16);
+        if constexpr (STATS) {
+            add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
+            float ss = __fadd_rn(x2.x, x2.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+            if (lane == 0) red_ss[j & 1][wib] = ss;
+            if (threadIdx.x == 0) {
+                const uint32_t nr = a.rows - tr * TILE < TILE ? a.rows - tr * TILE : TILE;
+                kap_amax = __fmul_rn(amax, p);
+                kap_inv_n = 1.0f / (float)(nr * TILE);
+            }
+        }
+    }
+    if (ok) {
+        __syncthreads();
+        if constexpr (STATS) {
+            if (threadIdx.x == 0 && j > 0) {
+                const uint32_t jp = j - 1;
+                float ss = red_ss[jp & 1][0];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) ss = __fadd_rn(ss, red_ss[jp & 1][w]);
+                kappa_add(acc, kap_amax, ss, kap_inv_n);
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        atomicAdd(&g_flat_wait_timeouts, 1u);
+        for (int k = 0; k < TILE_NST; ++k)
+            if (inflight >> k & 1u) (void)mbar_wait(bar0 + 8 * k, phase >> k & 1u);
+    }
+    if constexpr (STATS) finish_stats(acc, a.ws, a.stats, false, 0.0f, 0.0, true);
+}
+
+// ---------------------------------------------------------------------------
 // Launchers.
 // ---------------------------------------------------------------------------
 
@@ -1102,6 +1270,47 @@ cudaError_t run_rows_hs(bool had, bool stats, const RowsArgs& a, cudaStream_t st
     return stats ? run_rows<FMT, false, true, false>(a, st) : run_rows<FMT, false, false, false>(a, st);
 }
 
+// x seen as [rows][cols]: boxes of 128 rows x 64 columns, 128-byte swizzle, zero fill
+// past the last row.
+cudaError_t x_tiles_map(const uint32_t* x, uint32_t rows, uint32_t cols, CUtensorMap* map)
+{
+    *map = CUtensorMap{};
+    const EncodeTiled enc = encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, TILE};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint32_t*>(x), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int FMT, bool HAD, bool STATS, bool EXACT>
+cudaError_t run_tile2d(const Tile2dArgs& a, cudaStream_t st)
+{
+    constexpr int block = 256;
+    constexpr auto kern = k_quant_tile2d<FMT, HAD, STATS, EXACT>;
+    CUtensorMap map;
+    const cudaError_t e = x_tiles_map(a.x, a.rows, a.cols, &map);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = grid_for<kern, block, TILE2D_SMEM>(1, a.ntiles);
+    kern<<<grid, block, TILE2D_SMEM, st>>>(map, a);
+    return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t run_tile2d_hs(bool had, bool stats, const Tile2dArgs& a, cudaStream_t st)
+{
+    if (had) return stats ? run_tile2d<FMT, true, true, false>(a, st) : run_tile2d<FMT, true, false, false>(a, st);
+    if constexpr (can_exact<FMT>()) {
+        if (a.scale_fp16)
+            return stats ? run_tile2d<FMT, false, true, true>(a, st) : run_tile2d<FMT, false, false, true>(a, st);
+    }
+    return stats ? run_tile2d<FMT, false, true, false>(a, st) : run_tile2d<FMT, false, false, false>(a, st);
+}
+
 template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
@@ -1164,6 +1373,19 @@ cudaError_t launch_quant_rows(int fmt, bool had, bool stats, const RowsArgs& a, 
     case BQ_UINT4_ASYM: return run_rows_hs<BQ_UINT4_ASYM>(had, stats, a, st);
     case BQ_FP8_E4M3:   return run_rows_hs<BQ_FP8_E4M3>(had, stats, a, st);
     case BQ_FP8_E5M2:   return run_rows_hs<BQ_FP8_E5M2>(had, stats, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_quant_tile2d(int fmt, bool had, bool stats, const Tile2dArgs& a, cudaStream_t st)
+{
+    switch (fmt) {
+    case BQ_INT8_SYM:   return run_tile2d_hs<BQ_INT8_SYM>(had, stats, a, st);
+    case BQ_INT8_ASYM:  return run_tile2d_hs<BQ_INT8_ASYM>(had, stats, a, st);
+    case BQ_INT4_SYM:   return run_tile2d_hs<BQ_INT4_SYM>(had, stats, a, st);
+    case BQ_UINT4_ASYM: return run_tile2d_hs<BQ_UINT4_ASYM>(had, stats, a, st);
+    case BQ_FP8_E4M3:   return run_tile2d_hs<BQ_FP8_E4M3>(had, stats, a, st);
+    case BQ_FP8_E5M2:   return run_tile2d_hs<BQ_FP8_E5M2>(had, stats, a, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -51,9 +51,10 @@
  *  - codes: 8-bit formats uint8 [rows, cols]; 4-bit formats uint8 [rows, cols/2], element
  *    2j in the low nibble of byte j; FP6 formats one code per byte [rows, cols] (the low
  *    six bits, sign at bit 5); INT codes are two's complement (UINT4 unsigned);
- *  - scales: per tensor 1 value; per row [rows]; per group [rows, cols/block]; MX uint8
- *    [rows, cols/32] (UE8M0 codes); NV uint8 [rows, cols/16] (E4M3 codes);
- *    fp32 or fp16 as scheme.scale_dtype says for the first three;
+ *  - scales: per tensor 1 value; per row [rows]; per group [rows, cols/block]; 2-D
+ *    tiles [ceil(rows/128), cols/128] (tile (i, j) covers rows 128i.., columns 128j..);
+ *    MX uint8 [rows, cols/32] (UE8M0 codes); NV uint8 [rows, cols/16] (E4M3 codes);
+ *    fp32 or fp16 as scheme.scale_dtype says for the first four;
  *  - zero points (asymmetric formats only): same shape and dtype as the scales,
  *    holding exact integers;
  *  - tensor_scale: one fp32 (NV only).
@@ -104,13 +105,18 @@ enum {
     BQ_PER_ROW = 1,      /* one scale per row (output channel of a weight, or token)   */
     BQ_PER_GROUP = 2,    /* block in {16, 32, 64, 128, 256, 512} contiguous along a row */
     BQ_MX_BLOCK = 3,     /* block 32, UE8M0 scale: INT8_SYM, E4M3, E5M2, E2M1, E2M3, E3M2 */
-    BQ_NV_BLOCK = 4      /* block 16, E4M3 scale + fp32 tensor scale: E2M1, INT4_SYM    */
+    BQ_NV_BLOCK = 4,     /* block 16, E4M3 scale + fp32 tensor scale: E2M1, INT4_SYM    */
+    BQ_TILE_2D = 5       /* one scale per 128 x 128 tile (block 128; the last tile row  */
+                         /* may hold fewer rows), fp32 or fp16: every format but FP4 /  */
+                         /* FP6; cols % 128 == 0 ("Quantization survey" §4.4, the       */
+                         /* DeepSeek-V3 weight tiles)                                    */
 };
 
 typedef struct bq_scheme {
     int32_t format;       /* BQ_INT8_SYM ...                                     */
     int32_t granularity;  /* BQ_PER_TENSOR ...                                   */
     int32_t block;        /* group size for BQ_PER_GROUP; 32 for MX, 16 for NV;  */
+                          /* 128 (or 0) for BQ_TILE_2D;                          */
                           /* ignored (0) for per-tensor / per-row                */
     int32_t scale_dtype;  /* BQ_DT_FP32 or BQ_DT_FP16 (tensor/row/group),        */
                           /* BQ_DT_UE8M0 (MX), BQ_DT_E4M3 (NV)                    */
@@ -120,7 +126,7 @@ typedef struct bq_scheme {
 
 /* QSNR and crest-factor sums, written by the library into caller device memory.
  * err2 = sum (x - xhat)^2 and x2 = sum x^2 over the whole tensor (original domain);
- * kappa_* over the scaling units (block, group, row, or the tensor), each unit's
+ * kappa_* over the scaling units (block, group, row, 2-D tile, or the tensor), each unit's
  * kappa = amax / sqrt(mean of squares) of the values it quantizes (rotated values
  * when hadamard = 1); units whose sum of squares is zero are not counted. */
 typedef struct bq_stats {

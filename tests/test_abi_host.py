@@ -44,6 +44,7 @@ SCHEMES = [
     Scheme("e2m3", "mx"), Scheme("e3m2", "mx"),
     Scheme("e2m1", "nv"), Scheme("int4_sym", "nv"), Scheme("int4_sym", "nv", hadamard=True),
     Scheme("int8_sym", "group", 512), Scheme("e4m3", "group", 16, "fp16"),
+    Scheme("e4m3", "tile2d"), Scheme("uint4_asym", "tile2d", scale_dtype="fp16"), Scheme("int4_sym", "tile2d"),
 ]
 
 
@@ -87,6 +88,11 @@ def _status(fn, *args):
     (Scheme("int8_sym", "group", 128), (4, 64), 3),
     (Scheme("int8_sym", "row"), (1 << 20, 1 << 16), 3),      # 2^36 elements
     (Scheme("int8_sym", "row"), (4, 0), 3),
+    (Scheme("e2m1", "tile2d"), (4, 128), 2),
+    (Scheme("e2m3", "tile2d"), (4, 128), 2),
+    (Scheme("int8_sym", "tile2d", 64), (4, 128), 2),
+    (Scheme("int8_sym", "tile2d", scale_dtype="ue8m0"), (4, 128), 2),
+    (Scheme("int8_sym", "tile2d"), (4, 192), 3),
 ])
 def test_invalid_schemes_and_shapes(s, shape, want):
     assert _status(bq.bq_buffer_sizes, s, *shape) == want
@@ -95,7 +101,7 @@ def test_invalid_schemes_and_shapes(s, shape, want):
 def test_bad_enum_and_reserved():
     L = bq.lib()
     z = ctypes.c_size_t(0)
-    for f in [(9, 0, 0, 2, 0, 0), (0, 7, 0, 2, 0, 0), (0, 1, 0, 2, 2, 0), (0, 1, 0, 2, 0, 1), (0, 1, 0, 9, 0, 0)]:
+    for f in [(9, 0, 0, 2, 0, 0), (0, 7, 0, 2, 0, 0), (0, 6, 0, 2, 0, 0), (0, 1, 0, 2, 2, 0), (0, 1, 0, 2, 0, 1), (0, 1, 0, 9, 0, 0)]:
         sc = bq.BqScheme(*f)
         assert L.bq_buffer_sizes(ctypes.byref(sc), 4, 64, ctypes.byref(z), None, None, None) == 1
     assert L.bq_buffer_sizes(None, 4, 64, ctypes.byref(z), None, None, None) == 1

@@ -40,6 +40,10 @@ ALL_SCHEMES = [
     Scheme("int8_sym", "row", hadamard=True), Scheme("e4m3", "tensor", hadamard=True),
     Scheme("uint4_asym", "group", 128, "fp16", hadamard=True), Scheme("int8_sym", "mx", hadamard=True),
     Scheme("e2m3", "mx"), Scheme("e3m2", "mx"), Scheme("e2m3", "mx", hadamard=True),
+    Scheme("int8_sym", "tile2d"), Scheme("int8_asym", "tile2d", scale_dtype="fp16"),
+    Scheme("int4_sym", "tile2d", scale_dtype="fp16"), Scheme("uint4_asym", "tile2d"),
+    Scheme("e4m3", "tile2d"), Scheme("e5m2", "tile2d", scale_dtype="fp16"),
+    Scheme("e4m3", "tile2d", hadamard=True), Scheme("uint4_asym", "tile2d", scale_dtype="fp16", hadamard=True),
 ]
 
 
@@ -165,6 +169,8 @@ INPUTS = {
     "tail_3x2064": lambda: synth.weight_outliers(3, 2064, seed=107),
     "single_1x16": lambda: synth.uniform(1, 16, seed=104),
     "uniform_3x2048": lambda: synth.uniform(3, 2048, seed=105),
+    # three 128-row tile rows, the last of 44 rows; three tile columns
+    "tiles_300x384": lambda: synth.weight_outliers(300, 384, seed=108),
 }
 
 
@@ -189,11 +195,21 @@ def test_row_kernel_shapes(s, cols, ws):
     check(x, s, ws, f"rows9x{cols}")
 
 
+@pytest.mark.parametrize("rows", [1, 127, 128, 129, 640])
+@pytest.mark.parametrize("s", [Scheme("e4m3", "tile2d"), Scheme("uint4_asym", "tile2d", scale_dtype="fp16")], ids=str)
+def test_tile2d_shapes(s, rows, ws):
+    # tile rows of 1..128 rows, whole and ragged, over more tiles than one wave of CTAs
+    # at 640 x 8192 (320 tiles)
+    cols = 8192 if rows == 640 else 1152
+    x = synth.weight_outliers(rows, cols, seed=300 + rows)
+    check(x, s, ws, f"tiles{rows}x{cols}")
+
+
 def test_empty_input(ws, cuda_device):
-    for s in [Scheme("int8_sym", "tensor"), Scheme("e2m1", "nv"), Scheme("int8_sym", "row")]:
-        x = torch.empty((0, 64), dtype=torch.bfloat16, device=cuda_device)
+    for s in [Scheme("int8_sym", "tensor"), Scheme("e2m1", "nv"), Scheme("int8_sym", "row"), Scheme("e4m3", "tile2d")]:
+        x = torch.empty((0, 128), dtype=torch.bfloat16, device=cuda_device)
         st = torch.full((5,), 7.0, dtype=torch.float64, device=cuda_device)
-        q = bq.alloc_outputs(s, 0, 64, cuda_device)
+        q = bq.alloc_outputs(s, 0, 128, cuda_device)
         codes = torch.empty(0, dtype=torch.uint8, device=cuda_device)
         bq.bq_quantize(x, s, codes, q.scales, q.zero_points, q.tensor_scale, st, ws)
         torch.cuda.synchronize()
@@ -232,7 +248,8 @@ def test_tiny_weight_full(ws):
 
 def test_weight_outliers_full(ws):
     x = synth.weight_outliers()
-    for s in [Scheme("uint4_asym", "group", 128, "fp16"), Scheme("int8_sym", "row")]:
+    for s in [Scheme("uint4_asym", "group", 128, "fp16"), Scheme("int8_sym", "row"),
+              Scheme("e4m3", "tile2d"), Scheme("e4m3", "group", 128)]:
         check(x, s, ws, "weight_outliers")
 
 
