@@ -430,22 +430,25 @@ __device__ __noinline__ NvOut nv_general(float2 y0, float2 y1, float2 y2, float2
     return o;
 }
 
-// A lane's four NV blocks. Fast path per block: the exact quotient RN(x / d), d = s_b S,
-// by the reciprocal correction with rn = RN(1/d) (s_b, d and rn from the CTA's table
-// over the 127 block-scale codes); FP codes by cvt, INT4 codes rounded
-// half to even and clamped to [-7, 7]. x-hat = (code value * s_b) * S (the first
-// product is exact). The span's plain sums and crest factors are gathered in fp32 and
-// folded into the lane's doubles once per span.
+// A lane's four NV blocks. Fast path per block: the exact quotient q = RN(x / d),
+// d = s_b S, by the reciprocal correction with rn = RN(1/d) (s_b, d and rn from the CTA's
+// table over the 127 block-scale codes); FP codes by cvt, INT4 codes rounded half to
+// even (no clamp: the table admits only block scales under which no code passes +-7).
+// The error of an element is taken as (q - code value) d, the quotient's residual in
+// units of d: the sums gather the residuals' squares and scale by d^2 once per block.
+// The span's plain sums and crest factors are gathered in fp32 and folded into the
+// lane's doubles once per span.
 template <int FMT, bool HAD, bool STATS>
 __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const FlatArgs& a, const TensorCtx& tc,
                                         const float4* nvtab, Acc& acc, uint32_t (&span4)[8], uint32_t& scodes)
 {
     using F = Fmt<FMT>;
-    float2 se2 = splat(0.0f), sx2 = splat(0.0f);
+    float se2 = 0.0f;
+    float2 sx2 = splat(0.0f);
     float ksum = 0.0f, kmax = 0.0f;
     uint32_t kn = 0u;
     const float S = tc.S;
-    const float2 SS = splat(S), M = splat(MAGIC), M1 = splat(-1.0f);
+    const float2 M = splat(MAGIC), M1 = splat(-1.0f);
 #pragma unroll 1
     for (int k = 0; k < SPAN; ++k) {
         uint32_t w[8], q[2];
@@ -454,26 +457,26 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
         chunk_in<HAD>(w, y);
         const float amax = chunk_amax(y, 0.0f);
         const uint32_t sbc = nv_scale_code<FMT>(amax, S, tc.cS);
-        const float4 tb = nvtab[sbc];                  // s_b, d = s_b S, RN(1/d)
+        const float4 tb = nvtab[sbc];                  // s_b, d = s_b S, RN(1/d), clamp-free
         const float sbv = tb.x, d = tb.y, rn = tb.z;
         scodes |= sbc << (8 * k);
         // d = 0 codes every element as +0: INT4 gets that from the fast path, FP (where -0
         // would keep its sign) from the general path
-        const bool mk = (F::is_int && !(d > 0.0f)) || (d >= 0x1p-60f && d <= 0x1p100f && __fmul_rn(amax, rn) < 0x1p20f);
+        const bool mk = (F::is_int && !(d > 0.0f)) ||
+                        (d >= 0x1p-60f && d <= 0x1p100f && __fmul_rn(amax, rn) < 0x1p20f);
+        const bool fast = mk && (!F::is_int || tb.w != 0.0f);
         const bool scaled = STATS && !plain_sums_ok(amax);
-        if (!__any_sync(0xFFFFFFFFu, !mk || scaled)) {
-            const float2 RN = splat(rn), ND = splat(-d), NB = splat(-sbv);
-            float2 val[8];
+        if (!__any_sync(0xFFFFFFFFu, !fast || scaled)) {
+            const float2 RN = splat(rn), ND = splat(-d);
+            float2 r[8];                                   // q - code value
             if constexpr (F::is_int) {
                 float2 t[8];
-                const float cmin = MAGIC - 7.0f, cmax = MAGIC + 7.0f;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float2 q0 = mul2(y[i], RN);
                     const float2 q1 = fma2(fma2(q0, ND, y[i]), RN, q0);      // RN(x / d)
-                    float2 t0 = add2(q1, M);                                  // MAGIC + rne(q)
-                    t0 = make_float2(fminf(fmaxf(t0.x, cmin), cmax), fminf(fmaxf(t0.y, cmin), cmax));
-                    val[i] = mul2(fma2(t0, M1, M), NB);                       // q s_b, exact
+                    const float2 t0 = add2(q1, M);                            // MAGIC + rne(q)
+                    if constexpr (STATS) r[i] = add2(q1, fma2(t0, M1, M));    // q1 - rne(q), exact
                     t[i] = add2(t0, splat(8.0f));                             // + bias
                 }
                 pack_int<FMT>(t, q);
@@ -482,28 +485,28 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float2 q0 = mul2(y[i], RN);
-                    const float2 q1 = fma2(fma2(q0, ND, y[i]), RN, q0);      // RN(x / d)
-                    pr[i] = cvt_pair<FMT>(q1.y, q1.x);
+                    r[i] = fma2(fma2(q0, ND, y[i]), RN, q0);                  // RN(x / d)
+                    pr[i] = cvt_pair<FMT>(r[i].y, r[i].x);
                 }
                 pack_pairs<FMT>(pr, q);
                 if constexpr (STATS) {
+                    float2 val[8];
                     decode_pairs<FMT>(pr, val);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) val[i] = mul2(val[i], splat(sbv));
+                    for (int i = 0; i < 8; ++i) r[i] = sub2(r[i], val[i]);
                 }
             }
             if constexpr (STATS) {
                 float2 ea = splat(0.0f), eb = splat(0.0f), xa = splat(0.0f), xb = splat(0.0f);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
-                    const float2 d0 = fma2(val[i], splat(-S), y[i]), d1 = fma2(val[i + 1], splat(-S), y[i + 1]);
-                    ea = fma2(d0, d0, ea);
-                    eb = fma2(d1, d1, eb);
+                    ea = fma2(r[i], r[i], ea);
+                    eb = fma2(r[i + 1], r[i + 1], eb);
                     xa = fma2(y[i], y[i], xa);
                     xb = fma2(y[i + 1], y[i + 1], xb);
                 }
                 const float2 ce2 = add2(ea, eb), cx2 = add2(xa, xb);
-                se2 = add2(se2, ce2);
+                se2 = __fmaf_rn(__fadd_rn(ce2.x, ce2.y), __fmul_rn(d, d), se2);
                 sx2 = add2(sx2, cx2);
                 const float ss = __fadd_rn(cx2.x, cx2.y);
                 if (ss > 0.0f) {
@@ -531,7 +534,8 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
     }
     if constexpr (STATS) {
         // chunks past the tensor's end are zeros: they add nothing
-        add_unit_sums(acc, se2, sx2, 1.0);
+        acc.err2 += (double)se2;
+        acc.x2 += (double)__fadd_rn(sx2.x, sx2.y);
         acc.ksum += (double)ksum;
         acc.kmax = fmaxf(acc.kmax, kmax);
         acc.nunits += kn;
@@ -713,7 +717,9 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
     extern __shared__ uint8_t flat_smem[];
     __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    const uint32_t warp = blockIdx.x * FLAT_WARPS + wib;
+    // warps numbered across the CTAs first: the last, partly filled round of tiles (rows)
+    // spreads over every CTA, and so over every SM, instead of filling the first CTAs
+    const uint32_t warp = wib * gridDim.x + blockIdx.x;
     const uint32_t nwarps = gridDim.x * FLAT_WARPS;
     const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
     const uint32_t bar0 = smem_addr(&bars[wib][0]);
@@ -764,7 +770,10 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         for (int c = threadIdx.x; c < 128; c += blockDim.x) {
             const float sb = e4m3_value((uint32_t)c);
             const float d = __fmul_rn(sb, tc.S);
-            nvtab[c] = make_float4(sb, d, d > 0.0f ? __frcp_rn(d) : 0.0f, 0.0f);
+            // w = 1: no integer code can pass +-Qmax (a normal E4M3 s_b is at most 2^-4
+            // below (amax / Qmax) / S, so |x / d| < Qmax (1 + 1/15) < Qmax + 0.5; d = 0 codes 0)
+            const bool nc = !(d > 0.0f) || (c & 0x78) != 0;
+            nvtab[c] = make_float4(sb, d, d > 0.0f ? __frcp_rn(d) : 0.0f, nc ? 1.0f : 0.0f);
         }
         __syncthreads();
     }
@@ -869,7 +878,9 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_rows(co
     extern __shared__ uint8_t flat_smem[];
     __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    const uint32_t warp = blockIdx.x * FLAT_WARPS + wib;
+    // warps numbered across the CTAs first: the last, partly filled round of tiles (rows)
+    // spreads over every CTA, and so over every SM, instead of filling the first CTAs
+    const uint32_t warp = wib * gridDim.x + blockIdx.x;
     const uint32_t nwarps = gridDim.x * FLAT_WARPS;
     const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
     const uint32_t bar0 = smem_addr(&bars[wib][0]);
