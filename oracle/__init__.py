@@ -85,6 +85,14 @@ def lib() -> ctypes.CDLL:
         L.orc_f32_to_bf16_array.argtypes = [vp, vp, i64]
         L.orc_buffer_sizes.restype = i32
         L.orc_buffer_sizes.argtypes = [i32, i32, i32, i32, i32, i64, i64, vp]
+        L.orc_fwht.restype = None
+        L.orc_fwht.argtypes = [vp, i64]
+        L.orc_rotate_rows.restype = i32
+        L.orc_rotate_rows.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.orc_quantize_rt.restype = i32
+        L.orc_quantize_rt.argtypes = [vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.orc_dequantize_rt.restype = i32
+        L.orc_dequantize_rt.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp]
         _lib = L
     return _lib
 
@@ -238,4 +246,67 @@ def to_bf16_array(values_f32: np.ndarray) -> np.ndarray:
     a = np.ascontiguousarray(values_f32, dtype=np.float32)
     out = np.zeros(a.shape, dtype=np.uint16)
     lib().orc_f32_to_bf16_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Row transforms: a per-column factor (SmoothQuant) and the randomized full-row
+# Hadamard rotation (QuaRot); signs are bytes, nonzero = -1.
+# ---------------------------------------------------------------------------
+
+def _opt_f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _opt_u8(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def fwht(v: np.ndarray) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform (Sylvester order) of a float32 vector."""
+    v = np.array(v, dtype=np.float32)
+    lib().orc_fwht(_ptr(v), v.size)
+    return v
+
+
+def rotate_rows(x_bits: np.ndarray, col_scale=None, signs=None) -> np.ndarray:
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, cols = x_bits.shape
+    out = np.zeros((rows, cols), dtype=np.float32)
+    cs, sg = _opt_f32(col_scale), _opt_u8(signs)
+    _check(lib().orc_rotate_rows(_ptr(x_bits), rows, cols, _ptr(cs), _ptr(sg), _ptr(out)), "rotate_rows")
+    return out
+
+
+def quantize_rt(x_bits: np.ndarray, scheme: Scheme, col_scale=None, signs=None, stats: bool = True):
+    """quantize() after the row transforms (row, group and MX schemes)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, cols = x_bits.shape
+    s = scheme.resolved()
+    if s.hadamard:
+        raise ValueError("oracle quantize_rt: the block-16 Hadamard does not combine with the row transforms")
+    cb, sb, zb, tb = buffer_sizes(s, rows, cols)
+    sdt = _scale_np_dtype(s)
+    codes = np.zeros(cb, dtype=np.uint8)
+    scales = np.zeros(sb // np.dtype(sdt).itemsize, dtype=sdt)
+    zps = np.zeros(zb // np.dtype(sdt).itemsize, dtype=sdt) if zb else None
+    st = np.zeros(5, dtype=np.float64) if stats else None
+    cs, sg = _opt_f32(col_scale), _opt_u8(signs)
+    a = s.args()
+    rc = lib().orc_quantize_rt(_ptr(x_bits), rows, cols, a[0], a[1], a[2], a[3], _ptr(cs), _ptr(sg),
+                               _ptr(codes), _ptr(scales), _ptr(zps), _ptr(st))
+    _check(rc, "quantize_rt")
+    cols_b = cols // 2 if s.fmt in FOUR_BIT else cols
+    return {"codes": codes.reshape(rows, cols_b), "scales": scales, "zps": zps, "tensor_scale": None, "stats": st}
+
+
+def dequantize_rt(codes, scales, zps, rows: int, cols: int, scheme: Scheme, signs=None) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.zeros((rows, cols), dtype=np.float32)
+    sg = _opt_u8(signs)
+    a = scheme.resolved().args()
+    rc = lib().orc_dequantize_rt(_ptr(codes), _ptr(np.ascontiguousarray(scales)),
+                                 _ptr(None if zps is None else np.ascontiguousarray(zps)), rows, cols,
+                                 a[0], a[1], a[2], a[3], _ptr(sg), _ptr(out))
+    _check(rc, "dequantize_rt")
     return out

@@ -800,3 +800,155 @@ void orc_f32_to_bf16_array(const float* in, uint16_t* out, int64_t n)
 {
     for (int64_t i = 0; i < n; i++) out[i] = orc_f32_to_bf16(in[i]);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Row transforms before quantizing: SmoothQuant's per-channel factor          */
+/* ("Quantization survey" §3.2 and §5.2: W * s per input channel) and QuaRot's */
+/* randomized Hadamard rotation of the whole row (same page §5.3: an           */
+/* orthogonal +-1 rotation, R^T R = I, spreads outlier channels over all).     */
+/*                                                                            */
+/* Readings: x' = RN(x * m_j) with m the caller's per-column factor; the       */
+/* rotation is y = (x' * sigma) H_n c with sigma_j = -1 where the caller's     */
+/* sign byte is set, H_n the Sylvester-order Walsh-Hadamard matrix (n = cols,  */
+/* a power of two), taken as stages h = 1, 2, ..., n/2 of (a + b, a - b), and  */
+/* c = the fp32 value nearest 1/sqrt(n); dequantize applies the inverse        */
+/* (the same stages, * c, then the signs) and returns x' (the factor stays:    */
+/* the operand a GEMM would take); QSNR compares x' with that.                 */
+/* ------------------------------------------------------------------------- */
+
+/* Walsh-Hadamard transform (unnormalised) of n = 2^m values in place. */
+void orc_fwht(float* v, int64_t n)
+{
+    for (int64_t h = 1; h < n; h *= 2)
+        for (int64_t i = 0; i < n; i += 2 * h)
+            for (int64_t k = i; k < i + h; k++) {
+                float a = v[k], b = v[k + h];
+                v[k] = a + b;
+                v[k + h] = a - b;
+            }
+}
+
+static float rot_norm(int64_t n) { return (float)(1.0 / sqrt((double)n)); }
+
+static int pow2_in(int64_t n, int64_t lo, int64_t hi) { return n >= lo && n <= hi && (n & (n - 1)) == 0; }
+
+/* One row: xs = x' (pre-scaled), y = rotated (or x' when signs is NULL). */
+static void rt_forward(const uint16_t* xrow, int64_t n, const float* col_scale, const uint8_t* signs,
+                       float* xs, float* y)
+{
+    for (int64_t j = 0; j < n; j++) {
+        float v = orc_bf16_to_f32(xrow[j]);
+        if (col_scale) v = v * col_scale[j];
+        xs[j] = v;
+        y[j] = (signs && signs[j]) ? -v : v;
+    }
+    if (signs) {
+        const float c = rot_norm(n);
+        orc_fwht(y, n);
+        for (int64_t j = 0; j < n; j++) y[j] = y[j] * c;
+    }
+}
+
+static void rt_inverse(float* v, int64_t n, const uint8_t* signs)
+{
+    if (!signs) return;
+    const float c = rot_norm(n);
+    orc_fwht(v, n);
+    for (int64_t j = 0; j < n; j++) {
+        v[j] = v[j] * c;
+        if (signs[j]) v[j] = -v[j];
+    }
+}
+
+static int rt_check(const scheme* s, int gran, int64_t cols, const uint8_t* signs)
+{
+    if (!(gran == G_ROW || gran == G_GROUP || gran == G_MX)) return -1;
+    if (s->had) return -1;
+    if (signs && !pow2_in(cols, 16, 16384)) return -2;
+    return 0;
+}
+
+/* The transformed rows' fp32 values (x' rotated), [rows, cols]. */
+int orc_rotate_rows(const uint16_t* x, int64_t rows, int64_t cols, const float* col_scale,
+                    const uint8_t* signs, float* out)
+{
+    if (rows < 0 || cols <= 0) return -2;
+    if (signs && !pow2_in(cols, 16, 16384)) return -2;
+    float* xs = (float*)malloc(sizeof(float) * (size_t)cols);
+    if (!xs) return -3;
+    for (int64_t r = 0; r < rows; r++) rt_forward(x + r * cols, cols, col_scale, signs, xs, out + r * cols);
+    free(xs);
+    return 0;
+}
+
+/*
+ * Quantize x [rows, cols] after the row transforms (col_scale: NULL or [cols];
+ * signs: NULL for no rotation, else [cols] bytes, nonzero = -1). Per-row, per-group
+ * and MX schemes without the block-16 Hadamard. Outputs as orc_quantize; stats:
+ * err2 and x2 against x' in the original (unrotated) domain, kappa over the units'
+ * rotated values.
+ */
+int orc_quantize_rt(const uint16_t* x, int64_t rows, int64_t cols,
+                    int fmt, int gran, int block, int scale_dtype,
+                    const float* col_scale, const uint8_t* signs,
+                    uint8_t* codes, void* scales, void* zps, double* stats)
+{
+    scheme s;
+    int rc = make_scheme(fmt, gran, block, scale_dtype, 0, cols, &s);
+    if (rc) return rc;
+    rc = rt_check(&s, gran, cols, signs);
+    if (rc) return rc;
+    if (rows < 0) return -2;
+    if (stats) for (int i = 0; i < 5; i++) stats[i] = 0.0;
+    const int64_t unit = s.unit, upr = cols / unit;
+    float* xs = (float*)malloc(sizeof(float) * (size_t)cols);
+    float* y = (float*)malloc(sizeof(float) * (size_t)cols);
+    float* yh = (float*)malloc(sizeof(float) * (size_t)cols);
+    unsigned* cd = (unsigned*)malloc(sizeof(unsigned) * (size_t)cols);
+    if (!xs || !y || !yh || !cd) { free(xs); free(y); free(yh); free(cd); return -3; }
+    for (int64_t r = 0; r < rows; r++) {
+        rt_forward(x + r * cols, cols, col_scale, signs, xs, y);
+        for (int64_t u = 0; u < upr; u++) {
+            unit_range ur;
+            range_of(y + u * unit, unit, &ur);
+            ur.S = 0.0f;
+            float sc = 0.0f, zp = 0.0f;
+            uint8_t scode = 0;
+            quant_unit(&s, y + u * unit, unit, ur, cd + u * unit, &sc, &zp, &scode, yh + u * unit);
+            const int64_t si = r * upr + u;
+            if (gran == G_MX) ((uint8_t*)scales)[si] = scode;
+            else {
+                write_scale(scales, si, sc, s.sdt);
+                if (s.is_asym && zps) write_scale(zps, si, zp, s.sdt);
+            }
+            if (stats) kappa_add(stats, ur.amax, y + u * unit, unit);
+        }
+        for (int64_t j = 0; j < cols; j++) put_code(codes, r, cols, j, cd[j], s.bits4);
+        rt_inverse(yh, cols, signs);
+        if (stats)
+            for (int64_t j = 0; j < cols; j++) {
+                double e = (double)xs[j] - (double)yh[j];
+                stats[0] += e * e;
+                stats[1] += (double)xs[j] * (double)xs[j];
+            }
+    }
+    free(xs); free(y); free(yh); free(cd);
+    return 0;
+}
+
+/* Dequantize codes written by orc_quantize_rt: x-hat' [rows, cols] (the inverse
+ * rotation applied; the per-column factor kept). */
+int orc_dequantize_rt(const uint8_t* codes, const void* scales, const void* zps,
+                      int64_t rows, int64_t cols, int fmt, int gran, int block, int scale_dtype,
+                      const uint8_t* signs, float* out)
+{
+    scheme s;
+    int rc = make_scheme(fmt, gran, block, scale_dtype, 0, cols, &s);
+    if (rc) return rc;
+    rc = rt_check(&s, gran, cols, signs);
+    if (rc) return rc;
+    rc = orc_dequantize(codes, scales, zps, NULL, rows, cols, fmt, gran, block, scale_dtype, 0, out);
+    if (rc) return rc;
+    for (int64_t r = 0; r < rows; r++) rt_inverse(out + r * cols, cols, signs);
+    return 0;
+}

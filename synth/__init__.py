@@ -42,6 +42,8 @@ __all__ = [
     "ffn_lognormal",
     "weight_x50",
     "workload",
+    "random_signs",
+    "col_factors",
 ]
 
 
@@ -128,6 +130,18 @@ def weight_x50(rows: int = 8192, cols: int = 28672, seed: int = 4,
         pos = g.choice(n, size=k, replace=False)
         a.reshape(-1)[pos] *= np.float32(factor)
     return to_bf16(a)
+
+
+def random_signs(n: int, seed: int) -> np.ndarray:
+    """n fair coin flips as uint8 0/1 (1 = negate that column), the random diagonal of a
+    randomized Hadamard rotation."""
+    return _rng(seed).integers(0, 2, size=n, dtype=np.uint8)
+
+
+def col_factors(n: int, seed: int, sigma: float = 0.5) -> np.ndarray:
+    """n positive float32 per-column factors, lognormal(0, sigma): synthetic stand-ins
+    for smoothing factors derived from calibration statistics."""
+    return np.exp(_rng(seed).normal(0.0, sigma, size=n)).astype(np.float32)
 
 
 # name -> (generator, full shape, description)
