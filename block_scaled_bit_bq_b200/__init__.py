@@ -44,6 +44,10 @@ class BqScheme(ctypes.Structure):
                 ("scale_dtype", ctypes.c_int32), ("hadamard", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class BqRowTransform(ctypes.Structure):
+    _fields_ = [("col_scale", ctypes.c_void_p), ("sign_bits", ctypes.c_void_p), ("reserved", ctypes.c_int64)]
+
+
 class BqStats(ctypes.Structure):
     _fields_ = [("err2", ctypes.c_double), ("x2", ctypes.c_double), ("kappa_sum", ctypes.c_double),
                 ("kappa_max", ctypes.c_double), ("n_units", ctypes.c_double)]
@@ -81,6 +85,11 @@ def _lib() -> ctypes.CDLL:
         L.bq_stats_qsnr_db.argtypes = [ctypes.POINTER(BqStats)]
         L.bq_wait_timeouts.restype = ctypes.c_int
         L.bq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        rtp = ctypes.POINTER(BqRowTransform)
+        L.bq_quantize_rt.restype = ctypes.c_int
+        L.bq_quantize_rt.argtypes = [vp, i32, i64, i64, sp, rtp, vp, vp, vp, vp, vp, sz, vp]
+        L.bq_dequantize_rt.restype = ctypes.c_int
+        L.bq_dequantize_rt.argtypes = [vp, vp, vp, i64, i64, sp, rtp, vp, i32, vp]
         _L = L
     return _L
 
@@ -204,6 +213,42 @@ def bq_qsnr(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zero_poi
            "bq_qsnr")
 
 
+def _rt(col_scale: torch.Tensor | None, sign_bits: torch.Tensor | None) -> BqRowTransform:
+    return BqRowTransform(_ptr(col_scale), _ptr(sign_bits), 0)
+
+
+def bq_quantize_rt(x: torch.Tensor, scheme: Scheme, col_scale: torch.Tensor | None, sign_bits: torch.Tensor | None,
+                   codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor | None,
+                   stats: torch.Tensor | None, workspace: torch.Tensor | None, stream=None) -> None:
+    """x: bf16 [rows, cols]; col_scale: fp32 [cols] or None; sign_bits: int32 [cols / 32]
+    (bit j % 32 of word j / 32 negates column j) or None (no rotation)."""
+    rows, cols = x.shape
+    sc = scheme.c()
+    rt = _rt(col_scale, sign_bits)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().bq_quantize_rt(_ptr(x), DT["bf16"], rows, cols, ctypes.byref(sc), ctypes.byref(rt), _ptr(codes),
+                                 _ptr(scales), _ptr(zero_points), _ptr(stats), _ptr(workspace), ws_bytes,
+                                 _stream(stream)), "bq_quantize_rt")
+
+
+def bq_dequantize_rt(codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor | None, rows: int,
+                     cols: int, scheme: Scheme, col_scale: torch.Tensor | None, sign_bits: torch.Tensor | None,
+                     out: torch.Tensor, stream=None) -> None:
+    out_dt = {torch.bfloat16: DT["bf16"], torch.float32: DT["fp32"]}[out.dtype]
+    sc = scheme.c()
+    rt = _rt(col_scale, sign_bits)
+    _check(_lib().bq_dequantize_rt(_ptr(codes), _ptr(scales), _ptr(zero_points), rows, cols, ctypes.byref(sc),
+                                   ctypes.byref(rt), _ptr(out), out_dt, _stream(stream)), "bq_dequantize_rt")
+
+
+def pack_sign_bits(signs, device=None) -> torch.Tensor:
+    """Per-column 0/1 flags (1 = negate) -> int32 words, bit j % 32 of word j / 32."""
+    f = torch.as_tensor(signs).to(torch.int64).reshape(-1, 32)
+    w = (f << torch.arange(32, dtype=torch.int64)).sum(1)
+    w = torch.where(w >= 2 ** 31, w - 2 ** 32, w).to(torch.int32)
+    return w.to(device) if device is not None else w
+
+
 def bq_wait_timeouts(reset: bool = False) -> int:
     """Tile waits of the quantize kernels that gave up on the current device (each
     leaves its call's outputs incomplete); synchronizes with the device."""
@@ -290,6 +335,30 @@ def dequantize(q: Quantized, dtype=torch.bfloat16, out: torch.Tensor | None = No
     if out is None:
         out = torch.empty((q.rows, q.cols), dtype=dtype, device=q.codes.device)
     bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, q.rows, q.cols, q.scheme, out, stream)
+    return out
+
+
+def quantize_rt(x: torch.Tensor, scheme: Scheme, col_scale: torch.Tensor | None = None,
+                sign_bits: torch.Tensor | None = None, stats: bool = True, workspace: torch.Tensor | None = None,
+                stream=None) -> Quantized:
+    """Quantize a bf16 [rows, cols] CUDA tensor after the row transforms (per-column
+    factor, randomized full-row Hadamard rotation); per-row, per-group and MX schemes."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor")
+    x = x.contiguous()
+    rows, cols = x.shape
+    q = alloc_outputs(scheme, rows, cols, x.device, stats)
+    if stats and workspace is None:
+        workspace = new_workspace(x.device)
+    bq_quantize_rt(x, q.scheme, col_scale, sign_bits, q.codes, q.scales, q.zero_points,
+                   q.stats if stats else None, workspace, stream)
+    return q
+
+
+def dequantize_rt(q: Quantized, col_scale: torch.Tensor | None = None, sign_bits: torch.Tensor | None = None,
+                  dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    out = torch.empty((q.rows, q.cols), dtype=dtype, device=q.codes.device)
+    bq_dequantize_rt(q.codes, q.scales, q.zero_points, q.rows, q.cols, q.scheme, col_scale, sign_bits, out, stream)
     return out
 
 

@@ -345,6 +345,85 @@ bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void*
     return cuda_status(launch_qsnr(p.fmt, scale_kind(p), p.had != 0, a, s));
 }
 
+namespace {
+
+// Checks shared by the row-transform entry points: per-row, per-group and MX schemes
+// without the block-16 rotation; cols a multiple of 512 up to 16384 (a power of two
+// when rotating); the factor array 16-byte aligned.
+bq_status rt_check(const Plan& p, int64_t cols, const bq_row_transform* rt)
+{
+    if (!(p.gran == BQ_PER_ROW || p.gran == BQ_PER_GROUP || p.gran == BQ_MX_BLOCK) || p.had) return BQ_ERR_UNSUPPORTED;
+    if (cols % 512 != 0 || cols > 16384) return BQ_ERR_SHAPE;
+    if (rt && rt->sign_bits && (cols & (cols - 1)) != 0) return BQ_ERR_SHAPE;
+    if (rt && rt->reserved != 0) return BQ_ERR_INVALID_ARG;
+    if (rt && rt->col_scale && ((uintptr_t)rt->col_scale & 15u) != 0) return BQ_ERR_ALIGNMENT;
+    if (rt && rt->sign_bits && !aligned4(rt->sign_bits)) return BQ_ERR_ALIGNMENT;
+    return BQ_OK;
+}
+
+float rt_norm(int64_t cols) { return (float)(1.0 / std::sqrt((double)cols)); }
+
+}  // namespace
+
+bq_status bq_quantize_rt(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, const bq_scheme* scheme,
+                         const bq_row_transform* rt, void* codes, void* scales, void* zero_points,
+                         bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    st = rt_check(p, cols, rt);
+    if (st != BQ_OK) return st;
+    const bool want_stats = stats != nullptr;
+    if (want_stats && (!workspace || workspace_bytes < WS_BYTES)) return BQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (p.n == 0) {
+        if (want_stats) return cuda_status(cudaMemsetAsync(stats, 0, sizeof(bq_stats), s));
+        return BQ_OK;
+    }
+    if (!x || !codes || !scales) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points)) return BQ_ERR_ALIGNMENT;
+    RtArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.x = reinterpret_cast<const uint32_t*>(x); a.codes = reinterpret_cast<uint8_t*>(codes);
+    a.scales = scales; a.zps = zero_points; a.stats = stats; a.ws = reinterpret_cast<uint8_t*>(workspace);
+    a.col_scale = rt ? rt->col_scale : nullptr;
+    a.sign_bits = rt ? rt->sign_bits : nullptr;
+    a.rows = (uint32_t)rows; a.cols = (uint32_t)cols; a.cpr = (uint32_t)(cols / 16);
+    a.lanes = p.gran == BQ_PER_ROW ? 0u : (uint32_t)(p.block / 16);
+    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+    a.norm = rt_norm(cols);
+    a.inv_unit = 1.0f / (float)(p.gran == BQ_PER_ROW ? cols : p.block);
+    return cuda_status(launch_quant_rt(p.fmt, p.gran == BQ_MX_BLOCK, a, s));
+}
+
+bq_status bq_dequantize_rt(const void* codes, const void* scales, const void* zero_points, int64_t rows, int64_t cols,
+                           const bq_scheme* scheme, const bq_row_transform* rt, void* out, int32_t out_dtype,
+                           void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    st = rt_check(p, cols, rt);
+    if (st != BQ_OK) return st;
+    if (!rt || !rt->sign_bits)          // no rotation to invert: the plain dequantize
+        return bq_dequantize(codes, scales, zero_points, nullptr, rows, cols, scheme, out, out_dtype, stream);
+    if (out_dtype != BQ_DT_BF16 && out_dtype != BQ_DT_FP32) return BQ_ERR_UNSUPPORTED;
+    if (p.n == 0) return BQ_OK;
+    if (!codes || !scales || !out) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(codes) || !aligned32(out)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points)) return BQ_ERR_ALIGNMENT;
+    DequantArgs a = dequant_args(p, cols);
+    a.codes = reinterpret_cast<const uint8_t*>(codes);
+    a.scales = scales; a.zps = zero_points; a.out = out;
+    return cuda_status(launch_dequant_rt(p.fmt, scale_kind(p), out_dtype, a, rt->sign_bits, (uint32_t)rows,
+                                         (uint32_t)cols, rt_norm(cols), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 bq_status bq_wait_timeouts(uint32_t* count, int32_t reset)
 {
     if (!count) return BQ_ERR_INVALID_ARG;

@@ -275,9 +275,9 @@ __device__ __forceinline__ void widen16x2(const uint32_t (&w)[8], float2 (&v)[8]
     for (int i = 0; i < 8; ++i) v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
-// 16-point Walsh-Hadamard transform on pairs; the same additions in the same order as
-// fwht16 (stage h = 1 inside each pair, stages 2, 4, 8 across pairs), then * 0.25.
-__device__ __forceinline__ void fwht16x2(float2 (&v)[8])
+// 16-point Walsh-Hadamard stages on pairs, unnormalised: the same additions in the same
+// order as fwht16 (stage h = 1 inside each pair, stages 2, 4, 8 across pairs).
+__device__ __forceinline__ void wht16x2(float2 (&v)[8])
 {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -296,6 +296,12 @@ __device__ __forceinline__ void fwht16x2(float2 (&v)[8])
             }
         }
     }
+}
+
+// The block-16 rotation: those stages, then * 0.25.
+__device__ __forceinline__ void fwht16x2(float2 (&v)[8])
+{
+    wht16x2(v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = mul2(v[i], splat(0.25f));
 }

@@ -12,6 +12,7 @@
 // codes before decoding the current ones. A chunk's scale index is its chunk index
 // divided (multiply-high) by the chunks per scaling unit.
 #include "quant_ops.cuh"
+#include "rot.cuh"
 #include "internal.h"
 
 #include <atomic>
@@ -290,6 +291,60 @@ __global__ void __launch_bounds__(256) k_qsnr(const DequantArgs a)
     finish_stats(acc, a.ws, a.stats, false, 0.0f, 0.0, false);
 }
 
+// Dequantize with the inverse full-row rotation: a CTA per row at a time. Each chunk
+// is decoded, scaled and run through the first four Walsh-Hadamard stages in
+// registers; the row sits in shared memory (fp32) for the remaining stages; then each
+// value is multiplied by the normalisation, the signed columns negated and the result
+// written. The per-column factor is not undone (the codes stand for x times it).
+template <int FMT, int SK, int OUT>
+__global__ void __launch_bounds__(256) k_dequant_rt(const DequantArgs a, const uint32_t* sign_bits, uint32_t rows,
+                                                    uint32_t cols, float norm)
+{
+    constexpr int NC = SpanCodes<FMT, 1>::n;
+    extern __shared__ float4 rt_smem[];
+    float* v = reinterpret_cast<float*>(rt_smem);
+    const uint32_t cpr = cols / 16;
+    for (uint32_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        for (uint32_t c = threadIdx.x; c < cpr; c += blockDim.x) {
+            const uint32_t cg = r * cpr + c;
+            uint32_t w[NC];
+            float2 val[8], xh[8];
+            load_codes<FMT, 1>(a.codes, cg, a.n_chunks, w);
+            chunk_values<FMT, 1>(w, 0, val);
+            dequant_chunk<FMT, SK>(load_unit_scale<FMT, SK>(a, cg), val, xh);
+            wht16x2(xh);
+            store_chunk_f32(v, c, xh);
+        }
+        wht_smem_stages(v, cols);
+        for (uint32_t c = threadIdx.x; c < cpr; c += blockDim.x) {
+            float2 xh[8];
+            load_chunk_f32(v, c, norm, xh);
+            apply_signs(xh, chunk_sign_bits(sign_bits, c));
+            const size_t cg = (size_t)r * cpr + c;
+            if constexpr (OUT == BQ_DT_BF16) {
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const __nv_bfloat162 b = __floats2bfloat162_rn(xh[i].x, xh[i].y);
+                    o[i] = *reinterpret_cast<const uint32_t*>(&b);
+                }
+                st_v8(reinterpret_cast<uint8_t*>(a.out) + cg * 32, o);
+            } else {
+                uint32_t o0[8], o1[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    o0[2 * i] = __float_as_uint(xh[i].x); o0[2 * i + 1] = __float_as_uint(xh[i].y);
+                    o1[2 * i] = __float_as_uint(xh[4 + i].x); o1[2 * i + 1] = __float_as_uint(xh[4 + i].y);
+                }
+                uint8_t* p = reinterpret_cast<uint8_t*>(a.out) + cg * 64;
+                st_v8(p, o0);
+                st_v8(p + 32, o1);
+            }
+        }
+        __syncthreads();             // the row is written out; the next row may overwrite it
+    }
+}
+
 namespace {
 
 template <auto KERN, int BLOCK>
@@ -374,11 +429,41 @@ cudaError_t dispatch(int fmt, int sk, Fn&& fn)
     return cudaErrorInvalidValue;
 }
 
+template <auto KERN>
+cudaError_t launch_row_kernel(const DequantArgs& a, const uint32_t* sign_bits, uint32_t rows, uint32_t cols,
+                              float norm, cudaStream_t st)
+{
+    constexpr int block = 256;
+    const size_t smem = (size_t)cols * 4;
+    if (smem > 48u * 1024u) {
+        const cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, KERN, block, smem) != cudaSuccess || occ < 1) occ = 1;
+    uint64_t grid = (uint64_t)device_sm_count() * (uint64_t)occ;
+    if (grid > rows) grid = rows;
+    if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
+    if (grid < 1) grid = 1;
+    KERN<<<(unsigned)grid, block, smem, st>>>(a, sign_bits, rows, cols, norm);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_dequant(int fmt, int sk, bool had, int out_dtype, const DequantArgs& a, cudaStream_t st)
 {
     return dispatch(fmt, sk, [&]<int FMT, int SK>() { return run_dq<FMT, SK>(had, out_dtype, a, st); });
+}
+
+cudaError_t launch_dequant_rt(int fmt, int sk, int out_dtype, const DequantArgs& a, const uint32_t* sign_bits,
+                              uint32_t rows, uint32_t cols, float norm, cudaStream_t st)
+{
+    return dispatch(fmt, sk, [&]<int FMT, int SK>() {
+        return out_dtype == BQ_DT_BF16
+                   ? launch_row_kernel<k_dequant_rt<FMT, SK, BQ_DT_BF16>>(a, sign_bits, rows, cols, norm, st)
+                   : launch_row_kernel<k_dequant_rt<FMT, SK, BQ_DT_FP32>>(a, sign_bits, rows, cols, norm, st);
+    });
 }
 
 cudaError_t launch_qsnr(int fmt, int sk, bool had, const DequantArgs& a, cudaStream_t st)

@@ -76,6 +76,26 @@ struct Tile2dArgs {
     int32_t scale_fp16;
 };
 
+// Row transforms before quantizing (a per-column factor, a randomized full-row
+// Hadamard rotation): a CTA per row at a time, the row held in shared memory as fp32.
+struct RtArgs {
+    const uint32_t* x;
+    uint8_t* codes;
+    void* scales;
+    void* zps;
+    bq_stats* stats;            // may be null
+    uint8_t* ws;
+    const float* col_scale;     // [cols] or null
+    const uint32_t* sign_bits;  // [cols / 32] or null (no rotation)
+    uint32_t rows;
+    uint32_t cols;
+    uint32_t cpr;               // chunks per row = cols / 16
+    uint32_t lanes;             // chunks per scaling unit (1 .. 32); 0: the whole row
+    int32_t scale_fp16;
+    float norm;                 // rotation: the fp32 value nearest 1 / sqrt(cols)
+    float inv_unit;             // 1 / elements per unit (kappa)
+};
+
 struct DequantArgs {
     const uint8_t* codes;
     const void* scales;
@@ -107,6 +127,10 @@ cudaError_t launch_quant_flat(int fmt, int kind, bool hadamard, bool stats, cons
 cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& a, cudaStream_t st);
 cudaError_t launch_quant_rows(int fmt, bool hadamard, bool stats, const RowsArgs& a, cudaStream_t st);
 cudaError_t launch_quant_tile2d(int fmt, bool hadamard, bool stats, const Tile2dArgs& a, cudaStream_t st);
+cudaError_t launch_quant_rt(int fmt, bool mx, const RtArgs& a, cudaStream_t st);
+// Dequantize with the inverse full-row rotation (sign_bits [cols / 32], norm as RtArgs).
+cudaError_t launch_dequant_rt(int fmt, int sk, int out_dtype, const DequantArgs& a, const uint32_t* sign_bits,
+                              uint32_t rows, uint32_t cols, float norm, cudaStream_t st);
 cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
                            cudaStream_t st);
 cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);

@@ -20,6 +20,7 @@
 // work in the original domain).
 #include "quant_ops.cuh"
 #include "tma.cuh"
+#include "rot.cuh"
 #include "internal.h"
 
 #include <atomic>
@@ -1166,6 +1167,154 @@ __global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------
+// Row transforms, then quantize (per-row, per-group, MX): SmoothQuant's per-column
+// factor ("Quantization survey" §3.2, §5.2) and QuaRot's randomized full-row Hadamard
+// rotation (same page §5.3).
+//
+// A CTA of 256 threads owns a row at a time. Thread t loads chunks t, t + 256, ... of
+// the row, multiplies by the factors, negates the signed columns and runs the first
+// four Walsh-Hadamard stages in registers; the row then sits in shared memory as fp32
+// for the remaining stages (wht_smem_stages). The quantize phase reads each chunk back
+// times the normalisation and codes it through the general chunk path (clamping,
+// scaled sums): a scaling unit of L chunks is L adjacent threads, reduced with xor
+// shuffles; a per-row unit is reduced over the CTA. The fused QSNR sums are taken on
+// the rotated values (an orthogonal rotation keeps both sums).
+// ---------------------------------------------------------------------------
+
+template <int FMT, bool MX>
+__global__ void __launch_bounds__(256) k_quant_rt(const RtArgs a)
+{
+    using F = Fmt<FMT>;
+    constexpr int NW = CodeWords<FMT>::n;
+    extern __shared__ float4 rt_smem[];
+    float* v = reinterpret_cast<float*>(rt_smem);
+    __shared__ float4 red[8];
+    __shared__ float red_ss[8];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const bool rot = a.sign_bits != nullptr, f16 = a.scale_fp16 != 0;
+    const float norm = rot ? a.norm : 1.0f;
+    const uint32_t L = a.lanes;
+    Acc acc;
+
+    for (uint32_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+        // load, factor, signs, stages h = 1 .. 8
+        for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
+            uint32_t w[8];
+            float2 y[8];
+            ld_nc_v8(a.x + ((size_t)r * a.cpr + c) * 8, w);
+            widen16x2(w, y);
+            if (a.col_scale) {
+                const float4* m = reinterpret_cast<const float4*>(a.col_scale) + 4 * c;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = __ldg(m + i);
+                    y[2 * i] = mul2(y[2 * i], make_float2(f.x, f.y));
+                    y[2 * i + 1] = mul2(y[2 * i + 1], make_float2(f.z, f.w));
+                }
+            }
+            if (rot) {
+                apply_signs(y, chunk_sign_bits(a.sign_bits, c));
+                wht16x2(y);
+            }
+            store_chunk_f32(v, c, y);
+        }
+        if (rot) wht_smem_stages(v, a.cols);
+        else __syncthreads();
+
+        if (L == 0) {
+            // one unit: the whole row, reduced over the CTA
+            float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+            for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
+                float2 y[8];
+                load_chunk_f32(v, c, norm, y);
+                if constexpr (F::asym) chunk_minmax(y, mn, mx);
+                else amax = chunk_amax(y, amax);
+            }
+            if constexpr (F::asym) { mn = warp_minf(mn); mx = warp_maxf(mx); }
+            else amax = warp_maxf(amax);
+            if (lane == 0) red[wib] = make_float4(amax, mn, mx, 0.0f);
+            __syncthreads();
+            {
+                const float4 v0 = red[0];
+                amax = v0.x; mn = v0.y; mx = v0.z;
+                for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+                    const float4 q = red[w];
+                    amax = fmaxf(amax, q.x); mn = fminf(mn, q.y); mx = fmaxf(mx, q.z);
+                }
+                if constexpr (F::asym) amax = fmaxf(-mn, mx);
+            }
+            const bool scaled = !plain_sums_ok(amax);
+            const Pow2 pw = pow2_for(amax);
+            const float p = scaled ? pw.p : 1.0f;
+            const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+            const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+            float2 e2 = splat(0.0f), x2 = splat(0.0f);
+            for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
+                float2 y[8];
+                uint32_t q[NW];
+                load_chunk_f32(v, c, norm, y);
+                plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
+                store_codes<FMT>(a.codes, r * a.cpr + c, q);
+            }
+            if (threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, r, ps, f16);
+            add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
+            float ss = __fadd_rn(x2.x, x2.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+            if (lane == 0) red_ss[wib] = ss;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float t = red_ss[0];
+                for (int w = 1; w < (int)(blockDim.x >> 5); ++w) t = __fadd_rn(t, red_ss[w]);
+                kappa_add(acc, __fmul_rn(amax, p), t, a.inv_unit);
+            }
+        } else {
+            // units of L chunks = L adjacent threads (L divides 32; cpr is a multiple of 32)
+            for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
+                float2 y[8];
+                uint32_t q[NW];
+                load_chunk_f32(v, c, norm, y);
+                float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+                if constexpr (F::asym && !MX) chunk_minmax(y, mn, mx);
+                else amax = chunk_amax(y, 0.0f);
+                for (uint32_t o = 1; o < L; o <<= 1) {
+                    if constexpr (F::asym && !MX) {
+                        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                    } else {
+                        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                    }
+                }
+                if constexpr (F::asym && !MX) amax = fmaxf(-mn, mx);
+                const bool scaled = !plain_sums_ok(amax);
+                const Pow2 pw = pow2_for(amax);
+                const float p = scaled ? pw.p : 1.0f;
+                float2 e2 = splat(0.0f), x2 = splat(0.0f);
+                const uint32_t cg = r * a.cpr + c;            // chunk index in the tensor
+                const bool first = (c % L) == 0;
+                if constexpr (MX) {
+                    const int e = ue8m0_exponent<FMT>(amax);
+                    mx_chunk<FMT, K_MX, true>(y, exp2i(-e), exp2i(e), scaled, p, q, e2, x2);
+                    if (first) reinterpret_cast<uint8_t*>(a.scales)[cg / L] = (uint8_t)(e + 127);
+                } else {
+                    const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
+                    const PlainUnit<FMT> u = plain_unit<FMT>(ps);
+                    plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
+                    if (first) store_plain_scale<FMT>(a.scales, a.zps, cg / L, ps, f16);
+                }
+                store_codes<FMT>(a.codes, cg, q);
+                add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
+                float ss = __fadd_rn(x2.x, x2.y);
+                for (uint32_t o = 1; o < L; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+                if (first) kappa_add(acc, __fmul_rn(amax, p), ss, a.inv_unit);
+            }
+        }
+        __syncthreads();             // the row's values are read; the next row may overwrite them
+    }
+    if (a.stats) finish_stats(acc, a.ws, a.stats, false, 0.0f, 0.0, true);
+}
+
+// ---------------------------------------------------------------------------
 // Launchers.
 // ---------------------------------------------------------------------------
 
@@ -1322,6 +1471,26 @@ cudaError_t run_tile2d_hs(bool had, bool stats, const Tile2dArgs& a, cudaStream_
     return stats ? run_tile2d<FMT, false, true, false>(a, st) : run_tile2d<FMT, false, false, false>(a, st);
 }
 
+template <int FMT, bool MX>
+cudaError_t run_rt(const RtArgs& a, cudaStream_t st)
+{
+    constexpr int block = 256;
+    constexpr auto kern = k_quant_rt<FMT, MX>;
+    const size_t smem = (size_t)a.cols * 4;
+    if (smem > 48u * 1024u) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, block, smem) != cudaSuccess || occ < 1) occ = 1;
+    uint64_t grid = (uint64_t)device_sm_count() * (uint64_t)occ;
+    if (grid > a.rows) grid = a.rows;
+    if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, block, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
 template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
@@ -1397,6 +1566,30 @@ cudaError_t launch_quant_tile2d(int fmt, bool had, bool stats, const Tile2dArgs&
     case BQ_UINT4_ASYM: return run_tile2d_hs<BQ_UINT4_ASYM>(had, stats, a, st);
     case BQ_FP8_E4M3:   return run_tile2d_hs<BQ_FP8_E4M3>(had, stats, a, st);
     case BQ_FP8_E5M2:   return run_tile2d_hs<BQ_FP8_E5M2>(had, stats, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_quant_rt(int fmt, bool mx, const RtArgs& a, cudaStream_t st)
+{
+    if (mx) {
+        switch (fmt) {
+        case BQ_INT8_SYM: return run_rt<BQ_INT8_SYM, true>(a, st);
+        case BQ_FP8_E4M3: return run_rt<BQ_FP8_E4M3, true>(a, st);
+        case BQ_FP8_E5M2: return run_rt<BQ_FP8_E5M2, true>(a, st);
+        case BQ_FP4_E2M1: return run_rt<BQ_FP4_E2M1, true>(a, st);
+        case BQ_FP6_E2M3: return run_rt<BQ_FP6_E2M3, true>(a, st);
+        case BQ_FP6_E3M2: return run_rt<BQ_FP6_E3M2, true>(a, st);
+        default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (fmt) {
+    case BQ_INT8_SYM:   return run_rt<BQ_INT8_SYM, false>(a, st);
+    case BQ_INT8_ASYM:  return run_rt<BQ_INT8_ASYM, false>(a, st);
+    case BQ_INT4_SYM:   return run_rt<BQ_INT4_SYM, false>(a, st);
+    case BQ_UINT4_ASYM: return run_rt<BQ_UINT4_ASYM, false>(a, st);
+    case BQ_FP8_E4M3:   return run_rt<BQ_FP8_E4M3, false>(a, st);
+    case BQ_FP8_E5M2:   return run_rt<BQ_FP8_E5M2, false>(a, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -197,6 +197,50 @@ bq_status bq_qsnr(const void* x, int32_t x_dtype, const void* codes, const void*
                   bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Row transforms applied before quantizing ("Quantization survey" §3.2 and §5.2:
+ * SmoothQuant's per-channel factor; §5.3: QuaRot's randomized Hadamard rotation, an
+ * orthogonal R with R^T R = I that spreads outlier channels over the whole row).
+ *  - col_scale (device fp32 [cols], 16-byte aligned, or NULL): x'[i][j] = RN(x[i][j] *
+ *    col_scale[j]), e.g. SmoothQuant's 1/s on activations or s on weights;
+ *  - sign_bits (device uint32 [cols / 32], 4-byte aligned, or NULL for no rotation):
+ *    y = (x' * sigma) H c per row, sigma[j] = -1 where bit j % 32 of word j / 32 is set,
+ *    H the cols-point Walsh-Hadamard matrix in Sylvester order (taken as stages
+ *    h = 1, 2, ..., cols/2 of (a + b, a - b)), c = the fp32 value nearest 1/sqrt(cols).
+ *  - reserved: must be 0.
+ * The arrays are read only (caller-owned).
+ */
+typedef struct bq_row_transform {
+    const float* col_scale;
+    const uint32_t* sign_bits;
+    int64_t reserved;
+} bq_row_transform;
+
+/*
+ * bq_quantize after the row transforms rt (may be NULL: none). Per-row, per-group and
+ * MX schemes with hadamard = 0 (else BQ_ERR_UNSUPPORTED); cols a multiple of 512 up to
+ * 16384, a power of two when rotating (else BQ_ERR_SHAPE). The codes, scales and zero
+ * points are those of the transformed rows. stats (may be NULL; needs a workspace of
+ * bq_workspace_size(..., 1, ...) bytes) holds err2 and x2 summed on the rotated values
+ * (equal to the sums against x' up to fp32 rounding: the rotation is orthogonal) and
+ * kappa over the units' rotated values. One pass over x; a CTA per row at a time.
+ */
+bq_status bq_quantize_rt(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                         const bq_scheme* scheme, const bq_row_transform* rt,
+                         void* codes, void* scales, void* zero_points,
+                         bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dequantize codes written by bq_quantize_rt into out [rows, cols] (BQ_DT_BF16 or
+ * BQ_DT_FP32): the element values, then the inverse rotation (the same stages, times c,
+ * then the signs) when rt->sign_bits is given. The per-column factor is not undone:
+ * out estimates x' (the operand a GEMM with the inverse factor on the other side
+ * takes). Shapes and schemes as bq_quantize_rt.
+ */
+bq_status bq_dequantize_rt(const void* codes, const void* scales, const void* zero_points,
+                           int64_t rows, int64_t cols, const bq_scheme* scheme,
+                           const bq_row_transform* rt, void* out, int32_t out_dtype, void* stream);
+
+/*
  * bq_quantize without a caller-provided workspace, for callers that cannot allocate
  * device memory: code running under another component's allocator (a framework or
  * serving runtime that owns all device memory), code that must not call cudaMalloc

@@ -152,3 +152,30 @@ def test_stats_to_db():
 def test_status_strings():
     for k in range(7):
         assert bq.bq_status_string(k).startswith(bq.STATUS[k])
+
+
+def test_row_transform_checks_before_any_launch():
+    L = bq.lib()
+    fake = 1 << 40
+    ws = ctypes.c_void_p(fake)
+    row = Scheme("int8_sym", "row").c()
+    rt_rot = bq.BqRowTransform(None, fake, 0)
+    def q(scheme, cols, rt, x=fake):
+        return L.bq_quantize_rt(x, 0, 4, cols, ctypes.byref(scheme), rt and ctypes.byref(rt), fake, fake, fake,
+                                None, None, 0, None)
+    # tensor / NV / tile granularities and the block-16 Hadamard are not offered
+    for s in [Scheme("int8_sym", "tensor"), Scheme("e2m1", "nv"), Scheme("e4m3", "tile2d"),
+              Scheme("int8_sym", "row", hadamard=True)]:
+        assert q(s.c(), 512, rt_rot) == 2
+    # widths: a multiple of 512 up to 16384, a power of two when rotating
+    assert q(row, 256, rt_rot) == 3
+    assert q(row, 32768, rt_rot) == 3
+    assert q(row, 1536, rt_rot) == 3
+    # misaligned factor array, misaligned x, reserved field
+    assert q(row, 512, bq.BqRowTransform(fake + 4, None, 0)) == 4
+    assert q(row, 512, rt_rot, x=fake + 16) == 4
+    assert q(row, 512, bq.BqRowTransform(None, fake, 1)) == 1
+    # stats without a workspace
+    assert L.bq_quantize_rt(fake, 0, 4, 512, ctypes.byref(row), ctypes.byref(rt_rot), fake, fake, None,
+                            fake, None, 0, None) == 5
+    assert L.bq_dequantize_rt(fake, fake, None, 4, 1536, ctypes.byref(row), ctypes.byref(rt_rot), fake, 0, None) == 3
