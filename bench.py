@@ -1,7 +1,7 @@
 """Benchmark of the block-scaled quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_tiles_fp8|weight_x50]
+                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_tiles_fp8|weight_rotated|weight_x50]
 
 A step is one pass of the whole path over one synthetic tensor of the workload:
 quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
-KERNEL_SOURCES = ("common.cuh", "quant_ops.cuh", "tma.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu")
+KERNEL_SOURCES = ("common.cuh", "quant_ops.cuh", "tma.cuh", "rot.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu")
 
 # workload -> (generator kwargs, list of (label, scheme args))
 WORKLOADS = {
@@ -64,17 +64,30 @@ WORKLOADS = {
     # scale per 128 x 128 tile (weights), and per 1 x 128 tile (the activation tiling)
     "weight_tiles_fp8": [("e4m3_tile128x128", ("e4m3", "tile2d", 128, "fp32", False)),
                          ("e4m3_tile1x128", ("e4m3", "group", 128, "fp32", False))],
+    # QuaRot-style: the 4096 x 4096 outlier weight under a randomized full-row Hadamard
+    # rotation (random signs, seed 21), then MXFP4 and INT4 group-128
+    "weight_rotated": [("mxfp4_rot", ("e2m1", "mx", 32, "ue8m0", False)),
+                       ("int4_g128_rot", ("int4_sym", "group", 128, "fp32", False))],
     "weight_x50": [("nvfp4", ("e2m1", "nv", 16, "e4m3", False)),
                    ("nvint4", ("int4_sym", "nv", 16, "e4m3", False)),
                    ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
 }
 
 
+# workloads whose schemes all run after the randomized full-row rotation: sign seed
+ROTATED = {"weight_rotated": 21}
+
+
+def rotation_signs(workload: str, cols: int):
+    """The workload's per-column sign flags (uint8 0/1), or None."""
+    return synth.random_signs(cols, ROTATED[workload]) if workload in ROTATED else None
+
+
 def gen_input(workload: str, rank: int) -> torch.Tensor:
     """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
     if workload in ("ffn_lognormal", "ffn_mx_family"):
         return synth.ffn_lognormal(rank)
-    if workload == "weight_tiles_fp8":
+    if workload in ("weight_tiles_fp8", "weight_rotated"):
         return synth.weight_outliers(seed=1 + 1000 * rank)
     gen, _, _ = synth.WORKLOADS[workload]
     base = {"tiny_weight": 0, "weight_outliers": 1, "activations_t3": 2, "weight_x50": 4}[workload]
@@ -246,7 +259,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     schemes = [(lab, Scheme(*a)) for lab, a in WORKLOADS[args.workload]]
     x_host = gen_input(args.workload, rank)
     rows, cols = x_host.shape
+    signs = rotation_signs(args.workload, cols)
+    sign_bits = None if signs is None else bq.pack_sign_bits(signs, device)
     per_scheme_bytes = [kernel_bytes(bq.bq_buffer_sizes(s, rows, cols), rows, cols) for _, s in schemes]
+    if signs is not None:
+        # the sign words are read by both kernels
+        per_scheme_bytes = [(q + cols // 8, d + cols // 8) for q, d in per_scheme_bytes]
     step_bytes = sum(q + d for q, d in per_scheme_bytes)
 
     # buffer sets: inputs + outputs of every kernel, rotated so that each step touches
@@ -269,7 +287,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         """Kernel `kind` ("quantize" / "dequantize" / "qsnr") of scheme j on buffer set i."""
         xi, outs, deqs = sets[i % n_sets]
         s, q = schemes[j][1], outs[j]
-        if kind == "quantize":
+        if sign_bits is not None and kind == "quantize":
+            bq.bq_quantize_rt(xi, s, None, sign_bits, q.codes, q.scales, q.zero_points, q.stats, ws, st)
+        elif sign_bits is not None and kind == "dequantize":
+            bq.bq_dequantize_rt(q.codes, q.scales, q.zero_points, rows, cols, s, None, sign_bits, deqs[j], st)
+        elif kind == "quantize":
             bq.bq_quantize(xi, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, st)
         elif kind == "dequantize":
             bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, deqs[j], st)
@@ -342,7 +364,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for j, (lab, s) in enumerate(schemes):
         qb, db = per_scheme_bytes[j]
         # the standalone QSNR pass (not part of the step) reads what quantize reads and writes
-        for kind, nbytes in (("quantize", qb), ("dequantize", db), ("qsnr", qb)):
+        kinds = (("quantize", qb), ("dequantize", db), ("qsnr", qb))
+        if sign_bits is not None:
+            kinds = kinds[:2]            # the rotated schemes have no standalone QSNR pass
+        for kind, nbytes in kinds:
             def seq(st, j=j, kind=kind):
                 for i in range(n_per):
                     launch(j, kind, args.warmup + i, st)
@@ -385,9 +410,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
         def e2e_step():
             xd.copy_(x_pin, non_blocking=True)
-            for (lab, s), q, dq in zip(schemes, outs, deqs):
-                bq.bq_quantize(xd, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, stream)
-                bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, dq, stream)
+            for j in range(len(schemes)):
+                launch(j, "quantize", 0, stream)
+                launch(j, "dequantize", 0, stream)
             for hs in host_outs:
                 for pair in hs:
                     if pair is not None:
@@ -412,7 +437,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, schemes_args=WORKLOADS[args.workload], x_host=x_host,
-                           budget_s=args.cpu_seconds)
+                           budget_s=args.cpu_seconds, signs=signs)
 
     value = aggregate(step_bytes, world, ms_max)
     if rank != 0:
@@ -433,7 +458,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "data": "synthetic",
         "config": {
             "workload": f"{args.workload} {rows}x{cols} bf16: " + " + ".join(l for l, _ in schemes)
-                        + "; quantize with fused QSNR/kappa, then dequantize to bf16",
+                        + ("; randomized full-row Hadamard rotation," if signs is not None else ";")
+                        + " quantize with fused QSNR/kappa, then dequantize to bf16",
             "rows": rows, "cols": cols,
             "bytes_per_step_per_gpu": step_bytes,
             "l2": f"inputs larger than L2: {n_sets} rotating buffer sets of {set_bytes / 2**20:.1f} MiB",
@@ -460,12 +486,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_step(xb: np.ndarray, schemes_args):
+def oracle_step(xb: np.ndarray, schemes_args, signs=None):
     import oracle
     for _, a in schemes_args:
         s = oracle.Scheme(*a)
-        r = oracle.quantize(xb, s, stats=True)
-        xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], r["tensor_scale"], xb.shape[0], xb.shape[1], s)
+        if signs is not None:
+            r = oracle.quantize_rt(xb, s, signs=signs, stats=True)
+            xh = oracle.dequantize_rt(r["codes"], r["scales"], r["zps"], xb.shape[0], xb.shape[1], s, signs=signs)
+        else:
+            r = oracle.quantize(xb, s, stats=True)
+            xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], r["tensor_scale"], xb.shape[0], xb.shape[1], s)
         oracle.to_bf16_array(xh)
 
 
@@ -478,14 +508,14 @@ def oracle_bytes(schemes_args, rows, cols):
     return tot
 
 
-def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, rows_per_step=None):
+def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, rows_per_step=None, signs=None):
     """Time the oracle, as it stands, on this host (one thread) over whole steps of a
     row sample of the workload tensor, until budget_s is spent (at least 2 steps)."""
     xb = synth.bf16_bits(x_host)
     rows, cols = xb.shape
     if rows_per_step is None:
         t = time.perf_counter()
-        oracle_step(xb[: max(1, rows // 32)], schemes_args)
+        oracle_step(xb[: max(1, rows // 32)], schemes_args, signs)
         per_row = (time.perf_counter() - t) / max(1, rows // 32)
         rows_per_step = int(min(rows, max(16, budget_s / 4 / max(per_row, 1e-9))))
     sample = xb[:rows_per_step]
@@ -493,7 +523,7 @@ def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, rows_per_step=No
     t0 = time.perf_counter()
     n = 0
     while True:
-        oracle_step(sample, schemes_args)
+        oracle_step(sample, schemes_args, signs)
         n += 1
         if n >= 2 and time.perf_counter() - t0 >= budget_s:
             break
@@ -510,19 +540,20 @@ def run_reference(args, rank: int):
     x_host = gen_input(args.workload, 0)
     xb = synth.bf16_bits(x_host)
     rows, cols = xb.shape
+    signs = rotation_signs(args.workload, cols)
     # rows per step so that warmup + steps take about args.cpu_seconds * 6 in total
     t = time.perf_counter()
-    oracle_step(xb[: max(1, rows // 32)], schemes_args)
+    oracle_step(xb[: max(1, rows // 32)], schemes_args, signs)
     per_row = (time.perf_counter() - t) / max(1, rows // 32)
     total_budget = max(30.0, 6 * args.cpu_seconds)
     rows_per_step = int(min(rows, max(16, total_budget / (args.steps + args.warmup) / max(per_row, 1e-9))))
     sample = xb[:rows_per_step]
     nbytes = oracle_bytes(schemes_args, rows_per_step, cols)
     for _ in range(args.warmup):
-        oracle_step(sample, schemes_args)
+        oracle_step(sample, schemes_args, signs)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(sample, schemes_args)
+        oracle_step(sample, schemes_args, signs)
     dt = time.perf_counter() - t0
     value = nbytes * args.steps / dt / 1e9
     desc = (f"first {rows_per_step} of {rows} rows of the {args.workload} tensor per step, "
