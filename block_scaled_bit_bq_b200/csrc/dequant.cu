@@ -433,8 +433,8 @@ template <auto KERN>
 cudaError_t launch_row_kernel(const DequantArgs& a, const uint32_t* sign_bits, uint32_t rows, uint32_t cols,
                               float norm, cudaStream_t st)
 {
-    constexpr int block = 256;
-    const size_t smem = (size_t)cols * 4;
+    const int block = cols / 16 < 256u ? (int)(cols / 16) : 256;   // a thread per chunk, up to 256
+    const size_t smem = (size_t)rot_row_floats(cols) * 4;
     if (smem > 48u * 1024u) {
         const cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

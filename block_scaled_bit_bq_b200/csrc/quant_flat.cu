@@ -1171,18 +1171,35 @@ __global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__
 // factor ("Quantization survey" §3.2, §5.2) and QuaRot's randomized full-row Hadamard
 // rotation (same page §5.3).
 //
-// A CTA of 256 threads owns a row at a time. Thread t loads chunks t, t + 256, ... of
-// the row, multiplies by the factors, negates the signed columns and runs the first
-// four Walsh-Hadamard stages in registers; the row then sits in shared memory as fp32
-// for the remaining stages (wht_smem_stages). The quantize phase reads each chunk back
-// times the normalisation and codes it through the general chunk path (clamping,
-// scaled sums): a scaling unit of L chunks is L adjacent threads, reduced with xor
-// shuffles; a per-row unit is reduced over the CTA. The fused QSNR sums are taken on
-// the rotated values (an orthogonal rotation keeps both sums).
+// A CTA of B = min(256, cols / 16) threads owns a row at a time. Thread t loads chunks
+// t, t + B, ... of the row, multiplies by the factors, negates the signed columns and
+// runs the first four Walsh-Hadamard stages in registers; the row then sits in shared
+// memory as fp32 for the remaining stages (wht_smem_stages). The quantize phase reads
+// each chunk back times the normalisation and codes it (the fast chunk path when the
+// warp's units admit it, else the general one): a scaling unit of L chunks is L
+// adjacent threads, reduced with xor shuffles; a per-row unit is reduced over the
+// CTA. The fused QSNR sums are taken on the rotated values (an orthogonal rotation
+// keeps both sums).
 // ---------------------------------------------------------------------------
 
+// One chunk of a plain unit: the fast path when the warp's units admit it, else the
+// general one (sums added to e2 / x2).
+template <int FMT>
+__device__ __forceinline__ void rt_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, bool general, bool scaled,
+                                         float p, uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
+{
+    if (!general) {
+        float2 ce2, cx2;
+        (void)plain_chunk_fast<FMT, true, false>(y, u, q, ce2, cx2);
+        e2 = add2(e2, ce2);
+        x2 = add2(x2, cx2);
+    } else {
+        plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
+    }
+}
+
 template <int FMT, bool MX>
-__global__ void __launch_bounds__(256) k_quant_rt(const RtArgs a)
+__global__ void __launch_bounds__(256, 3) k_quant_rt(const RtArgs a)
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
@@ -1249,11 +1266,12 @@ __global__ void __launch_bounds__(256) k_quant_rt(const RtArgs a)
             const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
             const PlainUnit<FMT> u = plain_unit<FMT>(ps);
             float2 e2 = splat(0.0f), x2 = splat(0.0f);
+            const bool general = unit_general_fast<FMT, false>(u, scaled);
             for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
                 float2 y[8];
                 uint32_t q[NW];
                 load_chunk_f32(v, c, norm, y);
-                plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
+                rt_chunk<FMT>(y, u, general, scaled, p, q, e2, x2);
                 store_codes<FMT>(a.codes, r * a.cpr + c, q);
             }
             if (threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, r, ps, f16);
@@ -1299,7 +1317,7 @@ __global__ void __launch_bounds__(256) k_quant_rt(const RtArgs a)
                 } else {
                     const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
                     const PlainUnit<FMT> u = plain_unit<FMT>(ps);
-                    plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
+                    rt_chunk<FMT>(y, u, unit_general_fast<FMT, false>(u, scaled), scaled, p, q, e2, x2);
                     if (first) store_plain_scale<FMT>(a.scales, a.zps, cg / L, ps, f16);
                 }
                 store_codes<FMT>(a.codes, cg, q);
@@ -1474,9 +1492,10 @@ cudaError_t run_tile2d_hs(bool had, bool stats, const Tile2dArgs& a, cudaStream_
 template <int FMT, bool MX>
 cudaError_t run_rt(const RtArgs& a, cudaStream_t st)
 {
-    constexpr int block = 256;
+    // a thread per chunk of the row, up to 256 (narrow rows: more CTAs per SM)
+    const int block = a.cpr < 256u ? (int)a.cpr : 256;
     constexpr auto kern = k_quant_rt<FMT, MX>;
-    const size_t smem = (size_t)a.cols * 4;
+    const size_t smem = (size_t)rot_row_floats(a.cols) * 4;
     if (smem > 48u * 1024u) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

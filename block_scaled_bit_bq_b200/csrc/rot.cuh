@@ -8,49 +8,112 @@
 // pass) and runs stages S, 2S, ..., S R / 2 on each group in registers. Every output
 // is a + b or a - b of the same two values as in the sequential stage order, so the
 // result does not depend on how the threads split the work.
+//
+// Layout: element o of chunk c (index 16c + o) sits at
+//   16c + 16 (c >> 4) + 4 (((o >> 2) + (c >> 1)) & 3) + (o & 3),
+// i.e. the chunk's four 16-byte quarters rotated by (c >> 1) & 3, and 16 floats of
+// padding after every 16 chunks. Chunk stores and loads by consecutive threads, and
+// both kinds of pass below, then touch 32 distinct banks per 32 accesses.
 #pragma once
 
 #include "common.cuh"
 
 namespace bq {
 
-template <int R>
-__device__ __forceinline__ void wht_pass(float* v, uint32_t n, uint32_t S)
+// Floats of shared memory for a row of n values.
+__host__ __device__ constexpr uint32_t rot_row_floats(uint32_t n) { return n + n / 16; }
+
+__device__ __forceinline__ uint32_t rot_chunk_base(uint32_t c) { return 16u * c + 16u * (c >> 4); }
+
+// Quarter j of chunk c (its four floats are contiguous).
+__device__ __forceinline__ uint32_t rot_quarter(uint32_t c, uint32_t j)
 {
-    const uint32_t ngroups = n / R;
-    for (uint32_t g = threadIdx.x; g < ngroups; g += blockDim.x) {
-        const uint32_t base = (g % S) + (g / S) * S * R;
-        float t[R];
+    return rot_chunk_base(c) + 4u * ((j + (c >> 1)) & 3u);
+}
+
+// Stage h of R values, two independent groups at once (packed pairs).
+template <int R, int H>
+__device__ __forceinline__ void wht_stage2(float2 (&t)[R])
+{
 #pragma unroll
-        for (int k = 0; k < R; ++k) t[k] = v[base + S * k];
+    for (int i = 0; i < R; i += 2 * H) {
 #pragma unroll
-        for (int h = 1; h < R; h <<= 1) {
-#pragma unroll
-            for (int i = 0; i < R; i += 2 * h) {
-#pragma unroll
-                for (int j = i; j < i + h; ++j) {
-                    const float a = t[j], b = t[j + h];
-                    t[j] = __fadd_rn(a, b);
-                    t[j + h] = __fsub_rn(a, b);
-                }
-            }
+        for (int j = 0; j < H; ++j) {
+            const float2 a = t[i + j], b = t[i + j + H];
+            t[i + j] = add2(a, b);
+            t[i + j + H] = sub2(a, b);
         }
-#pragma unroll
-        for (int k = 0; k < R; ++k) v[base + S * k] = t[k];
     }
 }
 
-// Stages h = 16 .. n / 2 of v[0, n) (16 <= n <= 65536, a power of two). Called by every
-// thread of the block; synchronizes before each pass and at the end.
+// Stages 1 .. R / 2 of R values (R = 2, 4, 8 or 16), two groups at once.
+template <int R>
+__device__ __forceinline__ void wht_group2(float2 (&t)[R])
+{
+    wht_stage2<R, 1>(t);
+    if constexpr (R > 2) wht_stage2<R, 2>(t);
+    if constexpr (R > 4) wht_stage2<R, 4>(t);
+    if constexpr (R > 8) wht_stage2<R, 8>(t);
+}
+
+// A thread takes two adjacent groups at a time: groups 2q and 2q + 1 hold elements o
+// and o + 1 (o even) of the same chunks, which sit side by side (one 8-byte access).
+
+// Stages S .. S R / 2 for stride S >= 256: the chunks of a group are S / 16 apart, a
+// multiple of 16, so each value's quarter rotation is the group's and the k-th value
+// sits (S + S / 16) k floats after the first.
+template <int R>
+__device__ __forceinline__ void wht_pass_wide(float* v, uint32_t n, uint32_t S)
+{
+    const uint32_t npairs = n / (2 * R), step = S + S / 16;
+    for (uint32_t q = threadIdx.x; q < npairs; q += blockDim.x) {
+        const uint32_t g = 2 * q;
+        const uint32_t base = (g % S) + (g / S) * S * R;
+        const uint32_t c = base >> 4, o = base & 15u;
+        float2* p0 = reinterpret_cast<float2*>(v + rot_chunk_base(c) + 4u * (((o >> 2) + (c >> 1)) & 3u) + (o & 3u));
+        float2 t[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) t[k] = p0[(step / 2) * k];
+        wht_group2<R>(t);
+#pragma unroll
+        for (int k = 0; k < R; ++k) p0[(step / 2) * k] = t[k];
+    }
+}
+
+// Stages 16 .. 128 (S = 16, R = 16, n >= 256): group g holds element o = g % 16 of 16
+// consecutive chunks starting at a multiple of 16, so the quarter rotation of the k-th
+// value is ((k >> 1) & 3) past the element's own quarter.
+__device__ __forceinline__ void wht_pass_16(float* v, uint32_t n)
+{
+    const uint32_t npairs = n / 32;
+    for (uint32_t q = threadIdx.x; q < npairs; q += blockDim.x) {
+        const uint32_t o = (2 * q) & 15u, c0 = (q >> 3) * 16u;
+        const uint32_t p0 = rot_chunk_base(c0) + (o & 3u), oq = o >> 2;
+        float2* pm[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) pm[m] = reinterpret_cast<float2*>(v + p0 + 4u * ((oq + (uint32_t)m) & 3u));
+        float2 t[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) t[k] = pm[(k >> 1) & 3][8 * k];
+        wht_group2<16>(t);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pm[(k >> 1) & 3][8 * k] = t[k];
+    }
+}
+
+// Stages h = 16 .. n / 2 of the row in v (256 <= n <= 65536, a power of two). Called by
+// every thread of the block; synchronizes before each pass and at the end.
 __device__ __forceinline__ void wht_smem_stages(float* v, uint32_t n)
 {
-    for (uint32_t S = 16; S < n; S *= 16) {
+    __syncthreads();
+    wht_pass_16(v, n);
+    for (uint32_t S = 256; S < n; S *= 16) {
         const uint32_t R = n / S;
         __syncthreads();
-        if (R >= 16) wht_pass<16>(v, n, S);
-        else if (R == 8) wht_pass<8>(v, n, S);
-        else if (R == 4) wht_pass<4>(v, n, S);
-        else wht_pass<2>(v, n, S);
+        if (R >= 16) wht_pass_wide<16>(v, n, S);
+        else if (R == 8) wht_pass_wide<8>(v, n, S);
+        else if (R == 4) wht_pass_wide<4>(v, n, S);
+        else wht_pass_wide<2>(v, n, S);
     }
     __syncthreads();
 }
@@ -73,20 +136,21 @@ __device__ __forceinline__ uint32_t chunk_sign_bits(const uint32_t* sign_bits, u
 
 __device__ __forceinline__ void store_chunk_f32(float* v, uint32_t c, const float2 (&y)[8])
 {
-    float4* p = reinterpret_cast<float4*>(v + 16 * c);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = make_float4(y[2 * i].x, y[2 * i].y, y[2 * i + 1].x, y[2 * i + 1].y);
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4*>(v + rot_quarter(c, j)) =
+            make_float4(y[2 * j].x, y[2 * j].y, y[2 * j + 1].x, y[2 * j + 1].y);
 }
 
 // Chunk c from shared memory, times s.
 __device__ __forceinline__ void load_chunk_f32(const float* v, uint32_t c, float s, float2 (&y)[8])
 {
-    const float4* p = reinterpret_cast<const float4*>(v + 16 * c);
+    const float2 S = splat(s);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 q = p[i];
-        y[2 * i] = make_float2(__fmul_rn(q.x, s), __fmul_rn(q.y, s));
-        y[2 * i + 1] = make_float2(__fmul_rn(q.z, s), __fmul_rn(q.w, s));
+    for (int j = 0; j < 4; ++j) {
+        const float4 q = *reinterpret_cast<const float4*>(v + rot_quarter(c, j));
+        y[2 * j] = mul2(make_float2(q.x, q.y), S);
+        y[2 * j + 1] = mul2(make_float2(q.z, q.w), S);
     }
 }
 
