@@ -68,3 +68,22 @@ def test_single_process_helpers():
     b = bench.gen_input("tiny_weight", 0)
     import torch
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))   # same seed, same bytes
+
+
+def test_bench_oracle_arm_covers_every_workload():
+    # every bench workload's schemes are valid oracle schemes, and the oracle step (the
+    # cpu_baseline leg and the reference arm) runs on a few rows of each, with the
+    # rotation where the workload asks for it
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    for w, schemes in bench.WORKLOADS.items():
+        rows = 2
+        cols = {"tiny_weight": 1024}.get(w, 4096)
+        x = synth.bf16_bits(synth.normal(rows, cols, seed=5, sigma=0.02))
+        signs = bench.rotation_signs(w, cols)
+        bench.oracle_step(x, schemes, signs)
+        assert bench.oracle_bytes(schemes, rows, cols) > 2 * rows * cols * len(schemes)
+    assert bench.rotation_signs("weight_outliers", 4096) is None
+    s = bench.rotation_signs("weight_rotated", 4096)
+    assert s.shape == (4096,) and set(np.unique(s)) <= {0, 1}
