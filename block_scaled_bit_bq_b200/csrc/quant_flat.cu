@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
 #define BQ_FLAT_WARPS 8
 #endif
 #ifndef BQ_FLAT_NST
-#define BQ_FLAT_NST 3
+#define BQ_FLAT_NST 2
 #endif
 #ifndef BQ_FLAT_MINB
 #define BQ_FLAT_MINB 2
@@ -1012,7 +1012,7 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_rows(co
 // right there, and that tile's kappa is formed from the warps' sums of squares.
 // ---------------------------------------------------------------------------
 
-constexpr int TILE_NST = 3;                                 // tile buffers per CTA
+constexpr int TILE_NST = 2;                                 // tile buffers per CTA
 constexpr uint32_t TBOX_BYTES = TILE * ROW_BYTES;           // 128 rows x 64 bf16 = 16 KiB
 constexpr uint32_t TSTAGE_BYTES = 2 * TBOX_BYTES;           // a whole tile, 32 KiB
 constexpr uint32_t TILE2D_SMEM = TILE_NST * TSTAGE_BYTES + 1024;
