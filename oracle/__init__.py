@@ -93,6 +93,14 @@ def lib() -> ctypes.CDLL:
         L.orc_quantize_rt.argtypes = [vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
         L.orc_dequantize_rt.restype = i32
         L.orc_dequantize_rt.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp]
+        L.orc_gemm_scale_offset.restype = i64
+        L.orc_gemm_scale_offset.argtypes = [i64, i64, i64]
+        L.orc_gemm_scale_bytes.restype = i64
+        L.orc_gemm_scale_bytes.argtypes = [i64, i64]
+        L.orc_scales_to_gemm.restype = None
+        L.orc_scales_to_gemm.argtypes = [vp, i64, i64, vp]
+        L.orc_scales_from_gemm.restype = None
+        L.orc_scales_from_gemm.argtypes = [vp, i64, i64, vp]
         _lib = L
     return _lib
 
@@ -309,4 +317,31 @@ def dequantize_rt(codes, scales, zps, rows: int, cols: int, scheme: Scheme, sign
                                  _ptr(None if zps is None else np.ascontiguousarray(zps)), rows, cols,
                                  a[0], a[1], a[2], a[3], _ptr(sg), _ptr(out))
     _check(rc, "dequantize_rt")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# MX / NV block scales in a block-scaled GEMM's layout (128 x 4 tiles of 512 bytes)
+# ---------------------------------------------------------------------------
+
+def gemm_scale_bytes(rows: int, nb: int) -> int:
+    return int(lib().orc_gemm_scale_bytes(rows, nb))
+
+
+def gemm_scale_offset(r: int, c: int, nb: int) -> int:
+    return int(lib().orc_gemm_scale_offset(r, c, nb))
+
+
+def scales_to_gemm(scales: np.ndarray, rows: int, nb: int, fill: int = 0) -> np.ndarray:
+    """Row-major [rows, nb] uint8 scale codes -> the GEMM layout (padding = fill)."""
+    a = np.ascontiguousarray(scales, dtype=np.uint8).reshape(rows, nb)
+    out = np.full(gemm_scale_bytes(rows, nb), fill, dtype=np.uint8)
+    lib().orc_scales_to_gemm(_ptr(a), rows, nb, _ptr(out))
+    return out
+
+
+def scales_from_gemm(buf: np.ndarray, rows: int, nb: int) -> np.ndarray:
+    b = np.ascontiguousarray(buf, dtype=np.uint8)
+    out = np.zeros((rows, nb), dtype=np.uint8)
+    lib().orc_scales_from_gemm(_ptr(b), rows, nb, _ptr(out))
     return out

@@ -952,3 +952,42 @@ int orc_dequantize_rt(const uint8_t* codes, const void* scales, const void* zps,
     for (int64_t r = 0; r < rows; r++) rt_inverse(out + r * cols, cols, signs);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Block-scale factors in the layout a block-scaled GEMM reads them in          */
+/* ("Quantization survey" §4.3 and the MX/NV recipes: the consumer of the     */
+/* codes is a tensor-core GEMM that scales each 1 x 32 (MX) or 1 x 16 (NV)   */
+/* block). Reading (the scale-factor layout of NVIDIA's block-scaled MMA and  */
+/* its libraries): the scale matrix [rows, nb] (nb blocks per row) is padded   */
+/* to [ceil(rows/128) * 128, ceil(nb/4) * 4] and cut into 128 x 4 tiles of    */
+/* 512 bytes, tiles in row-major order; inside a tile, entry (r, c) sits at   */
+/* byte (r % 32) * 16 + (r / 32) * 4 + c. Padding bytes are not written.      */
+/* ------------------------------------------------------------------------- */
+
+int64_t orc_gemm_scale_offset(int64_t r, int64_t c, int64_t nb)
+{
+    const int64_t tiles_per_row = (nb + 3) / 4;
+    const int64_t tile = (r / 128) * tiles_per_row + c / 4;
+    const int64_t rr = r % 128;
+    return tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (c % 4);
+}
+
+int64_t orc_gemm_scale_bytes(int64_t rows, int64_t nb)
+{
+    return ((rows + 127) / 128) * 128 * ((nb + 3) / 4) * 4;
+}
+
+/* Row-major [rows, nb] scale bytes to the GEMM layout (out has
+ * orc_gemm_scale_bytes(rows, nb) bytes; padding left as it was). */
+void orc_scales_to_gemm(const uint8_t* in, int64_t rows, int64_t nb, uint8_t* out)
+{
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < nb; c++) out[orc_gemm_scale_offset(r, c, nb)] = in[r * nb + c];
+}
+
+/* And back. */
+void orc_scales_from_gemm(const uint8_t* in, int64_t rows, int64_t nb, uint8_t* out)
+{
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < nb; c++) out[r * nb + c] = in[orc_gemm_scale_offset(r, c, nb)];
+}
