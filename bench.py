@@ -1,7 +1,7 @@
 """Benchmark of the block-scaled quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|weight_tiles_fp8|weight_rotated|weight_x50]
+                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|ffn_mx_gemm_operands|weight_tiles_fp8|weight_rotated|weight_x50]
 
 A step is one pass of the whole path over one synthetic tensor of the workload:
 quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
@@ -64,6 +64,10 @@ WORKLOADS = {
     # scale per 128 x 128 tile (weights), and per 1 x 128 tile (the activation tiling)
     "weight_tiles_fp8": [("e4m3_tile128x128", ("e4m3", "tile2d", 128, "fp32", False)),
                          ("e4m3_tile1x128", ("e4m3", "group", 128, "fp32", False))],
+    # GEMM operands: MXFP8 and MXFP4 of the FFN tensor with the block scales written in
+    # the layout a block-scaled tensor-core GEMM reads (128 x 4 tiles)
+    "ffn_mx_gemm_operands": [("mxfp8_e4m3_gemm", ("e4m3", "mx", 32, "ue8m0", False, "gemm")),
+                             ("mxfp4_gemm", ("e2m1", "mx", 32, "ue8m0", False, "gemm"))],
     # QuaRot-style: the 4096 x 4096 outlier weight under a randomized full-row Hadamard
     # rotation (random signs, seed 21), then MXFP4 and INT4 group-128
     "weight_rotated": [("mxfp4_rot", ("e2m1", "mx", 32, "ue8m0", False)),
@@ -85,7 +89,7 @@ def rotation_signs(workload: str, cols: int):
 
 def gen_input(workload: str, rank: int) -> torch.Tensor:
     """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
-    if workload in ("ffn_lognormal", "ffn_mx_family"):
+    if workload in ("ffn_lognormal", "ffn_mx_family", "ffn_mx_gemm_operands"):
         return synth.ffn_lognormal(rank)
     if workload in ("weight_tiles_fp8", "weight_rotated"):
         return synth.weight_outliers(seed=1 + 1000 * rank)
@@ -489,7 +493,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 def oracle_step(xb: np.ndarray, schemes_args, signs=None):
     import oracle
     for _, a in schemes_args:
-        s = oracle.Scheme(*a)
+        s = oracle.Scheme(*a[:5])
         if signs is not None:
             r = oracle.quantize_rt(xb, s, signs=signs, stats=True)
             xh = oracle.dequantize_rt(r["codes"], r["scales"], r["zps"], xb.shape[0], xb.shape[1], s, signs=signs)
@@ -503,7 +507,7 @@ def oracle_bytes(schemes_args, rows, cols):
     import oracle
     tot = 0
     for _, a in schemes_args:
-        q, d = kernel_bytes(oracle.buffer_sizes(oracle.Scheme(*a), rows, cols), rows, cols)
+        q, d = kernel_bytes(oracle.buffer_sizes(oracle.Scheme(*a[:5]), rows, cols), rows, cols)
         tot += q + d
     return tot
 

@@ -26,6 +26,7 @@ DT = {"bf16": 0, "fp16": 1, "fp32": 2, "ue8m0": 3, "e4m3": 4}
 FORMATS = {"int8_sym": 0, "int8_asym": 1, "int4_sym": 2, "uint4_asym": 3, "e4m3": 4, "e5m2": 5, "e2m1": 6,
            "e2m3": 7, "e3m2": 8}
 GRANULARITIES = {"tensor": 0, "row": 1, "group": 2, "mx": 3, "nv": 4, "tile2d": 5}
+LAYOUTS = {"rows": 0, "gemm": 1}       # MX / NV block scales: row-major, or a block-scaled GEMM's tiles
 FOUR_BIT = {"int4_sym", "uint4_asym", "e2m1"}
 ASYMMETRIC = {"int8_asym", "uint4_asym"}
 
@@ -41,7 +42,7 @@ class BqError(RuntimeError):
 
 class BqScheme(ctypes.Structure):
     _fields_ = [("format", ctypes.c_int32), ("granularity", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("scale_dtype", ctypes.c_int32), ("hadamard", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("scale_dtype", ctypes.c_int32), ("hadamard", ctypes.c_int32), ("scale_layout", ctypes.c_int32)]
 
 
 class BqRowTransform(ctypes.Structure):
@@ -102,23 +103,26 @@ def lib() -> ctypes.CDLL:
 @dataclass(frozen=True)
 class Scheme:
     """A quantization scheme: element format, scaling granularity, group size, scale
-    dtype and the Hadamard flag. block / scale_dtype default to the granularity's own
-    (32 / ue8m0 for mx, 16 / e4m3 for nv, 128 / fp32 for tile2d (128 x 128 tiles),
-    fp32 otherwise)."""
+    dtype, the Hadamard flag and the layout of MX / NV block scales ("rows", or "gemm":
+    the tiles a block-scaled GEMM reads). block / scale_dtype default to the
+    granularity's own (32 / ue8m0 for mx, 16 / e4m3 for nv, 128 / fp32 for tile2d
+    (128 x 128 tiles), fp32 otherwise)."""
     fmt: str
     gran: str
     block: int = 0
     scale_dtype: str | None = None
     hadamard: bool = False
+    layout: str = "rows"
 
     def resolved(self) -> "Scheme":
         sd = self.scale_dtype or {"mx": "ue8m0", "nv": "e4m3"}.get(self.gran, "fp32")
         blk = self.block or {"mx": 32, "nv": 16, "tile2d": 128}.get(self.gran, 0)
-        return Scheme(self.fmt, self.gran, blk, sd, bool(self.hadamard))
+        return Scheme(self.fmt, self.gran, blk, sd, bool(self.hadamard), self.layout)
 
     def c(self) -> BqScheme:
         s = self.resolved()
-        return BqScheme(FORMATS[s.fmt], GRANULARITIES[s.gran], s.block, DT[s.scale_dtype], int(s.hadamard), 0)
+        return BqScheme(FORMATS[s.fmt], GRANULARITIES[s.gran], s.block, DT[s.scale_dtype], int(s.hadamard),
+                        LAYOUTS[s.layout])
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:

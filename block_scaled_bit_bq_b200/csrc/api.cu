@@ -23,6 +23,8 @@ struct Plan {
     uint64_t n_scales;
     size_t code_bytes, scale_bytes, zp_bytes, ts_bytes;
     bool needs_range;      // per-tensor and NV schemes take the range pass first
+    bool gemm_layout;      // MX / NV block scales in the GEMM layout
+    uint32_t nb;           // blocks per row (MX / NV)
 };
 
 bool fmt_is_int(int f) { return f == BQ_INT8_SYM || f == BQ_INT8_ASYM || f == BQ_INT4_SYM || f == BQ_UINT4_ASYM; }
@@ -32,7 +34,8 @@ bool fmt_asym(int f) { return f == BQ_INT8_ASYM || f == BQ_UINT4_ASYM; }
 bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
 {
     if (!s) return BQ_ERR_INVALID_ARG;
-    if (s->reserved != 0 || (s->hadamard != 0 && s->hadamard != 1)) return BQ_ERR_INVALID_ARG;
+    if ((s->scale_layout != BQ_LAYOUT_ROWS && s->scale_layout != BQ_LAYOUT_GEMM) ||
+        (s->hadamard != 0 && s->hadamard != 1)) return BQ_ERR_INVALID_ARG;
     if (s->format < BQ_INT8_SYM || s->format > BQ_FP6_E3M2) return BQ_ERR_INVALID_ARG;
     if (s->granularity < BQ_PER_TENSOR || s->granularity > BQ_TILE_2D) return BQ_ERR_INVALID_ARG;
     if (s->scale_dtype < BQ_DT_BF16 || s->scale_dtype > BQ_DT_E4M3) return BQ_ERR_INVALID_ARG;
@@ -73,6 +76,9 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
         p->block = TILE;
         break;
     }
+    p->gemm_layout = s->scale_layout == BQ_LAYOUT_GEMM;
+    if (p->gemm_layout && !(p->gran == BQ_MX_BLOCK || p->gran == BQ_NV_BLOCK)) return BQ_ERR_UNSUPPORTED;
+    if (p->gemm_layout && cols % 128 != 0) return BQ_ERR_SHAPE;
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return BQ_ERR_SHAPE;
     if (p->block && cols % p->block != 0) return BQ_ERR_SHAPE;
     if (rows > 0 && (uint64_t)rows > ((1ull << 36) - 16) / (uint64_t)cols) return BQ_ERR_SHAPE;
@@ -86,6 +92,9 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
     case BQ_TILE_2D: p->n_scales = (((uint64_t)rows + TILE - 1) / TILE) * ((uint64_t)cols / TILE); break;
     default: p->n_scales = p->n / (uint64_t)p->block; break;
     }
+    if (p->gran == BQ_MX_BLOCK || p->gran == BQ_NV_BLOCK) p->nb = (uint32_t)(cols / p->block);
+    if (p->gemm_layout)     // 128 x 4 tiles: rows padded to 128 (nb is a multiple of 4)
+        p->n_scales = (((uint64_t)rows + 127) / 128) * 128 * (uint64_t)p->nb;
     const size_t se = (p->sdt == BQ_DT_FP32) ? 4 : (p->sdt == BQ_DT_FP16) ? 2 : 1;
     p->code_bytes = p->four ? p->n / 2 : p->n;
     p->scale_bytes = p->n_scales * se;
@@ -137,6 +146,7 @@ DequantArgs dequant_args(const Plan& p, int64_t cols)
         a.fd_s = f.s;
     }
     a.tile_cols = p.gran == BQ_TILE_2D ? (uint32_t)(cols / TILE) : 0u;
+    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     return a;
 }
@@ -294,6 +304,7 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     a.n_elems = (double)p.n;
     a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
+    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
     return cuda_status(launch_quant_flat(p.fmt, kind_of(p.gran), p.had != 0, want_stats, a, s));
 }
 
@@ -397,6 +408,7 @@ bq_status bq_quantize_rt(const void* x, int32_t x_dtype, int64_t rows, int64_t c
     a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
     a.norm = rt_norm(cols);
     a.inv_unit = 1.0f / (float)(p.gran == BQ_PER_ROW ? cols : p.block);
+    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
     return cuda_status(launch_quant_rt(p.fmt, p.gran == BQ_MX_BLOCK, a, s));
 }
 

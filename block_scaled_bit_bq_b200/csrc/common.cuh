@@ -413,6 +413,21 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f)
     return (uint32_t)(t >> f.s);
 }
 
+// Block scales in a block-scaled GEMM's layout: the [rows, nb] scale matrix in 128 x 4
+// tiles of 512 bytes (row-major tile order), entry (r, c) of a tile at byte
+// (r % 32) * 16 + (r / 32) * 4 + c. nb is a multiple of 4 here.
+__host__ __device__ inline uint32_t gemm_scale_offset(uint32_t r, uint32_t c, uint32_t nb)
+{
+    return (((r >> 7) * (nb >> 2) + (c >> 2)) << 9) + ((r & 31u) << 4) + (((r >> 5) & 3u) << 2) + (c & 3u);
+}
+
+// The same for the flat unit index u = r * nb + c (nb_div: fast division by nb).
+__device__ __forceinline__ uint32_t gemm_unit_offset(uint32_t u, const FastDiv& nb_div)
+{
+    const uint32_t r = fast_div(u, nb_div);
+    return gemm_scale_offset(r, u - r * nb_div.d, nb_div.d);
+}
+
 // ---------------------------------------------------------------------------
 // Workspace layout and the cross-CTA reduction (last CTA finishes; no waiting).
 // ---------------------------------------------------------------------------

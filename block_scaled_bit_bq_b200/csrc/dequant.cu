@@ -110,6 +110,9 @@ template <int FMT, int SK>
 __device__ __forceinline__ UnitScale load_unit_scale(const DequantArgs& d, uint32_t c)
 {
     uint32_t u = d.chunks_per_unit == 0 ? 0u : (uint32_t)(((uint64_t)__umulhi(c, d.fd_m) + c) >> d.fd_s);
+    if constexpr (SK == SK_UE8M0 || SK == SK_NV) {
+        if (d.gemm_layout) u = gemm_unit_offset(u, d.gemm_nb);
+    }
     if constexpr (SK == SK_F32 || SK == SK_F16) {
         if (d.tile_cols) {
             // u is the chunk's row: tile (row / 128, column / 128), 8 chunks per tile column

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include "bq.h"
+#include "common.cuh"
 
 namespace bq {
 
@@ -25,6 +26,8 @@ struct FlatArgs {
     int32_t scale_fp16;         // 1: fp16 scales and zero points
     double n_elems;
     float inv_unit;             // 1 / elements per scaling unit (kappa)
+    FastDiv gemm_nb;            // MX / NV scales in the GEMM layout: division by blocks per row
+    int32_t gemm_layout;        // 1: scales in the GEMM layout; 0: row-major
 };
 
 // Per-row kernel: one CTA per row at a time.
@@ -94,6 +97,8 @@ struct RtArgs {
     int32_t scale_fp16;
     float norm;                 // rotation: the fp32 value nearest 1 / sqrt(cols)
     float inv_unit;             // 1 / elements per unit (kappa)
+    FastDiv gemm_nb;            // MX scales in the GEMM layout (see FlatArgs)
+    int32_t gemm_layout;
 };
 
 struct DequantArgs {
@@ -112,6 +117,8 @@ struct DequantArgs {
     uint32_t fd_m, fd_s;        // fast division by chunks_per_unit
     uint32_t tile_cols;         // 2-D tiles: tiles per tile row (cols / TILE); else 0
     int32_t scale_fp16;
+    FastDiv gemm_nb;            // MX / NV scales in the GEMM layout (see FlatArgs)
+    int32_t gemm_layout;
 };
 
 // Scale kinds for dequantize / QSNR.

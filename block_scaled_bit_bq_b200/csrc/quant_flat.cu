@@ -830,19 +830,27 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         store_span4<FMT>(a.codes, span, a.n_chunks, span4);
         const uint32_t c0 = SPAN * span;
         if constexpr (GK == K_NV) {
-            // four E4M3 block scales, one per chunk
+            // four E4M3 block scales, one per chunk (in the GEMM layout: four adjacent
+            // bytes, the span's first block being a multiple of 4 in its row)
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
-            if (c0 + SPAN <= a.n_chunks)
+            if (a.gemm_layout) {
+                if (c0 < a.n_chunks) *reinterpret_cast<uint32_t*>(sc + gemm_unit_offset(c0, a.gemm_nb)) = scodes;
+            } else if (c0 + SPAN <= a.n_chunks) {
                 *reinterpret_cast<uint32_t*>(sc + c0) = scodes;
-            else
+            } else {
                 for (int k = 0; k < SPAN; ++k)
                     if (c0 + k < a.n_chunks) sc[c0 + k] = (uint8_t)(scodes >> (8 * k));
+            }
         } else if constexpr (GK == K_MX) {
+            // two UE8M0 block scales (in the GEMM layout: two adjacent bytes)
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
-            if (c0 + SPAN <= a.n_chunks)
+            if (a.gemm_layout) {
+                if (c0 < a.n_chunks) *reinterpret_cast<uint16_t*>(sc + gemm_unit_offset(c0 / 2, a.gemm_nb)) = (uint16_t)scodes;
+            } else if (c0 + SPAN <= a.n_chunks) {
                 *reinterpret_cast<uint16_t*>(sc + c0 / 2) = (uint16_t)scodes;
-            else if (c0 < a.n_chunks)
+            } else if (c0 < a.n_chunks) {
                 sc[c0 / 2] = (uint8_t)scodes;
+            }
         }
     }
     if (!ok) {
@@ -1319,7 +1327,11 @@ __global__ void __launch_bounds__(256, 3) k_quant_rt(const RtArgs a)
                 if constexpr (MX) {
                     const int e = ue8m0_exponent<FMT>(amax);
                     mx_chunk<FMT, K_MX, true>(y, exp2i(-e), exp2i(e), scaled, p, q, e2, x2);
-                    if (first) reinterpret_cast<uint8_t*>(a.scales)[cg / L] = (uint8_t)(e + 127);
+                    if (first) {
+                        const uint32_t u = cg / L;
+                        reinterpret_cast<uint8_t*>(a.scales)[a.gemm_layout ? gemm_unit_offset(u, a.gemm_nb) : u] =
+                            (uint8_t)(e + 127);
+                    }
                 } else {
                     const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
                     const PlainUnit<FMT> u = plain_unit<FMT>(ps);

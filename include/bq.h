@@ -54,6 +54,7 @@
  *  - scales: per tensor 1 value; per row [rows]; per group [rows, cols/block]; 2-D
  *    tiles [ceil(rows/128), cols/128] (tile (i, j) covers rows 128i.., columns 128j..);
  *    MX uint8 [rows, cols/32] (UE8M0 codes); NV uint8 [rows, cols/16] (E4M3 codes);
+ *    MX / NV with scale_layout = BQ_LAYOUT_GEMM: the GEMM tile layout below;
  *    fp32 or fp16 as scheme.scale_dtype says for the first four;
  *  - zero points (asymmetric formats only): same shape and dtype as the scales,
  *    holding exact integers;
@@ -121,8 +122,20 @@ typedef struct bq_scheme {
     int32_t scale_dtype;  /* BQ_DT_FP32 or BQ_DT_FP16 (tensor/row/group),        */
                           /* BQ_DT_UE8M0 (MX), BQ_DT_E4M3 (NV)                    */
     int32_t hadamard;     /* 0 or 1: rotate each 16-run by H16/4 before scaling  */
-    int32_t reserved;     /* must be 0                                           */
+    int32_t scale_layout; /* BQ_LAYOUT_ROWS (0) or BQ_LAYOUT_GEMM (1, MX / NV)   */
 } bq_scheme;
+
+/* Layout of the MX / NV block scales (scale_layout):
+ *  - BQ_LAYOUT_ROWS: row-major [rows, nb] bytes (nb = cols / 32 for MX, cols / 16 for NV);
+ *  - BQ_LAYOUT_GEMM: the layout a block-scaled tensor-core GEMM reads its scale factors
+ *    in, so the codes and scales go to the GEMM as they are (the scale-factor layout of
+ *    NVIDIA's block-scaled MMA and its libraries, e.g. cuBLASLt's and torch's 32x4x4
+ *    swizzle): the matrix padded to [ceil(rows / 128) * 128, nb] and cut into 128 x 4
+ *    tiles of 512 bytes in row-major tile order; entry (r, c) of a tile sits at byte
+ *    (r % 32) * 16 + (r / 32) * 4 + c. Needs cols % 128 == 0 (nb a multiple of 4);
+ *    padding bytes (rows past the last) are not written. Dequantize and QSNR read the
+ *    same layout. Other granularities: BQ_ERR_UNSUPPORTED. */
+enum { BQ_LAYOUT_ROWS = 0, BQ_LAYOUT_GEMM = 1 };
 
 /* QSNR and crest-factor sums, written by the library into caller device memory.
  * err2 = sum (x - xhat)^2 and x2 = sum x^2 over the whole tensor (original domain);

@@ -47,6 +47,19 @@ SCHEMES = [
     Scheme("e4m3", "tile2d"), Scheme("uint4_asym", "tile2d", scale_dtype="fp16"), Scheme("int4_sym", "tile2d"),
 ]
 
+GEMM_SCHEMES = [Scheme("e4m3", "mx", layout="gemm"), Scheme("e2m1", "mx", layout="gemm"),
+                Scheme("e2m1", "nv", layout="gemm"), Scheme("int8_sym", "mx", layout="gemm")]
+
+
+@pytest.mark.parametrize("s", GEMM_SCHEMES, ids=str)
+@pytest.mark.parametrize("shape", [(1, 128), (130, 1024), (4096, 4096)])
+def test_gemm_layout_buffer_sizes(s, shape):
+    rows, cols = shape
+    o = oracle.Scheme(s.fmt, s.gran, s.block, s.scale_dtype, s.hadamard)
+    cb, sb, zb, tb = oracle.buffer_sizes(o, rows, cols)
+    nb = cols // (32 if s.gran == "mx" else 16)
+    assert bq.bq_buffer_sizes(s, rows, cols) == (cb, oracle.gemm_scale_bytes(rows, nb), zb, tb)
+
 
 @pytest.mark.parametrize("s", SCHEMES, ids=str)
 @pytest.mark.parametrize("shape", [(1, 512), (37, 1024), (4096, 4096), (0, 512)])
@@ -93,6 +106,10 @@ def _status(fn, *args):
     (Scheme("int8_sym", "tile2d", 64), (4, 128), 2),
     (Scheme("int8_sym", "tile2d", scale_dtype="ue8m0"), (4, 128), 2),
     (Scheme("int8_sym", "tile2d"), (4, 192), 3),
+    (Scheme("int8_sym", "row", layout="gemm"), (4, 128), 2),
+    (Scheme("e4m3", "group", 32, layout="gemm"), (4, 128), 2),
+    (Scheme("e4m3", "mx", layout="gemm"), (4, 96), 3),
+    (Scheme("e2m1", "nv", layout="gemm"), (4, 112), 3),
 ])
 def test_invalid_schemes_and_shapes(s, shape, want):
     assert _status(bq.bq_buffer_sizes, s, *shape) == want
@@ -101,7 +118,7 @@ def test_invalid_schemes_and_shapes(s, shape, want):
 def test_bad_enum_and_reserved():
     L = bq.lib()
     z = ctypes.c_size_t(0)
-    for f in [(9, 0, 0, 2, 0, 0), (0, 7, 0, 2, 0, 0), (0, 6, 0, 2, 0, 0), (0, 1, 0, 2, 2, 0), (0, 1, 0, 2, 0, 1), (0, 1, 0, 9, 0, 0)]:
+    for f in [(9, 0, 0, 2, 0, 0), (0, 7, 0, 2, 0, 0), (0, 6, 0, 2, 0, 0), (0, 1, 0, 2, 2, 0), (0, 1, 0, 2, 0, 2), (0, 1, 0, 9, 0, 0)]:
         sc = bq.BqScheme(*f)
         assert L.bq_buffer_sizes(ctypes.byref(sc), 4, 64, ctypes.byref(z), None, None, None) == 1
     assert L.bq_buffer_sizes(None, 4, 64, ctypes.byref(z), None, None, None) == 1
