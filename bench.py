@@ -284,10 +284,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         outs = [bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes]
         deqs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in schemes]
         sets.append((xi, outs, deqs))
-    ws = bq.new_workspace(device)
     stream = torch.cuda.current_stream(device)
+    # the schemes of a step are independent: with two or more, they run as two lanes
+    # (even schemes on the launching stream, odd ones on a side stream, each lane with its
+    # own workspace), forked and joined inside the step, so one lane's kernels fill the
+    # other's ramp and tail
+    n_lanes = 1 if (args.serial or len(schemes) < 2) else 2
+    wss = [bq.new_workspace(device) for _ in range(n_lanes)]
+    side = torch.cuda.Stream(device) if n_lanes > 1 else None
+    ws = wss[0]
 
-    def launch(j, kind, i, st):
+    def launch(j, kind, i, st, ws=ws):
         """Kernel `kind` ("quantize" / "dequantize" / "qsnr") of scheme j on buffer set i."""
         xi, outs, deqs = sets[i % n_sets]
         s, q = schemes[j][1], outs[j]
@@ -304,9 +311,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     def step(i, st=None):
         st = st or stream
+        if n_lanes == 1:
+            for j in range(len(schemes)):
+                launch(j, "quantize", i, st)
+                launch(j, "dequantize", i, st)
+            return
+        side.wait_stream(st)
         for j in range(len(schemes)):
-            launch(j, "quantize", i, st)
-            launch(j, "dequantize", i, st)
+            lane_st, lane_ws = (st, wss[0]) if j % 2 == 0 else (side, wss[1])
+            launch(j, "quantize", i, lane_st, lane_ws)
+            launch(j, "dequantize", i, lane_st, lane_ws)
+        st.wait_stream(side)
 
     for i in range(args.warmup):
         step(i)
@@ -414,9 +429,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
         def e2e_step():
             xd.copy_(x_pin, non_blocking=True)
-            for j in range(len(schemes)):
-                launch(j, "quantize", 0, stream)
-                launch(j, "dequantize", 0, stream)
+            step(0, stream)
             for hs in host_outs:
                 for pair in hs:
                     if pair is not None:
@@ -469,6 +482,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "l2": f"inputs larger than L2: {n_sets} rotating buffer sets of {set_bytes / 2**20:.1f} MiB",
             "parallelism": f"dp{world} (one independent tensor per GPU, no collective on the data path)",
             "launch": "eager" if graph is None else "CUDA graph of the K timed steps",
+            "streams": (f"{n_lanes} (the step's independent schemes alternate between two streams, "
+                        "forked and joined inside the step)") if n_lanes > 1 else "1",
             "kernel_timing": f"each kernel alone, {n_per} launches back to back over the rotating sets",
         },
         "pct_hbm_peak": round(100.0 * value / world / peak, 2),
@@ -592,6 +607,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="weight_outliers")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--serial", action="store_true", help="run the step's schemes one after another on one stream")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps one by one instead of as a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
