@@ -873,9 +873,10 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
 // The row reaches shared memory as M = ceil(cols / 2048) tiles of a 3-D tensor map (x
 // as [rows][cols / 64][64]; a box is 32 segments of 64 elements of one row, zero past
 // the row's end), lane l taking segment l of each tile (four chunks, as in the flat
-// kernel). The tiles pass through the warp's ring twice: for the row's range, then
-// (from L2) for the codes, so the ring needs no room for a whole row. One scale per
-// row, computed by every lane from the warp's reduced range.
+// kernel). A row of at most NST tiles is loaded once and read twice from the ring (range,
+// then codes); a longer row passes through the ring twice (the second time from L2), so
+// the ring needs no room for a whole row. One scale per row, computed by every lane
+// from the warp's reduced range.
 // ---------------------------------------------------------------------------
 
 // CTAs of 4 warps, 4 per SM (the same 16 warps per SM as the flat kernel): with 1-2
@@ -899,7 +900,11 @@ __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_
     const uint32_t nwarps = gridDim.x * ROWS_WARPS;
     const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
     const uint32_t bar0 = smem_addr(&bars[wib][0]);
-    const uint32_t M = a.tiles, L = 2 * a.tiles;         // tiles per row, loads per row
+    // tiles per row; a row of at most NST tiles stays in the ring for both passes
+    // (loaded once), a longer one is loaded again (from L2) for the codes
+    const uint32_t M = a.tiles;
+    const bool resident = M <= (uint32_t)NST;
+    const uint32_t L = resident ? M : 2 * M;             // loads per row
 
     if (lane == 0) {
         for (int s = 0; s < NST; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -935,6 +940,7 @@ __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_
     uint32_t k = 0;
     int s = 0;
     for (uint32_t r = warp; r < a.rows && ok; r += nwarps) {
+        const int s_row = s;                              // the row's first stage
         // pass 1: the lane's part of the row's range
         float amax = 0.0f, mn = 0.0f, mx = 0.0f;
         uint32_t plo = 0u, phi = 0u, pm = 0u;            // packed bf16 pairs
@@ -957,11 +963,14 @@ __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_
                 }
             }
             __syncwarp();
-            issue(k + NST, s);
-            ++k;
+            if (!resident) {
+                issue(k + NST, s);
+                ++k;
+            }
             s = (s + 1 == NST) ? 0 : s + 1;
         }
         if (!ok) break;
+        if (resident) s = s_row;                          // the codes read the same stages
         if constexpr (!HAD) {
             if constexpr (F::asym) { mn = pair_min(plo); mx = pair_max(phi); }
             else amax = pair_absmax(pm);
@@ -978,7 +987,7 @@ __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_
 
         // pass 2: codes
         for (uint32_t j = 0; j < M; ++j) {
-            if (!wait_stage(s)) { ok = false; break; }
+            if (!resident && !wait_stage(s)) { ok = false; break; }
             const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
             const uint32_t g = j * 32 + lane;                    // the lane's segment
             const bool seg_ok = g < a.nseg;
