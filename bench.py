@@ -17,7 +17,7 @@ e2e: the same bytes / step time when every step also copies its input from pinne
 memory and reads its quantized outputs and QSNR sums back.
 
 Under torchrun (N > 1) each rank drives cuda:LOCAL_RANK; times are the max over ranks.
---impl reference times the CPU oracle (the reference of this build) on rank 0.
+--impl reference times the CPU oracle (the reference implementation here) on rank 0.
 """
 
 from __future__ import annotations
