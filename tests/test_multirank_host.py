@@ -87,3 +87,21 @@ def test_bench_oracle_arm_covers_every_workload():
     assert bench.rotation_signs("weight_outliers", 4096) is None
     s = bench.rotation_signs("weight_rotated", 4096)
     assert s.shape == (4096,) and set(np.unique(s)) <= {0, 1}
+
+
+def test_reference_arm_prints_the_contract_line():
+    # bench.py --impl reference: the oracle timed on this host, one JSON line with the
+    # contract's keys (no GPU needed)
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "tiny_weight", "--steps", "3", "--warmup", "3", "--cpu-seconds", "1"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["steps"] == 3 and d["warmup"] == 3
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["value"] == d["value"] and "rows" in d["cpu_baseline"]["sample"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"].startswith("tiny_weight 256x1024")
