@@ -93,8 +93,10 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
     default: p->n_scales = p->n / (uint64_t)p->block; break;
     }
     if (p->gran == BQ_MX_BLOCK || p->gran == BQ_NV_BLOCK) p->nb = (uint32_t)(cols / p->block);
-    if (p->gemm_layout)     // 128 x 4 tiles: rows padded to 128 (nb is a multiple of 4)
+    if (p->gemm_layout) {   // 128 x 4 tiles: rows padded to 128 (nb is a multiple of 4)
         p->n_scales = (((uint64_t)rows + 127) / 128) * 128 * (uint64_t)p->nb;
+        if (p->n_scales > 0xFFFFFFFFull) return BQ_ERR_SHAPE;    // byte offsets are 32-bit
+    }
     const size_t se = (p->sdt == BQ_DT_FP32) ? 4 : (p->sdt == BQ_DT_FP16) ? 2 : 1;
     p->code_bytes = p->four ? p->n / 2 : p->n;
     p->scale_bytes = p->n_scales * se;

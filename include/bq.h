@@ -132,7 +132,8 @@ typedef struct bq_scheme {
  *    NVIDIA's block-scaled MMA and its libraries, e.g. cuBLASLt's and torch's 32x4x4
  *    swizzle): the matrix padded to [ceil(rows / 128) * 128, nb] and cut into 128 x 4
  *    tiles of 512 bytes in row-major tile order; entry (r, c) of a tile sits at byte
- *    (r % 32) * 16 + (r / 32) * 4 + c. Needs cols % 128 == 0 (nb a multiple of 4);
+ *    (r % 32) * 16 + (r / 32) * 4 + c. Needs cols % 128 == 0 (nb a multiple of 4) and
+ *    fewer than 2^32 padded scale bytes (else BQ_ERR_SHAPE);
  *    padding bytes (rows past the last) are not written. Dequantize and QSNR read the
  *    same layout. Other granularities: BQ_ERR_UNSUPPORTED. */
 enum { BQ_LAYOUT_ROWS = 0, BQ_LAYOUT_GEMM = 1 };

@@ -110,6 +110,8 @@ def _status(fn, *args):
     (Scheme("e4m3", "group", 32, layout="gemm"), (4, 128), 2),
     (Scheme("e4m3", "mx", layout="gemm"), (4, 96), 3),
     (Scheme("e2m1", "nv", layout="gemm"), (4, 112), 3),
+    # one row of 2^31 - 128 columns: 2^36 padded scale bytes, past 32-bit offsets
+    (Scheme("e2m1", "nv", layout="gemm"), (1, (1 << 31) - 128), 3),
 ])
 def test_invalid_schemes_and_shapes(s, shape, want):
     assert _status(bq.bq_buffer_sizes, s, *shape) == want
