@@ -237,6 +237,9 @@ typedef struct bq_row_transform {
  * bq_workspace_size(..., 1, ...) bytes) holds err2 and x2 summed on the rotated values
  * (equal to the sums against x' up to fp32 rounding: the rotation is orthogonal) and
  * kappa over the units' rotated values. One pass over x; a CTA per row at a time.
+ * Pointers and alignment as bq_quantize (tensor_scale is not used), plus the arrays'
+ * alignment above (BQ_ERR_ALIGNMENT); rt->reserved != 0 gives BQ_ERR_INVALID_ARG. MX
+ * scales may take scale_layout = BQ_LAYOUT_GEMM.
  */
 bq_status bq_quantize_rt(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
                          const bq_scheme* scheme, const bq_row_transform* rt,
