@@ -1,20 +1,31 @@
 """Benchmark of the block-scaled quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload weight_outliers|tiny_weight|activations_t3|ffn_lognormal|ffn_mx_family|ffn_mx_gemm_operands|weight_tiles_fp8|weight_rotated|weight_x50]
+                    [--workload ffn_lognormal|weight_outliers|tiny_weight|activations_t3|ffn_mx_family|
+                                ffn_mx_gemm_operands|weight_tiles_fp8|weight_rotated|weight_x50]
+                    [--tensors T]
 
-A step is one pass of the whole path over one synthetic tensor of the workload:
-quantize (with fused QSNR and crest-factor sums) under each of the workload's schemes,
-then dequantize each result to bf16. The default workload is the 4096 x 4096 weight
-(N(0, 0.02^2) with 0.1% entries +-U(0.1, 0.2)) under UINT4 group-128 asymmetric
-(fp16 scale + zero) and INT8 per-output-channel symmetric.
+The default workload is the FFN set at full size: 64 bf16 tensors of 4096 x 11008
+(N(0, 1) times a per-row lognormal(0, 0.5) gain, seeds 3..66; the Llama-7B FFN shape of
+"INT vs FP at fine granularity" §4.2) under MXINT8 and MXFP8 E4M3 (block 32 along rows,
+UE8M0 scales).
 
-value: algorithmic bytes of every kernel of a step (bytes each kernel must read plus
-bytes it must write) / step time, summed over ranks (weak scaling: each rank owns an
-independent tensor), with inputs resident in HBM. Inputs rotate over enough buffer sets
-that every step reads data last touched more than 4 x L2 ago.
-e2e: the same bytes / step time when every step also copies its input from pinned host
-memory and reads its quantized outputs and QSNR sums back.
+A step is one pass of the quantize path over the workload's tensors: for every tensor
+and every scheme, bq_quantize with the fused QSNR and crest-factor sums (bf16 load,
+optional block-16 rotation, ranges, scales, codes, packing and the QSNR partial sums;
+per-tensor and NV schemes take their range pass first).
+value: quantize GB/s = algorithmic bytes of every quantize call of a step (x read once,
+codes, scales, zero points and tensor scales written) / step time, summed over ranks
+(weak scaling: each rank owns its own tensors), with inputs resident in HBM. The 64
+distinct FFN tensors (5.8 GB) already exceed 4 x L2; single-tensor workloads rotate over
+enough copies that every step reads data last touched more than 4 x L2 ago.
+full_path: the same with the dequantize of every result to bf16 added to the step.
+kernels: each kernel alone (quantize; for per-tensor / NV schemes also the range pass
+and the quantize pass separately; dequantize; the standalone QSNR pass), launches back
+to back over inputs rotating with a reuse distance of more than 4 x L2 of that
+kernel's own bytes.
+e2e: quantize GB/s when every step also copies its inputs from pinned host memory and
+reads the codes, scales, zero points, tensor scales and QSNR sums back to the host.
 
 Under torchrun (N > 1) each rank drives cuda:LOCAL_RANK; times are the max over ranks.
 --impl reference times the CPU oracle (the reference implementation here) on rank 0.
@@ -32,6 +43,7 @@ import subprocess
 import sys
 import threading
 import time
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -44,8 +56,10 @@ import synth  # noqa: E402
 METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
 KERNEL_SOURCES = ("common.cuh", "quant_ops.cuh", "tma.cuh", "rot.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu")
 
-# workload -> (generator kwargs, list of (label, scheme args))
+# workload -> list of (label, scheme args)
 WORKLOADS = {
+    "ffn_lognormal": [("mxint8", ("int8_sym", "mx", 32, "ue8m0", False)),
+                      ("mxfp8_e4m3", ("e4m3", "mx", 32, "ue8m0", False))],
     "weight_outliers": [("uint4_g128_asym", ("uint4_asym", "group", 128, "fp16", False)),
                         ("int8_row_sym", ("int8_sym", "row", 0, "fp32", False))],
     "tiny_weight": [("int8_tensor_sym", ("int8_sym", "tensor", 0, "fp32", False)),
@@ -54,9 +68,7 @@ WORKLOADS = {
                        ("e5m2_tensor", ("e5m2", "tensor", 0, "fp32", False)),
                        ("e4m3_token", ("e4m3", "row", 0, "fp32", False)),
                        ("e5m2_token", ("e5m2", "row", 0, "fp32", False))],
-    "ffn_lognormal": [("mxint8", ("int8_sym", "mx", 32, "ue8m0", False)),
-                      ("mxfp8_e4m3", ("e4m3", "mx", 32, "ue8m0", False))],
-    # the rest of the MX family on the same FFN tensor (MXFP4 and MXFP6)
+    # the rest of the MX family on the FFN tensors (MXFP4 and MXFP6)
     "ffn_mx_family": [("mxfp4", ("e2m1", "mx", 32, "ue8m0", False)),
                       ("mxfp6_e2m3", ("e2m3", "mx", 32, "ue8m0", False)),
                       ("mxfp6_e3m2", ("e3m2", "mx", 32, "ue8m0", False))],
@@ -64,7 +76,7 @@ WORKLOADS = {
     # scale per 128 x 128 tile (weights), and per 1 x 128 tile (the activation tiling)
     "weight_tiles_fp8": [("e4m3_tile128x128", ("e4m3", "tile2d", 128, "fp32", False)),
                          ("e4m3_tile1x128", ("e4m3", "group", 128, "fp32", False))],
-    # GEMM operands: MXFP8 and MXFP4 of the FFN tensor with the block scales written in
+    # GEMM operands: MXFP8 and MXFP4 of the FFN tensors with the block scales written in
     # the layout a block-scaled tensor-core GEMM reads (128 x 4 tiles)
     "ffn_mx_gemm_operands": [("mxfp8_e4m3_gemm", ("e4m3", "mx", 32, "ue8m0", False, "gemm")),
                              ("mxfp4_gemm", ("e2m1", "mx", 32, "ue8m0", False, "gemm"))],
@@ -77,6 +89,9 @@ WORKLOADS = {
                    ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
 }
 
+FFN_WORKLOADS = ("ffn_lognormal", "ffn_mx_family", "ffn_mx_gemm_operands")
+# tensors per step: the FFN set is 64 tensors; the other workloads are one tensor
+DEFAULT_TENSORS = {"ffn_lognormal": 64, "ffn_mx_family": 64, "ffn_mx_gemm_operands": 64}
 
 # workloads whose schemes all run after the randomized full-row rotation: sign seed
 ROTATED = {"weight_rotated": 21}
@@ -87,15 +102,18 @@ def rotation_signs(workload: str, cols: int):
     return synth.random_signs(cols, ROTATED[workload]) if workload in ROTATED else None
 
 
-def gen_input(workload: str, rank: int) -> torch.Tensor:
-    """The rank's tensor: the workload's generator with its seed shifted by 1000 * rank."""
-    if workload in ("ffn_lognormal", "ffn_mx_family", "ffn_mx_gemm_operands"):
-        return synth.ffn_lognormal(rank)
+def gen_inputs(workload: str, rank: int, n_tensors: int):
+    """The rank's tensors (CPU bf16). FFN: tensors t = 64 * rank + i (seed 3 + t), drawn in
+    parallel; else one tensor with the workload's seed shifted by 1000 * rank."""
+    if workload in FFN_WORKLOADS:
+        ids = [n_tensors * rank + i for i in range(n_tensors)]
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            return list(ex.map(synth.ffn_lognormal, ids))
     if workload in ("weight_tiles_fp8", "weight_rotated"):
-        return synth.weight_outliers(seed=1 + 1000 * rank)
+        return [synth.weight_outliers(seed=1 + 1000 * rank)]
     gen, _, _ = synth.WORKLOADS[workload]
     base = {"tiny_weight": 0, "weight_outliers": 1, "activations_t3": 2, "weight_x50": 4}[workload]
-    return gen(seed=base + 1000 * rank)
+    return [gen(seed=base + 1000 * rank)]
 
 
 # ---------------------------------------------------------------------------
@@ -103,13 +121,14 @@ def gen_input(workload: str, rank: int) -> torch.Tensor:
 # ---------------------------------------------------------------------------
 
 def kernel_bytes(sizes, rows: int, cols: int):
-    """Algorithmic bytes of (quantize, dequantize-to-bf16) for one scheme.
+    """Algorithmic bytes of one scheme's kernels on one tensor: quantize (x read once,
+    outputs written), the range pass alone (x read), dequantize to bf16 (codes and
+    scales read, bf16 written), standalone QSNR (x, codes and scales read).
     sizes = (code, scale, zero point, tensor scale) bytes."""
     cb, sb, zb, tb = sizes
     x = 2 * rows * cols
-    q = x + cb + sb + zb + tb
-    dq = cb + sb + zb + tb + x
-    return q, dq
+    out = cb + sb + zb + tb
+    return {"quantize": x + out, "range": x, "quantize_pass": x + out, "dequantize": out + x, "qsnr": x + out}
 
 
 def aggregate(bytes_per_step_per_rank: float, n_ranks: int, max_ms_per_step: float) -> float:
@@ -145,11 +164,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.lines = []
         self.proc = None
-        self.t_on = self.t_off = None
+        self.windows = []
 
     def start(self):
         try:
@@ -169,11 +188,8 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
 
-    def mark_on(self):
-        self.t_on = time.time()
-
-    def mark_off(self):
-        self.t_off = time.time()
+    def mark(self, t_on: float, t_off: float):
+        self.windows.append((t_on, t_off))
 
     def stop(self):
         if self.proc is None:
@@ -190,7 +206,7 @@ class ClockSampler:
             if len(parts) < 10:
                 continue
             rows.append((t, parts))
-        window = [p for t, p in rows if self.t_on - 0.025 <= t <= self.t_off + 0.025]
+        window = [p for t, p in rows if any(a - 0.025 <= t <= b + 0.025 for a, b in self.windows)]
         use = window or [p for _, p in rows]
 
         def num(s):
@@ -234,8 +250,8 @@ def kernel_src_hash() -> str:
 
 
 def ncu_traffic(label: str, workload: str):
-    """DRAM bytes per launch of a kernel from the committed ncu summary, if that summary
-    was taken on the current kernel sources; else None."""
+    """DRAM bytes (read + write) per launch of a kernel from the committed ncu summary, if
+    that summary was taken on the current kernel sources; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -261,29 +277,36 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     schemes = [(lab, Scheme(*a)) for lab, a in WORKLOADS[args.workload]]
-    x_host = gen_input(args.workload, rank)
-    rows, cols = x_host.shape
+    n_tensors = args.tensors or DEFAULT_TENSORS.get(args.workload, 1)
+    hosts = gen_inputs(args.workload, rank, n_tensors)
+    rows, cols = hosts[0].shape
     signs = rotation_signs(args.workload, cols)
     sign_bits = None if signs is None else bq.pack_sign_bits(signs, device)
-    per_scheme_bytes = [kernel_bytes(bq.bq_buffer_sizes(s, rows, cols), rows, cols) for _, s in schemes]
+    kb = [kernel_bytes(bq.bq_buffer_sizes(s, rows, cols), rows, cols) for _, s in schemes]
     if signs is not None:
         # the sign words are read by both kernels
-        per_scheme_bytes = [(q + cols // 8, d + cols // 8) for q, d in per_scheme_bytes]
-    step_bytes = sum(q + d for q, d in per_scheme_bytes)
+        kb = [{k: v + cols // 8 for k, v in d.items()} for d in kb]
+    # per-tensor and NV schemes: the range pass and the quantize pass are two kernels
+    two_pass = [s.resolved().gran in ("tensor", "nv") for _, s in schemes]
 
-    # buffer sets: inputs + outputs of every kernel, rotated so that each step touches
-    # memory last used more than 4 x L2 ago
+    # units: the device copies of the inputs that the steps and the kernel timing rotate
+    # over. FFN: the distinct tensors. One-tensor workloads: enough copies that the
+    # smallest kernel's reuse distance exceeds 4 x L2.
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    set_bytes = step_bytes
-    n_sets = max(2, math.ceil(4 * l2 / set_bytes) + 1)
-    n_sets = min(n_sets, max(2, int(0.5 * torch.cuda.mem_get_info(device)[0] // max(set_bytes, 1))))
-    x_dev = x_host.to(device)
-    sets = []
-    for i in range(n_sets):
-        xi = x_dev if i == 0 else x_dev.clone()
-        outs = [bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes]
-        deqs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in schemes]
-        sets.append((xi, outs, deqs))
+    smallest = min(min(v for k, v in d.items() if k != "range") for d in kb)
+    if len(hosts) > 1:
+        srcs = hosts
+    else:
+        n_copies = max(2, math.ceil(4 * l2 / smallest) + 1)
+        free = torch.cuda.mem_get_info(device)[0]
+        unit_bytes = 2 * rows * cols * 2 + sum(d["quantize"] for d in kb)
+        n_copies = min(n_copies, max(2, int(0.5 * free // unit_bytes)))
+        srcs = hosts * n_copies
+    n_units = len(srcs)
+    xs = [h.to(device) for h in srcs]
+    outs = [[bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes] for _ in range(n_units)]
+    deqs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in range(n_units)]
+    rngs = [torch.zeros(3, dtype=torch.float32, device=device) for _ in range(n_units)]
     stream = torch.cuda.current_stream(device)
     # the schemes of a step are independent: with two or more, they run as two lanes
     # (even schemes on the launching stream, odd ones on a side stream, each lane with its
@@ -292,39 +315,51 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     n_lanes = 1 if (args.serial or len(schemes) < 2) else 2
     wss = [bq.new_workspace(device) for _ in range(n_lanes)]
     side = torch.cuda.Stream(device) if n_lanes > 1 else None
-    ws = wss[0]
 
-    def launch(j, kind, i, st, ws=ws):
-        """Kernel `kind` ("quantize" / "dequantize" / "qsnr") of scheme j on buffer set i."""
-        xi, outs, deqs = sets[i % n_sets]
-        s, q = schemes[j][1], outs[j]
+    def launch(j, kind, u, st, ws):
+        """Kernel `kind` of scheme j on unit u (mod n_units)."""
+        u %= n_units
+        xi, q, s = xs[u], outs[u][j], schemes[j][1]
         if sign_bits is not None and kind == "quantize":
             bq.bq_quantize_rt(xi, s, None, sign_bits, q.codes, q.scales, q.zero_points, q.stats, ws, st)
         elif sign_bits is not None and kind == "dequantize":
-            bq.bq_dequantize_rt(q.codes, q.scales, q.zero_points, rows, cols, s, None, sign_bits, deqs[j], st)
+            bq.bq_dequantize_rt(q.codes, q.scales, q.zero_points, rows, cols, s, None, sign_bits, deqs[u], st)
         elif kind == "quantize":
             bq.bq_quantize(xi, s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws, st)
+        elif kind == "range":
+            bq.bq_tensor_range(xi, s, rngs[u], ws, st)
+        elif kind == "quantize_pass":
+            bq.bq_quantize_with_range(xi, s, rngs[u], q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats,
+                                      ws, st)
         elif kind == "dequantize":
-            bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, deqs[j], st)
+            bq.bq_dequantize(q.codes, q.scales, q.zero_points, q.tensor_scale, rows, cols, s, deqs[u], st)
         else:
             bq.bq_qsnr(xi, q.codes, q.scales, q.zero_points, q.tensor_scale, s, q.stats, ws, st)
 
-    def step(i, st=None):
+    # units of step i: every FFN tensor, or the i-th copy of the one tensor
+    def step_units(i):
+        return list(range(n_units)) if len(hosts) > 1 else [i % n_units]
+
+    def step(i, st=None, dequant=False):
         st = st or stream
-        if n_lanes == 1:
+        lanes = [(st, wss[0])] if n_lanes == 1 else [(st, wss[0]), (side, wss[1])]
+        if n_lanes > 1:
+            side.wait_stream(st)
+        for u in step_units(i):
             for j in range(len(schemes)):
-                launch(j, "quantize", i, st)
-                launch(j, "dequantize", i, st)
-            return
-        side.wait_stream(st)
-        for j in range(len(schemes)):
-            lane_st, lane_ws = (st, wss[0]) if j % 2 == 0 else (side, wss[1])
-            launch(j, "quantize", i, lane_st, lane_ws)
-            launch(j, "dequantize", i, lane_st, lane_ws)
-        st.wait_stream(side)
+                lane_st, lane_ws = lanes[j % n_lanes]
+                launch(j, "quantize", u, lane_st, lane_ws)
+                if dequant:
+                    launch(j, "dequantize", u, lane_st, lane_ws)
+        if n_lanes > 1:
+            st.wait_stream(side)
+
+    units_per_step = len(step_units(0))
+    q_bytes = units_per_step * sum(d["quantize"] for d in kb)
+    full_bytes = units_per_step * sum(d["quantize"] + d["dequantize"] for d in kb)
 
     for i in range(args.warmup):
-        step(i)
+        step(i, dequant=True)
     torch.cuda.synchronize(device)
 
     def capture(fn):
@@ -337,154 +372,108 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize(device)
         return g
 
-    # The K timed steps are captured once into a CUDA graph and replayed once inside the
-    # timed region, so host-side launch overhead does not enter the device time.
-    graph = None
-    if not args.eager:
-        graph = capture(lambda st: [step(args.warmup + i, st) for i in range(args.steps)])
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     sampler = ClockSampler(vis.split(",")[local_rank].strip() if vis else device.index)
     if rank == 0:
         sampler.start()
-    barrier(device)
-    torch.cuda.synchronize(device)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    sampler.mark_on()
-    t0.record(stream)
-    if graph is not None:
-        graph.replay()
-    else:
-        for i in range(args.steps):
-            step(args.warmup + i)
-    t1.record(stream)
-    torch.cuda.synchronize(device)
-    sampler.mark_off()
-    barrier(device)
-    clocks = sampler.stop() if rank == 0 else None
-    ms = t0.elapsed_time(t1) / args.steps
-    ms_max = reduce_max(ms, device)
 
-    # QSNR of the last timed step (device sums read back before the per-kernel timing,
-    # whose standalone QSNR launches rewrite them)
+    def timed(fn_graph, fn_eager, n):
+        """Device ms per iteration of a graph replay (or eager loop) between two events."""
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        a = time.time()
+        t0.record(stream)
+        if fn_graph is not None:
+            fn_graph.replay()
+        else:
+            fn_eager()
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        sampler.mark(a, time.time())
+        barrier(device)
+        return reduce_max(t0.elapsed_time(t1) / n, device)
+
+    # The K timed steps are captured once into a CUDA graph and replayed once inside the
+    # timed region, so host-side launch overhead does not enter the device time.
+    graph = None if args.eager else capture(lambda st: [step(args.warmup + i, st) for i in range(args.steps)])
+    ms_max = timed(graph, lambda: [step(args.warmup + i) for i in range(args.steps)], args.steps)
+    del graph
+
+    # QSNR of the last timed step (read back before later launches rewrite the sums)
     qsnr = {}
-    xi, outs, _ = sets[(args.warmup + args.steps - 1) % n_sets]
-    for (lab, _), q in zip(schemes, outs):
-        st = q.stats.cpu().tolist()
-        qsnr[lab] = {"db": bq.bq_stats_qsnr_db(st), "mean_kappa": (st[2] / st[4]) if st[4] else None}
+    last = step_units(args.warmup + args.steps - 1)
+    for j, (lab, _) in enumerate(schemes):
+        dbs, kap = [], []
+        for u in last:
+            st = outs[u][j].stats.cpu().tolist()
+            dbs.append(bq.bq_stats_to_db(st))
+            if st[4]:
+                kap.append(st[2] / st[4])
+        qsnr[lab] = {"mean_db": statistics.fmean(dbs), "min_db": min(dbs), "max_db": max(dbs),
+                     "mean_kappa": statistics.fmean(kap) if kap else None, "tensors": len(dbs)}
 
-    # Per-kernel launch durations: each kernel of the step alone, K launches back to back
-    # over the same rotating buffer sets (a graph of them, or eager), between two events
-    # on the launching stream. (Events between the kernels of one graph would add their
-    # own gaps to every interval.)
-    n_k = 2 * len(schemes)
-    n_per = max(8, min(args.steps, 64))
+    # the whole path: quantize and dequantize of every tensor under every scheme
+    n_full = max(2, min(args.steps, 10))
+    g_full = None if args.eager else capture(
+        lambda st: [step(args.warmup + i, st, dequant=True) for i in range(n_full)])
+    ms_full = timed(g_full, lambda: [step(args.warmup + i, dequant=True) for i in range(n_full)], n_full)
+    del g_full
+
+    # Per-kernel launch durations: each kernel alone, n_per launches back to back over
+    # the rotating units, between two events on the launching stream. (Events between
+    # the kernels of one graph would add their own gaps to every interval.)
+    n_per = max(8, min(64, 2 * n_units))
     kernels = []
     for j, (lab, s) in enumerate(schemes):
-        qb, db = per_scheme_bytes[j]
-        # the standalone QSNR pass (not part of the step) reads what quantize reads and writes
-        kinds = (("quantize", qb), ("dequantize", db), ("qsnr", qb))
-        if sign_bits is not None:
-            kinds = kinds[:2]            # the rotated schemes have no standalone QSNR pass
-        for kind, nbytes in kinds:
+        kinds = ["quantize"]
+        if two_pass[j]:
+            kinds += ["range", "quantize_pass"]
+        kinds += ["dequantize"]
+        if sign_bits is None:
+            kinds += ["qsnr"]          # (the rotated schemes have no standalone QSNR pass)
+        for kind in kinds:
+            if kind == "quantize_pass":
+                for u in range(n_units):       # every unit's range, for its quantize pass
+                    launch(j, "range", u, stream, wss[0])
+
             def seq(st, j=j, kind=kind):
                 for i in range(n_per):
-                    launch(j, kind, args.warmup + i, st)
+                    launch(j, kind, i, st, wss[0])
             seq(stream)                                  # warm
             g = None if args.eager else capture(seq)
-            k0 = torch.cuda.Event(enable_timing=True)
-            k1 = torch.cuda.Event(enable_timing=True)
-            k0.record(stream)
-            if g is not None:
-                g.replay()
-            else:
-                seq(stream)
-            k1.record(stream)
-            torch.cuda.synchronize(device)
-            kms = reduce_max(k0.elapsed_time(k1) / n_per, device)
-            kernels.append({"kernel": f"{kind}:{lab}", "bytes": nbytes, "ms": kms,
-                            "gbs": nbytes / (kms * 1e-3) / 1e9})
+            kms = timed(g, lambda: seq(stream), n_per)
+            reuse = min(n_per, n_units) * kb[j][kind]
+            kernels.append({"kernel": f"{kind}:{lab}", "bytes": kb[j][kind], "ms": kms,
+                            "gbs": kb[j][kind] / (kms * 1e-3) / 1e9, "reuse_distance_bytes": reuse})
             del g
-    dom = max((k for k in kernels if not k["kernel"].startswith("qsnr:")), key=lambda k: k["ms"])
+    # the dominant kernel of the step: the slowest single kernel that the quantize step
+    # launches (for two-pass schemes the range pass and the quantize pass count apart)
+    is_two_pass = {lab: tp for (lab, _), tp in zip(schemes, two_pass)}
+
+    def in_step(k):
+        kind, lab = k["kernel"].split(":", 1)
+        return kind in ("range", "quantize_pass") if is_two_pass[lab] else kind == "quantize"
+    step_kernels = [k for k in kernels if in_step(k)]
+    dom = max(step_kernels, key=lambda k: k["ms"])
     peak, peak_kind = measured_peaks()
 
-    # end to end: pinned host input in, quantized outputs + sums out, every step. Steps
-    # alternate between two device buffer sets, so the input copy of one step, the
-    # kernels of the previous one and the output copy of the one before that overlap
-    # (host-to-device and device-to-host copies on their own streams, ordered by events).
     e2e = None
     if not args.no_e2e:
-        x_pin = x_host.pin_memory()
-        n_buf = 2
-        host_outs = []          # per buffer set: per scheme: (device tensor, pinned host tensor)
-        d2h = 0
-        for k in range(n_buf):
-            per = []
-            for q in sets[k][1]:
-                hs = []
-                for t in (q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats):
-                    if t is None:
-                        continue
-                    hs.append((t, torch.empty(t.shape, dtype=t.dtype).pin_memory()))
-                    if k == 0:
-                        d2h += t.numel() * t.element_size()
-                per.append(hs)
-            host_outs.append(per)
-        h2d = x_pin.numel() * x_pin.element_size()
-        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        ev_in = [torch.cuda.Event() for _ in range(n_buf)]
-        ev_comp = [torch.cuda.Event() for _ in range(n_buf)]
-        ev_out = [torch.cuda.Event() for _ in range(n_buf)]
+        e2e = run_e2e(args, bq, schemes, hosts, rows, cols, device, stream, wss, sign_bits, q_bytes, world)
 
-        def e2e_step(i):
-            k = i % n_buf
-            s_in.wait_event(ev_comp[k])          # set k's input is no longer read
-            with torch.cuda.stream(s_in):
-                sets[k][0].copy_(x_pin, non_blocking=True)
-            ev_in[k].record(s_in)
-            stream.wait_event(ev_in[k])
-            stream.wait_event(ev_out[k])         # set k's outputs are copied out
-            step(k, stream)
-            ev_comp[k].record(stream)
-            s_out.wait_event(ev_comp[k])
-            with torch.cuda.stream(s_out):
-                for hs in host_outs[k]:
-                    for t, h in hs:
-                        h.copy_(t, non_blocking=True)
-            ev_out[k].record(s_out)
-
-        def e2e_run(n):
-            s_in.wait_stream(stream)
-            s_out.wait_stream(stream)
-            for i in range(n):
-                e2e_step(i)
-            stream.wait_stream(s_out)
-
-        e2e_run(max(2, args.warmup))
-        torch.cuda.synchronize(device)
-        barrier(device)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        n_e2e = max(2, min(args.steps, 50))
-        e2e_run(n_e2e)
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
-        e2e = {"value": aggregate(step_bytes, world, e_ms), "unit": "GB/s", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "pipeline": "two buffer sets: a step's input copy, the previous step's kernels and the "
-                           "output copy of the one before overlap (copies on their own streams)"}
-
+    clocks = sampler.stop() if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, schemes_args=WORKLOADS[args.workload], x_host=x_host,
-                           budget_s=args.cpu_seconds, signs=signs)
+        cpu = cpu_baseline(args.workload, WORKLOADS[args.workload], hosts[0], budget_s=args.cpu_seconds,
+                           signs=signs)
 
-    value = aggregate(step_bytes, world, ms_max)
+    value = aggregate(q_bytes, world, ms_max)
     if rank != 0:
         return None
     traffic = ncu_traffic(dom["kernel"], args.workload)
+    n_launch_q = sum(2 if tp else 1 for tp in two_pass)
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -499,26 +488,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": f"{args.workload} {rows}x{cols} bf16: " + " + ".join(l for l, _ in schemes)
-                        + ("; randomized full-row Hadamard rotation," if signs is not None else ";")
-                        + " quantize with fused QSNR/kappa, then dequantize to bf16",
-            "rows": rows, "cols": cols,
-            "bytes_per_step_per_gpu": step_bytes,
-            "l2": f"inputs larger than L2: {n_sets} rotating buffer sets of {set_bytes / 2**20:.1f} MiB",
-            "parallelism": f"dp{world} (one independent tensor per GPU, no collective on the data path)",
-            "launch": "eager" if graph is None else "CUDA graph of the K timed steps",
+            "workload": (f"{args.workload}: {units_per_step} x bf16 {rows}x{cols} per step: "
+                         + " + ".join(l for l, _ in schemes)
+                         + ("; randomized full-row Hadamard rotation" if signs is not None else "")
+                         + "; quantize with fused QSNR/kappa"),
+            "tensors_per_step": units_per_step, "rows": rows, "cols": cols,
+            "bytes_per_step_per_gpu": q_bytes,
+            "l2": (f"inputs larger than L2: {n_units} distinct {'tensors' if len(hosts) > 1 else 'copies'} of "
+                   f"{2 * rows * cols / 2**20:.1f} MiB rotate (L2 {l2 / 2**20:.0f} MiB)"),
+            "parallelism": f"dp{world} (each GPU owns its own tensors, no collective on the data path)",
+            "launch": "eager" if args.eager else "CUDA graph of the K timed steps",
             "streams": (f"{n_lanes} (the step's independent schemes alternate between two streams, "
                         "forked and joined inside the step)") if n_lanes > 1 else "1",
-            "kernel_timing": f"each kernel alone, {n_per} launches back to back over the rotating sets",
+            "kernel_timing": (f"each kernel alone, {n_per} launches back to back over the rotating inputs "
+                              "(reuse distance per kernel in kernels[].reuse_distance_bytes)"),
         },
         "pct_hbm_peak": round(100.0 * value / world / peak, 2),
+        "full_path": {"value": round(aggregate(full_bytes, world, ms_full), 2), "unit": "GB/s",
+                      "ms_per_step": ms_full, "bytes_per_step_per_gpu": full_bytes,
+                      "what": "quantize with fused QSNR/kappa, then dequantize to bf16, of every tensor and scheme"},
         "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(dom["gbs"], 1),
                      "peak": peak, "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom["bytes"], "peak_source": peak_kind},
         "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kernels],
         "qsnr": qsnr,
-        # quantize: one kernel, plus the range pass for per-tensor and NV scales; dequantize: one
-        "gpu_launches": args.steps * sum((2 if s.gran in ("tensor", "nv") else 1) + 1 for _, s in schemes),
+        "gpu_launches": args.steps * units_per_step * n_launch_q,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,
@@ -526,82 +520,202 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return out
 
 
+def run_e2e(args, bq, schemes, hosts, rows, cols, device, stream, wss, sign_bits, q_bytes, world):
+    """Quantize GB/s end to end: each tensor's input is copied from pinned host memory and
+    its codes, scales, zero points, tensor scale and QSNR sums are read back, every step.
+    A ring of three device slots lets one tensor's input copy, another's kernels and a
+    third's output copy run at the same time (copies on their own streams, ordered by
+    events)."""
+    n_slots = 3
+    pins = [h.pin_memory() for h in hosts]
+    slot_x = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in range(n_slots)]
+    slot_q = [[bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes] for _ in range(n_slots)]
+
+    def out_tensors(qs):
+        return [t for q in qs for t in (q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats) if t is not None]
+
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in out_tensors(slot_q[k])]
+                for k in range(n_slots)]
+    h2d = sum(p.numel() * p.element_size() for p in pins[:1])
+    d2h = sum(t.numel() * t.element_size() for t in out_tensors(slot_q[0]))
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(n_slots)]
+    ev_comp = [torch.cuda.Event() for _ in range(n_slots)]
+    ev_out = [torch.cuda.Event() for _ in range(n_slots)]
+    for e in ev_comp + ev_out:
+        e.record(stream)
+    k_ring = [0]
+
+    def one(u):
+        k = k_ring[0] % n_slots
+        k_ring[0] += 1
+        s_in.wait_event(ev_comp[k])           # slot k's input is no longer read
+        with torch.cuda.stream(s_in):
+            slot_x[k].copy_(pins[u], non_blocking=True)
+        ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        stream.wait_event(ev_out[k])          # slot k's outputs are copied out
+        for j, (_, s) in enumerate(schemes):
+            q = slot_q[k][j]
+            if sign_bits is not None:
+                bq.bq_quantize_rt(slot_x[k], s, None, sign_bits, q.codes, q.scales, q.zero_points, q.stats,
+                                  wss[0], stream)
+            else:
+                bq.bq_quantize(slot_x[k], s, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, wss[0],
+                               stream)
+        ev_comp[k].record(stream)
+        s_out.wait_event(ev_comp[k])
+        with torch.cuda.stream(s_out):
+            for t, h in zip(out_tensors(slot_q[k]), host_out[k]):
+                h.copy_(t, non_blocking=True)
+        ev_out[k].record(s_out)
+
+    def run(n_steps):
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        for _ in range(n_steps):
+            for u in range(len(hosts)):
+                one(u)
+        stream.wait_stream(s_out)
+
+    n_e2e = max(2, min(args.steps, 3 if len(hosts) > 1 else 50))
+    run(1)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(n_e2e)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
+    return {"value": round(aggregate(q_bytes, world, e_ms), 2), "unit": "GB/s", "ms_per_step": e_ms,
+            "h2d_bytes_per_step": h2d * len(hosts), "d2h_bytes_per_step": d2h * len(hosts), "steps": n_e2e,
+            "pipeline": "three device slots: one tensor's input copy, another's quantize and a third's output "
+                        "copy overlap (copies on their own streams)"}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_step(xb: np.ndarray, schemes_args, signs=None):
+def _blocks(rows: int, n: int):
+    edges = [rows * i // n for i in range(n + 1)]
+    return [(a, b) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+
+
+def oracle_step(xb: np.ndarray, schemes_args, signs=None, threads: int = 1):
+    """Quantize (with QSNR / kappa sums) and dequantize to bf16 of one tensor under every
+    scheme with the oracle. threads > 1 splits the rows into blocks run concurrently (the
+    oracle's C calls release the interpreter lock); per-tensor and NV schemes first take
+    the whole tensor's range (blocks' ranges combined), then quantize each block against it."""
     import oracle
-    for _, a in schemes_args:
-        s = oracle.Scheme(*a[:5])
+    rows, cols = xb.shape
+    blocks = _blocks(rows, threads)
+
+    def one_block(args):
+        (a, b), s, tr = args
+        xp = xb[a:b]
         if signs is not None:
-            r = oracle.quantize_rt(xb, s, signs=signs, stats=True)
-            xh = oracle.dequantize_rt(r["codes"], r["scales"], r["zps"], xb.shape[0], xb.shape[1], s, signs=signs)
+            r = oracle.quantize_rt(xp, s, signs=signs, stats=True)
+            xh = oracle.dequantize_rt(r["codes"], r["scales"], r["zps"], b - a, cols, s, signs=signs)
         else:
-            r = oracle.quantize(xb, s, stats=True)
-            xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], r["tensor_scale"], xb.shape[0], xb.shape[1], s)
+            r = oracle.quantize(xp, s, tensor_range=tr, stats=True)
+            xh = oracle.dequantize(r["codes"], r["scales"], r["zps"], r["tensor_scale"], b - a, cols, s)
         oracle.to_bf16_array(xh)
+
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        for _, a in schemes_args:
+            s = oracle.Scheme(*a[:5])
+            tr = None
+            if s.gran in ("tensor", "nv") and signs is None and len(blocks) > 1:
+                parts = list(ex.map(lambda ab: oracle.tensor_range(xb[ab[0]:ab[1]], s.hadamard), blocks))
+                tr = (max(p[0] for p in parts), min(p[1] for p in parts), max(p[2] for p in parts))
+            list(ex.map(one_block, [(ab, s, tr) for ab in blocks]))
 
 
 def oracle_bytes(schemes_args, rows, cols):
+    """Algorithmic bytes of one oracle step: quantize and dequantize of every scheme."""
     import oracle
     tot = 0
     for _, a in schemes_args:
-        q, d = kernel_bytes(oracle.buffer_sizes(oracle.Scheme(*a[:5]), rows, cols), rows, cols)
-        tot += q + d
+        d = kernel_bytes(oracle.buffer_sizes(oracle.Scheme(*a[:5]), rows, cols), rows, cols)
+        tot += d["quantize"] + d["dequantize"]
     return tot
 
 
-def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, rows_per_step=None, signs=None):
-    """Time the oracle, as it stands, on this host (one thread) over whole steps of a
-    row sample of the workload tensor, until budget_s is spent (at least 2 steps)."""
-    xb = synth.bf16_bits(x_host)
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle(xb, schemes_args, budget_s, signs, threads):
+    """Whole oracle steps on a row sample sized so the timing takes about budget_s."""
     rows, cols = xb.shape
-    if rows_per_step is None:
-        t = time.perf_counter()
-        oracle_step(xb[: max(1, rows // 32)], schemes_args, signs)
-        per_row = (time.perf_counter() - t) / max(1, rows // 32)
-        rows_per_step = int(min(rows, max(16, budget_s / 4 / max(per_row, 1e-9))))
+    probe = max(threads, rows // 64)
+    t = time.perf_counter()
+    oracle_step(xb[:probe], schemes_args, signs, threads)
+    per_row = (time.perf_counter() - t) / probe
+    rows_per_step = int(min(rows, max(16 * threads, budget_s / 4 / max(per_row, 1e-9))))
     sample = xb[:rows_per_step]
     nbytes = oracle_bytes(schemes_args, rows_per_step, cols)
     t0 = time.perf_counter()
     n = 0
     while True:
-        oracle_step(sample, schemes_args, signs)
+        oracle_step(sample, schemes_args, signs, threads)
         n += 1
         if n >= 2 and time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(nbytes * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows_per_step} of {rows} rows of the {workload} tensor, {n} whole steps "
-                      f"(quantize + dequantize of every scheme) in {dt:.1f} s, single thread"}
+    return nbytes * n / dt / 1e9, rows_per_step, n, dt
+
+
+def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, signs=None):
+    """Time the oracle, as it stands, on this host: all cores (row blocks in parallel) and
+    one thread, each over whole steps (quantize with QSNR / kappa sums, then dequantize, of
+    every scheme) of a row sample of the workload's first tensor."""
+    xb = synth.bf16_bits(x_host)
+    rows, cols = xb.shape
+    cores = host_cores()
+    v_all, r_all, n_all, dt_all = time_oracle(xb, schemes_args, budget_s, signs, cores)
+    v_one, r_one, n_one, dt_one = time_oracle(xb, schemes_args, budget_s, signs, 1)
+    return {"value": round(v_all, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": (f"first {r_all} of {rows} rows of the {workload} tensor, {n_all} whole steps (quantize "
+                       f"with QSNR/kappa + dequantize of every scheme) in {dt_all:.1f} s, rows split over "
+                       f"{cores} threads"),
+            "single_thread": {"value": round(v_one, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"first {r_one} rows, {n_one} whole steps in {dt_one:.1f} s"}}
 
 
 def run_reference(args, rank: int):
     if rank != 0:
         return None
     schemes_args = WORKLOADS[args.workload]
-    x_host = gen_input(args.workload, 0)
+    x_host = gen_inputs(args.workload, 0, 1)[0]
     xb = synth.bf16_bits(x_host)
     rows, cols = xb.shape
     signs = rotation_signs(args.workload, cols)
+    cores = host_cores()
     # rows per step so that warmup + steps take about args.cpu_seconds * 6 in total
+    probe = max(cores, rows // 64)
     t = time.perf_counter()
-    oracle_step(xb[: max(1, rows // 32)], schemes_args, signs)
-    per_row = (time.perf_counter() - t) / max(1, rows // 32)
+    oracle_step(xb[:probe], schemes_args, signs, cores)
+    per_row = (time.perf_counter() - t) / probe
     total_budget = max(30.0, 6 * args.cpu_seconds)
-    rows_per_step = int(min(rows, max(16, total_budget / (args.steps + args.warmup) / max(per_row, 1e-9))))
+    rows_per_step = int(min(rows, max(16 * cores, total_budget / (args.steps + args.warmup) / max(per_row, 1e-9))))
     sample = xb[:rows_per_step]
     nbytes = oracle_bytes(schemes_args, rows_per_step, cols)
     for _ in range(args.warmup):
-        oracle_step(sample, schemes_args, signs)
+        oracle_step(sample, schemes_args, signs, cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(sample, schemes_args, signs)
+        oracle_step(sample, schemes_args, signs, cores)
     dt = time.perf_counter() - t0
     value = nbytes * args.steps / dt / 1e9
     desc = (f"first {rows_per_step} of {rows} rows of the {args.workload} tensor per step, "
-            f"{args.steps} steps in {dt:.1f} s, single thread")
+            f"{args.steps} steps in {dt:.1f} s, rows split over {cores} threads")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -616,10 +730,10 @@ def run_reference(args, rank: int):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload} {rows}x{cols} bf16: " + " + ".join(l for l, _ in schemes_args)
+        "config": {"workload": f"{args.workload}: bf16 {rows}x{cols}: " + " + ".join(l for l, _ in schemes_args)
                    + "; quantize with QSNR/kappa, then dequantize to bf16 (CPU oracle)",
-                   "rows": rows, "cols": cols, "parallelism": "host, one thread"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+                   "rows": rows, "cols": cols, "parallelism": f"host, {cores} threads"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -627,10 +741,11 @@ def run_reference(args, rank: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="weight_outliers")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="ffn_lognormal")
+    ap.add_argument("--tensors", type=int, default=0, help="tensors per step (FFN workloads; default 64)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--serial", action="store_true", help="run the step's schemes one after another on one stream")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps one by one instead of as a CUDA graph")

@@ -84,6 +84,14 @@ def _lib() -> ctypes.CDLL:
         L.bq_quantize_noalloc.argtypes = [vp, i32, i64, i64, sp, vp, vp, vp, vp, vp, vp]
         L.bq_stats_qsnr_db.restype = ctypes.c_double
         L.bq_stats_qsnr_db.argtypes = [ctypes.POINTER(BqStats)]
+        L.bq_stats_to_db.restype = ctypes.c_double
+        L.bq_stats_to_db.argtypes = [ctypes.POINTER(BqStats)]
+        L.bq_tensor_range.restype = ctypes.c_int
+        L.bq_tensor_range.argtypes = [vp, i32, i64, i64, sp, vp, vp, sz, vp]
+        L.bq_quantize_with_range.restype = ctypes.c_int
+        L.bq_quantize_with_range.argtypes = [vp, i32, i64, i64, sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.bq_debug_skip_tile_copy.restype = ctypes.c_int
+        L.bq_debug_skip_tile_copy.argtypes = [i32]
         L.bq_wait_timeouts.restype = ctypes.c_int
         L.bq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         rtp = ctypes.POINTER(BqRowTransform)
@@ -197,6 +205,38 @@ def bq_quantize_noalloc(x: torch.Tensor, scheme: Scheme, codes: torch.Tensor, sc
            "bq_quantize_noalloc")
 
 
+def bq_tensor_range(x: torch.Tensor, scheme: Scheme, range_out: torch.Tensor, workspace: torch.Tensor,
+                    stream=None) -> None:
+    """The range pass of a per-tensor / NV scheme alone: range_out (fp32 [3] on the
+    device) = {amax, min(min, 0), max(max, 0)} of the (rotated) tensor."""
+    rows, cols = x.shape
+    sc = scheme.c()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib().bq_tensor_range(_ptr(x), DT["bf16"], rows, cols, ctypes.byref(sc), _ptr(range_out),
+                                  _ptr(workspace), ws_bytes, _stream(stream)), "bq_tensor_range")
+
+
+def bq_quantize_with_range(x: torch.Tensor, scheme: Scheme, range_in: torch.Tensor, codes: torch.Tensor,
+                           scales: torch.Tensor, zero_points: torch.Tensor | None,
+                           tensor_scale: torch.Tensor | None, stats: torch.Tensor | None,
+                           workspace: torch.Tensor | None, stream=None) -> None:
+    """The quantize pass of a per-tensor / NV scheme against a given range (fp32 [3] on
+    the device: amax, min, max)."""
+    rows, cols = x.shape
+    sc = scheme.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().bq_quantize_with_range(_ptr(x), DT["bf16"], rows, cols, ctypes.byref(sc), _ptr(range_in),
+                                         _ptr(codes), _ptr(scales), _ptr(zero_points), _ptr(tensor_scale),
+                                         _ptr(stats), _ptr(workspace), ws_bytes, _stream(stream)),
+           "bq_quantize_with_range")
+
+
+def bq_debug_skip_tile_copy(tile: int) -> None:
+    """Test hook: the next flat quantize launch issues no copy for staged tile `tile`, so
+    the wait for it runs out (bounded) and bq_wait_timeouts counts it."""
+    _check(_lib().bq_debug_skip_tile_copy(int(tile)), "bq_debug_skip_tile_copy")
+
+
 def bq_dequantize(codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor | None,
                   tensor_scale: torch.Tensor | None, rows: int, cols: int, scheme: Scheme,
                   out: torch.Tensor, stream=None) -> None:
@@ -266,6 +306,13 @@ def bq_stats_qsnr_db(stats_host) -> float:
     v = [float(a) for a in (stats_host.tolist() if hasattr(stats_host, "tolist") else stats_host)]
     s = BqStats(*v[:5])
     return float(_lib().bq_stats_qsnr_db(ctypes.byref(s)))
+
+
+def bq_stats_to_db(stats_host) -> float:
+    """The same as bq_stats_qsnr_db (the C ABI exports both names)."""
+    v = [float(a) for a in (stats_host.tolist() if hasattr(stats_host, "tolist") else stats_host)]
+    s = BqStats(*v[:5])
+    return float(_lib().bq_stats_to_db(ctypes.byref(s)))
 
 
 # ---------------------------------------------------------------------------

@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 
 namespace bq {
@@ -155,6 +156,92 @@ DequantArgs dequant_args(const Plan& p, int64_t cols)
 
 bq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA; }
 
+// The range pass's result in the workspace header: {amax, min, max}.
+const float* ws_range_ptr(void* ws)
+{
+    return reinterpret_cast<const float*>(reinterpret_cast<uint8_t*>(ws) + offsetof(WsHeader, amax));
+}
+
+// Test hook (bq_debug_skip_tile_copy): the tile of the next flat quantize launch whose
+// copy is not issued; consumed by that launch.
+std::atomic<uint32_t> g_skip_tile{0xFFFFFFFFu};
+
+uint32_t take_skip_tile() { return g_skip_tile.exchange(0xFFFFFFFFu, std::memory_order_acq_rel); }
+
+// The quantize pass of bq_quantize / bq_quantize_with_range: every check done; range:
+// {amax, min, max} of the (rotated) tensor for per-tensor and NV schemes.
+bq_status quantize_pass(const Plan& p, const uint32_t* xw, int64_t rows, int64_t cols, void* codes, void* scales,
+                        void* zero_points, float* tensor_scale, bq_stats* stats, uint8_t* ws, const float* range,
+                        cudaStream_t s)
+{
+    const bool want_stats = stats != nullptr;
+    if (p.gran == BQ_TILE_2D) {
+        Tile2dArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols;
+        a.tpr = (uint32_t)(cols / TILE);
+        a.ntiles = (uint32_t)p.n_scales;
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        return cuda_status(launch_quant_tile2d(p.fmt, p.had != 0, want_stats, a, s));
+    }
+    const bool pow2_segments = cols % 64 == 0 && ((cols / 64) & (cols / 64 - 1)) == 0;
+    if (p.gran == BQ_PER_ROW && pow2_segments && cols <= 2048) {
+        // a row is a group of cols elements inside one warp tile (cols / 64 lanes)
+        FlatArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.n_chunks = p.n_chunks;
+        a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
+        a.lanes_per_group = (int32_t)(cols / 64);
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.n_elems = (double)p.n;
+        a.inv_unit = 1.0f / (float)cols;
+        a.skip_tile = take_skip_tile();
+        return cuda_status(launch_quant_flat(p.fmt, K_GROUP, p.had != 0, want_stats, a, s));
+    }
+    if (p.gran == BQ_PER_ROW && cols % 64 == 0) {
+        RowsArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols; a.cpr = (uint32_t)(cols / 16);
+        a.nseg = (uint32_t)(cols / 64); a.tiles = (a.nseg + 31u) / 32u;
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.inv_cols = 1.0f / (float)cols;
+        return cuda_status(launch_quant_rows(p.fmt, p.had != 0, want_stats, a, s));
+    }
+    if (p.gran == BQ_PER_ROW) {
+        RowArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+        a.stats = stats; a.ws = ws;
+        a.rows = (uint32_t)rows; a.cpr = (uint32_t)(cols / 16);
+        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+        a.inv_cols = 1.0f / (float)cols;
+        return cuda_status(launch_quant_row(p.fmt, p.had != 0, want_stats, a, s));
+    }
+    FlatArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
+    a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
+    a.n_chunks = p.n_chunks;
+    // a warp tile is 32 lanes x 4 chunks
+    a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
+    // groups: 16 elements -> 0 (four units per lane), 32 -> -1 (two per lane),
+    // 64 and up -> lanes per group (one unit over block / 64 lanes)
+    a.lanes_per_group = p.gran != BQ_PER_GROUP ? 1 : (p.block == 16 ? 0 : (p.block == 32 ? -1 : p.block / 64));
+    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+    a.n_elems = (double)p.n;
+    a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
+    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
+    a.range = range;
+    a.skip_tile = take_skip_tile();
+    return cuda_status(launch_quant_flat(p.fmt, kind_of(p.gran), p.had != 0, want_stats, a, s));
+}
+
 }  // namespace
 
 int device_sm_count()
@@ -243,71 +330,66 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
     const uint32_t* xw = reinterpret_cast<const uint32_t*>(x);
 
     if (p.needs_range) {
-        const cudaError_t e = launch_range(xw, p.n_chunks, p.had != 0, p.gran == BQ_PER_TENSOR && p.asym, ws, s);
+        const cudaError_t e = launch_range(xw, p.n_chunks, p.had != 0, p.gran == BQ_PER_TENSOR && p.asym, ws,
+                                           nullptr, s);
         if (e != cudaSuccess) return BQ_ERR_CUDA;
     }
-    if (p.gran == BQ_TILE_2D) {
-        Tile2dArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
-        a.stats = stats; a.ws = ws;
-        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols;
-        a.tpr = (uint32_t)(cols / TILE);
-        a.ntiles = (uint32_t)p.n_scales;
-        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
-        return cuda_status(launch_quant_tile2d(p.fmt, p.had != 0, want_stats, a, s));
+    return quantize_pass(p, xw, rows, cols, codes, scales, zero_points, tensor_scale, stats, ws,
+                         p.needs_range ? ws_range_ptr(ws) : nullptr, s);
+}
+
+bq_status bq_tensor_range(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, const bq_scheme* scheme,
+                          float* range, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    if (!p.needs_range) return BQ_ERR_UNSUPPORTED;
+    if (!range) return BQ_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < WS_BYTES) return BQ_ERR_WORKSPACE;
+    if (!aligned4(range)) return BQ_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (p.n == 0) return cuda_status(cudaMemsetAsync(range, 0, 3 * sizeof(float), s));
+    if (!x) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x)) return BQ_ERR_ALIGNMENT;
+    return cuda_status(launch_range(reinterpret_cast<const uint32_t*>(x), p.n_chunks, p.had != 0,
+                                    p.gran == BQ_PER_TENSOR && p.asym, reinterpret_cast<uint8_t*>(workspace), range,
+                                    s));
+}
+
+bq_status bq_quantize_with_range(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                                 const bq_scheme* scheme, const float* range,
+                                 void* codes, void* scales, void* zero_points, float* tensor_scale,
+                                 bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    if (!p.needs_range) return BQ_ERR_UNSUPPORTED;
+    const bool want_stats = stats != nullptr;
+    if (want_stats && (!workspace || workspace_bytes < WS_BYTES)) return BQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (p.n == 0) {
+        if (want_stats) return cuda_status(cudaMemsetAsync(stats, 0, sizeof(bq_stats), s));
+        return BQ_OK;
     }
-    const bool pow2_segments = cols % 64 == 0 && ((cols / 64) & (cols / 64 - 1)) == 0;
-    if (p.gran == BQ_PER_ROW && pow2_segments && cols <= 2048) {
-        // a row is a group of cols elements inside one warp tile (cols / 64 lanes)
-        FlatArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
-        a.stats = stats; a.ws = ws;
-        a.n_chunks = p.n_chunks;
-        a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
-        a.lanes_per_group = (int32_t)(cols / 64);
-        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
-        a.n_elems = (double)p.n;
-        a.inv_unit = 1.0f / (float)cols;
-        return cuda_status(launch_quant_flat(p.fmt, K_GROUP, p.had != 0, want_stats, a, s));
-    }
-    if (p.gran == BQ_PER_ROW && cols % 64 == 0) {
-        RowsArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
-        a.stats = stats; a.ws = ws;
-        a.rows = (uint32_t)rows; a.cols = (uint32_t)cols; a.cpr = (uint32_t)(cols / 16);
-        a.nseg = (uint32_t)(cols / 64); a.tiles = (a.nseg + 31u) / 32u;
-        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
-        a.inv_cols = 1.0f / (float)cols;
-        return cuda_status(launch_quant_rows(p.fmt, p.had != 0, want_stats, a, s));
-    }
-    if (p.gran == BQ_PER_ROW) {
-        RowArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
-        a.stats = stats; a.ws = ws;
-        a.rows = (uint32_t)rows; a.cpr = (uint32_t)(cols / 16);
-        a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
-        a.inv_cols = 1.0f / (float)cols;
-        return cuda_status(launch_quant_row(p.fmt, p.had != 0, want_stats, a, s));
-    }
-    FlatArgs a;
-    std::memset(&a, 0, sizeof a);
-    a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
-    a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
-    a.n_chunks = p.n_chunks;
-    // a warp tile is 32 lanes x 4 chunks
-    a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
-    // groups: 16 elements -> 0 (four units per lane), 32 -> -1 (two per lane),
-    // 64 and up -> lanes per group (one unit over block / 64 lanes)
-    a.lanes_per_group = p.gran != BQ_PER_GROUP ? 1 : (p.block == 16 ? 0 : (p.block == 32 ? -1 : p.block / 64));
-    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
-    a.n_elems = (double)p.n;
-    a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
-    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
-    return cuda_status(launch_quant_flat(p.fmt, kind_of(p.gran), p.had != 0, want_stats, a, s));
+    if (!x || !codes || !scales || !range) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (p.gran == BQ_NV_BLOCK && !tensor_scale) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points) || !aligned4(tensor_scale) || !aligned4(range))
+        return BQ_ERR_ALIGNMENT;
+    return quantize_pass(p, reinterpret_cast<const uint32_t*>(x), rows, cols, codes, scales, zero_points,
+                         tensor_scale, stats, reinterpret_cast<uint8_t*>(workspace), range, s);
+}
+
+bq_status bq_debug_skip_tile_copy(int32_t tile)
+{
+    if (tile < 0) return BQ_ERR_INVALID_ARG;
+    g_skip_tile.store((uint32_t)tile, std::memory_order_release);
+    return BQ_OK;
 }
 
 bq_status bq_dequantize(const void* codes, const void* scales, const void* zero_points,
@@ -453,5 +535,7 @@ double bq_stats_qsnr_db(const bq_stats* host_stats)
     if (host_stats->err2 == 0.0) return INFINITY;
     return -10.0 * std::log10(host_stats->err2 / host_stats->x2);
 }
+
+double bq_stats_to_db(const bq_stats* host_stats) { return bq_stats_qsnr_db(host_stats); }
 
 }  // extern "C"

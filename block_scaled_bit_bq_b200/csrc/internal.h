@@ -20,6 +20,7 @@ struct FlatArgs {
     float* tensor_scale;
     bq_stats* stats;
     uint8_t* ws;
+    const float* range;         // per-tensor / NV: {amax, min, max} of the (rotated) tensor
     uint32_t n_chunks;          // rows * cols / 16
     uint32_t n_dtiles;          // ceil(n_chunks / 128): a warp takes 128 chunks (one tile) per step
     int32_t lanes_per_group;    // per-group: 0 (block 16), -1 (block 32), block / 64 (64..512)
@@ -28,6 +29,8 @@ struct FlatArgs {
     float inv_unit;             // 1 / elements per scaling unit (kappa)
     FastDiv gemm_nb;            // MX / NV scales in the GEMM layout: division by blocks per row
     int32_t gemm_layout;        // 1: scales in the GEMM layout; 0: row-major
+    uint32_t skip_tile;         // fault injection for tests: the copy of this tile is never
+                                // issued (its wait runs out); 0xFFFFFFFF: none
 };
 
 // Per-row kernel: one CTA per row at a time.
@@ -127,8 +130,9 @@ enum { SK_F32 = 0, SK_F16 = 1, SK_UE8M0 = 2, SK_NV = 3 };
 int device_sm_count();
 size_t workspace_bytes();
 
+// Range pass into the workspace header (and into out[0..2] when out is not null).
 cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool hadamard, bool minmax,
-                         uint8_t* ws, cudaStream_t st);
+                         uint8_t* ws, float* out, cudaStream_t st);
 cudaError_t launch_quant_flat(int fmt, int kind, bool hadamard, bool stats, const FlatArgs& a,
                               cudaStream_t st);
 cudaError_t launch_quant_row(int fmt, bool hadamard, bool stats, const RowArgs& a, cudaStream_t st);

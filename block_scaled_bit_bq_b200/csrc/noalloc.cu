@@ -11,9 +11,6 @@
 #include "common.cuh"
 #include "internal.h"
 
-#include <atomic>
-#include <mutex>
-
 namespace bq {
 
 namespace {
@@ -23,28 +20,17 @@ namespace {
 // copy until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[WS_BYTES];
 
-constexpr int MAX_DEV = 64;
-std::atomic<void*> g_scratch_ptr[MAX_DEV];
-std::mutex g_scratch_mu;
-
-// Device address of the scratch on the current device (looked up once per device; in
-// host code the array's name is only a stand-in, not a device address).
+// Device address of the scratch on the current device. In host code the array's name is
+// only a stand-in, not a device address. The address is looked up on every call rather
+// than cached: after cudaDeviceReset (or any teardown of the primary context) the module
+// is loaded again and the array may sit elsewhere. The first lookup on a device loads the
+// library's device code there (lazy loading), which is why the first call should come
+// before any stream capture; later lookups are a host-side table read.
 cudaError_t scratch_address(void** out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEV) return cudaErrorInvalidDevice;
-    void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        std::lock_guard<std::mutex> lock(g_scratch_mu);
-        p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-        if (!p) {
-            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-            if (e != cudaSuccess) return e;
-            g_scratch_ptr[dev].store(p, std::memory_order_release);
-        }
-    }
     *out = p;
     return cudaSuccess;
 }

@@ -43,7 +43,8 @@ __device__ __forceinline__ void range_chunk(const uint32_t (&w)[8], float& amax,
 }
 
 template <bool HAD, bool MINMAX>
-__global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, uint32_t n_chunks, uint8_t* ws)
+__global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, uint32_t n_chunks, uint8_t* ws,
+                                               float* out)
 {
     float amax = 0.0f, mn = 0.0f, mx = 0.0f;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
     if (threadIdx.x == 0) {
         for (int w = 0; w < nw; ++w) { a = fmaxf(a, sh[0][w]); lo = fminf(lo, sh[1][w]); hi = fmaxf(hi, sh[2][w]); }
         h->amax = a; h->vmin = lo; h->vmax = hi;
+        if (out) { out[0] = a; out[1] = lo; out[2] = hi; }
         h->counter_range = 0u;
     }
 }
@@ -735,7 +737,8 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
     uint32_t inflight = 0, parity = 0;                  // per stage bits (warp-uniform)
     auto issue = [&](uint32_t t, int s) {
         if (t < a.n_dtiles && t * 32 < rows_mapped) {
-            if (lane == 0) {
+            // (t == skip_tile only under the test hook: no copy, so the wait runs out)
+            if (lane == 0 && t != a.skip_tile) {
                 mbar_arrive_expect_tx(bar0 + 8 * s, TILE_BYTES);
                 tma_load_2d(buf0 + s * TILE_BYTES, &xmap, bar0 + 8 * s, 0, (int)(t * 32));
             }
@@ -750,16 +753,18 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
     Pow2 tp{1.0f, 1.0};
     bool tscaled = false;
     if constexpr (GK == K_TENSOR || GK == K_NV) {
-        const WsHeader* h = ws_header(a.ws);
-        tc.amax = h->amax;
+        // {amax, min, max} of the (rotated) tensor: the range pass's result in the
+        // workspace header, or the caller's
+        const float r_amax = a.range[0], r_min = a.range[1], r_max = a.range[2];
+        tc.amax = r_amax;
         if constexpr (GK == K_TENSOR) {
-            tc.ps = plain_scale<FMT>(h->amax, h->vmin, h->vmax, a.scale_fp16 != 0);
+            tc.ps = plain_scale<FMT>(r_amax, r_min, r_max, a.scale_fp16 != 0);
             tu = plain_unit<FMT>(tc.ps);
             tp = pow2_for(tc.amax);
             tscaled = STATS && !plain_sums_ok(tc.amax);
             if (blockIdx.x == 0 && threadIdx.x == 0) store_plain_scale<FMT>(a.scales, a.zps, 0, tc.ps, a.scale_fp16 != 0);
         } else {
-            tc.S = div_rn_call(h->amax, F::qscale * 448.0f);
+            tc.S = div_rn_call(r_amax, F::qscale * 448.0f);
             tc.cS = rcp_approx(__fmul_rn(F::qscale, tc.S));
             if (blockIdx.x == 0 && threadIdx.x == 0) a.tensor_scale[0] = tc.S;
         }
@@ -788,10 +793,11 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
         const uint32_t span = t * 32 + lane;
         if (inflight >> s & 1u) {
-            const bool got = mbar_wait(bar0 + 8 * s, parity >> s & 1u);
+            const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, parity >> s & 1u));
+            // a stage whose wait gave up stays in flight: the drain below waits for it
+            if (!got) { ok = false; break; }
             parity ^= 1u << s;
             inflight &= ~(1u << s);
-            if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
         } else {
             // no row of this tile is covered by the tensor map
             const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -926,10 +932,12 @@ __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_
     };
     auto wait_stage = [&](int s) -> bool {
         if (!(inflight >> s & 1u)) return true;
-        const bool got = mbar_wait(bar0 + 8 * s, parity >> s & 1u);
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, parity >> s & 1u));
+        // a stage whose wait gave up stays in flight: the drain at the end waits for it
+        if (!got) return false;
         parity ^= 1u << s;
         inflight &= ~(1u << s);
-        return __all_sync(0xFFFFFFFFu, got);
+        return true;
     };
 #pragma unroll
     for (int s = 0; s < NST; ++s) issue((uint32_t)s, s);
@@ -1563,12 +1571,12 @@ cudaError_t run_flat_hs(bool had, bool stats, const FlatArgs& a, cudaStream_t st
 }
 
 template <bool HAD, bool MINMAX>
-cudaError_t run_range(const uint32_t* x, uint32_t n_chunks, uint8_t* ws, cudaStream_t st)
+cudaError_t run_range(const uint32_t* x, uint32_t n_chunks, uint8_t* ws, float* out, cudaStream_t st)
 {
     constexpr int block = 256;
     constexpr auto kern = k_range<HAD, MINMAX>;
     const unsigned grid = grid_for<kern, block, 0>((uint64_t)block * 4, n_chunks);
-    kern<<<grid, block, 0, st>>>(x, n_chunks, ws);
+    kern<<<grid, block, 0, st>>>(x, n_chunks, ws, out);
     return cudaGetLastError();
 }
 
@@ -1584,10 +1592,11 @@ cudaError_t flat_wait_timeouts(unsigned int* count, bool reset)
     return e;
 }
 
-cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool had, bool minmax, uint8_t* ws, cudaStream_t st)
+cudaError_t launch_range(const uint32_t* x, uint32_t n_chunks, bool had, bool minmax, uint8_t* ws, float* out,
+                         cudaStream_t st)
 {
-    if (had) return minmax ? run_range<true, true>(x, n_chunks, ws, st) : run_range<true, false>(x, n_chunks, ws, st);
-    return minmax ? run_range<false, true>(x, n_chunks, ws, st) : run_range<false, false>(x, n_chunks, ws, st);
+    if (had) return minmax ? run_range<true, true>(x, n_chunks, ws, out, st) : run_range<true, false>(x, n_chunks, ws, out, st);
+    return minmax ? run_range<false, true>(x, n_chunks, ws, out, st) : run_range<false, false>(x, n_chunks, ws, out, st);
 }
 
 cudaError_t launch_quant_rows(int fmt, bool had, bool stats, const RowsArgs& a, cudaStream_t st)

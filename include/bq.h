@@ -190,6 +190,38 @@ bq_status bq_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols
                       void* stream);
 
 /*
+ * The two passes of a per-tensor or NV scheme, as separate calls.
+ *
+ * bq_tensor_range: the range pass alone ("max calibration": the tensor's largest
+ * magnitude maps to the format's largest value, "2025 H2 quantization trends" §三;
+ * AbsMax, "INT vs FP at fine granularity" §2.1). Writes range[0] = amax = max |y|,
+ * range[1] = min(min y, 0) and range[2] = max(max y, 0) of the tensor's values y (each
+ * 16-run rotated by H16/4 first when scheme->hadamard is set); the last two only for
+ * asymmetric formats under BQ_PER_TENSOR (else 0). range: device fp32 [3], 4-byte
+ * aligned. Needs a workspace of bq_workspace_size() bytes (its header holds the
+ * cross-CTA hand-off). rows == 0 writes zeros.
+ *
+ * bq_quantize_with_range: the quantize pass alone, against range = {amax, min, max}
+ * (device fp32 [3]; min and max are used as min(min, 0) and max(max, 0)), e.g. from
+ * bq_tensor_range on this tensor (bq_tensor_range then bq_quantize_with_range gives
+ * exactly bq_quantize's results), from an earlier calibration (static scales), or
+ * combined over the row blocks of a tensor split across GPUs (MAX of amax and of max,
+ * MIN of min). Outputs, stats and alignment as bq_quantize; the workspace is needed only
+ * with stats (NULL / 0 otherwise).
+ *
+ * Both: per-tensor and NV schemes only (else BQ_ERR_UNSUPPORTED); a NULL range gives
+ * BQ_ERR_INVALID_ARG.
+ */
+bq_status bq_tensor_range(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                          const bq_scheme* scheme, float* range,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+bq_status bq_quantize_with_range(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                                 const bq_scheme* scheme, const float* range,
+                                 void* codes, void* scales, void* zero_points, float* tensor_scale,
+                                 bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dequantize codes (+ scales, zero_points, tensor_scale as written by bq_quantize)
  * into out [rows, cols] (device) of dtype out_dtype = BQ_DT_BF16 (round to nearest
  * even from the fp32 value) or BQ_DT_FP32. Applies the inverse rotation when
@@ -266,9 +298,10 @@ bq_status bq_dequantize_rt(const void* codes, const void* scales, const void* ze
  * Arguments and results are those of bq_quantize. The scratch is a file-scope device
  * array of 131328 bytes (the workspace size of every scheme and shape); every GPU that
  * loads the library holds one copy until the process exits. A call whose scheme would
- * need more returns BQ_ERR_WORKSPACE. The first call on a device looks the array's
- * device address up (cudaGetSymbolAddress); make that first call before any stream
- * capture. Every call shares the one array and zeroes its counters on the stream
+ * need more returns BQ_ERR_WORKSPACE. Every call looks the array's device address up
+ * (cudaGetSymbolAddress), so the address stays right after a device reset; the first
+ * call on a device also loads the library's device code there, so make that first
+ * call before any stream capture. Every call shares the one array and zeroes its counters on the stream
  * first: calls that may overlap on the GPU (other streams, other threads) race, and
  * must be serialized by the caller. No cudaMalloc or cudaFree is made.
  */
@@ -292,7 +325,25 @@ bq_status bq_quantize_noalloc(const void* x, int32_t x_dtype, int64_t rows, int6
  */
 bq_status bq_wait_timeouts(uint32_t* count, int32_t reset);
 
-/* -10 log10(err2 / x2) from a host copy of the stats (+inf when err2 = 0). */
+/*
+ * Fault injection for tests of the bounded waits (no counterpart on the pages). The next
+ * bq_quantize / bq_quantize_with_range call that runs the flat quantize kernel (per-tensor,
+ * per-group, MX and NV schemes, and per-row schemes of at most 2048 power-of-two-many
+ * 64-element segments) issues no copy for its staged tile number `tile` (tile t holds
+ * chunks 128 t .. 128 t + 127 of the tensor seen as 16-element chunks; tile 0 is the
+ * first tile of the first warp). The warp that waits for it gives up after the
+ * one-second limit, waits (bounded) for its other copies in flight and stops; the call's
+ * outputs are then incomplete and bq_wait_timeouts counts one more. Nothing faults and
+ * nothing is left in flight; a following call on the same workspace runs normally.
+ * One-shot: the call that consumes it resets it. tile < 0: BQ_ERR_INVALID_ARG.
+ */
+bq_status bq_debug_skip_tile_copy(int32_t tile);
+
+/* QSNR = -10 log10(err2 / x2) in dB from a host copy of the stats ("INT vs FP at fine
+ * granularity" §4.1): +inf when err2 = 0, NaN when x2 = 0 with err2 > 0 or for a NULL
+ * pointer. host_stats: host memory, read only. bq_stats_to_db and bq_stats_qsnr_db are
+ * the same function under two names. */
+double bq_stats_to_db(const bq_stats* host_stats);
 double bq_stats_qsnr_db(const bq_stats* host_stats);
 
 #ifdef __cplusplus

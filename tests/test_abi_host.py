@@ -164,8 +164,47 @@ def test_empty_dequantize_is_a_no_op():
 
 
 def test_stats_to_db():
-    assert abs(bq.bq_stats_qsnr_db([0.0234375, 2.9453125, 0, 0, 0]) - 20.99219) < 1e-4
-    assert bq.bq_stats_qsnr_db([0.0, 1.0, 0, 0, 0]) == float("inf")
+    # -10 log10(0.0234375 / 2.9453125) = 20.99219 dB
+    for f in (bq.bq_stats_qsnr_db, bq.bq_stats_to_db):
+        assert abs(f([0.0234375, 2.9453125, 0, 0, 0]) - 20.99219) < 1e-4
+        assert f([0.0, 1.0, 0, 0, 0]) == float("inf")
+    # the C symbol bq_stats_to_db itself, through ctypes
+    L = bq.lib()
+    s = bq.BqStats(1.0, 1000.0, 0.0, 0.0, 0.0)
+    assert abs(L.bq_stats_to_db(ctypes.byref(s)) - 30.0) < 1e-12
+    assert L.bq_stats_to_db(None) != L.bq_stats_to_db(None)        # NaN for a NULL pointer
+
+
+def test_range_split_checks_before_any_launch():
+    L = bq.lib()
+    fake = 1 << 40
+    ws = ctypes.c_void_p(fake)
+    t = Scheme("e4m3", "tensor").c()
+    row = Scheme("int8_sym", "row").c()
+    # only per-tensor and NV schemes have a range pass
+    assert L.bq_tensor_range(fake, 0, 4, 64, ctypes.byref(row), fake, ws, 1 << 20, None) == 2
+    assert L.bq_quantize_with_range(fake, 0, 4, 64, ctypes.byref(row), fake, fake, fake, None, None, None,
+                                    None, 0, None) == 2
+    # range output / input required; workspace required for the range pass
+    assert L.bq_tensor_range(fake, 0, 4, 64, ctypes.byref(t), None, ws, 1 << 20, None) == 1
+    assert L.bq_tensor_range(fake, 0, 4, 64, ctypes.byref(t), fake, None, 0, None) == 5
+    assert L.bq_quantize_with_range(fake, 0, 4, 64, ctypes.byref(t), None, fake, fake, None, None, None,
+                                    None, 0, None) == 1
+    # alignment: x 32 bytes, the range 4 bytes
+    assert L.bq_tensor_range(fake + 16, 0, 4, 64, ctypes.byref(t), fake, ws, 1 << 20, None) == 4
+    assert L.bq_tensor_range(fake, 0, 4, 64, ctypes.byref(t), fake + 2, ws, 1 << 20, None) == 4
+    assert L.bq_quantize_with_range(fake, 0, 4, 64, ctypes.byref(t), fake + 1, fake, fake, None, None, None,
+                                    None, 0, None) == 4
+    # stats need a workspace; an NV scheme needs its tensor scale output
+    assert L.bq_quantize_with_range(fake, 0, 4, 64, ctypes.byref(t), fake, fake, fake, None, None, fake,
+                                    None, 0, None) == 5
+    nv = Scheme("e2m1", "nv").c()
+    assert L.bq_quantize_with_range(fake, 0, 4, 64, ctypes.byref(nv), fake, fake, fake, None, None, None,
+                                    None, 0, None) == 1
+
+
+def test_debug_hook_rejects_negative_tiles():
+    assert bq.lib().bq_debug_skip_tile_copy(-1) == 1
 
 
 def test_status_strings():

@@ -267,20 +267,51 @@ def test_ffn_lognormal_full(t, ws):
 
 
 def test_weight_x50_full(ws):
+    # every row of the 8192 x 28672 tensor: codes, block scales, the tensor scale, the fp32
+    # and bf16 dequantized values, the fused and standalone QSNR sums and the kappa sums
     x = synth.weight_x50()
-    rows = x.shape[0]
-    g = np.random.default_rng(11)
-    sample = np.unique(np.concatenate([[0, rows - 1], g.choice(rows, 48, replace=False)]))
-    xb = synth.bf16_bits(x)
     for s in [Scheme("e2m1", "nv"), Scheme("int4_sym", "nv"), Scheme("int4_sym", "nv", hadamard=True)]:
-        tr = oracle.tensor_range(xb, s.hadamard)
-        q = check(x, s, ws, "weight_x50", tensor_range=tr, rows_sample=sample)
-        # QSNR of the whole tensor against the oracle's standalone sums on the GPU codes
-        # is not an independent check; the full oracle pass is:
-        o = oracle.quantize(xb, _o(s))
-        st = q.stats.cpu().numpy()
-        assert abs(bq.bq_stats_qsnr_db(st) - oracle.qsnr_db(o["stats"][0], o["stats"][1])) < QSNR_TOL_DB
-        assert st[4] == o["stats"][4] and _close(st[2], o["stats"][2])
+        check(x, s, ws, "weight_x50")
+
+
+RANGE_SCHEMES = [Scheme("int8_sym", "tensor"), Scheme("int8_asym", "tensor"), Scheme("uint4_asym", "tensor", scale_dtype="fp16"),
+                 Scheme("e4m3", "tensor"), Scheme("e5m2", "tensor", hadamard=True), Scheme("e2m1", "nv"),
+                 Scheme("int4_sym", "nv", hadamard=True)]
+
+
+@pytest.mark.parametrize("s", RANGE_SCHEMES, ids=str)
+def test_range_split(s, ws, cuda_device):
+    """bq_tensor_range then bq_quantize_with_range gives bq_quantize's results; a row block
+    quantized against the whole tensor's range gives the oracle's codes for those rows."""
+    x = synth.activations_t3(300, 1024, seed=400, n_outlier_channels=2)
+    xb = synth.bf16_bits(x)
+    xd = x.to(cuda_device)
+    rng = torch.empty(3, dtype=torch.float32, device=cuda_device)
+    bq.bq_tensor_range(xd, s, rng, ws)
+    ref = bq.quantize(xd, s, workspace=ws)
+    q = bq.alloc_outputs(s, 300, 1024, cuda_device)
+    bq.bq_quantize_with_range(xd, s, rng, q.codes, q.scales, q.zero_points, q.tensor_scale, q.stats, ws)
+    torch.cuda.synchronize()
+    tr = oracle.tensor_range(xb, s.hadamard)
+    r = rng.cpu().numpy()
+    asym_tensor = s.fmt in ("int8_asym", "uint4_asym") and s.gran == "tensor"
+    want = np.array([tr[0], min(tr[1], 0.0) if asym_tensor else 0.0, max(tr[2], 0.0) if asym_tensor else 0.0],
+                    dtype=np.float32)
+    assert np.array_equal(r.view(np.uint32), want.view(np.uint32)), (r, tr)
+    for a, b in [(q.codes, ref.codes), (q.scales, ref.scales), (q.zero_points, ref.zero_points),
+                 (q.tensor_scale, ref.tensor_scale), (q.stats, ref.stats)]:
+        if a is not None:
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), s
+    # rows 100..227 of the tensor under the whole tensor's range (one shard of a split tensor)
+    part = xd[100:228].contiguous()
+    qp = bq.alloc_outputs(s, 128, 1024, cuda_device)
+    bq.bq_quantize_with_range(part, s, rng, qp.codes, qp.scales, qp.zero_points, qp.tensor_scale, None, None)
+    torch.cuda.synchronize()
+    o = oracle.quantize(xb[100:228], _o(s), tensor_range=tr, stats=False)
+    assert np.array_equal(qp.codes.cpu().numpy(), o["codes"]), s
+    assert np.array_equal(_bytes(qp.scales), _bytes(o["scales"])), s
+    if o["tensor_scale"] is not None:
+        assert np.array_equal(_bytes(qp.tensor_scale), _bytes(o["tensor_scale"])), s
 
 
 def test_no_tile_wait_gave_up(cuda_device):

@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
         ms = 1.0 + 0.5 * rank                     # this rank's step time
         m = bench.reduce_max(ms)
         bench.barrier()
-        x = bench.gen_input("tiny_weight", rank)
+        x = bench.gen_inputs("tiny_weight", rank, 1)[0]
         out.put((rank, m, bench.aggregate(1.0e9, world, m), float(x.float().abs().sum())))
     finally:
         dist.destroy_process_group()
@@ -61,13 +61,23 @@ def test_single_process_helpers():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.reduce_max(3.0) == 3.0          # no process group: identity
-    q, d = bench.kernel_bytes((1 << 20, 4096, 0, 0), 1024, 2048)
-    assert q == 2 * 1024 * 2048 + (1 << 20) + 4096
-    assert d == (1 << 20) + 4096 + 2 * 1024 * 2048
-    a = bench.gen_input("tiny_weight", 0)
-    b = bench.gen_input("tiny_weight", 0)
+    kb = bench.kernel_bytes((1 << 20, 4096, 0, 0), 1024, 2048)
+    assert kb["quantize"] == kb["quantize_pass"] == 2 * 1024 * 2048 + (1 << 20) + 4096
+    assert kb["dequantize"] == (1 << 20) + 4096 + 2 * 1024 * 2048
+    assert kb["range"] == 2 * 1024 * 2048
+    a = bench.gen_inputs("tiny_weight", 0, 1)[0]
+    b = bench.gen_inputs("tiny_weight", 0, 1)[0]
     import torch
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))   # same seed, same bytes
+    # the FFN set: rank r owns tensors 64 r .. 64 r + 63 (seed 3 + t); rank 0 owns the
+    # 64 tensors of the workload, drawn in parallel but identical to one-by-one draws
+    import synth
+    f = bench.gen_inputs("ffn_lognormal", 0, 3)
+    assert len(f) == 3 and torch.equal(f[2].view(torch.int16), synth.ffn_lognormal(2).view(torch.int16))
+    g = bench.gen_inputs("ffn_lognormal", 1, 3)
+    assert torch.equal(g[0].view(torch.int16), synth.ffn_lognormal(3).view(torch.int16))
+    assert [(a, b) for a, b in bench._blocks(10, 4)] == [(0, 2), (2, 5), (5, 7), (7, 10)]
+    assert bench._blocks(2, 8) == [(0, 1), (1, 2)]
 
 
 def test_bench_oracle_arm_covers_every_workload():
@@ -83,6 +93,7 @@ def test_bench_oracle_arm_covers_every_workload():
         x = synth.bf16_bits(synth.normal(rows, cols, seed=5, sigma=0.02))
         signs = bench.rotation_signs(w, cols)
         bench.oracle_step(x, schemes, signs)
+        bench.oracle_step(x, schemes, signs, threads=2)        # row blocks on two threads
         assert bench.oracle_bytes(schemes, rows, cols) > 2 * rows * cols * len(schemes)
     assert bench.rotation_signs("weight_outliers", 4096) is None
     s = bench.rotation_signs("weight_rotated", 4096)
@@ -101,7 +112,13 @@ def test_reference_arm_prints_the_contract_line():
     d = json.loads(r.stdout.strip().splitlines()[-1])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["higher_is_better"] is True and d["steps"] == 3 and d["warmup"] == 3
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == bench_cores()
     assert d["cpu_baseline"]["value"] == d["value"] and "rows" in d["cpu_baseline"]["sample"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"].startswith("tiny_weight 256x1024")
+    assert d["config"]["workload"].startswith("tiny_weight: bf16 256x1024")
+
+
+def bench_cores():
+    sys.path.insert(0, ROOT)
+    import bench
+    return bench.host_cores()
