@@ -11,9 +11,11 @@ The default workload is the FFN set at full size: 64 bf16 tensors of 4096 x 1100
 UE8M0 scales).
 
 A step is one pass of the quantize path over the workload's tensors: for every tensor
-and every scheme, bq_quantize with the fused QSNR and crest-factor sums (bf16 load,
+and every scheme, the quantize with the fused QSNR and crest-factor sums (bf16 load,
 optional block-16 rotation, ranges, scales, codes, packing and the QSNR partial sums;
-per-tensor and NV schemes take their range pass first).
+per-tensor and NV schemes take their range pass first). The FFN set takes one
+bq_quantize_batch launch per scheme over its 64 tensors (--per-tensor: one bq_quantize
+call per tensor); the other workloads one bq_quantize call per scheme.
 value: quantize GB/s = algorithmic bytes of every quantize call of a step (x read once,
 codes, scales, zero points and tensor scales written) / step time, summed over ranks
 (weak scaling: each rank owns its own tensors), with inputs resident in HBM. The 64
@@ -88,6 +90,10 @@ WORKLOADS = {
                    ("nvint4", ("int4_sym", "nv", 16, "e4m3", False)),
                    ("nvint4_hadamard", ("int4_sym", "nv", 16, "e4m3", True))],
 }
+
+# block-scaled GEMM workloads: D = A B^T of the 8192 x 8192 activations (Student-t(3) with
+# outlier channels) and an 8192 x 8192 weight, both quantized (GEMM-layout scales)
+GEMM_WORKLOADS = {"gemm_mxfp8": ("e4m3", "mx"), "gemm_nvfp4": ("e2m1", "nv")}
 
 FFN_WORKLOADS = ("ffn_lognormal", "ffn_mx_family", "ffn_mx_gemm_operands")
 # tensors per step: the FFN set is 64 tensors; the other workloads are one tensor
@@ -270,12 +276,87 @@ def ncu_traffic(label: str, workload: str):
 # our arm
 # ---------------------------------------------------------------------------
 
+def measured_tensor_peak(fmt: str):
+    """Dense tensor-core peak for the GEMM's element type: the measured bf16 burst figure
+    times the nominal ratio (FP8 2x, FP4 4x bf16)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    ratio = 4.0 if fmt == "e2m1" else 2.0
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]) * ratio, "measured bf16 x nominal ratio"
+    return 1590.0 * ratio, "fallback bf16 x nominal ratio"
+
+
+def run_gemm_bench(args, rank: int, world: int, device):
+    """TFLOP/s of bq_gemm (and of the library's block-scaled GEMM on the same operands)."""
+    import block_scaled_bit_bq_b200 as bq
+    from block_scaled_bit_bq_b200 import Scheme
+    fmt, gran = GEMM_WORKLOADS[args.workload]
+    s = Scheme(fmt, gran, layout="gemm")
+    M = N = K = 8192
+    a = synth.activations_t3(M, K, seed=2 + 1000 * rank)
+    b = synth.weight_outliers(N, K, seed=41 + 1000 * rank)
+    qa = bq.quantize(a.to(device), s, stats=False)
+    qb = bq.quantize(b.to(device), s, stats=False)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    flops = 2.0 * M * N * K
+
+    def time_fn(fn, reps):
+        for _ in range(3):
+            fn()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        return reduce_max(e0.elapsed_time(e1) / reps, device)
+
+    reps = max(5, args.steps)
+    ms = time_fn(lambda: bq.bq_gemm(qa, qb, d), reps)
+    lib = None
+    F = torch.nn.functional
+    if fmt == "e4m3" and hasattr(F, "scaled_mm") and hasattr(torch, "float8_e8m0fnu"):
+        dt = torch.float8_e4m3fn
+
+        def lib_gemm():
+            return F.scaled_mm(qa.codes.view(dt), qb.codes.view(dt).t(),
+                               qa.scales.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                               qb.scales.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                               swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                               output_dtype=torch.bfloat16)
+        try:
+            lib_ms = time_fn(lib_gemm, reps)
+            lib = {"kernel": "cuBLASLt scaled_mm (torch)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12}
+        except RuntimeError as e:
+            lib = {"kernel": "cuBLASLt scaled_mm (torch)", "unavailable": str(e).splitlines()[0][:200]}
+    if rank != 0:
+        return None
+    peak, src = measured_tensor_peak(fmt)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {
+        "metric": "block-scaled GEMM TFLOP/s (bq_gemm, D = A B^T)", "value": round(tf * world, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": reps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": fmt, "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {M}x{N}x{K}, {fmt} {gran} block scales in the GEMM layout, bf16 out",
+                   "operands": "A: activations_t3 8192x8192 (Student-t(3) with outlier channels); B: weight_outliers 8192x8192"},
+        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tf / peak, 4), "traffic": None, "peak_source": src},
+        "library_gemm": lib, "gpu_launches": reps,
+    }
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import block_scaled_bit_bq_b200 as bq
     from block_scaled_bit_bq_b200 import Scheme
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    if args.workload in GEMM_WORKLOADS:
+        return run_gemm_bench(args, rank, world, device)
     schemes = [(lab, Scheme(*a)) for lab, a in WORKLOADS[args.workload]]
     n_tensors = args.tensors or DEFAULT_TENSORS.get(args.workload, 1)
     hosts = gen_inputs(args.workload, rank, n_tensors)
@@ -303,8 +384,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         n_copies = min(n_copies, max(2, int(0.5 * free // unit_bytes)))
         srcs = hosts * n_copies
     n_units = len(srcs)
-    xs = [h.to(device) for h in srcs]
-    outs = [[bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes] for _ in range(n_units)]
+    # the units as one contiguous [n_units, rows, cols] tensor (a batch call takes it whole)
+    X = torch.empty((n_units, rows, cols), dtype=torch.bfloat16, device=device)
+    for u, h in enumerate(srcs):
+        X[u].copy_(h)
+    xs = [X[u] for u in range(n_units)]
+    # FFN sets quantize all their tensors in one bq_quantize_batch launch per scheme
+    batched = len(hosts) > 1 and not args.per_tensor and signs is None and not any(two_pass)
+    if batched:
+        qbs = [bq.alloc_batch_outputs(s, n_units, rows, cols, device, stats=True) for _, s in schemes]
+        outs = [[qbs[j].tensor(u) for j in range(len(schemes))] for u in range(n_units)]
+    else:
+        qbs = None
+        outs = [[bq.alloc_outputs(s, rows, cols, device, stats=True) for _, s in schemes] for _ in range(n_units)]
     deqs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=device) for _ in range(n_units)]
     rngs = [torch.zeros(3, dtype=torch.float32, device=device) for _ in range(n_units)]
     stream = torch.cuda.current_stream(device)
@@ -317,10 +409,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     side = torch.cuda.Stream(device) if n_lanes > 1 else None
 
     def launch(j, kind, u, st, ws):
-        """Kernel `kind` of scheme j on unit u (mod n_units)."""
+        """Kernel `kind` of scheme j on unit u (mod n_units); "quantize_batch": every unit."""
         u %= n_units
         xi, q, s = xs[u], outs[u][j], schemes[j][1]
-        if sign_bits is not None and kind == "quantize":
+        if kind == "quantize_batch":
+            qb = qbs[j]
+            bq.bq_quantize_batch(X, s, qb.codes, qb.scales, qb.zero_points, qb.stats, ws, st)
+        elif sign_bits is not None and kind == "quantize":
             bq.bq_quantize_rt(xi, s, None, sign_bits, q.codes, q.scales, q.zero_points, q.stats, ws, st)
         elif sign_bits is not None and kind == "dequantize":
             bq.bq_dequantize_rt(q.codes, q.scales, q.zero_points, rows, cols, s, None, sign_bits, deqs[u], st)
@@ -345,12 +440,20 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         lanes = [(st, wss[0])] if n_lanes == 1 else [(st, wss[0]), (side, wss[1])]
         if n_lanes > 1:
             side.wait_stream(st)
-        for u in step_units(i):
+        if batched:
             for j in range(len(schemes)):
                 lane_st, lane_ws = lanes[j % n_lanes]
-                launch(j, "quantize", u, lane_st, lane_ws)
+                launch(j, "quantize_batch", 0, lane_st, lane_ws)
                 if dequant:
-                    launch(j, "dequantize", u, lane_st, lane_ws)
+                    for u in step_units(i):
+                        launch(j, "dequantize", u, lane_st, lane_ws)
+        else:
+            for u in step_units(i):
+                for j in range(len(schemes)):
+                    lane_st, lane_ws = lanes[j % n_lanes]
+                    launch(j, "quantize", u, lane_st, lane_ws)
+                    if dequant:
+                        launch(j, "dequantize", u, lane_st, lane_ws)
         if n_lanes > 1:
             st.wait_stream(side)
 
@@ -427,7 +530,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     n_per = max(8, min(64, 2 * n_units))
     kernels = []
     for j, (lab, s) in enumerate(schemes):
-        kinds = ["quantize"]
+        kinds = ["quantize_batch", "quantize"] if batched else ["quantize"]
         if two_pass[j]:
             kinds += ["range", "quantize_pass"]
         kinds += ["dequantize"]
@@ -438,15 +541,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 for u in range(n_units):       # every unit's range, for its quantize pass
                     launch(j, "range", u, stream, wss[0])
 
-            def seq(st, j=j, kind=kind):
-                for i in range(n_per):
+            reps = max(3, min(8, n_per)) if kind == "quantize_batch" else n_per
+
+            def seq(st, j=j, kind=kind, reps=reps):
+                for i in range(reps):
                     launch(j, kind, i, st, wss[0])
             seq(stream)                                  # warm
             g = None if args.eager else capture(seq)
-            kms = timed(g, lambda: seq(stream), n_per)
-            reuse = min(n_per, n_units) * kb[j][kind]
-            kernels.append({"kernel": f"{kind}:{lab}", "bytes": kb[j][kind], "ms": kms,
-                            "gbs": kb[j][kind] / (kms * 1e-3) / 1e9, "reuse_distance_bytes": reuse})
+            kms = timed(g, lambda: seq(stream), reps)
+            nbytes = kb[j]["quantize"] * n_units if kind == "quantize_batch" else kb[j][kind]
+            reuse = nbytes if kind == "quantize_batch" else min(n_per, n_units) * kb[j][kind]
+            kernels.append({"kernel": f"{kind}:{lab}", "bytes": nbytes, "ms": kms,
+                            "gbs": nbytes / (kms * 1e-3) / 1e9, "reuse_distance_bytes": reuse,
+                            **({"tensors": n_units} if kind == "quantize_batch" else {})})
             del g
     # the dominant kernel of the step: the slowest single kernel that the quantize step
     # launches (for two-pass schemes the range pass and the quantize pass count apart)
@@ -454,6 +561,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     def in_step(k):
         kind, lab = k["kernel"].split(":", 1)
+        if batched:
+            return kind == "quantize_batch"
         return kind in ("range", "quantize_pass") if is_two_pass[lab] else kind == "quantize"
     step_kernels = [k for k in kernels if in_step(k)]
     dom = max(step_kernels, key=lambda k: k["ms"])
@@ -474,6 +583,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         return None
     traffic = ncu_traffic(dom["kernel"], args.workload)
     n_launch_q = sum(2 if tp else 1 for tp in two_pass)
+    launches_per_step = len(schemes) if batched else units_per_step * n_launch_q
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -497,7 +607,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "l2": (f"inputs larger than L2: {n_units} distinct {'tensors' if len(hosts) > 1 else 'copies'} of "
                    f"{2 * rows * cols / 2**20:.1f} MiB rotate (L2 {l2 / 2**20:.0f} MiB)"),
             "parallelism": f"dp{world} (each GPU owns its own tensors, no collective on the data path)",
-            "launch": "eager" if args.eager else "CUDA graph of the K timed steps",
+            "launch": ("eager" if args.eager else "CUDA graph of the K timed steps")
+                      + ("; one bq_quantize_batch launch per scheme over the step's tensors" if batched
+                         else "; one bq_quantize call per tensor and scheme"),
             "streams": (f"{n_lanes} (the step's independent schemes alternate between two streams, "
                         "forked and joined inside the step)") if n_lanes > 1 else "1",
             "kernel_timing": (f"each kernel alone, {n_per} launches back to back over the rotating inputs "
@@ -512,7 +624,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "traffic": traffic, "algorithmic_bytes": dom["bytes"], "peak_source": peak_kind},
         "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in kk.items()} for kk in kernels],
         "qsnr": qsnr,
-        "gpu_launches": args.steps * units_per_step * n_launch_q,
+        "gpu_launches": args.steps * launches_per_step,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,
@@ -692,6 +804,9 @@ def cpu_baseline(workload, schemes_args, x_host, budget_s=10.0, signs=None):
 def run_reference(args, rank: int):
     if rank != 0:
         return None
+    if args.workload in GEMM_WORKLOADS:
+        return {"impl": "reference", "unavailable": "the GEMM workloads have no CPU arm (the oracle's float64 GEMM "
+                                                   "reference serves the parity tests only)"}
     schemes_args = WORKLOADS[args.workload]
     x_host = gen_inputs(args.workload, 0, 1)[0]
     xb = synth.bf16_bits(x_host)
@@ -744,8 +859,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="ffn_lognormal")
+    ap.add_argument("--workload", choices=list(WORKLOADS) + list(GEMM_WORKLOADS), default="ffn_lognormal")
     ap.add_argument("--tensors", type=int, default=0, help="tensors per step (FFN workloads; default 64)")
+    ap.add_argument("--per-tensor", action="store_true",
+                    help="FFN sets: one bq_quantize call per tensor instead of one batch call per scheme")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--serial", action="store_true", help="run the step's schemes one after another on one stream")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps one by one instead of as a CUDA graph")

@@ -90,6 +90,10 @@ def _lib() -> ctypes.CDLL:
         L.bq_tensor_range.argtypes = [vp, i32, i64, i64, sp, vp, vp, sz, vp]
         L.bq_quantize_with_range.restype = ctypes.c_int
         L.bq_quantize_with_range.argtypes = [vp, i32, i64, i64, sp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.bq_quantize_batch.restype = ctypes.c_int
+        L.bq_quantize_batch.argtypes = [vp, i32, i64, i64, i64, sp, vp, vp, vp, vp, vp, sz, vp]
+        L.bq_gemm.restype = ctypes.c_int
+        L.bq_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, sp, vp, i32, vp]
         L.bq_debug_skip_tile_copy.restype = ctypes.c_int
         L.bq_debug_skip_tile_copy.argtypes = [i32]
         L.bq_wait_timeouts.restype = ctypes.c_int
@@ -231,10 +235,42 @@ def bq_quantize_with_range(x: torch.Tensor, scheme: Scheme, range_in: torch.Tens
            "bq_quantize_with_range")
 
 
-def bq_debug_skip_tile_copy(tile: int) -> None:
-    """Test hook: the next flat quantize launch issues no copy for staged tile `tile`, so
-    the wait for it runs out (bounded) and bq_wait_timeouts counts it."""
-    _check(_lib().bq_debug_skip_tile_copy(int(tile)), "bq_debug_skip_tile_copy")
+def bq_quantize_batch(x: torch.Tensor, scheme: Scheme, codes: torch.Tensor, scales: torch.Tensor,
+                      zero_points: torch.Tensor | None, stats: torch.Tensor | None,
+                      workspace: torch.Tensor | None, stream=None) -> None:
+    """x: bf16 [batch, rows, cols] on the device; outputs preallocated (see alloc_batch_outputs);
+    stats: float64 [batch, 5] or None."""
+    batch, rows, cols = x.shape
+    sc = scheme.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().bq_quantize_batch(_ptr(x), DT["bf16"], batch, rows, cols, ctypes.byref(sc), _ptr(codes),
+                                    _ptr(scales), _ptr(zero_points), _ptr(stats), _ptr(workspace), ws_bytes,
+                                    _stream(stream)), "bq_quantize_batch")
+
+
+def bq_gemm(a: "Quantized", b: "Quantized", d: torch.Tensor, stream=None) -> None:
+    """D[m, n] = A[m, k] B[n, k]^T on the tensor cores from two quantized operands (same
+    MXFP8 or NVFP4 scheme, GEMM-layout scales); d: fp32 or bf16 [m, n] on the device."""
+    if a.scheme != b.scheme or a.cols != b.cols:
+        raise ValueError("operands need the same scheme and the same k")
+    m, n, k = a.rows, b.rows, a.cols
+    d_dt = {torch.bfloat16: DT["bf16"], torch.float32: DT["fp32"]}[d.dtype]
+    sc = a.scheme.c()
+    _check(_lib().bq_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(a.tensor_scale), _ptr(b.codes), _ptr(b.scales),
+                          _ptr(b.tensor_scale), m, n, k, ctypes.byref(sc), _ptr(d), d_dt, _stream(stream)), "bq_gemm")
+
+
+def gemm(a: "Quantized", b: "Quantized", dtype=torch.float32, stream=None) -> torch.Tensor:
+    """A B^T of two quantized operands (MXFP8 / NVFP4, GEMM-layout scales)."""
+    d = torch.empty((a.rows, b.rows), dtype=dtype, device=a.codes.device)
+    bq_gemm(a, b, d, stream)
+    return d
+
+
+def bq_debug_skip_tile_copy(warp: int) -> None:
+    """Test hook: in the next flat quantize launch, warp `warp` issues no copy for its first
+    staged tile, so its wait runs out (bounded) and bq_wait_timeouts counts it."""
+    _check(_lib().bq_debug_skip_tile_copy(int(warp)), "bq_debug_skip_tile_copy")
 
 
 def bq_dequantize(codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor | None,
@@ -364,6 +400,52 @@ def alloc_outputs(scheme: Scheme, rows: int, cols: int, device, stats: bool = Tr
     ts = torch.empty(1, dtype=torch.float32, device=device) if tb else None
     st = torch.empty(5, dtype=torch.float64, device=device) if stats else None
     return Quantized(s, rows, cols, codes, scales, zps, ts, st)
+
+
+@dataclass
+class QuantizedBatch:
+    scheme: Scheme
+    batch: int
+    rows: int
+    cols: int
+    codes: torch.Tensor             # uint8 [batch, rows, cols] (4-bit: [batch, rows, cols / 2])
+    scales: torch.Tensor            # [batch, one tensor's scales]
+    zero_points: torch.Tensor | None
+    stats: torch.Tensor | None      # float64 [batch, 5]
+
+    def tensor(self, b: int) -> Quantized:
+        """Tensor b's outputs as a Quantized (views, no copy)."""
+        return Quantized(self.scheme, self.rows, self.cols, self.codes[b], self.scales[b],
+                         None if self.zero_points is None else self.zero_points[b], None,
+                         None if self.stats is None else self.stats[b])
+
+
+def alloc_batch_outputs(scheme: Scheme, batch: int, rows: int, cols: int, device, stats: bool = True) -> QuantizedBatch:
+    s = scheme.resolved()
+    cb, sb, zb, _ = bq_buffer_sizes(s, rows, cols)
+    sdt = _scale_dtype_torch(s)
+    esz = torch.tensor([], dtype=sdt).element_size()
+    cols_b = cols // 2 if s.fmt in FOUR_BIT else cols
+    codes = torch.empty((batch, rows, cols_b), dtype=torch.uint8, device=device)
+    scales = torch.empty((batch, max(sb // esz, 1)), dtype=sdt, device=device)
+    zps = torch.empty((batch, zb // esz), dtype=sdt, device=device) if zb else None
+    st = torch.empty((batch, 5), dtype=torch.float64, device=device) if stats else None
+    return QuantizedBatch(s, batch, rows, cols, codes, scales, zps, st)
+
+
+def quantize_batch(x: torch.Tensor, scheme: Scheme, stats: bool = True, workspace: torch.Tensor | None = None,
+                   out: QuantizedBatch | None = None, stream=None) -> QuantizedBatch:
+    """Quantize a bf16 [batch, rows, cols] CUDA tensor (same-shape tensors, one launch);
+    per-tensor QSNR / kappa sums in stats[b]."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 3:
+        raise ValueError("x must be a 3-D bf16 CUDA tensor")
+    x = x.contiguous()
+    batch, rows, cols = x.shape
+    q = out or alloc_batch_outputs(scheme, batch, rows, cols, x.device, stats)
+    if stats and workspace is None:
+        workspace = new_workspace(x.device)
+    bq_quantize_batch(x, q.scheme, q.codes, q.scales, q.zero_points, q.stats if stats else None, workspace, stream)
+    return q
 
 
 def quantize(x: torch.Tensor, scheme: Scheme, stats: bool = True, workspace: torch.Tensor | None = None,

@@ -4,6 +4,7 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstddef>
@@ -14,6 +15,9 @@ namespace bq {
 namespace {
 
 constexpr int MAX_DEVICES = 64;
+// elements per call (per launch of a batch): chunk indices stay below 2^32 - 4 with room
+// for the flat kernel's "no span" index
+constexpr uint64_t MAX_ELEMS = (1ull << 36) - 2048;
 std::atomic<int> g_sm_count[MAX_DEVICES];
 
 struct Plan {
@@ -82,7 +86,7 @@ bq_status make_plan(const bq_scheme* s, int64_t rows, int64_t cols, Plan* p)
     if (p->gemm_layout && cols % 128 != 0) return BQ_ERR_SHAPE;
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return BQ_ERR_SHAPE;
     if (p->block && cols % p->block != 0) return BQ_ERR_SHAPE;
-    if (rows > 0 && (uint64_t)rows > ((1ull << 36) - 16) / (uint64_t)cols) return BQ_ERR_SHAPE;
+    if (rows > 0 && (uint64_t)rows > MAX_ELEMS / (uint64_t)cols) return BQ_ERR_SHAPE;
     if (rows >= (1ll << 31) || cols >= (1ll << 31)) return BQ_ERR_SHAPE;
 
     p->n = (uint64_t)rows * (uint64_t)cols;
@@ -194,11 +198,13 @@ bq_status quantize_pass(const Plan& p, const uint32_t* xw, int64_t rows, int64_t
         a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
         a.stats = stats; a.ws = ws;
         a.n_chunks = p.n_chunks;
-        a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
         a.lanes_per_group = (int32_t)(cols / 64);
         a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
         a.n_elems = (double)p.n;
         a.inv_unit = 1.0f / (float)cols;
+        a.batch = 1;
+        a.spans_per_tensor = (p.n_chunks + 3u) / 4u;
+        a.unit_oct = a.lanes_per_group > 8 ? (uint32_t)a.lanes_per_group / 8u : 1u;
         a.skip_tile = take_skip_tile();
         return cuda_status(launch_quant_flat(p.fmt, K_GROUP, p.had != 0, want_stats, a, s));
     }
@@ -228,8 +234,6 @@ bq_status quantize_pass(const Plan& p, const uint32_t* xw, int64_t rows, int64_t
     a.x = xw; a.codes = reinterpret_cast<uint8_t*>(codes); a.scales = scales; a.zps = zero_points;
     a.tensor_scale = tensor_scale; a.stats = stats; a.ws = ws;
     a.n_chunks = p.n_chunks;
-    // a warp tile is 32 lanes x 4 chunks
-    a.n_dtiles = (uint32_t)((p.n_chunks + 127u) / 128u);
     // groups: 16 elements -> 0 (four units per lane), 32 -> -1 (two per lane),
     // 64 and up -> lanes per group (one unit over block / 64 lanes)
     a.lanes_per_group = p.gran != BQ_PER_GROUP ? 1 : (p.block == 16 ? 0 : (p.block == 32 ? -1 : p.block / 64));
@@ -238,8 +242,30 @@ bq_status quantize_pass(const Plan& p, const uint32_t* xw, int64_t rows, int64_t
     a.inv_unit = p.block ? 1.0f / (float)p.block : 0.0f;
     if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
     a.range = range;
+    a.batch = 1;
+    a.spans_per_tensor = (p.n_chunks + 3u) / 4u;
+    a.unit_oct = a.lanes_per_group > 8 ? (uint32_t)a.lanes_per_group / 8u : 1u;
     a.skip_tile = take_skip_tile();
     return cuda_status(launch_quant_flat(p.fmt, kind_of(p.gran), p.had != 0, want_stats, a, s));
+}
+
+// Flat-kernel arguments of a batch of `batch` tensors of one plan (p describes one tensor).
+FlatArgs batch_args(const Plan& p, int64_t cols, uint32_t batch)
+{
+    FlatArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.n_chunks = p.n_chunks * batch;
+    a.lanes_per_group = p.gran == BQ_PER_ROW ? (int32_t)(cols / 64)
+                      : p.gran != BQ_PER_GROUP ? 1 : (p.block == 16 ? 0 : (p.block == 32 ? -1 : p.block / 64));
+    a.scale_fp16 = p.sdt == BQ_DT_FP16 ? 1 : 0;
+    a.n_elems = (double)p.n;
+    a.inv_unit = p.gran == BQ_PER_ROW ? 1.0f / (float)cols : 1.0f / (float)p.block;
+    if (p.gemm_layout) { a.gemm_layout = 1; a.gemm_nb = make_fastdiv(p.nb); }
+    a.batch = batch;
+    a.spans_per_tensor = p.n_chunks / 4u;
+    a.unit_oct = a.lanes_per_group > 8 ? (uint32_t)a.lanes_per_group / 8u : 1u;
+    a.skip_tile = take_skip_tile();
+    return a;
 }
 
 }  // namespace
@@ -385,10 +411,56 @@ bq_status bq_quantize_with_range(const void* x, int32_t x_dtype, int64_t rows, i
                          tensor_scale, stats, reinterpret_cast<uint8_t*>(workspace), range, s);
 }
 
-bq_status bq_debug_skip_tile_copy(int32_t tile)
+bq_status bq_debug_skip_tile_copy(int32_t warp)
 {
-    if (tile < 0) return BQ_ERR_INVALID_ARG;
-    g_skip_tile.store((uint32_t)tile, std::memory_order_release);
+    if (warp < 0) return BQ_ERR_INVALID_ARG;
+    g_skip_tile.store((uint32_t)warp, std::memory_order_release);
+    return BQ_OK;
+}
+
+bq_status bq_quantize_batch(const void* x, int32_t x_dtype, int64_t batch, int64_t rows, int64_t cols,
+                            const bq_scheme* scheme, void* codes, void* scales, void* zero_points,
+                            bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Plan p;
+    bq_status st = make_plan(scheme, rows, cols, &p);
+    if (st != BQ_OK) return st;
+    if (x_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    // row-local schemes that run on the flat kernel
+    const bool pow2_segments = cols % 64 == 0 && ((cols / 64) & (cols / 64 - 1)) == 0;
+    if (!(p.gran == BQ_PER_GROUP || p.gran == BQ_MX_BLOCK || (p.gran == BQ_PER_ROW && pow2_segments && cols <= 2048)))
+        return BQ_ERR_UNSUPPORTED;
+    if (batch < 0) return BQ_ERR_SHAPE;
+    if (batch > 1 && p.n % 64 != 0) return BQ_ERR_SHAPE;           // tensors of whole 64-element spans
+    if (batch > 1 && p.gemm_layout && rows % 128 != 0) return BQ_ERR_SHAPE;
+    const bool want_stats = stats != nullptr;
+    if (want_stats && (!workspace || workspace_bytes < WS_BYTES)) return BQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (batch == 0) return BQ_OK;
+    if (p.n == 0) {
+        if (want_stats) return cuda_status(cudaMemsetAsync(stats, 0, sizeof(bq_stats) * (size_t)batch, s));
+        return BQ_OK;
+    }
+    if (!x || !codes || !scales) return BQ_ERR_INVALID_ARG;
+    if (p.asym && !zero_points) return BQ_ERR_INVALID_ARG;
+    if (!aligned32(x) || !aligned32(codes)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(scales) || !aligned4(zero_points)) return BQ_ERR_ALIGNMENT;
+    // launches of at most one tensor per stats slot and MAX_ELEMS elements
+    const uint64_t per = std::min<uint64_t>((uint64_t)MAX_STAT_SLOTS, MAX_ELEMS / p.n);
+    const size_t scale_b = p.scale_bytes, zp_b = p.zp_bytes, code_b = p.code_bytes, x_b = p.n * 2;
+    for (uint64_t b0 = 0; b0 < (uint64_t)batch; b0 += per) {
+        const uint32_t nb = (uint32_t)std::min<uint64_t>(per, (uint64_t)batch - b0);
+        FlatArgs a = batch_args(p, cols, nb);
+        a.x = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(x) + b0 * x_b);
+        a.codes = reinterpret_cast<uint8_t*>(codes) + b0 * code_b;
+        a.scales = reinterpret_cast<uint8_t*>(scales) + b0 * scale_b;
+        a.zps = zero_points ? reinterpret_cast<uint8_t*>(zero_points) + b0 * zp_b : nullptr;
+        a.stats = want_stats ? stats + b0 : nullptr;
+        a.ws = reinterpret_cast<uint8_t*>(workspace);
+        const int kind = p.gran == BQ_MX_BLOCK ? K_MX : K_GROUP;
+        const cudaError_t e = launch_quant_flat(p.fmt, kind, p.had != 0, want_stats, a, s);
+        if (e != cudaSuccess) return BQ_ERR_CUDA;
+    }
     return BQ_OK;
 }
 
@@ -523,10 +595,60 @@ bq_status bq_dequantize_rt(const void* codes, const void* scales, const void* ze
 bq_status bq_wait_timeouts(uint32_t* count, int32_t reset)
 {
     if (!count) return BQ_ERR_INVALID_ARG;
-    unsigned int c = 0;
+    unsigned int c = 0, g = 0;
     if (bq::flat_wait_timeouts(&c, reset != 0) != cudaSuccess) return BQ_ERR_CUDA;
-    *count = c;
+    if (bq::gemm_wait_timeouts(&g, reset != 0) != cudaSuccess) return BQ_ERR_CUDA;
+    *count = c + g;
     return BQ_OK;
+}
+
+bq_status bq_gemm(const void* a_codes, const void* a_scales, const float* a_tensor_scale,
+                  const void* b_codes, const void* b_scales, const float* b_tensor_scale,
+                  int64_t m, int64_t n, int64_t k, const bq_scheme* scheme,
+                  void* d, int32_t d_dtype, void* stream)
+{
+    if (!scheme) return BQ_ERR_INVALID_ARG;
+    Plan p;
+    bq_status st = make_plan(scheme, 1, k, &p);
+    if (st != BQ_OK) return st;
+    int kind;
+    uint32_t fmt_code;
+    if (p.gran == BQ_MX_BLOCK && (p.fmt == BQ_FP8_E4M3 || p.fmt == BQ_FP8_E5M2)) {
+        kind = GEMM_MXF8;
+        fmt_code = p.fmt == BQ_FP8_E4M3 ? 0u : 1u;
+    } else if (p.gran == BQ_NV_BLOCK && p.fmt == BQ_FP4_E2M1) {
+        kind = GEMM_NVF4;
+        fmt_code = 1u;
+    } else {
+        return BQ_ERR_UNSUPPORTED;
+    }
+    if (!p.gemm_layout) return BQ_ERR_UNSUPPORTED;
+    if (d_dtype != BQ_DT_FP32 && d_dtype != BQ_DT_BF16) return BQ_ERR_UNSUPPORTED;
+    const int64_t kstep = kind == GEMM_MXF8 ? 128 : 256;
+    if (m < 0 || n < 0 || k <= 0 || m % 128 != 0 || n % 128 != 0 || k % kstep != 0) return BQ_ERR_SHAPE;
+    if (m >= (1ll << 31) || n >= (1ll << 31) || k >= (1ll << 31) || (uint64_t)m * (uint64_t)n >= (1ull << 40))
+        return BQ_ERR_SHAPE;
+    if (m == 0 || n == 0) return BQ_OK;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !d) return BQ_ERR_INVALID_ARG;
+    if (kind == GEMM_NVF4 && (!a_tensor_scale || !b_tensor_scale)) return BQ_ERR_INVALID_ARG;
+    auto al16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+    if (!al16(a_codes) || !al16(b_codes) || !al16(a_scales) || !al16(b_scales) || !al16(d)) return BQ_ERR_ALIGNMENT;
+    if (!aligned4(a_tensor_scale) || !aligned4(b_tensor_scale)) return BQ_ERR_ALIGNMENT;
+    GemmArgs g;
+    std::memset(&g, 0, sizeof g);
+    g.a = a_codes; g.b = b_codes;
+    g.sfa = reinterpret_cast<const uint8_t*>(a_scales);
+    g.sfb = reinterpret_cast<const uint8_t*>(b_scales);
+    g.a_tensor_scale = a_tensor_scale; g.b_tensor_scale = b_tensor_scale;
+    g.d = d;
+    g.m = (uint32_t)m; g.n = (uint32_t)n;
+    g.kb = (uint32_t)(kind == GEMM_MXF8 ? k : k / 2);
+    g.k_stages = g.kb / 128u;
+    g.sf_tiles_per_row = p.nb / 4u;
+    g.ldd = (uint32_t)n;
+    g.elem_fmt = fmt_code;
+    g.d_bf16 = d_dtype == BQ_DT_BF16 ? 1 : 0;
+    return cuda_status(launch_gemm(kind, g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 double bq_stats_qsnr_db(const bq_stats* host_stats)

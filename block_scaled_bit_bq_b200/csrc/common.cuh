@@ -225,6 +225,8 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 // a - b, rounded once (fma with -1 is exactly the subtraction)
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, splat(-1.0f), a); }
+// -a (exact, sign bits flipped)
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
 // max(a, |b|, |c|) in one three-input max
 __device__ __forceinline__ float amax3(float a, float b, float c)
@@ -445,10 +447,12 @@ struct RangeSlot { float amax, vmin, vmax, pad; };
 
 struct StatSlot { double err2, x2, ksum, kmax, nunits, ss; };
 
+// stats slots: one per CTA (MAX_GRID), or one per warp for the flat kernel's batches
+constexpr int MAX_STAT_SLOTS = 4096;
 constexpr size_t WS_HEADER_BYTES = 256;
 constexpr size_t WS_RANGE_OFF = WS_HEADER_BYTES;
 constexpr size_t WS_STAT_OFF = WS_RANGE_OFF + sizeof(RangeSlot) * MAX_GRID;
-constexpr size_t WS_BYTES = WS_STAT_OFF + sizeof(StatSlot) * MAX_GRID;
+constexpr size_t WS_BYTES = WS_STAT_OFF + sizeof(StatSlot) * MAX_STAT_SLOTS;
 
 __device__ __forceinline__ WsHeader* ws_header(uint8_t* ws) { return reinterpret_cast<WsHeader*>(ws); }
 __device__ __forceinline__ RangeSlot* ws_range(uint8_t* ws) { return reinterpret_cast<RangeSlot*>(ws + WS_RANGE_OFF); }

@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(256) k_qsnr(const DequantArgs a)
 // value is multiplied by the normalisation, the signed columns negated and the result
 // written. The per-column factor is not undone (the codes stand for x times it).
 template <int FMT, int SK, int OUT>
-__global__ void __launch_bounds__(256) k_dequant_rt(const DequantArgs a, const uint32_t* sign_bits, uint32_t rows,
+__global__ void __launch_bounds__(RT_THREADS, 8) k_dequant_rt(const DequantArgs a, const uint32_t* sign_bits, uint32_t rows,
                                                     uint32_t cols, float norm)
 {
     constexpr int NC = SpanCodes<FMT, 1>::n;
@@ -436,7 +436,7 @@ template <auto KERN>
 cudaError_t launch_row_kernel(const DequantArgs& a, const uint32_t* sign_bits, uint32_t rows, uint32_t cols,
                               float norm, cudaStream_t st)
 {
-    const int block = cols / 16 < 256u ? (int)(cols / 16) : 256;   // a thread per chunk, up to 256
+    const int block = cols / 16 < (uint32_t)RT_THREADS ? (int)(cols / 16) : RT_THREADS;   // a thread per chunk, up to RT_THREADS
     const size_t smem = (size_t)rot_row_floats(cols) * 4;
     if (smem > 48u * 1024u) {
         const cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -21,16 +21,18 @@ struct FlatArgs {
     bq_stats* stats;
     uint8_t* ws;
     const float* range;         // per-tensor / NV: {amax, min, max} of the (rotated) tensor
-    uint32_t n_chunks;          // rows * cols / 16
-    uint32_t n_dtiles;          // ceil(n_chunks / 128): a warp takes 128 chunks (one tile) per step
+    uint32_t n_chunks;          // rows * cols / 16 (of the whole batch)
+    uint32_t batch;             // tensors (1: one tensor; > 1: contiguous, same shape, no ragged span)
+    uint32_t spans_per_tensor;  // 64-element spans of one tensor (the last one may be partial)
+    uint32_t unit_oct;          // octets (8 spans) per partition unit: 1, or lanes_per_group / 8
     int32_t lanes_per_group;    // per-group: 0 (block 16), -1 (block 32), block / 64 (64..512)
     int32_t scale_fp16;         // 1: fp16 scales and zero points
     double n_elems;
     float inv_unit;             // 1 / elements per scaling unit (kappa)
     FastDiv gemm_nb;            // MX / NV scales in the GEMM layout: division by blocks per row
     int32_t gemm_layout;        // 1: scales in the GEMM layout; 0: row-major
-    uint32_t skip_tile;         // fault injection for tests: the copy of this tile is never
-                                // issued (its wait runs out); 0xFFFFFFFF: none
+    uint32_t skip_tile;         // fault injection for tests: this warp issues no copy for its
+                                // first tile (its wait runs out); 0xFFFFFFFF: none
 };
 
 // Per-row kernel: one CTA per row at a time.
@@ -123,6 +125,30 @@ struct DequantArgs {
     FastDiv gemm_nb;            // MX / NV scales in the GEMM layout (see FlatArgs)
     int32_t gemm_layout;
 };
+
+// Block-scaled GEMM D = A B^T on the tensor cores (codes and GEMM-layout scales as
+// bq_quantize writes them).
+enum { GEMM_MXF8 = 0, GEMM_NVF4 = 1 };
+
+struct GemmArgs {
+    const void* a;              // codes [m, kb] bytes, K-major
+    const void* b;              // codes [n, kb] bytes, K-major
+    const uint8_t* sfa;         // GEMM-layout scales of A (512-byte tiles)
+    const uint8_t* sfb;
+    const float* a_tensor_scale;  // NV: fp32 tensor scales (else unused)
+    const float* b_tensor_scale;
+    void* d;                    // [m, n] row-major, fp32 or bf16
+    uint32_t m, n, kb;          // kb: bytes of a row of codes (k, or k / 2 for FP4)
+    uint32_t k_stages;          // kb / 128
+    uint32_t sf_tiles_per_row;  // scale tiles per 128-row tile (blocks per row / 4)
+    uint32_t ldd;               // elements per row of D (n)
+    uint32_t elem_fmt;          // MMA element format code (E4M3 0, E5M2 1; E2M1 1 for NV)
+    int32_t d_bf16;
+};
+
+cudaError_t launch_gemm(int kind, const GemmArgs& g, cudaStream_t st);
+// Waits of the GEMM kernel that gave up (each leaves that call's D incomplete). Synchronous.
+cudaError_t gemm_wait_timeouts(unsigned int* count, bool reset);
 
 // Scale kinds for dequantize / QSNR.
 enum { SK_F32 = 0, SK_F16 = 1, SK_UE8M0 = 2, SK_NV = 3 };

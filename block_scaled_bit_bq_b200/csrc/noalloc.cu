@@ -15,7 +15,7 @@ namespace bq {
 
 namespace {
 
-// The scratch every bq_quantize_noalloc call uses: WS_BYTES (128 KiB + 256 B), enough
+// The scratch every bq_quantize_noalloc call uses: WS_BYTES (224 KiB + 256 B), enough
 // for the largest grid the kernels launch. Every GPU that loads the library holds one
 // copy until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[WS_BYTES];

@@ -485,10 +485,12 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
                 pack_int<FMT>(t, q);
             } else {
                 uint32_t pr[8];
+                const float2 D = splat(d), NRN = splat(-rn);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
+                    // RN(x / d), the residual taken negated so that -0 keeps its sign
                     const float2 q0 = mul2(y[i], RN);
-                    r[i] = fma2(fma2(q0, ND, y[i]), RN, q0);                  // RN(x / d)
+                    r[i] = fma2(fma2(q0, D, neg2(y[i])), NRN, q0);
                     pr[i] = cvt_pair<FMT>(r[i].y, r[i].x);
                 }
                 pack_pairs<FMT>(pr, q);
@@ -699,7 +701,7 @@ __device__ __forceinline__ void store_span4(uint8_t* codes, uint32_t span, uint3
 {
     if constexpr (Fmt<FMT>::four) {
         const uint32_t c0 = SPAN * span;
-        if (c0 + SPAN <= n_chunks) {
+        if (c0 < n_chunks && n_chunks - c0 >= (uint32_t)SPAN) {
             st_v8(codes + (size_t)span * 32, v);
         } else {
 #pragma unroll
@@ -712,21 +714,96 @@ __device__ __forceinline__ void store_span4(uint8_t* codes, uint32_t span, uint3
     }
 }
 
+// The part of the work a warp owns. The tensor (or each tensor of a batch) is a run of
+// spans of 64 elements; spans are grouped into octets of 8 (1 KiB, one tensor-map box),
+// and octets into partition units of `unit_oct` octets (a group of more than 8 lanes
+// needs its whole tile). A batch gives each tensor its own group of warps (every warp
+// sees one tensor); a tensor's units are split evenly over its warps, so the warps of a
+// launch finish within one unit of each other.
+struct WarpRange {
+    uint32_t tensor;        // index in the batch
+    uint64_t base;          // global span index of the tensor's first span
+    uint32_t oct0, oct1;    // the warp's octets of that tensor, [oct0, oct1)
+};
+
+__device__ __forceinline__ WarpRange warp_range(uint32_t w, uint32_t nw, const FlatArgs& a)
+{
+    WarpRange r;
+    const uint64_t B = a.batch, W = nw;
+    // tensor b's warps are [floor(W b / B), floor(W (b + 1) / B)) (B <= W)
+    const uint32_t b = (uint32_t)(((uint64_t)(w + 1) * B - 1) / W);
+    const uint32_t g0 = (uint32_t)(W * b / B), g1 = (uint32_t)(W * (b + 1) / B);
+    const uint64_t octs = ((uint64_t)a.spans_per_tensor + 7) / 8;
+    const uint64_t units = octs / a.unit_oct, i = w - g0, n = g1 - g0;
+    r.tensor = b;
+    r.base = (uint64_t)b * a.spans_per_tensor;
+    r.oct0 = (uint32_t)(units * i / n * a.unit_oct);
+    r.oct1 = (uint32_t)(units * (i + 1) / n * a.unit_oct);
+    return r;
+}
+
+// Batched stats: every warp's sums go to its own slot; the last CTA sums, for each tensor,
+// the slots of that tensor's warps in warp order (a warp of the last CTA per tensor, its
+// lanes over the slots, then a fixed xor tree), so the result is bit-reproducible.
+__device__ __forceinline__ void finish_stats_batch(Acc mine, uint8_t* ws, bq_stats* out, uint32_t w, uint32_t nw,
+                                                   uint32_t batch)
+{
+    __shared__ bool is_last;
+    AccD m;
+    m.err2 = mine.err2; m.x2 = mine.x2; m.ksum = mine.ksum; m.kmax = (double)mine.kmax; m.nunits = (double)mine.nunits;
+    const AccD t = warp_reduce_acc(m);
+    StatSlot* slots = ws_stats(ws);
+    WsHeader* h = ws_header(ws);
+    if ((threadIdx.x & 31) == 0) {
+        slots[w] = StatSlot{t.err2, t.x2, t.ksum, t.kmax, t.nunits, 0.0};
+        __threadfence();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomic_add_acq_rel(&h->counter_stats, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!is_last) return;
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, nwib = blockDim.x >> 5;
+    for (uint32_t b = wib; b < batch; b += nwib) {
+        const uint32_t g0 = (uint32_t)((uint64_t)nw * b / batch), g1 = (uint32_t)((uint64_t)nw * (b + 1) / batch);
+        AccD a;
+        for (uint32_t i = g0 + lane; i < g1; i += 32) {
+            const double* p = reinterpret_cast<const double*>(&slots[i]);
+            a.err2 += __ldcg(p + 0); a.x2 += __ldcg(p + 1); a.ksum += __ldcg(p + 2);
+            a.kmax = fmax(a.kmax, __ldcg(p + 3)); a.nunits += __ldcg(p + 4);
+        }
+        a = warp_reduce_acc(a);
+        if (lane == 0) {
+            bq_stats r;
+            r.err2 = a.err2; r.x2 = a.x2; r.kappa_sum = a.ksum; r.kappa_max = a.kmax; r.n_units = a.nunits;
+            out[b] = r;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) h->counter_stats = 0u;   // ready for the next call on this workspace
+}
+
 template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(const __grid_constant__ CUtensorMap xmap,
+                                                                  const __grid_constant__ CUtensorMap xmap32,
                                                                   const FlatArgs a)
 {
     using F = Fmt<FMT>;
     extern __shared__ uint8_t flat_smem[];
     __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    // warps numbered across the CTAs first: the last, partly filled round of tiles (rows)
-    // spreads over every CTA, and so over every SM, instead of filling the first CTAs
-    const uint32_t warp = wib * gridDim.x + blockIdx.x;
+    // warps numbered CTA by CTA: a CTA's warps own neighbouring ranges
+    const uint32_t warp = blockIdx.x * FLAT_WARPS + wib;
     const uint32_t nwarps = gridDim.x * FLAT_WARPS;
     const uint32_t buf0 = ((smem_addr(flat_smem) + 1023u) & ~1023u) + (uint32_t)wib * NST * TILE_BYTES;
     const uint32_t bar0 = smem_addr(&bars[wib][0]);
-    const uint32_t rows_mapped = a.n_chunks / SPAN;     // whole rows the tensor map covers
+    const uint32_t rows_mapped = a.n_chunks / SPAN;     // whole spans the tensor map covers
+    const WarpRange wr = warp_range(warp, nwarps, a);
+    // the warp's spans, global indices [first_span, end_span) (32-bit: a launch has fewer
+    // than 2^30 spans); tile k: spans first_span + 32 k .., octets oct0 + 4 k ..
+    const uint32_t first_span = (uint32_t)wr.base + 8u * wr.oct0;
+    const uint32_t end_span = (uint32_t)wr.base + min(8u * wr.oct1, a.spans_per_tensor);
+    const uint32_t n_oct = wr.oct1 - wr.oct0;
+    const uint32_t n_tiles = (n_oct + 3) / 4;
 
     if (lane == 0) {
         for (int s = 0; s < NST; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -735,18 +812,29 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
     __syncwarp();
 
     uint32_t inflight = 0, parity = 0;                  // per stage bits (warp-uniform)
-    auto issue = [&](uint32_t t, int s) {
-        if (t < a.n_dtiles && t * 32 < rows_mapped) {
-            // (t == skip_tile only under the test hook: no copy, so the wait runs out)
-            if (lane == 0 && t != a.skip_tile) {
-                mbar_arrive_expect_tx(bar0 + 8 * s, TILE_BYTES);
-                tma_load_2d(buf0 + s * TILE_BYTES, &xmap, bar0 + 8 * s, 0, (int)(t * 32));
+    // tile k goes in as one 32-span box when it is whole, else as one 8-span box per
+    // octet that the map covers (boxes past the map's last span are filled with zeros by
+    // the lanes that own them)
+    auto issue = [&](uint32_t k, int s) {
+        if (k >= n_tiles) return;
+        const uint32_t n = min(4u, n_oct - 4 * k), first = first_span + 32 * k;
+        if (first >= rows_mapped) return;
+        // (the test hook: warp skip_tile issues no copy for its first tile, so its wait runs out)
+        if (lane == 0 && !(k == 0 && warp == a.skip_tile)) {
+            const uint32_t dst = buf0 + s * TILE_BYTES, bar = bar0 + 8 * s;
+            if (n == 4) {
+                mbar_arrive_expect_tx(bar, TILE_BYTES);
+                tma_load_2d(dst, &xmap32, bar, 0, (int)first);
+            } else {
+                const uint32_t boxes = min(n, (rows_mapped - first + 7) / 8);
+                mbar_arrive_expect_tx(bar, boxes * 1024u);
+                for (uint32_t j = 0; j < boxes; ++j) tma_load_2d(dst + j * 1024u, &xmap, bar, 0, (int)(first + 8 * j));
             }
-            inflight |= 1u << s;
         }
+        inflight |= 1u << s;
     };
 #pragma unroll
-    for (int s = 0; s < NST; ++s) issue(warp + s * nwarps, s);
+    for (int s = 0; s < NST; ++s) issue((uint32_t)s, s);
 
     TensorCtx tc{};
     PlainUnit<FMT> tu{};
@@ -785,32 +873,45 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
     }
     // per-group units: 16 elements (one chunk), 32 (two), 64 and up (the span, T lanes)
     const int T = (GK == K_GROUP && a.lanes_per_group > 0) ? a.lanes_per_group : 1;
+    // span index of lanes with nothing to do: its chunks (from 0xFFFFFFF8 on) lie past every
+    // tensor's end (at most 2^32 - 128 chunks), and no guard on them wraps around
+    constexpr uint32_t NO_SPAN = 0xFFFFFFFFu / SPAN - 1u;
 
     Acc acc;
     bool ok = true;
     int s = 0;
-    for (uint32_t t = warp; t < a.n_dtiles; t += nwarps) {
+    for (uint32_t k = 0; k < n_tiles; ++k) {
         const Row row{buf0 + s * TILE_BYTES + lane * ROW_BYTES, (uint32_t)(lane & 7)};
-        const uint32_t span = t * 32 + lane;
+        const uint32_t n = min(4u, n_oct - 4 * k), tspan = first_span + 32 * k;
+        const uint32_t gspan = tspan + (uint32_t)lane;            // the lane's span
+        const bool mine = gspan < end_span;
+        const uint32_t span = mine ? gspan : NO_SPAN;
         if (inflight >> s & 1u) {
             const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, parity >> s & 1u));
             // a stage whose wait gave up stays in flight: the drain below waits for it
             if (!got) { ok = false; break; }
             parity ^= 1u << s;
             inflight &= ~(1u << s);
-        } else {
-            // no row of this tile is covered by the tensor map
-            const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int k = 0; k < SPAN; ++k) row_put_chunk(row, k, z);
         }
-        if (span == rows_mapped && rows_mapped * SPAN < a.n_chunks) {
-            // the ragged end: chunks past the last whole row come from global memory
-            for (int k = 0; k < SPAN; ++k) {
+        if ((uint32_t)lane >= 8 * n || (n < 4 && tspan + 8u * ((uint32_t)lane / 8) >= rows_mapped) ||
+            tspan >= rows_mapped) {
+            // the lane's row is outside this tile, or its box was not issued (past the
+            // map's last span): zeros (fast paths sum every lane's values), or for the span
+            // holding the ragged end, its chunks from global memory
+            const uint32_t c0 = SPAN * gspan;
+#pragma unroll 1
+            for (int kk = 0; kk < SPAN; ++kk) {
                 uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                const uint32_t c = SPAN * span + k;
+                if (mine && c0 + kk < a.n_chunks) ld_nc_v8(a.x + (size_t)(c0 + kk) * 8, w);
+                row_put_chunk(row, kk, w);
+            }
+        } else if (mine && gspan == rows_mapped && rows_mapped * SPAN < a.n_chunks) {
+            // the ragged end inside a mapped box (zero filled there): from global memory
+            for (int kk = 0; kk < SPAN; ++kk) {
+                uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                const uint32_t c = SPAN * span + kk;
                 if (c < a.n_chunks) ld_nc_v8(a.x + (size_t)c * 8, w);
-                row_put_chunk(row, k, w);
+                row_put_chunk(row, kk, w);
             }
         }
         fence_proxy_async();
@@ -830,7 +931,7 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
             else span_n4<FMT, HAD, STATS, EXACT>(row, span, a, acc, lane, T, span4);
         }
         __syncwarp();                       // every lane is done with the buffer
-        issue(t + NST * nwarps, s);
+        issue(k + NST, s);
         s = (s + 1 == NST) ? 0 : s + 1;
 
         store_span4<FMT>(a.codes, span, a.n_chunks, span4);
@@ -841,18 +942,18 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
             if (a.gemm_layout) {
                 if (c0 < a.n_chunks) *reinterpret_cast<uint32_t*>(sc + gemm_unit_offset(c0, a.gemm_nb)) = scodes;
-            } else if (c0 + SPAN <= a.n_chunks) {
+            } else if (c0 < a.n_chunks && a.n_chunks - c0 >= (uint32_t)SPAN) {
                 *reinterpret_cast<uint32_t*>(sc + c0) = scodes;
             } else {
-                for (int k = 0; k < SPAN; ++k)
-                    if (c0 + k < a.n_chunks) sc[c0 + k] = (uint8_t)(scodes >> (8 * k));
+                for (int kk = 0; kk < SPAN; ++kk)
+                    if (c0 + kk < a.n_chunks) sc[c0 + kk] = (uint8_t)(scodes >> (8 * kk));
             }
         } else if constexpr (GK == K_MX) {
             // two UE8M0 block scales (in the GEMM layout: two adjacent bytes)
             uint8_t* sc = reinterpret_cast<uint8_t*>(a.scales);
             if (a.gemm_layout) {
                 if (c0 < a.n_chunks) *reinterpret_cast<uint16_t*>(sc + gemm_unit_offset(c0 / 2, a.gemm_nb)) = (uint16_t)scodes;
-            } else if (c0 + SPAN <= a.n_chunks) {
+            } else if (c0 < a.n_chunks && a.n_chunks - c0 >= (uint32_t)SPAN) {
                 *reinterpret_cast<uint16_t*>(sc + c0 / 2) = (uint16_t)scodes;
             } else if (c0 < a.n_chunks) {
                 sc[c0 / 2] = (uint8_t)scodes;
@@ -863,13 +964,17 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
         // a tile never arrived: record it, give the other loads in flight their chance
         // to land (bounded) and stop; the results of this call are incomplete
         if (lane == 0) atomicAdd(&g_flat_wait_timeouts, 1u);
-        for (int k = 0; k < NST; ++k)
-            if (inflight >> k & 1u) (void)mbar_wait(bar0 + 8 * k, parity >> k & 1u);
+        for (int kk = 0; kk < NST; ++kk)
+            if (inflight >> kk & 1u) (void)mbar_wait(bar0 + 8 * kk, parity >> kk & 1u);
     }
 
     if constexpr (STATS) {
-        // per-tensor kappa comes from the totals: amax / sqrt(sum y^2 / n)
-        finish_stats(acc, a.ws, a.stats, GK == K_TENSOR, tc.amax, a.n_elems, true);
+        if (a.batch > 1) {
+            finish_stats_batch(acc, a.ws, a.stats, warp, nwarps, a.batch);
+        } else {
+            // per-tensor kappa comes from the totals: amax / sqrt(sum y^2 / n)
+            finish_stats(acc, a.ws, a.stats, GK == K_TENSOR, tc.amax, a.n_elems, true);
+        }
     }
 }
 
@@ -1230,7 +1335,7 @@ __device__ __forceinline__ void rt_chunk(const float2 (&y)[8], const PlainUnit<F
 }
 
 template <int FMT, bool MX>
-__global__ void __launch_bounds__(256, 3) k_quant_rt(const RtArgs a)
+__global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
@@ -1401,9 +1506,7 @@ unsigned grid_for(uint64_t min_items_per_cta, uint64_t total_items)
     return (unsigned)g;
 }
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
 EncodeTiled encode_tiled()
@@ -1420,9 +1523,12 @@ EncodeTiled encode_tiled()
     return reinterpret_cast<EncodeTiled>(f);
 }
 
-// x seen as rows of 64 bf16 (128 bytes): boxes of 32 rows, 128-byte swizzle, zero fill
-// past the last row. rows = 0: a zeroed map that no launch reads.
-cudaError_t x_rows_map(const uint32_t* x, uint32_t rows, CUtensorMap* map)
+namespace {
+
+// x seen as rows of 64 bf16 (128 bytes): boxes of box_rows rows (8: one octet, 1 KiB;
+// 32: a whole tile), 128-byte swizzle, zero fill past the last row. rows = 0: a zeroed
+// map that no launch reads.
+cudaError_t x_rows_map(const uint32_t* x, uint32_t rows, uint32_t box_rows, CUtensorMap* map)
 {
     *map = CUtensorMap{};
     if (rows == 0) return cudaSuccess;
@@ -1430,7 +1536,7 @@ cudaError_t x_rows_map(const uint32_t* x, uint32_t rows, CUtensorMap* map)
     if (!enc) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {64, rows};
     const cuuint64_t strides[1] = {ROW_BYTES};
-    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint32_t*>(x), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1527,8 +1633,8 @@ cudaError_t run_tile2d_hs(bool had, bool stats, const Tile2dArgs& a, cudaStream_
 template <int FMT, bool MX>
 cudaError_t run_rt(const RtArgs& a, cudaStream_t st)
 {
-    // a thread per chunk of the row, up to 256 (narrow rows: more CTAs per SM)
-    const int block = a.cpr < 256u ? (int)a.cpr : 256;
+    // a thread per chunk of the row, up to RT_THREADS (narrow rows: more CTAs per SM)
+    const int block = a.cpr < (uint32_t)RT_THREADS ? (int)a.cpr : RT_THREADS;
     constexpr auto kern = k_quant_rt<FMT, MX>;
     const size_t smem = (size_t)rot_row_floats(a.cols) * 4;
     if (smem > 48u * 1024u) {
@@ -1550,12 +1656,20 @@ cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
 {
     constexpr int block = FLAT_WARPS * 32;
     constexpr auto kern = k_quant_flat<FMT, GK, HAD, STATS, EXACT>;
-    CUtensorMap map;
-    const cudaError_t e = x_rows_map(a.x, a.n_chunks / SPAN, &map);
+    CUtensorMap map, map32;
+    cudaError_t e = x_rows_map(a.x, a.n_chunks / SPAN, 8u, &map);
     if (e != cudaSuccess) return e;
-    // one tile per warp at least
-    const unsigned grid = grid_for<kern, block, FLAT_SMEM>(FLAT_WARPS, a.n_dtiles);
-    kern<<<grid, block, FLAT_SMEM, st>>>(map, a);
+    e = x_rows_map(a.x, a.n_chunks / SPAN, 32u, &map32);
+    if (e != cudaSuccess) return e;
+    // one partition unit per warp at least, and (a batch) a warp per tensor at least;
+    // at most one stats slot per warp
+    const uint64_t units = (uint64_t)a.batch * ((((uint64_t)a.spans_per_tensor + 7) / 8) / a.unit_oct);
+    unsigned grid = grid_for<kern, block, FLAT_SMEM>(FLAT_WARPS, units);
+    const unsigned min_grid = (a.batch + FLAT_WARPS - 1) / FLAT_WARPS;
+    if (grid < min_grid) grid = min_grid;
+    if (grid > MAX_STAT_SLOTS / FLAT_WARPS) grid = MAX_STAT_SLOTS / FLAT_WARPS;
+    if (grid * FLAT_WARPS < a.batch) return cudaErrorInvalidValue;
+    kern<<<grid, block, FLAT_SMEM, st>>>(map, map32, a);
     return cudaGetLastError();
 }
 

@@ -826,11 +826,13 @@ __device__ __forceinline__ bool fp_chunk_fast(const float2 (&y)[8], const FpQ& u
                                               float2& ce2, float2& cx2)
 {
     uint32_t pr[8];
-    const float2 RN = splat(u.rn), NS = splat(-u.s);
+    const float2 RN = splat(u.rn), NS = splat(-u.s), S = splat(u.s), NRN = splat(-u.rn);
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
+        // RN(x / s) = RN(q0 - (q0 s - x) rn): the residual is taken negated so that a -0
+        // input keeps its sign (-0 + -0); every nonzero result is the same either way
         const float2 q0 = mul2(y[p], RN);
-        const float2 q1 = fma2(fma2(q0, NS, y[p]), RN, q0);       // RN(x / s)
+        const float2 q1 = fma2(fma2(q0, S, neg2(y[p])), NRN, q0);
         pr[p] = cvt_pair<FMT>(q1.y, q1.x);
     }
     pack_pairs<FMT>(pr, w);

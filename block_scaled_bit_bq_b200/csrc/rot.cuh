@@ -20,6 +20,11 @@
 
 namespace bq {
 
+// Threads per CTA of the row-transform kernels (a row at a time): 128 keeps every thread
+// busy in both passes of a 4096-column row (n / 32 pairs each) and lets 6-8 CTAs, so as
+// many rows, share an SM.
+constexpr int RT_THREADS = 128;
+
 // Floats of shared memory for a row of n values.
 __host__ __device__ constexpr uint32_t rot_row_floats(uint32_t n) { return n + n / 16; }
 

@@ -60,8 +60,8 @@
  *    holding exact integers;
  *  - tensor_scale: one fp32 (NV only).
  *
- * Shapes: rows >= 0, cols > 0, cols % 16 == 0 (and cols % block == 0); rows * cols <
- * 2^36. rows == 0 is a valid empty call. Alignment: x, codes and out 32-byte aligned;
+ * Shapes: rows >= 0, cols > 0, cols % 16 == 0 (and cols % block == 0); rows * cols <=
+ * 2^36 - 2048. rows == 0 is a valid empty call. Alignment: x, codes and out 32-byte aligned;
  * scales, zero points and the tensor scale 4-byte aligned.
  */
 #ifndef BQ_H
@@ -222,6 +222,29 @@ bq_status bq_quantize_with_range(const void* x, int32_t x_dtype, int64_t rows, i
                                  bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * A batch of same-shape tensors in one call: x is [batch, rows, cols] bf16, contiguous;
+ * tensor b is quantized exactly as bq_quantize would quantize it alone (the same codes,
+ * scales and zero points), with its QSNR and kappa sums in stats[b] (device, [batch],
+ * or NULL). The experiment of "INT vs FP at fine granularity" §4.2 compares formats on
+ * thousands of weight tensors of one model; a batch serves such sets (e.g. all FFN
+ * weights of a layer type) with one launch instead of one per tensor.
+ * Outputs: codes [batch, rows, cols] (4-bit formats [batch, rows, cols / 2]), scales and
+ * zero points [batch] x the one-tensor size (bq_buffer_sizes(rows, cols) each), tensor b's
+ * at b times that size. Schemes: per-group and MX (either scale layout), and per-row
+ * schemes with cols a power-of-two multiple of 64 up to 2048, each with or without the
+ * block-16 rotation (else BQ_ERR_UNSUPPORTED: per-tensor and NV schemes need a range
+ * per tensor first, use bq_quantize per tensor). batch > 1 needs rows * cols % 64 == 0,
+ * and rows % 128 == 0 for scale_layout = BQ_LAYOUT_GEMM (else BQ_ERR_SHAPE). The stats
+ * of a tensor are reduced in a fixed order, bit-reproducible for a given batch size on a
+ * given GPU (the order differs from a one-tensor call's: the sums agree to rounding).
+ * workspace: bq_workspace_size() bytes when stats is given (it does not grow with the
+ * batch). batch == 0 does nothing. Alignment as bq_quantize.
+ */
+bq_status bq_quantize_batch(const void* x, int32_t x_dtype, int64_t batch, int64_t rows, int64_t cols,
+                            const bq_scheme* scheme, void* codes, void* scales, void* zero_points,
+                            bq_stats* stats, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dequantize codes (+ scales, zero_points, tensor_scale as written by bq_quantize)
  * into out [rows, cols] (device) of dtype out_dtype = BQ_DT_BF16 (round to nearest
  * even from the fp32 value) or BQ_DT_FP32. Applies the inverse rotation when
@@ -296,7 +319,7 @@ bq_status bq_dequantize_rt(const void* codes, const void* scales, const void* ze
  * in the middle of an asynchronous pipeline, or code with a fixed memory budget.
  * The paper has no counterpart of this call (it serves such callers, not the method).
  * Arguments and results are those of bq_quantize. The scratch is a file-scope device
- * array of 131328 bytes (the workspace size of every scheme and shape); every GPU that
+ * array of 229632 bytes (the workspace size of every scheme and shape); every GPU that
  * loads the library holds one copy until the process exits. A call whose scheme would
  * need more returns BQ_ERR_WORKSPACE. Every call looks the array's device address up
  * (cudaGetSymbolAddress), so the address stays right after a device reset; the first
@@ -309,6 +332,36 @@ bq_status bq_quantize_noalloc(const void* x, int32_t x_dtype, int64_t rows, int6
                               const bq_scheme* scheme,
                               void* codes, void* scales, void* zero_points, float* tensor_scale,
                               bq_stats* stats, void* stream);
+
+/*
+ * Block-scaled GEMM on the tensor cores: D[m, n] = sum_k A[m, k] B[n, k], with A and B
+ * quantized by bq_quantize (or bq_quantize_batch) along k under the same scheme, scales
+ * in the GEMM layout (scale_layout = BQ_LAYOUT_GEMM), codes and scales passed as
+ * bq_quantize wrote them. This is the consumer block scaling serves: "Quantization survey"
+ * §4.3 (MX and NV formats feed Blackwell's block-scaled tensor cores) and the FP8
+ * training recipe's fp8_matmul of two FP8 operands with fp32 accumulation.
+ *  - MXFP8 (scheme: BQ_FP8_E4M3 or BQ_FP8_E5M2, BQ_MX_BLOCK): each product of codes is
+ *    scaled by both blocks' 2^e on the tensor cores; k % 128 == 0.
+ *  - NVFP4 (BQ_FP4_E2M1, BQ_NV_BLOCK): the E4M3 block scales on the tensor cores, then
+ *    D = acc * S_a * S_b with the operands' fp32 tensor scales (a_tensor_scale,
+ *    b_tensor_scale: device, one fp32 each); k % 256 == 0.
+ *  - scheme->hadamard = 1: both operands carry the block-16 rotation along k; H16/4 is
+ *    orthogonal, so the product equals that of the unrotated operands up to rounding.
+ * a_codes: [m, k] (FP4: [m, k / 2] bytes), b_codes: [n, k] likewise, row-major (k
+ * contiguous: a weight W[out, in] is B with n = out); a_scales / b_scales: the GEMM-layout
+ * scale buffers of those tensors (bq_buffer_sizes(scheme, m or n, k)). d: device
+ * [m, n] row-major, fp32 (BQ_DT_FP32) or bf16 (BQ_DT_BF16, round to nearest even).
+ * Accumulation is fp32 on the tensor cores (not bit-exact with any CPU order).
+ * Shapes: m % 128 == 0, n % 128 == 0 (else BQ_ERR_SHAPE); m == 0 or n == 0 does nothing.
+ * Alignment: codes, scales and d 16-byte aligned (else BQ_ERR_ALIGNMENT). Other schemes
+ * (INT formats, MXFP4 / MXFP6, row-major scales): BQ_ERR_UNSUPPORTED. Every wait in the
+ * kernel is bounded as described under bq_wait_timeouts below (which counts the GEMM's
+ * too). No workspace; enqueued on stream.
+ */
+bq_status bq_gemm(const void* a_codes, const void* a_scales, const float* a_tensor_scale,
+                  const void* b_codes, const void* b_scales, const float* b_tensor_scale,
+                  int64_t m, int64_t n, int64_t k, const bq_scheme* scheme,
+                  void* d, int32_t d_dtype, void* stream);
 
 /*
  * Bounded waits. The quantize kernels stage their input tiles in shared memory with
@@ -327,17 +380,17 @@ bq_status bq_wait_timeouts(uint32_t* count, int32_t reset);
 
 /*
  * Fault injection for tests of the bounded waits (no counterpart on the pages). The next
- * bq_quantize / bq_quantize_with_range call that runs the flat quantize kernel (per-tensor,
- * per-group, MX and NV schemes, and per-row schemes of at most 2048 power-of-two-many
- * 64-element segments) issues no copy for its staged tile number `tile` (tile t holds
- * chunks 128 t .. 128 t + 127 of the tensor seen as 16-element chunks; tile 0 is the
- * first tile of the first warp). The warp that waits for it gives up after the
- * one-second limit, waits (bounded) for its other copies in flight and stops; the call's
- * outputs are then incomplete and bq_wait_timeouts counts one more. Nothing faults and
- * nothing is left in flight; a following call on the same workspace runs normally.
- * One-shot: the call that consumes it resets it. tile < 0: BQ_ERR_INVALID_ARG.
+ * call that runs the flat quantize kernel (bq_quantize, bq_quantize_with_range or
+ * bq_quantize_batch with a per-tensor, per-group, MX or NV scheme, or a per-row scheme
+ * of at most 2048 columns, a power-of-two multiple of 64) issues no copy for the first
+ * staged tile of its warp number `warp` (warps are numbered CTA by CTA from 0; warp 0
+ * always has work). That warp's wait gives up after the one-second limit, it waits
+ * (bounded) for its other copies in flight and stops; the call's outputs are then
+ * incomplete and bq_wait_timeouts counts one more. Nothing faults and nothing is left in
+ * flight; a following call on the same workspace runs normally. One-shot: the call that
+ * consumes it resets it. warp < 0: BQ_ERR_INVALID_ARG.
  */
-bq_status bq_debug_skip_tile_copy(int32_t tile);
+bq_status bq_debug_skip_tile_copy(int32_t warp);
 
 /* QSNR = -10 log10(err2 / x2) in dB from a host copy of the stats ("INT vs FP at fine
  * granularity" §4.1): +inf when err2 = 0, NaN when x2 = 0 with err2 > 0 or for a NULL

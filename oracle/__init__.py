@@ -202,6 +202,27 @@ def qsnr_sums(x_bits, codes, scales, zps, tensor_scale, scheme: Scheme) -> np.nd
     return st
 
 
+def gemm(a: dict, b: dict, m: int, n: int, k: int, scheme: Scheme) -> np.ndarray:
+    """D[m, n] = sum_k A[m, k] B[n, k] in float64 of the two operands as quantized (the
+    oracle's own quantize outputs a and b, row-layout scales): each operand dequantized
+    by the oracle (fp32 values, NV tensor scale and inverse rotation included), then one
+    float64 matrix product. This is the block-scaled GEMM's definition: "Quantization
+    survey" §4.3.2 (x = x_q s_block S_tensor) and the FP8 recipe's fp8_matmul, whose
+    result the tensor cores approximate with fp32 accumulation. A weight W[out, in] is B
+    (n = out), so D = A W^T."""
+    da = dequantize(a["codes"], a["scales"], a["zps"], a["tensor_scale"], m, k, scheme).astype(np.float64)
+    db = dequantize(b["codes"], b["scales"], b["zps"], b["tensor_scale"], n, k, scheme).astype(np.float64)
+    return da @ db.T
+
+
+def gemm_magnitude(a: dict, b: dict, m: int, n: int, k: int, scheme: Scheme) -> np.ndarray:
+    """sum_k |A[m, k]| |B[n, k]| of the dequantized operands (the scale of the rounding
+    error of any order of summation)."""
+    da = np.abs(dequantize(a["codes"], a["scales"], a["zps"], a["tensor_scale"], m, k, scheme).astype(np.float64))
+    db = np.abs(dequantize(b["codes"], b["scales"], b["zps"], b["tensor_scale"], n, k, scheme).astype(np.float64))
+    return da @ db.T
+
+
 def tensor_range(x_bits: np.ndarray, hadamard: bool = False):
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     rows, cols = x_bits.shape

@@ -203,6 +203,27 @@ def test_range_split_checks_before_any_launch():
                                     None, 0, None) == 1
 
 
+def test_batch_checks_before_any_launch():
+    L = bq.lib()
+    fake = 1 << 40
+    ws = ctypes.c_void_p(fake)
+    mx = Scheme("int8_sym", "mx").c()
+    def q(scheme, batch, rows, cols, x=fake, codes=fake, stats=None, wsb=0):
+        return L.bq_quantize_batch(x, 0, batch, rows, cols, ctypes.byref(scheme), codes, fake, None, stats,
+                                   ws if wsb else None, wsb, None)
+    # per-tensor, NV and 2-D tile schemes, and per-row widths off the flat kernel, are not offered
+    for s, cols in [(Scheme("e4m3", "tensor"), 64), (Scheme("e2m1", "nv"), 64), (Scheme("e4m3", "tile2d"), 128),
+                    (Scheme("int8_sym", "row"), 4096), (Scheme("int8_sym", "row"), 192)]:
+        assert q(s.c(), 2, 4, cols) == 2
+    assert q(mx, -1, 4, 64) == 3                                 # negative batch
+    assert q(mx, 2, 1, 32) == 3                                  # tensors of a partial 64-element span
+    assert q(Scheme("e4m3", "mx", layout="gemm").c(), 2, 64, 128) == 3    # GEMM layout: rows % 128
+    assert q(mx, 2, 4, 64, x=None) == 1
+    assert q(mx, 2, 4, 64, x=fake + 16) == 4
+    assert q(mx, 2, 4, 64, stats=fake) == 5                      # stats without a workspace
+    assert q(mx, 0, 4, 64, x=None, codes=None) == 0              # an empty batch is a no-op
+
+
 def test_debug_hook_rejects_negative_tiles():
     assert bq.lib().bq_debug_skip_tile_copy(-1) == 1
 

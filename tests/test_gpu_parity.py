@@ -317,3 +317,16 @@ def test_range_split(s, ws, cuda_device):
 def test_no_tile_wait_gave_up(cuda_device):
     # every staged tile of every call above arrived (bounded waits never ran out)
     assert bq.bq_wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("s", [Scheme("e4m3", "tensor"), Scheme("e4m3", "row"), Scheme("e5m2", "group", 128),
+                               Scheme("e4m3", "group", 32, "fp16"), Scheme("e2m1", "nv"), Scheme("e4m3", "mx"),
+                               Scheme("e2m1", "mx")], ids=str)
+def test_negative_zero_keeps_its_sign(s, ws):
+    # a tensor of one row: -0.0 and tiny negatives next to ordinary values, alone in its
+    # warp, so the fast FP path (not the general one) codes it; the oracle keeps the sign
+    # of a zero result (codes 0x80 / 0x8)
+    a = np.full((1, 512), -0.0, dtype=np.float32)
+    a[0, ::4] = np.linspace(-2.0, 2.0, 128, dtype=np.float32)
+    a[0, 1::16] = -1e-30
+    check(synth.to_bf16(a), s, ws, "negative zeros")
