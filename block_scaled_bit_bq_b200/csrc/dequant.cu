@@ -307,6 +307,9 @@ __global__ void __launch_bounds__(RT_THREADS, 8) k_dequant_rt(const DequantArgs 
     extern __shared__ float4 rt_smem[];
     float* v = reinterpret_cast<float*>(rt_smem);
     const uint32_t cpr = cols / 16;
+    uint32_t* smask = reinterpret_cast<uint32_t*>(v + rot_row_floats(cols));
+    build_sign_masks(smask, sign_bits, cols);
+    __syncthreads();
     for (uint32_t r = blockIdx.x; r < rows; r += gridDim.x) {
         for (uint32_t c = threadIdx.x; c < cpr; c += blockDim.x) {
             const uint32_t cg = r * cpr + c;
@@ -322,22 +325,27 @@ __global__ void __launch_bounds__(RT_THREADS, 8) k_dequant_rt(const DequantArgs 
         for (uint32_t c = threadIdx.x; c < cpr; c += blockDim.x) {
             float2 xh[8];
             load_chunk_f32(v, c, norm, xh);
-            apply_signs(xh, chunk_sign_bits(sign_bits, c));
             const size_t cg = (size_t)r * cpr + c;
+            // the signs last: a flip of the sign bit (rounding to bf16 is odd-symmetric, so
+            // flipping after the rounding gives the same bits as before it)
+            uint32_t m[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            flip_words(smask, c, m);
             if constexpr (OUT == BQ_DT_BF16) {
                 uint32_t o[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const __nv_bfloat162 b = __floats2bfloat162_rn(xh[i].x, xh[i].y);
-                    o[i] = *reinterpret_cast<const uint32_t*>(&b);
+                    o[i] = *reinterpret_cast<const uint32_t*>(&b) ^ m[i];
                 }
                 st_v8(reinterpret_cast<uint8_t*>(a.out) + cg * 32, o);
             } else {
                 uint32_t o0[8], o1[8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    o0[2 * i] = __float_as_uint(xh[i].x); o0[2 * i + 1] = __float_as_uint(xh[i].y);
-                    o1[2 * i] = __float_as_uint(xh[4 + i].x); o1[2 * i + 1] = __float_as_uint(xh[4 + i].y);
+                    o0[2 * i] = __float_as_uint(xh[i].x) ^ (m[i] << 16);
+                    o0[2 * i + 1] = __float_as_uint(xh[i].y) ^ (m[i] & 0x80000000u);
+                    o1[2 * i] = __float_as_uint(xh[4 + i].x) ^ (m[4 + i] << 16);
+                    o1[2 * i + 1] = __float_as_uint(xh[4 + i].y) ^ (m[4 + i] & 0x80000000u);
                 }
                 uint8_t* p = reinterpret_cast<uint8_t*>(a.out) + cg * 64;
                 st_v8(p, o0);
@@ -437,7 +445,7 @@ cudaError_t launch_row_kernel(const DequantArgs& a, const uint32_t* sign_bits, u
                               float norm, cudaStream_t st)
 {
     const int block = cols / 16 < (uint32_t)RT_THREADS ? (int)(cols / 16) : RT_THREADS;   // a thread per chunk, up to RT_THREADS
-    const size_t smem = (size_t)rot_row_floats(cols) * 4;
+    const size_t smem = rot_smem_bytes(cols, true);
     if (smem > 48u * 1024u) {
         const cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

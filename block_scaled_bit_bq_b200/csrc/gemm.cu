@@ -39,6 +39,7 @@ constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_NS = 4;                   // pipeline stages
 constexpr uint32_t TMEM_COLS = 512;          // the whole tensor memory of the SM (one CTA per SM)
 constexpr uint32_t SF_TMEM_COL = 256;        // scale-factor columns start here (accumulator below)
+constexpr uint32_t GEMM_GROUP_M = 8;         // row tiles per group of the tile order
 
 template <int KIND, int BN>
 struct GemmCfg {
@@ -142,7 +143,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t base = (smem_addr(gemm_smem) + 1023u) & ~1023u;
-    const uint32_t n_tile = blockIdx.x, m_tile = blockIdx.y;
+    // tile order: groups of GEMM_GROUP_M row tiles, column by column inside a group, so the
+    // CTAs in flight at a time share a few bands of A and of B (they stay in L2)
+    uint32_t m_tile, n_tile;
+    {
+        const uint32_t num_m = g.m / 128u, num_n = g.n / (uint32_t)BN;
+        const uint32_t per_group = GEMM_GROUP_M * num_n, grp = blockIdx.x / per_group;
+        const uint32_t first_m = grp * GEMM_GROUP_M, gm = min(GEMM_GROUP_M, num_m - first_m);
+        const uint32_t local = blockIdx.x - grp * per_group;
+        m_tile = first_m + local % gm;
+        n_tile = local / gm;
+    }
     const uint32_t KT = g.k_stages;
 
     auto a_smem = [&](uint32_t s) { return base + s * C::STAGE; };
@@ -318,7 +329,7 @@ cudaError_t run_gemm(const GemmArgs& g, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = operand_map(g.b, g.n, g.kb, (uint32_t)BN, &bm);
     if (e != cudaSuccess) return e;
-    const dim3 grid(g.n / BN, g.m / 128u);
+    const unsigned grid = (g.n / BN) * (g.m / 128u);
     kern<<<grid, GEMM_THREADS, C::SMEM, st>>>(am, bm, g);
     return cudaGetLastError();
 }

@@ -1335,7 +1335,7 @@ __device__ __forceinline__ void rt_chunk(const float2 (&y)[8], const PlainUnit<F
 }
 
 template <int FMT, bool MX>
-__global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
+__global__ void __launch_bounds__(RT_THREADS, Fmt<FMT>::asym ? 4 : 5) k_quant_rt(const RtArgs a)
 {
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
@@ -1347,6 +1347,11 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
     const bool rot = a.sign_bits != nullptr, f16 = a.scale_fp16 != 0;
     const float norm = rot ? a.norm : 1.0f;
     const uint32_t L = a.lanes;
+    uint32_t* smask = reinterpret_cast<uint32_t*>(v + rot_row_floats(a.cols));
+    if (rot) {
+        build_sign_masks(smask, a.sign_bits, a.cols);
+        __syncthreads();
+    }
     Acc acc;
 
     for (uint32_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
@@ -1355,6 +1360,9 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
             uint32_t w[8];
             float2 y[8];
             ld_nc_v8(a.x + ((size_t)r * a.cpr + c) * 8, w);
+            // the signs flip bf16 sign bits before the factor: the same values as flipping
+            // the products' signs (a product's sign is its factors' signs combined)
+            if (rot) flip_words(smask, c, w);
             widen16x2(w, y);
             if (a.col_scale) {
                 const float4* m = reinterpret_cast<const float4*>(a.col_scale) + 4 * c;
@@ -1365,10 +1373,7 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
                     y[2 * i + 1] = mul2(y[2 * i + 1], make_float2(f.z, f.w));
                 }
             }
-            if (rot) {
-                apply_signs(y, chunk_sign_bits(a.sign_bits, c));
-                wht16x2(y);
-            }
+            if (rot) wht16x2(y);
             store_chunk_f32(v, c, y);
         }
         if (rot) wht_smem_stages(v, a.cols);
@@ -1423,7 +1428,9 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
                 kappa_add(acc, __fmul_rn(amax, p), t, a.inv_unit);
             }
         } else {
-            // units of L chunks = L adjacent threads (L divides 32; cpr is a multiple of 32)
+            // units of L chunks = L adjacent threads (L a power of two dividing 32; cpr is a
+            // multiple of 32): unit index and first chunk by shifts
+            const uint32_t lgL = (uint32_t)(__ffs((int)L) - 1);
             for (uint32_t c = threadIdx.x; c < a.cpr; c += blockDim.x) {
                 float2 y[8];
                 uint32_t q[NW];
@@ -1445,12 +1452,12 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
                 const float p = scaled ? pw.p : 1.0f;
                 float2 e2 = splat(0.0f), x2 = splat(0.0f);
                 const uint32_t cg = r * a.cpr + c;            // chunk index in the tensor
-                const bool first = (c % L) == 0;
+                const bool first = (c & (L - 1u)) == 0;
                 if constexpr (MX) {
                     const int e = ue8m0_exponent<FMT>(amax);
                     mx_chunk<FMT, K_MX, true>(y, exp2i(-e), exp2i(e), scaled, p, q, e2, x2);
                     if (first) {
-                        const uint32_t u = cg / L;
+                        const uint32_t u = cg >> lgL;
                         reinterpret_cast<uint8_t*>(a.scales)[a.gemm_layout ? gemm_unit_offset(u, a.gemm_nb) : u] =
                             (uint8_t)(e + 127);
                     }
@@ -1458,7 +1465,7 @@ __global__ void __launch_bounds__(RT_THREADS, 6) k_quant_rt(const RtArgs a)
                     const PlainScale ps = plain_scale<FMT>(amax, mn, mx, f16);
                     const PlainUnit<FMT> u = plain_unit<FMT>(ps);
                     rt_chunk<FMT>(y, u, unit_general_fast<FMT, false>(u, scaled), scaled, p, q, e2, x2);
-                    if (first) store_plain_scale<FMT>(a.scales, a.zps, cg / L, ps, f16);
+                    if (first) store_plain_scale<FMT>(a.scales, a.zps, cg >> lgL, ps, f16);
                 }
                 store_codes<FMT>(a.codes, cg, q);
                 add_unit_sums(acc, e2, x2, scaled ? pw.inv_p2 : 1.0);
@@ -1636,7 +1643,7 @@ cudaError_t run_rt(const RtArgs& a, cudaStream_t st)
     // a thread per chunk of the row, up to RT_THREADS (narrow rows: more CTAs per SM)
     const int block = a.cpr < (uint32_t)RT_THREADS ? (int)a.cpr : RT_THREADS;
     constexpr auto kern = k_quant_rt<FMT, MX>;
-    const size_t smem = (size_t)rot_row_floats(a.cols) * 4;
+    const size_t smem = rot_smem_bytes(a.cols, a.sign_bits != nullptr);
     if (smem > 48u * 1024u) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

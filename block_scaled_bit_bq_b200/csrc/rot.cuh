@@ -70,10 +70,12 @@ __device__ __forceinline__ void wht_group2(float2 (&t)[R])
 template <int R>
 __device__ __forceinline__ void wht_pass_wide(float* v, uint32_t n, uint32_t S)
 {
+    // S is a power of two: the group's position by shifts and masks, not divisions
+    const uint32_t lg = (uint32_t)(__ffs((int)S) - 1);
     const uint32_t npairs = n / (2 * R), step = S + S / 16;
     for (uint32_t q = threadIdx.x; q < npairs; q += blockDim.x) {
         const uint32_t g = 2 * q;
-        const uint32_t base = (g % S) + (g / S) * S * R;
+        const uint32_t base = (g & (S - 1u)) + ((g >> lg) << lg) * R;
         const uint32_t c = base >> 4, o = base & 15u;
         float2* p0 = reinterpret_cast<float2*>(v + rot_chunk_base(c) + 4u * (((o >> 2) + (c >> 1)) & 3u) + (o & 3u));
         float2 t[R];
@@ -123,20 +125,29 @@ __device__ __forceinline__ void wht_smem_stages(float* v, uint32_t n)
     __syncthreads();
 }
 
-// Negate element i of a chunk where bit i of the chunk's 16 sign bits is set.
-__device__ __forceinline__ void apply_signs(float2 (&y)[8], uint32_t bits)
+// The random signs as XOR masks of bf16 pairs, one 32-bit word per two columns (bit 15:
+// column 2j, bit 31: column 2j + 1), built once per CTA in shared memory after the row's
+// floats: a chunk's signs are then two 16-byte loads and one XOR per pair of values.
+__host__ __device__ constexpr uint32_t rot_smem_bytes(uint32_t n, bool signs)
 {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        y[i].x = __uint_as_float(__float_as_uint(y[i].x) ^ (((bits >> (2 * i)) & 1u) << 31));
-        y[i].y = __uint_as_float(__float_as_uint(y[i].y) ^ (((bits >> (2 * i + 1)) & 1u) << 31));
+    return rot_row_floats(n) * 4u + (signs ? n / 2 * 4u : 0u);
+}
+
+__device__ __forceinline__ void build_sign_masks(uint32_t* m, const uint32_t* sign_bits, uint32_t n)
+{
+    for (uint32_t j = threadIdx.x; j < n / 2; j += blockDim.x) {
+        const uint32_t b = (__ldg(sign_bits + (j >> 4)) >> ((2u * j) & 31u)) & 3u;
+        m[j] = ((b & 1u) << 15) | ((b & 2u) << 30);
     }
 }
 
-// The 16 sign bits of chunk c (columns 16c .. 16c + 15).
-__device__ __forceinline__ uint32_t chunk_sign_bits(const uint32_t* sign_bits, uint32_t c)
+// XOR the 8 bf16-pair words of chunk c with their sign masks.
+__device__ __forceinline__ void flip_words(const uint32_t* m, uint32_t c, uint32_t (&w)[8])
 {
-    return (__ldg(sign_bits + (c >> 1)) >> (16u * (c & 1u))) & 0xFFFFu;
+    const uint4 a = *reinterpret_cast<const uint4*>(m + 8 * c);
+    const uint4 b = *reinterpret_cast<const uint4*>(m + 8 * c + 4);
+    w[0] ^= a.x; w[1] ^= a.y; w[2] ^= a.z; w[3] ^= a.w;
+    w[4] ^= b.x; w[5] ^= b.y; w[6] ^= b.z; w[7] ^= b.w;
 }
 
 __device__ __forceinline__ void store_chunk_f32(float* v, uint32_t c, const float2 (&y)[8])
