@@ -131,3 +131,29 @@ def test_gemm_argument_checks(cuda_device):
     with pytest.raises(bq.BqError, match="BQ_ERR_UNSUPPORTED"):
         bq.bq_gemm(i8, i8, d)
     assert bq.bq_wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("s", [MX, NV], ids=str)
+def test_gemm_bench_size_sampled(s):
+    """The bench's GEMM (8192 x 8192 x 8192, bf16 out, the same operands): every code of
+    both operands against the oracle, and 64 sampled rows of D (every column) against the
+    oracle's float64 product of those rows."""
+    M = N = K = 8192
+    a = synth.activations_t3(M, K, seed=2)
+    b = synth.weight_outliers(N, K, seed=41)
+    qa = bq.quantize(a.cuda(), s, stats=False)
+    qb = bq.quantize(b.cuda(), s, stats=False)
+    d = bq.gemm(qa, qb, torch.bfloat16)
+    torch.cuda.synchronize()
+    os_ = _o(s)
+    oa = oracle.quantize(synth.bf16_bits(a), os_, stats=False)
+    ob = oracle.quantize(synth.bf16_bits(b), os_, stats=False)
+    assert np.array_equal(qa.codes.cpu().numpy(), oa["codes"]) and np.array_equal(qb.codes.cpu().numpy(), ob["codes"])
+    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], np.random.default_rng(5).choice(M, 60, replace=False)]))
+    da = oracle.dequantize(oa["codes"], oa["scales"], None, oa["tensor_scale"], M, K, os_)[rows].astype(np.float64)
+    db = oracle.dequantize(ob["codes"], ob["scales"], None, ob["tensor_scale"], N, K, os_).astype(np.float64)
+    ref = da @ db.T
+    mag = np.abs(da) @ np.abs(db).T
+    got = d.float().cpu().numpy()[rows].astype(np.float64)
+    bad = np.abs(got - ref) > REL * mag + 2.0 ** -8 * np.abs(ref) + 1e-30
+    assert not bad.any(), (s, np.argwhere(bad)[:5])

@@ -122,3 +122,43 @@ def bench_cores():
     sys.path.insert(0, ROOT)
     import bench
     return bench.host_cores()
+
+
+def _combine_worker(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from block_scaled_bit_bq_b200 import sharded
+        # rank 0's block: amax 3, min -3, max 1; rank 1's: amax 5, min 0, max 5
+        local = torch.tensor([[3.0, -3.0, 1.0], [5.0, 0.0, 5.0]][rank])
+        rng = sharded.combine_ranges(local)
+        st = torch.tensor([[1.0, 10.0, 2.0, 1.5, 4.0], [3.0, 30.0, 6.0, 2.5, 8.0]][rank], dtype=torch.float64)
+        blocks = sharded.combine_stats(st, None, 100)
+        tensor = sharded.combine_stats(st, 5.0, 100)
+        out.put((rank, rng.tolist(), blocks.tolist(), tensor.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_combine_ranges_and_stats():
+    # the split-tensor path's two collectives: ranges (MAX of amax and max, MIN of min) and
+    # stats (sums added, kappa max taken; a per-tensor scheme's one kappa from the totals)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_combine_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, rng, blocks, tensor in res:
+        assert rng == [5.0, -3.0, 5.0]
+        assert blocks == [4.0, 40.0, 8.0, 2.5, 12.0]
+        k = 5.0 / (40.0 / 100) ** 0.5
+        assert tensor[:2] == [4.0, 40.0] and abs(tensor[2] - k) < 1e-12 and tensor[3] == tensor[2] and tensor[4] == 1.0
