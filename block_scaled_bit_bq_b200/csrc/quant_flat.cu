@@ -21,6 +21,7 @@
 #include "quant_ops.cuh"
 #include "tma.cuh"
 #include "rot.cuh"
+#include "rot64.cuh"
 #include "internal.h"
 
 #include <atomic>
@@ -548,27 +549,6 @@ __device__ __forceinline__ void span_nv(const Row& row, uint32_t span, const Fla
 }
 
 // ---- two-chunk units: MX block 32, groups of 32 -------------------------------
-
-template <int FMT, int GK, bool STATS>
-__device__ __forceinline__ void mx_chunk(const float2 (&y)[8], float p2, float pe, bool scaled, float p,
-                                         uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
-{
-    using F = Fmt<FMT>;
-    float2 z[8];
-    if constexpr (F::is_int) {
-        int8_chunk_pow2<STATS>(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
-        if constexpr (STATS) {
-            if (scaled) int_sums<true>(y, z, pe, p, e2, x2);
-            else int_sums<false>(y, z, pe, p, e2, x2);
-        }
-    } else {
-        fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
-        if constexpr (STATS) {
-            if (scaled) val_sums<true>(y, z, pe, p, e2, x2);
-            else val_sums<false>(y, z, pe, p, e2, x2);
-        }
-    }
-}
 
 template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
 __device__ __forceinline__ void span_n2(const Row& row, uint32_t span, const FlatArgs& a, Acc& acc,
@@ -1318,22 +1298,6 @@ __global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__
 // keeps both sums).
 // ---------------------------------------------------------------------------
 
-// One chunk of a plain unit: the fast path when the warp's units admit it, else the
-// general one (sums added to e2 / x2).
-template <int FMT>
-__device__ __forceinline__ void rt_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, bool general, bool scaled,
-                                         float p, uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
-{
-    if (!general) {
-        float2 ce2, cx2;
-        (void)plain_chunk_fast<FMT, true, false>(y, u, q, ce2, cx2);
-        e2 = add2(e2, ce2);
-        x2 = add2(x2, cx2);
-    } else {
-        plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
-    }
-}
-
 template <int FMT, bool MX>
 __global__ void __launch_bounds__(RT_THREADS, Fmt<FMT>::asym ? 4 : 5) k_quant_rt(const RtArgs a)
 {
@@ -1748,6 +1712,8 @@ cudaError_t launch_quant_tile2d(int fmt, bool had, bool stats, const Tile2dArgs&
 
 cudaError_t launch_quant_rt(int fmt, bool mx, const RtArgs& a, cudaStream_t st)
 {
+    // rotated rows of 1024, 2048 or 4096 columns: the two-pass kernels
+    if (a.sign_bits && rt64_cols(a.cols) && a.rows > 0) return launch_quant_rt64(fmt, mx, a, st);
     if (mx) {
         switch (fmt) {
         case BQ_INT8_SYM: return run_rt<BQ_INT8_SYM, true>(a, st);

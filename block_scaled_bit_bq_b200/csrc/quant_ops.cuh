@@ -703,8 +703,8 @@ __device__ __forceinline__ void plain_chunk(const float2 (&y)[8], const PlainUni
 template <int FMT>
 __device__ __forceinline__ bool unit_general(const PlainUnit<FMT>& u, bool scaled)
 {
-    if constexpr (Fmt<FMT>::is_int) return scaled || __any_sync(0xFFFFFFFFu, u.iq.clamp);
-    else return scaled;
+    if constexpr (Fmt<FMT>::is_int) return __any_sync(0xFFFFFFFFu, scaled || u.iq.clamp);
+    else return __any_sync(0xFFFFFFFFu, scaled);
 }
 
 // Call f(std::integral_constant<bool, EXACT>, std::integral_constant<bool, GENERAL>) with
@@ -863,16 +863,57 @@ __device__ __forceinline__ bool plain_chunk_fast(const float2 (&y)[8], const Pla
     else return int_chunk_fast<FMT, STATS>(y, u.iq, w, ce2, cx2);
 }
 
-// Whether a plain unit must take the general path as a whole (warp-uniform): scaled
-// sums, clamping, or a scale outside the fast paths' range.
+// Whether a plain unit must take the general path as a whole (warp-uniform: any lane
+// with scaled sums, clamping, or a scale outside the fast paths' range).
 template <int FMT, bool EXACT>
 __device__ __forceinline__ bool unit_general_fast(const PlainUnit<FMT>& u, bool scaled)
 {
+    // every lane votes (scaled may differ between the lanes' units): the general chunk
+    // path is itself warp-collective, so all lanes must take the same path
     if constexpr (Fmt<FMT>::is_int) {
         const bool g = u.iq.clamp || !u.iq.fast || (EXACT ? !u.iq.br : !u.iq.mk);
-        return scaled || __any_sync(0xFFFFFFFFu, g);
+        return __any_sync(0xFFFFFFFFu, scaled || g);
     } else {
-        return scaled || __any_sync(0xFFFFFFFFu, !u.fq.mk);
+        return __any_sync(0xFFFFFFFFu, scaled || !u.fq.mk);
+    }
+}
+
+// One chunk of an MX block (power-of-two scale 2^e: p2 = 2^-e, pe = 2^e); STATS adds
+// its sums (scaled form when `scaled`).
+template <int FMT, int GK, bool STATS>
+__device__ __forceinline__ void mx_chunk(const float2 (&y)[8], float p2, float pe, bool scaled, float p,
+                                         uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
+{
+    using F = Fmt<FMT>;
+    float2 z[8];
+    if constexpr (F::is_int) {
+        int8_chunk_pow2<STATS>(y, p2, *reinterpret_cast<uint32_t(*)[4]>(&q), z);
+        if constexpr (STATS) {
+            if (scaled) int_sums<true>(y, z, pe, p, e2, x2);
+            else int_sums<false>(y, z, pe, p, e2, x2);
+        }
+    } else {
+        fp_chunk_pow2<FMT, STATS>(y, p2, q, z);
+        if constexpr (STATS) {
+            if (scaled) val_sums<true>(y, z, pe, p, e2, x2);
+            else val_sums<false>(y, z, pe, p, e2, x2);
+        }
+    }
+}
+
+// One chunk of a plain unit: the fast path when the warp's units admit it, else the
+// general one (sums added to e2 / x2).
+template <int FMT>
+__device__ __forceinline__ void rt_chunk(const float2 (&y)[8], const PlainUnit<FMT>& u, bool general, bool scaled,
+                                         float p, uint32_t (&q)[CodeWords<FMT>::n], float2& e2, float2& x2)
+{
+    if (!general) {
+        float2 ce2, cx2;
+        (void)plain_chunk_fast<FMT, true, false>(y, u, q, ce2, cx2);
+        e2 = add2(e2, ce2);
+        x2 = add2(x2, cx2);
+    } else {
+        plain_chunk<FMT, true, false, true>(y, u, scaled, p, q, e2, x2);
     }
 }
 

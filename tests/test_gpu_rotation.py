@@ -21,7 +21,7 @@ SCHEMES = [Scheme("int8_sym", "row"), Scheme("uint4_asym", "group", 128, "fp16")
            Scheme("e4m3", "group", 128), Scheme("int8_asym", "row", scale_dtype="fp16"), Scheme("int8_sym", "mx"),
            Scheme("e2m1", "mx"), Scheme("e5m2", "group", 16), Scheme("e2m3", "mx")]
 
-SHAPES = [(37, 4096), (9, 512), (5, 16384), (300, 2048)]
+SHAPES = [(37, 4096), (9, 512), (5, 16384), (300, 2048), (203, 1024), (2501, 2048)]
 TRANSFORMS = ["signs", "factor", "both", "none"]
 
 
@@ -90,19 +90,23 @@ def test_rt_parity(s, shape, kind, ws):
 
 
 def test_rt_edge_values(ws):
-    # zero rows, tiny and huge values, exact ties under power-of-two factors
+    # zero rows, tiny and huge values (whole rows and half rows), exact ties under
+    # power-of-two factors
     g = np.random.default_rng(9)
     a = (g.standard_t(3, size=(6, 1024)) * 0.5).astype(np.float32)
     a[0] = 0.0
     a[1] *= 1e-30
     a[2] = g.uniform(-1, 1, 1024).astype(np.float32) * 1e30
     a[3] = g.integers(-64, 65, 1024).astype(np.float32) * 0.5
+    a[4, 512:] *= 1e-30          # units of one row (and of one warp) on both sides of
+    a[5, :512] *= 1e30           # the plain-sums range: the scaled and unscaled forms mix
     x = synth.to_bf16(a)
     signs = synth.random_signs(1024, 7)
     factor = np.ldexp(np.ones(1024, np.float32), g.integers(-2, 3, 1024)).astype(np.float32)
     for s in [Scheme("int8_sym", "row"), Scheme("uint4_asym", "group", 64, "fp16"), Scheme("e4m3", "mx")]:
         check_rt(x, s, signs, factor, ws, "edge")
         check_rt(x, s, signs, None, ws, "edge")
+        check_rt(x, s, None, factor, ws, "edge, no rotation")
 
 
 def test_rt_full_size_weight(ws):
