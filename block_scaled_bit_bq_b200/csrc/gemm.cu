@@ -9,17 +9,22 @@
 // with fp32 accumulation. The tensor cores apply the block scales themselves; the
 // epilogue applies NV's two tensor scales (D = acc * S_a * S_b).
 //
-// A CTA computes one 128 x BN tile of D with 6 warps:
-//  - warp 0, one lane: loads. Per stage (128 bytes of k: 128 FP8 or 256 FP4 elements)
-//    a tensor-map copy of the A tile [128 rows x 128 B] and the B tile [BN rows x 128 B]
-//    (128-byte swizzle), and bulk copies of the scale tiles: the GEMM layout keeps the
-//    scales of 128 rows x 4 blocks in one 512-byte tile, which is exactly the shared-
-//    memory form tcgen05.cp's 32x128b.warpx4 shape moves into tensor memory;
-//  - warp 1, one lane: tensor memory allocation, then per stage the scale tiles into
-//    tensor memory (tcgen05.cp) and 4 MMAs (k of 32 FP8 or 64 FP4 elements each) into
-//    the fp32 accumulator in tensor memory; a commit per stage frees the stage;
+// One CTA per SM, persistent over 128 x BN tiles of D (taken in a grouped order that keeps
+// a few bands of A and B in L2), with 6 warps:
+//  - warp 0, one lane: loads, one stage ring running across the CTA's tiles (the next
+//    tile's stages fill while the current one finishes). Per stage (128 bytes of k: 128
+//    FP8 or 256 FP4 elements) a tensor-map copy of the A tile [128 rows x 128 B] and the B
+//    tile [BN rows x 128 B] (128-byte swizzle), and bulk copies of the scale tiles: the GEMM
+//    layout keeps the scales of 128 rows x 4 blocks in one 512-byte tile, which is exactly
+//    the shared-memory form tcgen05.cp's 32x128b.warpx4 shape moves into tensor memory;
+//  - warp 1, one lane: tensor memory allocation; per tile, once the epilogue has read the
+//    previous accumulator, per stage the scale tiles into tensor memory (tcgen05.cp) and 4
+//    MMAs (k of 32 FP8 or 64 FP4 elements each) into the fp32 accumulator; a commit per
+//    stage frees the stage, one per tile hands the accumulator to the epilogue;
 //  - warps 2-5: the epilogue. Each reads its 32-lane quarter of the accumulator
-//    (tcgen05.ld), scales (NV) and stores rows of D (fp32 or bf16).
+//    (tcgen05.ld), scales (NV), rounds to bf16 into a swizzled staging buffer, releases the
+//    accumulator, and writes whole rows of D from the buffer (fp32 output: straight from
+//    registers, the accumulator released after the stores).
 // Every wait on an mbarrier gives up after about a second (counted in g_gemm_wait_timeouts);
 // the CTA then lets its copies and MMAs in flight finish (bounded), frees its tensor
 // memory and returns, leaving D incomplete.
@@ -36,10 +41,15 @@ __device__ unsigned int g_gemm_wait_timeouts = 0;
 namespace {
 
 constexpr int GEMM_THREADS = 192;
-constexpr int GEMM_NS = 4;                   // pipeline stages
 constexpr uint32_t TMEM_COLS = 512;          // the whole tensor memory of the SM (one CTA per SM)
 constexpr uint32_t SF_TMEM_COL = 256;        // scale-factor columns start here (accumulator below)
 constexpr uint32_t GEMM_GROUP_M = 8;         // row tiles per group of the tile order
+
+// The bf16 epilogue's staging buffer: per epilogue warp, 32 rows x 128 columns (256-byte
+// rows, 16-byte granule g of row r at g ^ (r & 15), so that a warp's row-wise writes and
+// its column-wise reads both touch every bank once per 8 lanes).
+constexpr uint32_t OUT_WARP_BYTES = 32u * 256u;
+constexpr uint32_t OUT_BYTES = 4u * OUT_WARP_BYTES;
 
 template <int KIND, int BN>
 struct GemmCfg {
@@ -55,9 +65,15 @@ struct GemmCfg {
     // a stage starts on a 1024-byte boundary: the 128-byte swizzle repeats every 1024 bytes
     // and the operand descriptors assume the tiles start on it
     static constexpr uint32_t STAGE = (TX_BYTES + 1023u) & ~1023u;
-    static constexpr uint32_t SMEM = GEMM_NS * STAGE + 1024u;
     static constexpr uint32_t SF_COLS = 4u * SFT * (1u + BT);    // tensor-memory columns of a stage's scales
-    static_assert(SF_TMEM_COL + GEMM_NS * SF_COLS <= TMEM_COLS, "tensor memory");
+    // as many stages as shared memory (less the epilogue buffer, the alignment slack and
+    // the barriers) and tensor memory hold, at most 6
+    static constexpr uint32_t NS_SMEM = (232448u - OUT_BYTES - 1024u - 512u) / STAGE;
+    static constexpr uint32_t NS_TMEM = (TMEM_COLS - SF_TMEM_COL) / SF_COLS;
+    static constexpr int NS = (int)(NS_SMEM < NS_TMEM ? (NS_SMEM < 6u ? NS_SMEM : 6u) : (NS_TMEM < 6u ? NS_TMEM : 6u));
+    static constexpr uint32_t SMEM = (uint32_t)NS * STAGE + OUT_BYTES + 1024u;
+    static_assert(NS >= 2, "pipeline depth");
+    static_assert(SF_TMEM_COL + NS * SF_COLS <= TMEM_COLS, "tensor memory");
     static_assert(SMEM <= 232448u, "shared memory");
 };
 
@@ -131,6 +147,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+// The tile order: groups of GEMM_GROUP_M row tiles, column by column inside a group, so
+// the tiles in flight at a time share a few bands of A and of B (they stay in L2).
+__device__ __forceinline__ void tile_coords(uint32_t t, uint32_t num_m, uint32_t num_n, uint32_t& m_tile,
+                                            uint32_t& n_tile)
+{
+    const uint32_t per_group = GEMM_GROUP_M * num_n, grp = t / per_group;
+    const uint32_t first_m = grp * GEMM_GROUP_M, gm = min(GEMM_GROUP_M, num_m - first_m);
+    const uint32_t local = t - grp * per_group;
+    m_tile = first_m + local % gm;
+    n_tile = local / gm;
+}
+
 template <int KIND, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_constant__ CUtensorMap amap,
                                                            const __grid_constant__ CUtensorMap bmap,
@@ -138,22 +171,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
 {
     using C = GemmCfg<KIND, BN>;
     extern __shared__ uint8_t gemm_smem[];
-    __shared__ __align__(8) uint64_t full_bar[GEMM_NS], empty_bar[GEMM_NS], done_bar;
+    __shared__ __align__(8) uint64_t full_bar[C::NS], empty_bar[C::NS], acc_full, acc_empty, done_bar;
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t base = (smem_addr(gemm_smem) + 1023u) & ~1023u;
-    // tile order: groups of GEMM_GROUP_M row tiles, column by column inside a group, so the
-    // CTAs in flight at a time share a few bands of A and of B (they stay in L2)
-    uint32_t m_tile, n_tile;
-    {
-        const uint32_t num_m = g.m / 128u, num_n = g.n / (uint32_t)BN;
-        const uint32_t per_group = GEMM_GROUP_M * num_n, grp = blockIdx.x / per_group;
-        const uint32_t first_m = grp * GEMM_GROUP_M, gm = min(GEMM_GROUP_M, num_m - first_m);
-        const uint32_t local = blockIdx.x - grp * per_group;
-        m_tile = first_m + local % gm;
-        n_tile = local / gm;
-    }
+    const uint32_t out_base = base + C::NS * C::STAGE;
+    const uint32_t num_m = g.m / 128u, num_n = g.n / (uint32_t)BN, num_tiles = num_m * num_n;
     const uint32_t KT = g.k_stages;
 
     auto a_smem = [&](uint32_t s) { return base + s * C::STAGE; };
@@ -162,10 +186,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
     auto sfb_smem = [&](uint32_t s) { return base + s * C::STAGE + C::A_BYTES + C::B_BYTES + C::SFA_BYTES; };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < GEMM_NS; ++s) {
+        for (int s = 0; s < C::NS; ++s) {
             mbar_init(smem_addr(&full_bar[s]), 1);
             mbar_init(smem_addr(&empty_bar[s]), 1);
         }
+        mbar_init(smem_addr(&acc_full), 1);
+        mbar_init(smem_addr(&acc_empty), 4);          // one arrival per epilogue warp
         mbar_init(smem_addr(&done_bar), 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -181,109 +207,158 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
     const uint32_t tmem = tmem_holder;
 
     if (warp == 0 && lane == 0) {
-        // ---- loads ----
-        const uint8_t* sfa_row = g.sfa + (size_t)m_tile * g.sf_tiles_per_row * 512u;
-        uint32_t issued = 0;
-        for (uint32_t kk = 0; kk < KT; ++kk) {
-            const uint32_t s = kk % GEMM_NS;
-            if (kk >= GEMM_NS && !mbar_wait(smem_addr(&empty_bar[s]), ((kk / GEMM_NS) - 1) & 1u)) {
-                abort_flag = 1;
-                break;
+        // ---- loads: one stage ring over all of the CTA's tiles ----
+        uint32_t it = 0;
+        for (uint32_t t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x) {
+            uint32_t m_tile, n_tile;
+            tile_coords(t, num_m, num_n, m_tile, n_tile);
+            const uint8_t* sfa_row = g.sfa + (size_t)m_tile * g.sf_tiles_per_row * 512u;
+            for (uint32_t kk = 0; kk < KT; ++kk, ++it) {
+                const uint32_t s = it % C::NS;
+                if (it >= C::NS && !mbar_wait(smem_addr(&empty_bar[s]), ((it / C::NS) - 1) & 1u)) {
+                    abort_flag = 1;
+                    break;
+                }
+                if (abort_flag) break;
+                const uint32_t fb = smem_addr(&full_bar[s]);
+                mbar_arrive_expect_tx(fb, C::TX_BYTES);
+                tma_load_2d(a_smem(s), &amap, fb, (int)(kk * 128u), (int)(m_tile * 128u));
+                tma_load_2d(b_smem(s), &bmap, fb, (int)(kk * 128u), (int)(n_tile * (uint32_t)BN));
+                bulk_load(sfa_smem(s), sfa_row + (size_t)kk * C::SFT * 512u, C::SFA_BYTES, fb);
+                for (uint32_t i = 0; i < C::BT; ++i) {
+                    const uint8_t* src = g.sfb + ((size_t)(n_tile * C::BT + i) * g.sf_tiles_per_row + kk * C::SFT) * 512u;
+                    bulk_load(sfb_smem(s) + i * C::SFT * 512u, src, C::SFT * 512u, fb);
+                }
             }
-            if (abort_flag) break;
-            const uint32_t fb = smem_addr(&full_bar[s]);
-            mbar_arrive_expect_tx(fb, C::TX_BYTES);
-            tma_load_2d(a_smem(s), &amap, fb, (int)(kk * 128u), (int)(m_tile * 128u));
-            tma_load_2d(b_smem(s), &bmap, fb, (int)(kk * 128u), (int)(n_tile * (uint32_t)BN));
-            bulk_load(sfa_smem(s), sfa_row + (size_t)kk * C::SFT * 512u, C::SFA_BYTES, fb);
-            for (uint32_t i = 0; i < C::BT; ++i) {
-                const uint8_t* src = g.sfb + ((size_t)(n_tile * C::BT + i) * g.sf_tiles_per_row + kk * C::SFT) * 512u;
-                bulk_load(sfb_smem(s) + i * C::SFT * 512u, src, C::SFT * 512u, fb);
-            }
-            issued = kk + 1;
         }
         if (abort_flag) {
             // let the copies in flight land before the CTA can exit (bounded)
-            const uint32_t first = issued > (uint32_t)GEMM_NS ? issued - GEMM_NS : 0u;
-            for (uint32_t kk = first; kk < issued; ++kk)
-                (void)mbar_wait(smem_addr(&full_bar[kk % GEMM_NS]), (kk / GEMM_NS) & 1u);
+            const uint32_t first = it > (uint32_t)C::NS ? it - C::NS : 0u;
+            for (uint32_t j = first; j < it; ++j)
+                (void)mbar_wait(smem_addr(&full_bar[j % C::NS]), (j / C::NS) & 1u);
         }
     } else if (warp == 1 && lane == 0) {
-        // ---- MMAs ----
-        uint32_t acc = 0;
-        for (uint32_t kk = 0; kk < KT; ++kk) {
-            const uint32_t s = kk % GEMM_NS;
-            if (!mbar_wait(smem_addr(&full_bar[s]), (kk / GEMM_NS) & 1u)) { abort_flag = 1; break; }
-            if (abort_flag) break;
+        // ---- MMAs: a tile's k stages into the accumulator, once the epilogue has read
+        // the previous tile's ----
+        uint32_t it = 0, i = 0;
+        for (uint32_t t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x, ++i) {
+            if (i > 0 && !mbar_wait(smem_addr(&acc_empty), (i - 1) & 1u)) { abort_flag = 1; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // scale tiles into tensor memory: A's tiles j at columns 4 j, B's (row tile i,
-            // tile j) at 4 (j BT + i), so the BN / 128 tiles of one block group sit side by side
-            const uint32_t sf = tmem + SF_TMEM_COL + s * C::SF_COLS;
-            const uint32_t sfb_col = 4u * C::SFT;
-            for (uint32_t j = 0; j < C::SFT; ++j) {
-                tc_cp_scales(sf + 4u * j, scale_desc(sfa_smem(s) + 512u * j));
-                for (uint32_t i = 0; i < C::BT; ++i)
-                    tc_cp_scales(sf + sfb_col + 4u * (j * C::BT + i), scale_desc(sfb_smem(s) + (i * C::SFT + j) * 512u));
-            }
-            const uint64_t ad = operand_desc(a_smem(s)), bd = operand_desc(b_smem(s));
+            uint32_t acc = 0;
+            for (uint32_t kk = 0; kk < KT; ++kk, ++it) {
+                const uint32_t s = it % C::NS;
+                if (!mbar_wait(smem_addr(&full_bar[s]), (it / C::NS) & 1u)) { abort_flag = 1; break; }
+                if (abort_flag) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                // scale tiles into tensor memory: A's tiles j at columns 4 j, B's (row tile
+                // i, tile j) at 4 (j BT + i), so the BN / 128 tiles of one block group sit side
+                // by side
+                const uint32_t sf = tmem + SF_TMEM_COL + s * C::SF_COLS;
+                const uint32_t sfb_col = 4u * C::SFT;
+                for (uint32_t j = 0; j < C::SFT; ++j) {
+                    tc_cp_scales(sf + 4u * j, scale_desc(sfa_smem(s) + 512u * j));
+                    for (uint32_t b = 0; b < C::BT; ++b)
+                        tc_cp_scales(sf + sfb_col + 4u * (j * C::BT + b), scale_desc(sfb_smem(s) + (b * C::SFT + j) * 512u));
+                }
+                const uint64_t ad = operand_desc(a_smem(s)), bd = operand_desc(b_smem(s));
 #pragma unroll
-            for (uint32_t k = 0; k < 4; ++k) {
-                // MX: one 32-bit scale column per 128 rows holds the 4 blocks of the stage,
-                // MMA k reads byte k; NV: MMA k reads all 4 bytes of tile k
-                const uint32_t id = KIND == GEMM_MXF8 ? k : 0u;
-                const uint32_t ta = sf + (KIND == GEMM_MXF8 ? 0u : 4u * k);
-                const uint32_t tb = sf + sfb_col + (KIND == GEMM_MXF8 ? 0u : 4u * k * C::BT);
-                tc_mma<KIND>(tmem, ad + 2u * k, bd + 2u * k, instr_desc<KIND, BN>(g.elem_fmt, id),
-                             ta | (id << 30), tb | (id << 30), acc);
-                acc = 1;
+                for (uint32_t k = 0; k < 4; ++k) {
+                    // MX: one 32-bit scale column per 128 rows holds the 4 blocks of the
+                    // stage, MMA k reads byte k; NV: MMA k reads all 4 bytes of tile k
+                    const uint32_t id = KIND == GEMM_MXF8 ? k : 0u;
+                    const uint32_t ta = sf + (KIND == GEMM_MXF8 ? 0u : 4u * k);
+                    const uint32_t tb = sf + sfb_col + (KIND == GEMM_MXF8 ? 0u : 4u * k * C::BT);
+                    tc_mma<KIND>(tmem, ad + 2u * k, bd + 2u * k, instr_desc<KIND, BN>(g.elem_fmt, id),
+                                 ta | (id << 30), tb | (id << 30), acc);
+                    acc = 1;
+                }
+                tc_commit(smem_addr(&empty_bar[s]));     // the stage is free once these MMAs are done
             }
-            tc_commit(smem_addr(&empty_bar[s]));     // the stage is free once these MMAs are done
+            if (abort_flag) break;
+            tc_commit(smem_addr(&acc_full));             // the tile's accumulator is complete
         }
         // every MMA issued so far completes before done_bar's phase does
         tc_commit(smem_addr(&done_bar));
         if (!mbar_wait(smem_addr(&done_bar), 0u)) abort_flag = 1;
     } else if (warp >= 2) {
-        // ---- epilogue ----
-        const uint32_t q = (uint32_t)warp & 3u;       // the warp's quarter of tensor memory's lanes
-        bool ok = mbar_wait(smem_addr(&done_bar), 0u);
-        ok = __all_sync(0xFFFFFFFFu, ok) && !abort_flag;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (ok) {
-            const uint32_t row = m_tile * 128u + q * 32u + (uint32_t)lane;
-            const float sc = KIND == GEMM_NVF4 ? __fmul_rn(g.a_tensor_scale ? *g.a_tensor_scale : 1.0f,
-                                                            g.b_tensor_scale ? *g.b_tensor_scale : 1.0f) : 1.0f;
+        // ---- epilogue: warp w reads lanes 32 (w % 4) .. + 31 of the accumulator ----
+        const uint32_t q = (uint32_t)warp & 3u;
+        const uint32_t ob = out_base + q * OUT_WARP_BYTES;
+        const float sc = KIND == GEMM_NVF4 ? __fmul_rn(g.a_tensor_scale ? *g.a_tensor_scale : 1.0f,
+                                                        g.b_tensor_scale ? *g.b_tensor_scale : 1.0f) : 1.0f;
+        uint32_t i = 0;
+        for (uint32_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
+            uint32_t m_tile, n_tile;
+            tile_coords(t, num_m, num_n, m_tile, n_tile);
+            bool ok = mbar_wait(smem_addr(&acc_full), i & 1u);
+            ok = __all_sync(0xFFFFFFFFu, ok) && !abort_flag;
+            if (!ok) { abort_flag = 1; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t row0 = m_tile * 128u + q * 32u;
+            if (g.d_bf16) {
+                // two halves of 128 columns: accumulator -> bf16 -> staging buffer, then
+                // coalesced rows to D; the accumulator is released once its last columns are
+                // read, before the second half's stores
 #pragma unroll 1
-            for (uint32_t c0 = 0; c0 < (uint32_t)BN; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((q * 32u) << 16) + c0, r);
-                const size_t off = (size_t)row * g.ldd + n_tile * (uint32_t)BN + c0;
-                if (g.d_bf16) {
-                    uint32_t w[16];
+                for (uint32_t h = 0; h < (uint32_t)BN / 128u; ++h) {
+#pragma unroll 1
+                    for (uint32_t c = 0; c < 4; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tmem + ((q * 32u) << 16) + 128u * h + 32u * c, r);
+                        uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float x0 = __uint_as_float(r[2 * i]), x1 = __uint_as_float(r[2 * i + 1]);
-                        if (KIND == GEMM_NVF4) { x0 = __fmul_rn(x0, sc); x1 = __fmul_rn(x1, sc); }
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-                        w[i] = *reinterpret_cast<const uint32_t*>(&h);
-                    }
-                    uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(g.d) + off);
+                        for (int e = 0; e < 16; ++e) {
+                            float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                            if (KIND == GEMM_NVF4) { x0 = __fmul_rn(x0, sc); x1 = __fmul_rn(x1, sc); }
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                        // row = lane; granules 4 c .. 4 c + 3 of the row's 16
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t v[4] = {w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]};
-                        st_v4(dst + 4 * i, v);
+                        for (uint32_t e = 0; e < 4; ++e) {
+                            const uint32_t gi = (4u * c + e) ^ ((uint32_t)lane & 15u);
+                            sts_v4(ob + (uint32_t)lane * 256u + gi * 16u, w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                        }
                     }
-                } else {
+                    if (h + 1u == (uint32_t)BN / 128u) {
+                        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_addr(&acc_empty));
+                    }
+                    __syncwarp();
+                    // rows 2 j and 2 j + 1: lanes 0-15 and 16-31, a granule each
+#pragma unroll 4
+                    for (uint32_t j = 0; j < 16; ++j) {
+                        const uint32_t rr = 2u * j + ((uint32_t)lane >> 4), gi = (uint32_t)lane & 15u;
+                        uint32_t v0, v1, v2, v3;
+                        lds_v4(ob + rr * 256u + ((gi ^ (rr & 15u)) * 16u), v0, v1, v2, v3);
+                        const uint32_t v[4] = {v0, v1, v2, v3};
+                        const size_t off = (size_t)(row0 + rr) * g.ldd + n_tile * (uint32_t)BN + 128u * h + 8u * gi;
+                        st_v4(reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(g.d) + off), v);
+                    }
+                    __syncwarp();        // the buffer is read before the next half refills it
+                }
+            } else {
+                const uint32_t row = row0 + (uint32_t)lane;
+#pragma unroll 1
+                for (uint32_t c0 = 0; c0 < (uint32_t)BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((q * 32u) << 16) + c0, r);
+                    const size_t off = (size_t)row * g.ldd + n_tile * (uint32_t)BN + c0;
                     uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<float*>(g.d) + off);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int e8 = 0; e8 < 8; ++e8) {
                         uint32_t v[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            v[e] = KIND == GEMM_NVF4 ? __float_as_uint(__fmul_rn(__uint_as_float(r[4 * i + e]), sc))
-                                                     : r[4 * i + e];
-                        st_v4(dst + 4 * i, v);
+                            v[e] = KIND == GEMM_NVF4 ? __float_as_uint(__fmul_rn(__uint_as_float(r[4 * e8 + e]), sc))
+                                                     : r[4 * e8 + e];
+                        st_v4(dst + 4 * e8, v);
                     }
                 }
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&acc_empty));
             }
         }
     }
@@ -329,7 +404,10 @@ cudaError_t run_gemm(const GemmArgs& g, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = operand_map(g.b, g.n, g.kb, (uint32_t)BN, &bm);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (g.n / BN) * (g.m / 128u);
+    // persistent: a CTA per SM (tensor memory and shared memory admit one), tiles strided
+    const unsigned tiles = (g.n / BN) * (g.m / 128u);
+    const unsigned sms = (unsigned)device_sm_count();
+    const unsigned grid = tiles < sms ? tiles : sms;
     kern<<<grid, GEMM_THREADS, C::SMEM, st>>>(am, bm, g);
     return cudaGetLastError();
 }

@@ -76,6 +76,16 @@ def test_gemm_bf16_output(s):
     _run(s, 256, 256, 1024, seed=830, dtype=torch.bfloat16)
 
 
+# more tiles than SMs: CTAs take several tiles in turn (the stage ring runs on across
+# them, the accumulator is handed back and forth); 256- and 128-column tiles
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2560, 2048, 512), (1536, 1920, 512)], ids=lambda t: "x".join(map(str, t)))
+@pytest.mark.parametrize("s", [MX, NV], ids=str)
+def test_gemm_several_tiles_per_cta(s, shape, dtype):
+    m, n, k = shape
+    _run(s, m, n, k, seed=850 + m + n, dtype=dtype)
+
+
 @pytest.mark.parametrize("s", [Scheme("e4m3", "mx", hadamard=True, layout="gemm"),
                                Scheme("e2m1", "nv", hadamard=True, layout="gemm")], ids=str)
 def test_gemm_rotated_operands(s):
