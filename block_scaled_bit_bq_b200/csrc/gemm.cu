@@ -22,9 +22,9 @@
 //    MMAs (k of 32 FP8 or 64 FP4 elements each) into the fp32 accumulator; a commit per
 //    stage frees the stage, one per tile hands the accumulator to the epilogue;
 //  - warps 2-5: the epilogue. Each reads its 32-lane quarter of the accumulator
-//    (tcgen05.ld), scales (NV), rounds to bf16 into a swizzled staging buffer, releases the
-//    accumulator, and writes whole rows of D from the buffer (fp32 output: straight from
-//    registers, the accumulator released after the stores).
+//    (tcgen05.ld) 32 columns at a time, scales (NV), rounds to bf16 through a small
+//    swizzled staging buffer into row pieces of D, and releases the accumulator as soon as
+//    its last columns are read (fp32 output: straight from registers).
 // Every wait on an mbarrier gives up after about a second (counted in g_gemm_wait_timeouts);
 // the CTA then lets its copies and MMAs in flight finish (bounded), frees its tensor
 // memory and returns, leaving D incomplete.
@@ -45,10 +45,11 @@ constexpr uint32_t TMEM_COLS = 512;          // the whole tensor memory of the S
 constexpr uint32_t SF_TMEM_COL = 256;        // scale-factor columns start here (accumulator below)
 constexpr uint32_t GEMM_GROUP_M = 8;         // row tiles per group of the tile order
 
-// The bf16 epilogue's staging buffer: per epilogue warp, 32 rows x 128 columns (256-byte
-// rows, 16-byte granule g of row r at g ^ (r & 15), so that a warp's row-wise writes and
-// its column-wise reads both touch every bank once per 8 lanes).
-constexpr uint32_t OUT_WARP_BYTES = 32u * 256u;
+// The bf16 epilogue's staging buffer: per epilogue warp, 32 rows x 32 columns (64-byte
+// rows; 16-byte granule g of row r at g ^ ((r >> 1) & 3), so that a warp's row-wise
+// writes and its row-block reads both touch 8 distinct 16-byte bank groups per 8 lanes).
+// Small, so that the stage ring keeps four stages of 256-column tiles.
+constexpr uint32_t OUT_WARP_BYTES = 32u * 64u;
 constexpr uint32_t OUT_BYTES = 4u * OUT_WARP_BYTES;
 
 template <int KIND, int BN>
@@ -296,47 +297,43 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t row0 = m_tile * 128u + q * 32u;
             if (g.d_bf16) {
-                // two halves of 128 columns: accumulator -> bf16 -> staging buffer, then
-                // coalesced rows to D; the accumulator is released once its last columns are
-                // read, before the second half's stores
+                // chunks of 32 columns: accumulator -> bf16 -> staging buffer -> whole
+                // 64-byte row pieces of D; the accumulator is released once its last
+                // columns are read, before that chunk's stores
 #pragma unroll 1
-                for (uint32_t h = 0; h < (uint32_t)BN / 128u; ++h) {
-#pragma unroll 1
-                    for (uint32_t c = 0; c < 4; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem + ((q * 32u) << 16) + 128u * h + 32u * c, r);
-                        uint32_t w[16];
+                for (uint32_t c0 = 0; c0 < (uint32_t)BN; c0 += 32u) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((q * 32u) << 16) + c0, r);
+                    uint32_t w[16];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
-                            if (KIND == GEMM_NVF4) { x0 = __fmul_rn(x0, sc); x1 = __fmul_rn(x1, sc); }
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
-                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        // row = lane; granules 4 c .. 4 c + 3 of the row's 16
-#pragma unroll
-                        for (uint32_t e = 0; e < 4; ++e) {
-                            const uint32_t gi = (4u * c + e) ^ ((uint32_t)lane & 15u);
-                            sts_v4(ob + (uint32_t)lane * 256u + gi * 16u, w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-                        }
+                    for (int e = 0; e < 16; ++e) {
+                        float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                        if (KIND == GEMM_NVF4) { x0 = __fmul_rn(x0, sc); x1 = __fmul_rn(x1, sc); }
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
                     }
-                    if (h + 1u == (uint32_t)BN / 128u) {
+                    if (c0 + 32u == (uint32_t)BN) {
                         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                         __syncwarp();
                         if (lane == 0) mbar_arrive(smem_addr(&acc_empty));
                     }
+                    // row = lane: its 4 granules
+                    const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+                    for (uint32_t e = 0; e < 4; ++e)
+                        sts_v4(ob + (uint32_t)lane * 64u + ((e ^ sw) * 16u), w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
                     __syncwarp();
-                    // rows 2 j and 2 j + 1: lanes 0-15 and 16-31, a granule each
-#pragma unroll 4
-                    for (uint32_t j = 0; j < 16; ++j) {
-                        const uint32_t rr = 2u * j + ((uint32_t)lane >> 4), gi = (uint32_t)lane & 15u;
+                    // 8 rows per store: lane l takes granule l % 4 of row 8 j + l / 4
+#pragma unroll
+                    for (uint32_t j = 0; j < 4; ++j) {
+                        const uint32_t rr = 8u * j + ((uint32_t)lane >> 2), gi = (uint32_t)lane & 3u;
                         uint32_t v0, v1, v2, v3;
-                        lds_v4(ob + rr * 256u + ((gi ^ (rr & 15u)) * 16u), v0, v1, v2, v3);
+                        lds_v4(ob + rr * 64u + ((gi ^ ((rr >> 1) & 3u)) * 16u), v0, v1, v2, v3);
                         const uint32_t v[4] = {v0, v1, v2, v3};
-                        const size_t off = (size_t)(row0 + rr) * g.ldd + n_tile * (uint32_t)BN + 128u * h + 8u * gi;
+                        const size_t off = (size_t)(row0 + rr) * g.ldd + n_tile * (uint32_t)BN + c0 + 8u * gi;
                         st_v4(reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(g.d) + off), v);
                     }
-                    __syncwarp();        // the buffer is read before the next half refills it
+                    __syncwarp();        // the buffer is read before the next chunk refills it
                 }
             } else {
                 const uint32_t row = row0 + (uint32_t)lane;
