@@ -56,7 +56,9 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
-KERNEL_SOURCES = ("common.cuh", "quant_ops.cuh", "tma.cuh", "rot.cuh", "quant_flat.cu", "quant_row.cu", "dequant.cu")
+# every kernel source: a traffic figure is used only while none of them has changed since its capture
+KERNEL_SOURCES = tuple(sorted(n for n in os.listdir(os.path.join(ROOT, "block_scaled_bit_bq_b200", "csrc"))
+                              if n.endswith((".cu", ".cuh", ".h"))))
 
 # workload -> list of (label, scheme args)
 WORKLOADS = {

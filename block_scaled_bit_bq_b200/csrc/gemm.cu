@@ -10,17 +10,20 @@
 // epilogue applies NV's two tensor scales (D = acc * S_a * S_b).
 //
 // One CTA per SM, persistent over 128 x BN tiles of D (taken in a grouped order that keeps
-// a few bands of A and B in L2), with 6 warps:
+// a few bands of A and B in L2), with 7 warps:
 //  - warp 0, one lane: loads, one stage ring running across the CTA's tiles (the next
 //    tile's stages fill while the current one finishes). Per stage (128 bytes of k: 128
 //    FP8 or 256 FP4 elements) a tensor-map copy of the A tile [128 rows x 128 B] and the B
 //    tile [BN rows x 128 B] (128-byte swizzle), and bulk copies of the scale tiles: the GEMM
 //    layout keeps the scales of 128 rows x 4 blocks in one 512-byte tile, which is exactly
 //    the shared-memory form tcgen05.cp's 32x128b.warpx4 shape moves into tensor memory;
+//  - warp 6, one lane: per stage, once its copies landed, the scale tiles into tensor
+//    memory (tcgen05.cp), then a commit that lets the stage's MMAs start (a separate
+//    issuer: NVFP4 moves 12 scale tiles a stage);
 //  - warp 1, one lane: tensor memory allocation; per tile, once the epilogue has read the
-//    previous accumulator, per stage the scale tiles into tensor memory (tcgen05.cp) and 4
-//    MMAs (k of 32 FP8 or 64 FP4 elements each) into the fp32 accumulator; a commit per
-//    stage frees the stage, one per tile hands the accumulator to the epilogue;
+//    previous accumulator, per stage 4 MMAs (k of 32 FP8 or 64 FP4 elements each) into the
+//    fp32 accumulator; a commit per stage frees the stage, one per tile hands the
+//    accumulator to the epilogue;
 //  - warps 2-5: the epilogue. Each reads its 32-lane quarter of the accumulator
 //    (tcgen05.ld) 32 columns at a time, scales (NV), rounds to bf16 through a small
 //    swizzled staging buffer into row pieces of D, and releases the accumulator as soon as
@@ -40,7 +43,7 @@ __device__ unsigned int g_gemm_wait_timeouts = 0;
 
 namespace {
 
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 224;
 constexpr uint32_t TMEM_COLS = 512;          // the whole tensor memory of the SM (one CTA per SM)
 constexpr uint32_t SF_TMEM_COL = 256;        // scale-factor columns start here (accumulator below)
 constexpr uint32_t GEMM_GROUP_M = 8;         // row tiles per group of the tile order
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
 {
     using C = GemmCfg<KIND, BN>;
     extern __shared__ uint8_t gemm_smem[];
-    __shared__ __align__(8) uint64_t full_bar[C::NS], empty_bar[C::NS], acc_full, acc_empty, done_bar;
+    __shared__ __align__(8) uint64_t full_bar[C::NS], sf_bar[C::NS], empty_bar[C::NS], acc_full, acc_empty, done_bar, sf_done;
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,11 +192,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
             mbar_init(smem_addr(&full_bar[s]), 1);
+            mbar_init(smem_addr(&sf_bar[s]), 1);
             mbar_init(smem_addr(&empty_bar[s]), 1);
         }
         mbar_init(smem_addr(&acc_full), 1);
         mbar_init(smem_addr(&acc_empty), 4);          // one arrival per epilogue warp
         mbar_init(smem_addr(&done_bar), 1);
+        mbar_init(smem_addr(&sf_done), 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -240,7 +245,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMAs: a tile's k stages into the accumulator, once the epilogue has read
-        // the previous tile's ----
+        // the previous tile's; a stage is taken once its scale tiles are in tensor memory
+        // (which the scale warp moves only after the stage's copies landed) ----
         uint32_t it = 0, i = 0;
         for (uint32_t t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x, ++i) {
             if (i > 0 && !mbar_wait(smem_addr(&acc_empty), (i - 1) & 1u)) { abort_flag = 1; break; }
@@ -248,19 +254,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
             uint32_t acc = 0;
             for (uint32_t kk = 0; kk < KT; ++kk, ++it) {
                 const uint32_t s = it % C::NS;
-                if (!mbar_wait(smem_addr(&full_bar[s]), (it / C::NS) & 1u)) { abort_flag = 1; break; }
+                if (!mbar_wait(smem_addr(&sf_bar[s]), (it / C::NS) & 1u)) { abort_flag = 1; break; }
                 if (abort_flag) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                // scale tiles into tensor memory: A's tiles j at columns 4 j, B's (row tile
-                // i, tile j) at 4 (j BT + i), so the BN / 128 tiles of one block group sit side
-                // by side
                 const uint32_t sf = tmem + SF_TMEM_COL + s * C::SF_COLS;
                 const uint32_t sfb_col = 4u * C::SFT;
-                for (uint32_t j = 0; j < C::SFT; ++j) {
-                    tc_cp_scales(sf + 4u * j, scale_desc(sfa_smem(s) + 512u * j));
-                    for (uint32_t b = 0; b < C::BT; ++b)
-                        tc_cp_scales(sf + sfb_col + 4u * (j * C::BT + b), scale_desc(sfb_smem(s) + (b * C::SFT + j) * 512u));
-                }
                 const uint64_t ad = operand_desc(a_smem(s)), bd = operand_desc(b_smem(s));
 #pragma unroll
                 for (uint32_t k = 0; k < 4; ++k) {
@@ -281,7 +279,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) k_bs_gemm(const __grid_consta
         // every MMA issued so far completes before done_bar's phase does
         tc_commit(smem_addr(&done_bar));
         if (!mbar_wait(smem_addr(&done_bar), 0u)) abort_flag = 1;
-    } else if (warp >= 2) {
+    } else if (warp == 6 && lane == 0) {
+        // ---- scale tiles into tensor memory, a stage at a time once its copies landed:
+        // A's tiles j at columns 4 j, B's (row tile b, tile j) at 4 (j BT + b), so the
+        // BN / 128 tiles of one block group sit side by side. The stage's tensor-memory
+        // columns are free: its previous MMAs completed before the loads refilled it ----
+        uint32_t it = 0;
+        for (uint32_t t = blockIdx.x; t < num_tiles && !abort_flag; t += gridDim.x) {
+            for (uint32_t kk = 0; kk < KT; ++kk, ++it) {
+                const uint32_t s = it % C::NS;
+                if (!mbar_wait(smem_addr(&full_bar[s]), (it / C::NS) & 1u)) { abort_flag = 1; break; }
+                if (abort_flag) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t sf = tmem + SF_TMEM_COL + s * C::SF_COLS;
+                const uint32_t sfb_col = 4u * C::SFT;
+                for (uint32_t j = 0; j < C::SFT; ++j) {
+                    tc_cp_scales(sf + 4u * j, scale_desc(sfa_smem(s) + 512u * j));
+                    for (uint32_t b = 0; b < C::BT; ++b)
+                        tc_cp_scales(sf + sfb_col + 4u * (j * C::BT + b), scale_desc(sfb_smem(s) + (b * C::SFT + j) * 512u));
+                }
+                tc_commit(smem_addr(&sf_bar[s]));        // the MMAs of the stage may start
+            }
+        }
+        // every copy issued so far completes before sf_done's phase does
+        tc_commit(smem_addr(&sf_done));
+        if (!mbar_wait(smem_addr(&sf_done), 0u)) abort_flag = 1;
+    } else if (warp >= 2 && warp <= 5) {
         // ---- epilogue: warp w reads lanes 32 (w % 4) .. + 31 of the accumulator ----
         const uint32_t q = (uint32_t)warp & 3u;
         const uint32_t ob = out_base + q * OUT_WARP_BYTES;
