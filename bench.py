@@ -56,9 +56,9 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantize GB/s (bytes in+out) and % of B200 HBM peak; QSNR dB matching oracle"
-# every kernel source: a traffic figure is used only while none of them has changed since its capture
-KERNEL_SOURCES = tuple(sorted(n for n in os.listdir(os.path.join(ROOT, "block_scaled_bit_bq_b200", "csrc"))
-                              if n.endswith((".cu", ".cuh", ".h"))))
+# the sources the quantize kernels are built from (quant_flat.cu and what it includes): a traffic
+# figure is used only while none of them has changed since its capture
+KERNEL_SOURCES = ("common.cuh", "internal.h", "quant_flat.cu", "quant_ops.cuh", "rot.cuh", "rot64.cuh", "tma.cuh")
 
 # workload -> list of (label, scheme args)
 WORKLOADS = {

@@ -13,7 +13,6 @@
 // divided (multiply-high) by the chunks per scaling unit.
 #include "dequant_ops.cuh"
 #include "rot.cuh"
-#include "rot64.cuh"
 #include "internal.h"
 
 #include <atomic>
@@ -311,7 +310,6 @@ cudaError_t launch_dequant(int fmt, int sk, bool had, int out_dtype, const Dequa
 cudaError_t launch_dequant_rt(int fmt, int sk, int out_dtype, const DequantArgs& a, const uint32_t* sign_bits,
                               uint32_t rows, uint32_t cols, float norm, cudaStream_t st)
 {
-    if (rt64_cols(cols) && rows > 0) return launch_dequant_rt64(fmt, sk, out_dtype, a, sign_bits, rows, cols, norm, st);
     return dispatch(fmt, sk, [&]<int FMT, int SK>() {
         return out_dtype == BQ_DT_BF16
                    ? launch_row_kernel<k_dequant_rt<FMT, SK, BQ_DT_BF16>>(a, sign_bits, rows, cols, norm, st)

@@ -170,9 +170,6 @@ cudaError_t launch_quant_rt64(int fmt, bool mx, const RtArgs& a, cudaStream_t st
 // Dequantize with the inverse full-row rotation (sign_bits [cols / 32], norm as RtArgs).
 cudaError_t launch_dequant_rt(int fmt, int sk, int out_dtype, const DequantArgs& a, const uint32_t* sign_bits,
                               uint32_t rows, uint32_t cols, float norm, cudaStream_t st);
-// rows of 1024, 2048 or 4096 columns (rot_dequant.cu)
-cudaError_t launch_dequant_rt64(int fmt, int sk, int out_dtype, const DequantArgs& a, const uint32_t* sign_bits,
-                              uint32_t rows, uint32_t cols, float norm, cudaStream_t st);
 cudaError_t launch_dequant(int fmt, int sk, bool hadamard, int out_dtype, const DequantArgs& a,
                            cudaStream_t st);
 cudaError_t launch_qsnr(int fmt, int sk, bool hadamard, const DequantArgs& a, cudaStream_t st);

@@ -14,7 +14,7 @@
 // Shared-memory layout (one row): element (m, p) at
 //     64 m + 4 ((p >> 2) ^ (m & 7)) + (p & 3),
 // the 16-byte granules of matrix row m permuted by m & 7. Row-wise 16-byte accesses by
-// consecutive threads (pass A stores, the reads of the quantize / output phase) and
+// consecutive threads (pass A stores, the quantize phase's reads) and
 // column-wise 4-byte accesses (pass B) both touch 32 distinct banks per 32 accesses.
 // Rows of one CTA sit n + 16 floats apart (the 16-float shift keeps two rows read by
 // one warp, T = 16, on different banks). A pass-B thread reads and writes back the same
@@ -25,7 +25,7 @@
 
 namespace bq {
 
-// Threads per CTA of the two-pass row kernels: 64 / T rows at a time.
+// Threads per CTA of the two-pass row kernel: 64 / T rows at a time.
 constexpr int RT64_THREADS = 64;
 
 __host__ __device__ constexpr uint32_t rt64_row_floats(uint32_t n) { return n + 16u; }
@@ -36,7 +36,7 @@ __host__ __device__ constexpr uint32_t rt64_smem_bytes(uint32_t n)
     return (RT64_THREADS / (n / 64u)) * rt64_row_floats(n) * 4u + n / 2u * 4u;
 }
 
-// Whether a row length takes the two-pass kernels.
+// Whether a row length takes the two-pass kernel.
 __host__ __device__ constexpr bool rt64_cols(uint32_t n) { return n == 1024u || n == 2048u || n == 4096u; }
 
 __device__ __forceinline__ uint32_t la64(uint32_t m, uint32_t p)
@@ -170,15 +170,6 @@ __device__ __forceinline__ void build_sign_masks64(uint32_t* msk, const uint32_t
         const uint32_t b = (__ldg(sign_bits + (j >> 4)) >> ((2u * j) & 31u)) & 3u;
         msk[mask64(j >> 5, j & 31u)] = ((b & 1u) << 15) | ((b & 2u) << 30);
     }
-}
-
-// Words 8 k .. 8 k + 7 of thread m's masks (piece k's 16 columns).
-__device__ __forceinline__ void piece_masks64(const uint32_t* msk, uint32_t m, int k, uint32_t (&w)[8])
-{
-    const uint4 a = *reinterpret_cast<const uint4*>(msk + mask64(m, 8u * k));
-    const uint4 b = *reinterpret_cast<const uint4*>(msk + mask64(m, 8u * k + 4u));
-    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
 }
 
 }  // namespace bq
