@@ -335,6 +335,32 @@ def run_gemm_bench(args, rank: int, world: int, device):
             lib = {"kernel": "cuBLASLt scaled_mm (torch)", "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12}
         except RuntimeError as e:
             lib = {"kernel": "cuBLASLt scaled_mm (torch)", "unavailable": str(e).splitlines()[0][:200]}
+    elif fmt == "e2m1" and hasattr(F, "scaled_mm") and hasattr(torch, "float4_e2m1fn_x2") \
+            and hasattr(F.ScalingType, "BlockWise1x16"):
+        fp4, e4 = torch.float4_e2m1fn_x2, torch.float8_e4m3fn
+        ca, cb = qa.codes.view(fp4), qb.codes.view(fp4).t()
+        sa, sb = qa.scales.view(e4), qb.scales.view(e4)
+
+        def lib_gemm():
+            # the two-level NVFP4 form: block scales and each operand's tensor scale
+            return F.scaled_mm(ca, cb, [sa, qa.tensor_scale], [F.ScalingType.BlockWise1x16, F.ScalingType.TensorWise],
+                               [sb, qb.tensor_scale], [F.ScalingType.BlockWise1x16, F.ScalingType.TensorWise],
+                               swizzle_a=[F.SwizzleType.SWIZZLE_32_4_4, F.SwizzleType.NO_SWIZZLE],
+                               swizzle_b=[F.SwizzleType.SWIZZLE_32_4_4, F.SwizzleType.NO_SWIZZLE],
+                               output_dtype=torch.bfloat16)
+        def lib_gemm_blocks():
+            # block scales only (the tensor scales would multiply the result)
+            return F.scaled_mm(ca, cb, sa, F.ScalingType.BlockWise1x16, sb, F.ScalingType.BlockWise1x16,
+                               swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                               output_dtype=torch.bfloat16)
+        for name, fn in (("cuBLASLt scaled_mm NVFP4 (torch)", lib_gemm),
+                         ("cuBLASLt scaled_mm NVFP4, block scales only (torch)", lib_gemm_blocks)):
+            try:
+                lib_ms = time_fn(fn, reps)
+                lib = {"kernel": name, "ms": lib_ms, "tflops": flops / (lib_ms * 1e-3) / 1e12}
+                break
+            except (RuntimeError, TypeError, ValueError) as e:
+                lib = {"kernel": name, "unavailable": str(e).splitlines()[0][:200]}
     if rank != 0:
         return None
     peak, src = measured_tensor_peak(fmt)

@@ -130,6 +130,52 @@ def test_gemm_matches_the_library_gemm():
     assert np.all(np.abs(d.cpu().numpy().astype(np.float64) - c.cpu().numpy()) <= 2 * REL * mag)
 
 
+def _library_nvfp4(qa, qb, out_dtype):
+    """D = A B^T through cuBLASLt's NVFP4 GEMM (torch scaled_mm: E2M1 codes, E4M3 block scales
+    in the 32x4x4 tile layout, and the two fp32 tensor scales), or None where this torch
+    takes no such call."""
+    F = torch.nn.functional
+    if not (hasattr(F, "scaled_mm") and hasattr(torch, "float4_e2m1fn_x2") and
+            hasattr(F.ScalingType, "BlockWise1x16")):
+        return None
+    fp4, e4 = torch.float4_e2m1fn_x2, torch.float8_e4m3fn
+    a, b = qa.codes.view(fp4), qb.codes.view(fp4).t()
+    sa, sb = qa.scales.view(e4), qb.scales.view(e4)
+    try:
+        # two-level form: the block scales and the tensor scale of each operand
+        return F.scaled_mm(a, b, [sa, qa.tensor_scale], [F.ScalingType.BlockWise1x16, F.ScalingType.TensorWise],
+                           [sb, qb.tensor_scale], [F.ScalingType.BlockWise1x16, F.ScalingType.TensorWise],
+                           swizzle_a=[F.SwizzleType.SWIZZLE_32_4_4, F.SwizzleType.NO_SWIZZLE],
+                           swizzle_b=[F.SwizzleType.SWIZZLE_32_4_4, F.SwizzleType.NO_SWIZZLE], output_dtype=out_dtype)
+    except (RuntimeError, TypeError, ValueError):
+        pass
+    try:
+        # block scales only; the tensor scales multiply the result
+        c = F.scaled_mm(a, b, sa, F.ScalingType.BlockWise1x16, sb, F.ScalingType.BlockWise1x16,
+                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                        output_dtype=torch.float32)
+        return (c * (qa.tensor_scale * qb.tensor_scale)).to(out_dtype)
+    except (RuntimeError, TypeError, ValueError):
+        return None
+
+
+def test_gemm_nvfp4_matches_the_library_gemm():
+    # the same NVFP4 operands through cuBLASLt, where this torch has the call
+    a, b = _operands(NV, 256, 384, 2048, 860)
+    qa = bq.quantize(a.cuda(), NV, stats=False)
+    qb = bq.quantize(b.cuda(), NV, stats=False)
+    d = bq.gemm(qa, qb)
+    c = _library_nvfp4(qa, qb, torch.float32)
+    if c is None:
+        pytest.skip("no NVFP4 scaled_mm in this torch")
+    torch.cuda.synchronize()
+    os_ = _o(NV)
+    oa = oracle.quantize(synth.bf16_bits(a), os_, stats=False)
+    ob = oracle.quantize(synth.bf16_bits(b), os_, stats=False)
+    mag = oracle.gemm_magnitude(oa, ob, 256, 384, 2048, os_)
+    assert np.all(np.abs(d.cpu().numpy().astype(np.float64) - c.cpu().numpy()) <= 2 * REL * mag)
+
+
 def test_gemm_argument_checks(cuda_device):
     q = bq.quantize(synth.normal(128, 256, seed=1).cuda(), MX, stats=False)
     d = torch.empty((128, 128), dtype=torch.float32, device=cuda_device)
