@@ -185,14 +185,23 @@ def test_parity_small(s, name, ws):
     check(x, s, ws, name)
 
 
-@pytest.mark.parametrize("cols", [16, 96, 640, 2112, 3136, 4096, 8192, 12288, 16384, 20480])
+@pytest.mark.parametrize("cols", [16, 96, 640, 2112, 3136, 4096, 4160, 6144, 8192, 12288, 16384, 20480])
 @pytest.mark.parametrize("s", [Scheme("int8_sym", "row"), Scheme("uint4_asym", "row", scale_dtype="fp16"),
                                Scheme("e5m2", "row", hadamard=True)], ids=str)
 def test_row_kernel_shapes(s, cols, ws):
     # cols % 64 != 0 (16, 96): a CTA per row; other widths: a warp per row through the
-    # segment tensor map, with a partly filled last tile (640, 2112, 3136) or whole tiles
+    # segment tensor map, with a partly filled last tile (640, 2112, 3136, 4160) or whole tiles;
+    # rows of 3-4 tiles (4160, 6144, 8192) take the four-stage ring
     x = synth.activations_t3(9, cols, seed=200 + cols, n_outlier_channels=1)
     check(x, s, ws, f"rows9x{cols}")
+
+
+@pytest.mark.parametrize("s", [Scheme("int8_sym", "row"), Scheme("e4m3", "row")], ids=str)
+def test_row_kernel_rows_through_the_ring(s, ws):
+    # more rows than warps: each warp takes several 6144-column rows (three tiles) through
+    # the four-stage ring that keeps a row resident for both passes
+    x = synth.activations_t3(2000, 6144, seed=260, n_outlier_channels=2)
+    check(x, s, ws, "rows2000x6144")
 
 
 @pytest.mark.parametrize("rows", [1, 127, 128, 129, 640])
