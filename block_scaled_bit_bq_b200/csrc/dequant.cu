@@ -28,6 +28,7 @@ constexpr int DQ_CPL = 2;
 template <int FMT, int SK, bool HAD, int OUT>
 __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
 {
+    pdl_wait();
     constexpr int NC = SpanCodes<FMT, DQ_CPL>::n;
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(256) k_dequant(const DequantArgs a)
 template <int FMT, int SK, bool HAD>
 __global__ void __launch_bounds__(256) k_qsnr(const DequantArgs a)
 {
+    pdl_wait();
     constexpr int NC = SpanCodes<FMT>::n;
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -143,6 +145,7 @@ template <int FMT, int SK, int OUT>
 __global__ void __launch_bounds__(RT_THREADS, 8) k_dequant_rt(const DequantArgs a, const uint32_t* sign_bits, uint32_t rows,
                                                     uint32_t cols, float norm)
 {
+    pdl_wait();
     constexpr int NC = SpanCodes<FMT, 1>::n;
     extern __shared__ float4 rt_smem[];
     float* v = reinterpret_cast<float*>(rt_smem);
@@ -219,8 +222,7 @@ cudaError_t launch_flat_kernel(const DequantArgs& a, cudaStream_t st)
     if (need < 1) need = 1;
     uint64_t grid = need < waves ? need : waves;
     if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
-    KERN<<<(unsigned)grid, block, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(KERN, (unsigned)grid, (unsigned)block, 0, st, a);
 }
 
 template <int FMT, int SK>
@@ -296,8 +298,7 @@ cudaError_t launch_row_kernel(const DequantArgs& a, const uint32_t* sign_bits, u
     if (grid > rows) grid = rows;
     if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
     if (grid < 1) grid = 1;
-    KERN<<<(unsigned)grid, block, smem, st>>>(a, sign_bits, rows, cols, norm);
-    return cudaGetLastError();
+    return launch_pdl(KERN, (unsigned)grid, (unsigned)block, smem, st, a, sign_bits, rows, cols, norm);
 }
 
 }  // namespace

@@ -47,6 +47,7 @@ template <bool HAD, bool MINMAX>
 __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, uint32_t n_chunks, uint8_t* ws,
                                                float* out)
 {
+    pdl_wait();
     float amax = 0.0f, mn = 0.0f, mx = 0.0f;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -67,6 +68,7 @@ __global__ void __launch_bounds__(256) k_range(const uint32_t* __restrict__ x, u
         range_chunk<HAD, MINMAX>(w0, amax, mn, mx);
     }
     // min / max start from 0: only min(min, 0) and max(max, 0) are ever used.
+    pdl_release();                   // the CTA's loads are done
     amax = warp_maxf(amax);
     if constexpr (MINMAX) { mn = warp_minf(mn); mx = warp_maxf(mx); }
     __shared__ float sh[3][32];
@@ -767,6 +769,7 @@ __global__ void __launch_bounds__(FLAT_WARPS * 32, BQ_FLAT_MINB) k_quant_flat(co
                                                                   const __grid_constant__ CUtensorMap xmap32,
                                                                   const FlatArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     extern __shared__ uint8_t flat_smem[];
     __shared__ __align__(8) uint64_t bars[FLAT_WARPS][NST];
@@ -982,6 +985,7 @@ template <int FMT, bool HAD, bool STATS, bool EXACT, int RN>
 __global__ void __launch_bounds__(ROWS_WARPS * 32, 4) k_quant_rows(const __grid_constant__ CUtensorMap xmap,
                                                                  const RowsArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     extern __shared__ uint8_t flat_smem[];
@@ -1139,6 +1143,7 @@ template <int FMT, bool HAD, bool STATS, bool EXACT>
 __global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__ CUtensorMap xmap,
                                                          const Tile2dArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     extern __shared__ uint8_t tile_smem[];
     __shared__ __align__(8) uint64_t bars[TILE_NST];
@@ -1303,6 +1308,7 @@ __global__ void __launch_bounds__(256, 2) k_quant_tile2d(const __grid_constant__
 template <int FMT, bool MX>
 __global__ void __launch_bounds__(RT_THREADS, Fmt<FMT>::asym ? 4 : 5) k_quant_rt(const RtArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     extern __shared__ float4 rt_smem[];
@@ -1545,14 +1551,13 @@ cudaError_t run_rows(const RowsArgs& a, cudaStream_t st)
         constexpr auto kern = k_quant_rows<FMT, HAD, STATS, EXACT, 4>;
         constexpr uint32_t smem = rows_smem(4);            // above 48 KiB: resident_ctas opts in
         const unsigned grid = grid_for<kern, block, smem>(ROWS_WARPS, a.rows);
-        kern<<<grid, block, smem, st>>>(map, a);
+        return launch_pdl(kern, grid, block, smem, st, map, a);
     } else {
         constexpr auto kern = k_quant_rows<FMT, HAD, STATS, EXACT, 2>;
         constexpr uint32_t smem = rows_smem(2);
         const unsigned grid = grid_for<kern, block, smem>(ROWS_WARPS, a.rows);
-        kern<<<grid, block, smem, st>>>(map, a);
+        return launch_pdl(kern, grid, block, smem, st, map, a);
     }
-    return cudaGetLastError();
 }
 
 // The exact (value-domain) integer path: integer formats, fp16 scales, unrotated input.
@@ -1596,8 +1601,7 @@ cudaError_t run_tile2d(const Tile2dArgs& a, cudaStream_t st)
     const cudaError_t e = x_tiles_map(a.x, a.rows, a.cols, &map);
     if (e != cudaSuccess) return e;
     const unsigned grid = grid_for<kern, block, TILE2D_SMEM>(1, a.ntiles);
-    kern<<<grid, block, TILE2D_SMEM, st>>>(map, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, block, TILE2D_SMEM, st, map, a);
 }
 
 template <int FMT>
@@ -1628,8 +1632,7 @@ cudaError_t run_rt(const RtArgs& a, cudaStream_t st)
     if (grid > a.rows) grid = a.rows;
     if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, block, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)grid, (unsigned)block, smem, st, a);
 }
 
 template <int FMT, int GK, bool HAD, bool STATS, bool EXACT>
@@ -1650,8 +1653,7 @@ cudaError_t run_flat(const FlatArgs& a, cudaStream_t st)
     if (grid < min_grid) grid = min_grid;
     if (grid > MAX_STAT_SLOTS / FLAT_WARPS) grid = MAX_STAT_SLOTS / FLAT_WARPS;
     if (grid * FLAT_WARPS < a.batch) return cudaErrorInvalidValue;
-    kern<<<grid, block, FLAT_SMEM, st>>>(map, map32, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, block, FLAT_SMEM, st, map, map32, a);
 }
 
 template <int FMT, int GK>
@@ -1671,8 +1673,7 @@ cudaError_t run_range(const uint32_t* x, uint32_t n_chunks, uint8_t* ws, float* 
     constexpr int block = 256;
     constexpr auto kern = k_range<HAD, MINMAX>;
     const unsigned grid = grid_for<kern, block, 0>((uint64_t)block * 4, n_chunks);
-    kern<<<grid, block, 0, st>>>(x, n_chunks, ws, out);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, block, 0, st, x, n_chunks, ws, out);
 }
 
 }  // namespace

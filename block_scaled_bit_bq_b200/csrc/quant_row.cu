@@ -24,6 +24,7 @@ namespace bq {
 template <int FMT, bool HAD, bool STATS, int K>
 __global__ void __launch_bounds__(256) k_quant_row(const RowArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     __shared__ float red[2][8][4];
@@ -198,8 +199,7 @@ cudaError_t run_row(const RowArgs& a, int block, cudaStream_t st)
     if (grid > a.rows) grid = a.rows;
     if (grid > (uint64_t)MAX_GRID) grid = MAX_GRID;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, block, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)grid, (unsigned)block, 0, st, a);
 }
 
 template <int FMT, bool HAD, bool STATS>

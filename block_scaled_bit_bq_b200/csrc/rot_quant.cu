@@ -69,6 +69,7 @@ __device__ __forceinline__ float row_sum(float s, float (&red)[2])
 template <int FMT, bool MX, int MB>
 __global__ void __launch_bounds__(RT64_THREADS, 6) k_quant_rt64(const RtArgs a)
 {
+    pdl_wait();
     using F = Fmt<FMT>;
     constexpr int NW = CodeWords<FMT>::n;
     constexpr uint32_t T = 1u << MB, N = 64u * T, RS = 64u / T, CPR = N / 16u;
@@ -276,8 +277,7 @@ cudaError_t run_rt64(const RtArgs& a, cudaStream_t st)
     // every CTA slot busy, the row groups split evenly over them
     const uint64_t groups = ((uint64_t)a.rows + RS - 1) / RS;
     const uint64_t grid = groups < slots ? groups : slots;
-    kern<<<(unsigned)grid, RT64_THREADS, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)grid, (unsigned)RT64_THREADS, smem, st, a);
 }
 
 template <int FMT, bool MX>
