@@ -7,7 +7,11 @@
  * legacy default stream) and results are valid after the caller synchronizes that
  * stream. No entry point allocates device memory, throws, or falls back to the CPU.
  * Argument, shape and alignment checks run on the host before any launch; a failed
- * check launches nothing. A launch failure returns BQ_ERR_CUDA.
+ * check launches nothing. A launch failure returns BQ_ERR_CUDA. The quantize, dequantize
+ * and QSNR kernels are launched with programmatic stream serialization (programmatic
+ * dependent launch): a kernel may become resident while the work ahead of it in the
+ * stream is finishing, but it reads and writes no memory before that work has completed,
+ * so ordinary stream order holds, in eager use and inside CUDA graphs.
  *
  * Method (source pages cited by title and section):
  *  - AbsMax scale s = max|X| / Qmax and Xq = clip(round(X/s), Qmin, Qmax) * s:
