@@ -110,9 +110,11 @@ def test_batch_of_one_and_empty(cuda_device):
     assert e.stats.abs().sum().item() == 0.0
 
 
-@pytest.mark.parametrize("s", [Scheme("int8_sym", "mx"), Scheme("e4m3", "mx")], ids=str)
+@pytest.mark.parametrize("s", [Scheme("int8_sym", "mx"), Scheme("e4m3", "mx"), Scheme("e4m3", "mx", layout="gemm")],
+                         ids=str)
 def test_ffn_batch_full(s, cuda_device):
-    """The 64 FFN tensors of 4096 x 11008 in one call (the bench's launch): every tensor
+    """The 64 FFN tensors of 4096 x 11008 in one call (the bench's launch; with GEMM-layout
+    scales the call runs as several launches of at most 16 MiB of scales): every tensor
     against the one-tensor call; tensors 0 and 63 against the oracle."""
     from concurrent.futures import ThreadPoolExecutor
     with ThreadPoolExecutor(8) as ex:
